@@ -1,0 +1,407 @@
+"""Throughput of the kernelized linear attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload multi_head] [--dtype bf16]
+
+One step is one pass of every form of the path over one batch of the
+workload: non-causal (KV summary + readout), causal (chunked), prefix mask
+(queries binned by m_i) and one decode step on the state the non-causal pass
+produced. The default workload is multi-head attention with B=2, H=8,
+N=4096, d=64 (the lineartile quick-start shape), phi = relu+1, normalized,
+bf16, chunk 64, m_i uniform in [0, N-1].
+
+Tokens counted per step: B*N for each of the three full-sequence forms plus
+B for the decode step. ``value`` is tokens/s over all ranks (weak scaling:
+each rank runs its own batch; the path has no exchange step, so there is no
+data-path collective). Timing: CUDA events around every step on the
+launching stream, L2 flushed (a 256 MiB write) between steps outside the
+events, W untimed warm-up steps, max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from kernelized_linear_attention_phi_b200 import workloads as W  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+
+# Kernels each library call launches (memsets excluded); kept in step with
+# la_api.cu's dispatch and checked against the ncu launch list.
+LAUNCHES = {"noncausal": 3, "causal": 3, "prefix": 4, "decode": 1}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="multi_head")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "f32"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling (NVML reads only; no setting is changed)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            pr = torch.cuda.get_device_properties(device)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _sample(self):
+        self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+        try:
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.reasons |= int(r) & ~0x1
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.nv or not self.samples:
+            return None
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples),
+                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b]}
+
+
+# ---------------------------------------------------------------------------
+# The step
+# ---------------------------------------------------------------------------
+
+class Step:
+    """Device buffers and the four library calls of one step."""
+
+    def __init__(self, wl, dtype, seed, device):
+        from kernelized_linear_attention_phi_b200 import binding as la
+        self.la = la
+        B, H, N, d = wl.B, wl.H, wl.N, wl.d
+        self.wl, self.B, self.H, self.N, self.d = wl, B, H, N, d
+        self.phi, self.normalize, self.chunk = wl.phi, wl.normalize, wl.chunk
+        self.q, self.k, self.v = W.qkv(B, H, N, d, wl.sigma, seed, dtype, device)
+        self.m = W.prefix_mask_uniform(B, N, seed, device)
+        q1, k1, v1 = W.decode_tokens(1, B, H, d, wl.sigma, seed, dtype, device)
+        self.q1, self.k1, self.v1 = q1[0].contiguous(), k1[0].contiguous(), v1[0].contiguous()
+        self.out_nc = torch.empty_like(self.q)
+        self.out_c = torch.empty_like(self.q)
+        self.out_m = torch.empty_like(self.q)
+        self.out_d = torch.empty_like(self.q1)
+        self.S = torch.empty(B, H, d, d, dtype=torch.float32, device=device)
+        self.z = torch.empty(B, H, d, dtype=torch.float32, device=device)
+        desc = la._desc_of(self.q, self.phi, self.normalize)
+        self.ws = {op: la.workspace(desc, op, self.chunk, device) for op in ("noncausal", "causal", "prefix")}
+        self.tokens = 3 * B * N + B
+        self.elem = self.q.element_size()
+
+    def calls(self):
+        la = self.la
+        return [
+            ("noncausal", lambda: la.la_noncausal(self.q, self.k, self.v, self.out_nc, self.S, self.z,
+                                                  self.phi, self.normalize, self.ws["noncausal"])),
+            ("causal", lambda: la.la_causal_chunked(self.q, self.k, self.v, self.out_c, self.chunk,
+                                                    self.phi, self.normalize, self.ws["causal"])),
+            ("prefix", lambda: la.la_prefix_mask(self.q, self.k, self.v, self.m, self.out_m, self.chunk,
+                                                 self.phi, self.normalize, self.ws["prefix"])),
+            ("decode", lambda: la.la_decode_step(self.q1, self.k1, self.v1, self.S, self.z, self.out_d,
+                                                 self.phi, self.normalize)),
+        ]
+
+    def algorithmic_bytes(self):
+        """Bytes each call must move at least: its inputs once and outputs once."""
+        t = self.B * self.H * self.N * self.d * self.elem     # one [B,H,N,d] tensor
+        st = self.B * self.H * (self.d * self.d + self.d) * 4  # fp32 (S, z)
+        one = self.B * self.H * self.d * self.elem
+        return {"noncausal": 4 * t + st, "causal": 4 * t, "prefix": 4 * t + self.B * self.N * 4,
+                "decode": 2 * st + 4 * one}
+
+    def host_io(self):
+        ins = [self.q, self.k, self.v, self.m, self.q1, self.k1, self.v1]
+        outs = [self.out_nc, self.out_c, self.out_m, self.out_d]
+        return ins, outs
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+def run_ours(args, rank, world, local_rank):
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    from kernelized_linear_attention_phi_b200 import build as build_mod
+    if rank == 0 or world == 1:
+        build_mod.build()
+    if world > 1:
+        torch.distributed.barrier()
+    wl = W.WORKLOADS[args.workload]
+    dtype = args.dtype
+    step = Step(wl, dtype, wl.seed + 1000 * rank, device)
+    calls = step.calls()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    for _ in range(max(args.warmup, 3)):
+        for _, fn in calls:
+            fn()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(K)]
+    sampler = ClockSampler(device)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(K):
+            flush_l2(flush)
+            ev[i][0].record(stream)
+            for j, (_, fn) in enumerate(calls):
+                fn()
+                ev[i][j + 1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    per_call = {name: 0.0 for name, _ in calls}
+    total_ms = 0.0
+    for i in range(K):
+        total_ms += ev[i][0].elapsed_time(ev[i][-1])
+        for j, (name, _) in enumerate(calls):
+            per_call[name] += ev[i][j].elapsed_time(ev[i][j + 1])
+    t_s = total_ms / 1e3
+
+    # end to end through the public API: pinned host inputs in, outputs back
+    ins, outs = step.host_io()
+    h_ins = [t.cpu().pin_memory() for t in ins]
+    h_outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in h_ins)
+    d2h = sum(t.numel() * t.element_size() for t in h_outs)
+    Ke = max(1, min(K, 50))
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+    torch.cuda.synchronize()
+    for i in range(Ke):
+        flush_l2(flush)
+        e_ev[i][0].record(stream)
+        for d_t, h_t in zip(ins, h_ins):
+            d_t.copy_(h_t, non_blocking=True)
+        for _, fn in calls:
+            fn()
+        for h_t, d_t in zip(h_outs, outs):
+            h_t.copy_(d_t, non_blocking=True)
+        e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_s = sum(a.elapsed_time(b) for a, b in e_ev) / 1e3
+
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([t_s, e2e_s], dtype=torch.float64, device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_s, e2e_s = float(tt[0]), float(tt[1])
+
+    tokens_all = step.tokens * K * world
+    value = tokens_all / t_s
+    e2e_value = step.tokens * Ke * world / e2e_s
+
+    # roofline of the dominant call (its kernels together), bytes per launch
+    alg = step.algorithmic_bytes()
+    dom = max(per_call, key=per_call.get)
+    dom_s = per_call[dom] / 1e3 / K
+    achieved = alg[dom] / dom_s / 1e9
+    peaks = load_peaks()
+    peak = peaks.get("hbm_gbs", 6650.0)
+    per_kernel = {}
+    for name in per_call:
+        s = per_call[name] / 1e3 / K
+        per_kernel[name] = {"us": round(s * 1e6, 2), "GB_s": round(alg[name] / s / 1e9, 1),
+                            "frac_hbm": round(alg[name] / s / 1e9 / peak, 3),
+                            "share": round(per_call[name] / sum(per_call.values()), 3)}
+
+    result = {
+        "metric": "tokens/sec (fwd, 1xB200) and % of HBM / bf16 tensor-core roofline per kernel",
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": total_ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": dtype,
+        "data": "synthetic",
+        "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} N={wl.N} d={wl.d} {dtype} phi={wl.phi} "
+                               f"normalize={int(wl.normalize)} chunk={wl.chunk}; step = noncausal + "
+                               f"causal + prefix mask (m uniform) + 1 decode step",
+                   "global_batch": wl.B * world, "seq_len": wl.N, "parallelism": f"dp{world}",
+                   "l2": "flushed between steps (256 MiB write)",
+                   "tokens_per_step_per_gpu": step.tokens},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": sum(LAUNCHES[n] for n, _ in calls) * K,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": f"la_{dom} (all its kernels)", "peak_source": peaks.get("_src")},
+        "per_call": per_kernel,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(step, heads=2)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        d["_src"] = "measured (MEASURED_PEAKS.json)"
+        return d
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "_src": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# The oracle on the host cores (CPU baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+def _blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return 1
+
+
+def oracle_sample(q, k, v, m, q1, k1, v1, phi, normalize, heads):
+    """Runs the oracle's four forms on the first `heads` heads of sequence 0.
+    Returns (tokens processed, seconds)."""
+    import oracle
+    f = lambda t: t.detach().to(torch.float64).cpu().numpy()
+    Q, K, V = f(q[0, :heads]), f(k[0, :heads]), f(v[0, :heads])
+    M = m[0].cpu().numpy()
+    q1_, k1_, v1_ = f(q1[0, :heads, 0]), f(k1[0, :heads, 0]), f(v1[0, :heads, 0])
+    t0 = time.perf_counter()
+    for h in range(heads):
+        _, S, z = oracle.noncausal(Q[h], K[h], V[h], phi, normalize)
+        oracle.causal(Q[h], K[h], V[h], phi, normalize)
+        oracle.prefix_mask(Q[h], K[h], V[h], M, phi, normalize)
+        oracle.decode_step(S, z, q1_[h], k1_[h], v1_[h], phi, normalize)
+    dt = time.perf_counter() - t0
+    N = Q.shape[1]
+    # tokens are counted per sequence over all its heads, so a sample of
+    # `heads` heads of one sequence processes heads/H of each sequence's tokens
+    return dt, N, heads
+
+
+def cpu_baseline(step, heads=2):
+    dt, N, h = oracle_sample(step.q, step.k, step.v, step.m, step.q1, step.k1, step.v1,
+                             step.phi, step.normalize, heads)
+    tokens = (3 * N + 1) * h / step.H
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"oracle (numpy fp64) on {h} of {step.H} heads of sequence 0, all four forms, "
+                      f"N={N}; tokens scaled by heads/H; {dt:.2f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl = W.WORKLOADS[args.workload]
+    dtype = args.dtype
+    q, k, v = W.qkv(1, wl.H, wl.N, wl.d, wl.sigma, wl.seed, dtype, "cpu")
+    m = W.prefix_mask_uniform(1, wl.N, wl.seed, "cpu")
+    q1, k1, v1 = (t[0] for t in W.decode_tokens(1, 1, wl.H, wl.d, wl.sigma, wl.seed, dtype, "cpu"))
+    heads = 1
+    for _ in range(args.warmup):
+        oracle_sample(q, k, v, m, q1, k1, v1, wl.phi, wl.normalize, heads)
+    total = 0.0
+    for _ in range(args.steps):
+        dt, N, h = oracle_sample(q, k, v, m, q1, k1, v1, wl.phi, wl.normalize, heads)
+        total += dt
+    tokens = (3 * wl.N + 1) * heads / wl.H * args.steps
+    value = tokens / total
+    cores = _blas_threads()
+    sample = (f"oracle (numpy fp64) on {heads} of {wl.H} heads of one sequence per step, all four "
+              f"forms, N={wl.N}; tokens scaled by heads/H")
+    print(json.dumps({
+        "impl": "reference",
+        "metric": "tokens/sec (fwd, 1xB200) and % of HBM / bf16 tensor-core roofline per kernel",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} N={wl.N} d={wl.d} {dtype} inputs",
+                   "global_batch": wl.B, "seq_len": wl.N, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,164 @@
+/*
+ * la.h -- C ABI of the B200 (sm_100a) kernelized linear attention library
+ *         (libla_b200.so).
+ *
+ * The method. A positive feature map phi is applied to queries and keys.
+ * The keys and values of a head are folded into the KV summary
+ *     S = sum_j phi(K_j) (x) V_j      (d x d, row-major S[a*d + b])
+ *     z = sum_j phi(K_j)              (d)
+ * and each query reads out
+ *     out_i = phi(Q_i) S / (phi(Q_i) . z)        (normalize = 1)
+ *     out_i = phi(Q_i) S                         (normalize = 0)
+ * with no 1/sqrt(d) scale and no epsilon. Sources:
+ *   - "nx_f32_linear_attention.nx source": header comment (definitions of phi,
+ *     S, z, out), function la_phi (phi = relu(x)+1, relu by the sign bit),
+ *     the KV-summary loop and the per-query loop;
+ *   - "trim-transformer 0.1.0": introduction (unnormalized Q K^T V with the
+ *     identity map), "Masking" (query i sees keys 0..m_i, m_i in [0, n-1];
+ *     causal = arange(n)), "Key-value caching" (decode on a stored state);
+ *   - "lineartile 1.0.1", "How It Works" (O = phi(Q)(phi(K)^T V)).
+ *
+ * Conventions shared by every entry point.
+ *   - Tensors q, k, v, out are dense, contiguous [B, H, N, d] in the element
+ *     type desc->dtype (out has the same type as the inputs). d_k = d_v = d.
+ *   - S and z are float32: S [B, H, d, d] row-major per head, z [B, H, d].
+ *   - All pointers are device pointers owned by the caller, 16-byte aligned.
+ *     The library never allocates device memory and keeps no pointer after
+ *     a call returns; scratch space is the caller's workspace (ws), sized by
+ *     la_workspace_size().
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream). Buffers must stay valid until the stream
+ *     reaches the call's work.
+ *   - Validation is fail-closed: on any status other than LA_OK nothing was
+ *     launched, except LA_ERR_CUDA, which reports a failed launch.
+ *   - Supported: d in {16, 32, 64, 128}; dtype LA_F32 or LA_BF16;
+ *     phi LA_PHI_RELU1 or LA_PHI_IDENTITY; normalize in {0, 1}, with
+ *     normalize = 1 only for LA_PHI_RELU1 (with the identity map the
+ *     denominator phi(q).z can be zero or negative). Device: compute
+ *     capability 10.x (B200).
+ *   - Results are deterministic: every reduction runs in a fixed order, so
+ *     repeated calls on the same inputs give bit-identical outputs.
+ */
+#ifndef LA_B200_H
+#define LA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LA_API __attribute__((visibility("default")))
+#else
+#define LA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = 1,  /* NULL pointer, size <= 0, unknown enum value */
+    LA_ERR_UNSUPPORTED = 2,  /* valid request outside the supported set, or not a CC 10.x device */
+    LA_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
+    LA_ERR_WORKSPACE = 4,    /* ws is NULL or smaller than la_workspace_size() */
+    LA_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */
+    LA_ERR_MASK_RANGE = 6    /* (la_last_error) some m_i was outside [0, N-1] */
+} la_status;
+
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+
+typedef enum {
+    LA_PHI_RELU1 = 0,    /* phi(x) = relu(x) + 1, relu by the sign bit (-0.0 -> 1) */
+    LA_PHI_IDENTITY = 1  /* phi(x) = x (unnormalized Q K^T V form) */
+} la_phi;
+
+typedef enum {
+    LA_OP_KV_SUMMARY = 0,
+    LA_OP_NONCAUSAL = 1,
+    LA_OP_CAUSAL = 2,
+    LA_OP_PREFIX = 3,
+    LA_OP_DECODE = 4
+} la_op;
+
+/* Problem description. d is both d_k and d_v. */
+typedef struct {
+    int32_t B, H, N, d;
+    int32_t dtype;      /* la_dtype */
+    int32_t phi;        /* la_phi */
+    int32_t normalize;  /* 1: divide by phi(q).z; 0: unnormalized */
+} la_desc;
+
+/* Bytes of workspace `op` needs for `desc` (chunk is used by LA_OP_CAUSAL and
+ * LA_OP_PREFIX only). Returns 0 when the request is invalid or unsupported,
+ * and for ops that need none (LA_OP_DECODE). A valid request that needs a
+ * workspace always gets a non-zero size. Pure host function. */
+LA_API size_t la_workspace_size(const la_desc* desc, int32_t op, int32_t chunk);
+
+/* KV summary of every head (nx source, KV-summary loop):
+ *   S[b,h] = sum_j phi(K[b,h,j]) (x) V[b,h,j],  z[b,h] = sum_j phi(K[b,h,j]).
+ * k, v: [B,H,N,d] inputs. S_out [B,H,d,d], z_out [B,H,d]: float32 outputs,
+ * overwritten. desc->normalize is ignored. This is the prefill of a decode
+ * state. */
+LA_API la_status la_kv_summary(const la_desc* desc, const void* k, const void* v,
+                        float* S_out, float* z_out,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* Non-causal attention: every query sees every key of its head.
+ *   out_i = phi(q_i) S / (phi(q_i) . z)   (or the numerator alone).
+ * q, k, v: [B,H,N,d] inputs; out: [B,H,N,d] output.
+ * S_out, z_out: optional (may be NULL) float32 outputs receiving the KV
+ * summary used, so that a decode can continue from it. */
+LA_API la_status la_noncausal(const la_desc* desc, const void* q, const void* k,
+                       const void* v, void* out, float* S_out, float* z_out,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Causal attention: query i sees keys 0..i (inclusive; trim-transformer
+ * "Masking": the causal mask is arange(n)). Computed chunk by chunk: the
+ * intra-chunk part (phi(Q_c) phi(K_c)^T, lower triangle with diagonal) times
+ * V_c, plus phi(Q_c) times the state of all earlier chunks.
+ * chunk: 64 or 128 tokens. The result does not depend on it beyond rounding.
+ * q, k, v: [B,H,N,d] inputs; out: [B,H,N,d] output. */
+LA_API la_status la_causal_chunked(const la_desc* desc, int32_t chunk, const void* q,
+                            const void* k, const void* v, void* out,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Prefix-mask attention (trim-transformer 0.1.0, "Masking"): query i of
+ * sequence b sees keys 0..m[b*N + i], inclusive. m: int32 [B, N] device
+ * array with values in [0, N-1], one mask per sequence shared by its heads.
+ * An m_i outside that range is clamped into it and recorded in the
+ * workspace's error word (read it with la_last_error). m = arange(N) is the
+ * causal mask; m = N-1 everywhere is non-causal.
+ * chunk: 64 or 128 (queries are binned by floor((m_i+1)/chunk)). */
+LA_API la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q,
+                         const void* k, const void* v, const int32_t* m,
+                         void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* One recurrent decode step for every (b, h), on a cached state
+ * (trim-transformer 0.1.0, "Key-value caching"; update first, so the new
+ * token sees itself):
+ *   S += phi(k) (x) v;  z += phi(k);  out = phi(q) S / (phi(q) . z).
+ * q, k, v: [B,H,1,d] inputs (desc->N is ignored); S [B,H,d,d] and
+ * z [B,H,d]: float32 state, updated in place; out: [B,H,1,d] output.
+ * Zero-filled S and z are the empty cache. Needs no workspace. */
+LA_API la_status la_decode_step(const la_desc* desc, const void* q, const void* k,
+                         const void* v, float* S, float* z, void* out,
+                         void* stream);
+
+/* Waits for `stream`, then reads and clears the error word of workspace `ws`
+ * (written by la_prefix_mask). *flags_out (may be NULL) receives the raw
+ * bits: bit 0 = a mask value was out of range. Returns LA_ERR_MASK_RANGE
+ * when bit 0 was set, LA_OK when no bit was set, LA_ERR_CUDA on a CUDA
+ * failure. */
+LA_API la_status la_last_error(void* ws, void* stream, uint32_t* flags_out);
+
+/* Static string naming a status. */
+LA_API const char* la_status_string(la_status status);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+LA_API int32_t la_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_B200_H */

@@ -1,0 +1,61 @@
+// Internal interfaces between the host API (la_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace la {
+
+struct Problem {
+    int B, H, N, d;
+    int dtype;      // DT_F32 / DT_BF16
+    int phi;        // PHI_RELU1 / PHI_IDENTITY
+    int normalize;  // 0 / 1
+    long long bh() const { return (long long)B * H; }
+    size_t elem_bytes() const { return dtype == 0 ? 4 : 2; }
+    // floats in one (S, z) state record: S (d*d) followed by z (d)
+    size_t state_floats() const { return (size_t)d * d + d; }
+};
+
+// ---- CUDA-core kernels (simt.cu) -------------------------------------------
+// Partial KV summaries. Head bh, split s covers tokens
+// [s*tokens_per_split, min(N, (s+1)*tokens_per_split)) and writes the state
+// record part[(bh*nsplit + s) * state_floats()].
+cudaError_t simt_kv_partial(const Problem& p, const void* k, const void* v, int tokens_per_split,
+                            int nsplit, float* part, cudaStream_t st);
+// Sums the nsplit records of each head in split order into S [bh][d*d] and
+// z [bh][d].
+cudaError_t state_reduce(const Problem& p, const float* part, int nsplit, float* S, float* z,
+                         cudaStream_t st);
+// In place: record b of each head becomes the sum of records 0..b-1 (zero for
+// b = 0). If S_total/z_total are non-null they receive the sum of all records.
+cudaError_t state_exclusive_scan(const Problem& p, float* part, int nblk, float* S_total,
+                                 float* z_total, cudaStream_t st);
+// out = phi(q) S / (phi(q).z) (or numerator only) for every token.
+cudaError_t simt_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,
+                         cudaStream_t st);
+// Chunked causal / prefix-mask outputs. Block blk of head bh covers tokens
+// [blk*block_tokens, ...) and starts from record blk of `prefix` (the state of
+// all earlier keys). With perm == nullptr the queries of chunk c are the
+// tokens of chunk c (causal); otherwise the queries answered at chunk c are
+// perm[b*N + bin_start[b*(nbins+1) + c] ...] with key limits m.
+cudaError_t simt_chunked(const Problem& p, const void* q, const void* k, const void* v,
+                         const float* prefix, int block_tokens, int nblk, const int32_t* perm,
+                         const int32_t* bin_start, const int32_t* m, int nbins, void* out,
+                         cudaStream_t st);
+
+// ---- prefix-mask binning (bin.cu) -------------------------------------------
+// For each sequence b: clamp m into [0, N-1] (setting FLAG_MASK_RANGE in
+// *flags when it had to), bin query i by floor((m_i + 1) / chunk) and write a
+// counting-sort permutation perm[b*N ...] plus bin offsets
+// bin_start[b*(nbins+1) ...] (nbins = N / chunk + 1). mclamped receives the
+// clamped mask.
+cudaError_t bin_queries(const Problem& p, const int32_t* m, int chunk, int nbins, int32_t* perm,
+                        int32_t* bin_start, int32_t* mclamped, uint32_t* flags, cudaStream_t st);
+
+// ---- decode (decode.cu) -------------------------------------------------------
+cudaError_t decode_step(const Problem& p, const void* q, const void* k, const void* v, float* S,
+                        float* z, void* out, cudaStream_t st);
+
+}  // namespace la

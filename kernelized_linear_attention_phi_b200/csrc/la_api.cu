@@ -1,0 +1,315 @@
+// C ABI of libla_b200 (declared in include/la.h): argument validation,
+// workspace planning and kernel dispatch. Validation is fail-closed: a bad
+// request returns a status before anything is launched.
+
+#include <la.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.h"
+
+namespace la {
+namespace {
+
+constexpr int kSimtChunk = 64;     // chunk length the SIMT chunked kernel runs at
+constexpr int kNumSMs = 148;       // B200
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+la_status check_desc(const la_desc* d) {
+    if (d == nullptr) return LA_ERR_INVALID_ARG;
+    if (d->B <= 0 || d->H <= 0 || d->N <= 0 || d->d <= 0) return LA_ERR_INVALID_ARG;
+    if (d->dtype != LA_F32 && d->dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (d->phi != LA_PHI_RELU1 && d->phi != LA_PHI_IDENTITY) return LA_ERR_INVALID_ARG;
+    if (d->normalize != 0 && d->normalize != 1) return LA_ERR_INVALID_ARG;
+    if (d->d != 16 && d->d != 32 && d->d != 64 && d->d != 128) return LA_ERR_UNSUPPORTED;
+    if (d->normalize == 1 && d->phi == LA_PHI_IDENTITY) return LA_ERR_UNSUPPORTED;
+    if ((long long)d->B * d->H > 65535) return LA_ERR_UNSUPPORTED;  // grid.y limit
+    if ((long long)d->B * d->H * d->N * d->d > (1LL << 40)) return LA_ERR_UNSUPPORTED;
+    return LA_OK;
+}
+
+la_status check_chunk(int chunk) { return (chunk == 64 || chunk == 128) ? LA_OK : LA_ERR_UNSUPPORTED; }
+
+// The library's kernels are built for sm_100a only.
+la_status check_device() {
+    static std::atomic<uint64_t> ok{0}, bad{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    const uint64_t bit = 1ull << (dev & 63);
+    if (ok.load() & bit) return LA_OK;
+    if (bad.load() & bit) return LA_ERR_UNSUPPORTED;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    if (major != 10) {
+        bad.fetch_or(bit);
+        return LA_ERR_UNSUPPORTED;
+    }
+    ok.fetch_or(bit);
+    return LA_OK;
+}
+
+Problem to_problem(const la_desc* d) {
+    return Problem{d->B, d->H, d->N, d->d, d->dtype, d->phi, d->normalize};
+}
+
+// ---- work plans (pure functions of the problem, shared by sizing and launch) ----
+
+struct SplitPlan {
+    int nsplit, tps;  // splits per head, tokens per split
+};
+SplitPlan kv_plan(const Problem& p) {
+    const long long target = std::max(1LL, cdiv(2 * kNumSMs, p.bh()));
+    const long long max_splits = std::max(1LL, cdiv(p.N, 256));
+    long long ns = std::min(target, max_splits);
+    const long long tps = (long long)round_up((size_t)cdiv(p.N, ns), 128);
+    ns = cdiv(p.N, tps);
+    return SplitPlan{(int)ns, (int)tps};
+}
+
+struct BlockPlan {
+    int block_tokens, nblk;
+};
+BlockPlan block_plan(const Problem& p) {
+    const long long target = std::max(1LL, cdiv(2 * kNumSMs, p.bh()));
+    long long bt = (long long)round_up((size_t)cdiv(p.N, target), 128);
+    bt = std::max(bt, 256LL);
+    return BlockPlan{(int)bt, (int)cdiv(p.N, bt)};
+}
+
+int prefix_nbins(const Problem& p, int kchunk) { return p.N / kchunk + 1; }
+
+struct WsLayout {
+    size_t part = 0, sz = 0, perm = 0, mcl = 0, bins = 0, total = 0;
+};
+
+WsLayout ws_layout(const Problem& p, int op) {
+    WsLayout L;
+    size_t off = WS_HEADER;
+    const size_t rec = p.state_floats() * sizeof(float);
+    if (op == LA_OP_KV_SUMMARY || op == LA_OP_NONCAUSAL) {
+        const SplitPlan sp = kv_plan(p);
+        L.part = off;
+        off = round_up(off + (size_t)p.bh() * sp.nsplit * rec, kAlign);
+        if (op == LA_OP_NONCAUSAL) {
+            L.sz = off;
+            off = round_up(off + (size_t)p.bh() * rec, kAlign);
+        }
+    } else if (op == LA_OP_CAUSAL || op == LA_OP_PREFIX) {
+        const BlockPlan bp = block_plan(p);
+        L.part = off;
+        off = round_up(off + (size_t)p.bh() * bp.nblk * rec, kAlign);
+        if (op == LA_OP_PREFIX) {
+            const int nbins = prefix_nbins(p, kSimtChunk);
+            L.perm = off;
+            off = round_up(off + sizeof(int32_t) * (size_t)p.B * p.N, kAlign);
+            L.mcl = off;
+            off = round_up(off + sizeof(int32_t) * (size_t)p.B * p.N, kAlign);
+            L.bins = off;
+            off = round_up(off + sizeof(int32_t) * (size_t)p.B * (nbins + 1), kAlign);
+        }
+    } else {
+        return L;
+    }
+    L.total = off;
+    return L;
+}
+
+template <typename P>
+P* at(void* ws, size_t off) {
+    return reinterpret_cast<P*>(static_cast<char*>(ws) + off);
+}
+
+la_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return LA_OK;
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+}
+
+la_status check_ws(const WsLayout& L, void* ws, size_t ws_bytes) {
+    if (ws == nullptr || ws_bytes < L.total) return LA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return LA_ERR_MISALIGNED;
+    return LA_OK;
+}
+
+#define LA_TRY(expr)                      \
+    do {                                  \
+        la_status s__ = (expr);           \
+        if (s__ != LA_OK) return s__;     \
+    } while (0)
+
+la_status kv_summary_impl(const Problem& p, const void* k, const void* v, float* S, float* z,
+                          void* ws, cudaStream_t st) {
+    const SplitPlan sp = kv_plan(p);
+    float* part = at<float>(ws, ws_layout(p, LA_OP_KV_SUMMARY).part);
+    if (tc_supported(p)) {
+        LA_TRY(cuda_status(tc_kv_partial(p, k, v, sp.tps, sp.nsplit, part, st)));
+    } else {
+        LA_TRY(cuda_status(simt_kv_partial(p, k, v, sp.tps, sp.nsplit, part, st)));
+    }
+    return cuda_status(state_reduce(p, part, sp.nsplit, S, z, st));
+}
+
+}  // namespace
+}  // namespace la
+
+using namespace la;
+
+extern "C" {
+
+int32_t la_version(void) { return 100; }
+
+const char* la_status_string(la_status s) {
+    switch (s) {
+        case LA_OK: return "LA_OK";
+        case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED";
+        case LA_ERR_MISALIGNED: return "LA_ERR_MISALIGNED";
+        case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA";
+        case LA_ERR_MASK_RANGE: return "LA_ERR_MASK_RANGE";
+    }
+    return "LA_ERR_UNKNOWN";
+}
+
+size_t la_workspace_size(const la_desc* desc, int32_t op, int32_t chunk) {
+    if (check_desc(desc) != LA_OK) return 0;
+    if ((op == LA_OP_CAUSAL || op == LA_OP_PREFIX) && check_chunk(chunk) != LA_OK) return 0;
+    if (op < LA_OP_KV_SUMMARY || op > LA_OP_DECODE) return 0;
+    return ws_layout(to_problem(desc), op).total;
+}
+
+la_status la_kv_summary(const la_desc* desc, const void* k, const void* v, float* S_out,
+                        float* z_out, void* ws, size_t ws_bytes, void* stream) {
+    LA_TRY(check_desc(desc));
+    if (!k || !v || !S_out || !z_out) return LA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(S_out) || !aligned16(z_out))
+        return LA_ERR_MISALIGNED;
+    const Problem p = to_problem(desc);
+    LA_TRY(check_ws(ws_layout(p, LA_OP_KV_SUMMARY), ws, ws_bytes));
+    LA_TRY(check_device());
+    return kv_summary_impl(p, k, v, S_out, z_out, ws, static_cast<cudaStream_t>(stream));
+}
+
+la_status la_noncausal(const la_desc* desc, const void* q, const void* k, const void* v, void* out,
+                       float* S_out, float* z_out, void* ws, size_t ws_bytes, void* stream) {
+    LA_TRY(check_desc(desc));
+    if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
+    if ((S_out == nullptr) != (z_out == nullptr)) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_MISALIGNED;
+    if (S_out && (!aligned16(S_out) || !aligned16(z_out))) return LA_ERR_MISALIGNED;
+    const Problem p = to_problem(desc);
+    const WsLayout L = ws_layout(p, LA_OP_NONCAUSAL);
+    LA_TRY(check_ws(L, ws, ws_bytes));
+    LA_TRY(check_device());
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* S = S_out;
+    float* z = z_out;
+    if (S == nullptr) {
+        S = at<float>(ws, L.sz);
+        z = S + (size_t)p.bh() * p.d * p.d;
+    }
+    LA_TRY(kv_summary_impl(p, k, v, S, z, ws, st));
+    if (tc_supported(p)) return cuda_status(tc_readout(p, q, S, z, out, st));
+    return cuda_status(simt_readout(p, q, S, z, out, st));
+}
+
+la_status la_causal_chunked(const la_desc* desc, int32_t chunk, const void* q, const void* k,
+                            const void* v, void* out, void* ws, size_t ws_bytes, void* stream) {
+    LA_TRY(check_desc(desc));
+    LA_TRY(check_chunk(chunk));
+    if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_MISALIGNED;
+    const Problem p = to_problem(desc);
+    const WsLayout L = ws_layout(p, LA_OP_CAUSAL);
+    LA_TRY(check_ws(L, ws, ws_bytes));
+    LA_TRY(check_device());
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const BlockPlan bp = block_plan(p);
+    float* part = at<float>(ws, L.part);
+    // phase 1: per-block states; phase 2: exclusive prefix over blocks;
+    // phase 3: each block's outputs from its prefix state.
+    if (tc_supported(p)) {
+        LA_TRY(cuda_status(tc_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
+    } else {
+        LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
+    }
+    LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
+    if (tc_supported(p))
+        return cuda_status(tc_causal(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, out, st));
+    return cuda_status(simt_chunked(p, q, k, v, part, bp.block_tokens, bp.nblk, nullptr, nullptr,
+                                    nullptr, 0, out, st));
+}
+
+la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, const void* k,
+                         const void* v, const int32_t* m, void* out, void* ws, size_t ws_bytes,
+                         void* stream) {
+    LA_TRY(check_desc(desc));
+    LA_TRY(check_chunk(chunk));
+    if (!q || !k || !v || !m || !out) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(m))
+        return LA_ERR_MISALIGNED;
+    const Problem p = to_problem(desc);
+    if (p.N > (1 << 21)) return LA_ERR_UNSUPPORTED;  // bin table must fit in shared memory
+    const WsLayout L = ws_layout(p, LA_OP_PREFIX);
+    LA_TRY(check_ws(L, ws, ws_bytes));
+    LA_TRY(check_device());
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const BlockPlan bp = block_plan(p);
+    const int nbins = prefix_nbins(p, kSimtChunk);
+    uint32_t* flags = at<uint32_t>(ws, 0);
+    int32_t* perm = at<int32_t>(ws, L.perm);
+    int32_t* mcl = at<int32_t>(ws, L.mcl);
+    int32_t* bins = at<int32_t>(ws, L.bins);
+    float* part = at<float>(ws, L.part);
+    LA_TRY(cuda_status(cudaMemsetAsync(flags, 0, sizeof(uint32_t), st)));
+    LA_TRY(cuda_status(bin_queries(p, m, kSimtChunk, nbins, perm, bins, mcl, flags, st)));
+    LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
+    LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
+    return cuda_status(simt_chunked(p, q, k, v, part, bp.block_tokens, bp.nblk, perm, bins, mcl,
+                                    nbins, out, st));
+}
+
+la_status la_decode_step(const la_desc* desc, const void* q, const void* k, const void* v, float* S,
+                         float* z, void* out, void* stream) {
+    if (desc == nullptr) return LA_ERR_INVALID_ARG;
+    la_desc d1 = *desc;
+    d1.N = 1;  // N is not used by a decode step
+    LA_TRY(check_desc(&d1));
+    if (!q || !k || !v || !S || !z || !out) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(S) || !aligned16(z) ||
+        !aligned16(out))
+        return LA_ERR_MISALIGNED;
+    LA_TRY(check_device());
+    return cuda_status(decode_step(to_problem(&d1), q, k, v, S, z, out,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+la_status la_last_error(void* ws, void* stream, uint32_t* flags_out) {
+    if (ws == nullptr) return LA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t host = 0;
+    LA_TRY(cuda_status(cudaMemcpyAsync(&host, ws, sizeof(uint32_t), cudaMemcpyDeviceToHost, st)));
+    LA_TRY(cuda_status(cudaMemsetAsync(ws, 0, sizeof(uint32_t), st)));
+    LA_TRY(cuda_status(cudaStreamSynchronize(st)));
+    if (flags_out) *flags_out = host;
+    if (host & FLAG_MASK_RANGE) return LA_ERR_MASK_RANGE;
+    return LA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,21 @@
+// Tensor-core (tcgen05 / TMEM / TMA) kernels for bf16 inputs, d in {64, 128}.
+#pragma once
+
+#include "internal.h"
+
+namespace la {
+
+// True when the tcgen05 path handles this problem (bf16, d = 64 or 128).
+bool tc_supported(const Problem& p);
+
+// Same contract as simt_kv_partial.
+cudaError_t tc_kv_partial(const Problem& p, const void* k, const void* v, int tokens_per_split,
+                          int nsplit, float* part, cudaStream_t st);
+// Same contract as simt_readout.
+cudaError_t tc_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,
+                       cudaStream_t st);
+// Causal outputs of every block from its prefix state (chunk 64 or 128).
+cudaError_t tc_causal(const Problem& p, int chunk, const void* q, const void* k, const void* v,
+                      const float* prefix, int block_tokens, int nblk, void* out, cudaStream_t st);
+
+}  // namespace la

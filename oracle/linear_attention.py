@@ -151,10 +151,11 @@ def attention_rows(Q, K, V, rows, form=FORM_NONCAUSAL, m=None,
     Q, K, V = _f64(Q), _f64(K), _f64(V)
     n = Q.shape[0]
     lim = key_limits(n, form, m)
+    pk = phi(K, phi_kind)
     out = np.empty((len(rows), V.shape[1]))
     for r, i in enumerate(rows):
         last = int(lim[i])
-        w = phi(K[: last + 1], phi_kind) @ phi(Q[i], phi_kind)
+        w = pk[: last + 1] @ phi(Q[i], phi_kind)
         num = w @ V[: last + 1]
         out[r] = num / w.sum() if normalize else num
     return out

@@ -1,0 +1,111 @@
+"""C ABI checks that need no GPU: the library loads, exports every symbol
+include/la.h declares, sizes workspaces, and rejects bad requests before it
+touches the device (fail-closed validation)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from kernelized_linear_attention_phi_b200 import binding as B
+from kernelized_linear_attention_phi_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "la.h")).read()
+    return sorted(set(re.findall(r"LA_API\s+[\w\s\*]+?\b(la_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("la_kv_summary", "la_noncausal", "la_causal_chunked", "la_prefix_mask",
+              "la_decode_step", "la_workspace_size", "la_last_error", "la_status_string",
+              "la_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    # and nothing else: internal symbols stay hidden
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = sorted(l.split()[-1] for l in out.splitlines() if l.strip())
+    assert exported == declared_functions()
+
+
+def test_status_strings(lib):
+    for code, name in B.STATUS_NAMES.items():
+        assert B.la_status_string(code) == name
+    assert B.la_version() == 100
+
+
+def desc(B_=2, H=3, N=100, d=64, dtype=1, phi=0, normalize=1):
+    return B.la_desc(B_, H, N, d, dtype, phi, normalize)
+
+
+def test_workspace_sizes(lib):
+    for op in ("kv_summary", "noncausal", "causal", "prefix"):
+        for d in (16, 32, 64, 128):
+            n = B.la_workspace_size(desc(d=d), op, 64)
+            assert n > 0 and n % 256 == 0
+    assert B.la_workspace_size(desc(), "decode", 64) == 0
+    # the state records dominate: at least one (S, z) record per head
+    assert B.la_workspace_size(desc(d=128), "kv_summary") >= 2 * 3 * (128 * 128 + 128) * 4
+    # invalid or unsupported requests size to 0
+    assert B.la_workspace_size(desc(d=48), "noncausal") == 0
+    assert B.la_workspace_size(desc(phi=1, normalize=1), "noncausal") == 0
+    assert B.la_workspace_size(desc(N=0), "noncausal") == 0
+    assert B.la_workspace_size(desc(), "causal", 96) == 0
+    assert B.la_workspace_size(desc(), 7, 64) == 0
+
+
+P16 = ctypes.c_void_p(1 << 20)          # an aligned, never-dereferenced address
+P_MIS = ctypes.c_void_p((1 << 20) + 4)  # misaligned
+NULL = None
+
+
+def call_noncausal(lib, dsc, q=P16, ws_bytes=1 << 30, ws=P16):
+    return lib.la_noncausal(ctypes.byref(dsc), q, P16, P16, P16, NULL, NULL, ws, ws_bytes, NULL)
+
+
+def test_validation_statuses(lib):
+    assert lib.la_noncausal(None, P16, P16, P16, P16, NULL, NULL, P16, 1 << 30, NULL) == 1
+    assert call_noncausal(lib, desc(d=48)) == 2
+    assert call_noncausal(lib, desc(phi=1, normalize=1)) == 2
+    assert call_noncausal(lib, desc(N=0)) == 1
+    assert call_noncausal(lib, desc(dtype=5)) == 1
+    assert call_noncausal(lib, desc(normalize=2)) == 1
+    assert call_noncausal(lib, desc(), q=NULL) == 1
+    assert call_noncausal(lib, desc(), q=P_MIS) == 3
+    assert call_noncausal(lib, desc(), ws_bytes=16) == 4
+    assert call_noncausal(lib, desc(), ws=NULL) == 4
+    dsc = desc()
+    # causal / prefix chunk values
+    assert lib.la_causal_chunked(ctypes.byref(dsc), 96, P16, P16, P16, P16, P16, 1 << 30, NULL) == 2
+    assert lib.la_prefix_mask(ctypes.byref(dsc), 32, P16, P16, P16, P16, P16, P16, 1 << 30, NULL) == 2
+    assert lib.la_prefix_mask(ctypes.byref(dsc), 64, P16, P16, P16, NULL, P16, P16, 1 << 30, NULL) == 1
+    assert lib.la_prefix_mask(ctypes.byref(dsc), 64, P16, P16, P16, P_MIS, P16, P16, 1 << 30, NULL) == 3
+    # decode: N is ignored, other fields validated
+    assert lib.la_decode_step(ctypes.byref(desc(N=0)), P16, P16, P16, P16, P16, P_MIS, NULL) == 3
+    assert lib.la_decode_step(ctypes.byref(desc(d=8)), P16, P16, P16, P16, P16, P16, NULL) == 2
+    assert lib.la_kv_summary(ctypes.byref(dsc), P16, P16, NULL, P16, P16, 1 << 30, NULL) == 1
+    assert lib.la_last_error(NULL, NULL, None) == 1
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful on a machine with no GPU")
+def test_valid_request_without_gpu_reports_cuda_error(lib):
+    """A request that passes validation reaches the device check, which fails
+    cleanly with LA_ERR_CUDA when no GPU is present (nothing is launched)."""
+    assert call_noncausal(lib, desc()) == 5

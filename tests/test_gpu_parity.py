@@ -1,0 +1,200 @@
+"""GPU results against the fp64 oracle, element by element, at sizes the
+oracle finishes in seconds: several tiles, ragged tails, every head size and
+element type, and the edge cases (N = 1, degenerate masks, empty cache,
+out-of-range mask values)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kernelized_linear_attention_phi_b200 import binding as la
+from kernelized_linear_attention_phi_b200 import workloads
+
+from gpu_util import DT, TOL, f64, qkv
+
+pytestmark = pytest.mark.gpu
+
+DS = (16, 32, 64, 128)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from kernelized_linear_attention_phi_b200 import build
+    build.build()
+    la.lib()
+
+
+def _modes():
+    return [("relu1", True), ("relu1", False), ("identity", False)]
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("d", DS)
+@pytest.mark.parametrize("N", [1, 77, 1000])
+@pytest.mark.parametrize("phi,normalize", _modes())
+def test_noncausal(dt, d, N, phi, normalize):
+    sigma = 1.0 if phi == "relu1" else d ** -0.5
+    q, k, v = qkv(2, 3, N, d, dt, seed=N + d, sigma=sigma)
+    S = torch.empty(2, 3, d, d, device="cuda")
+    z = torch.empty(2, 3, d, device="cuda")
+    out = la.la_noncausal(q, k, v, S_out=S, z_out=z, phi=phi, normalize=normalize)
+    Q, K, V = f64(q), f64(k), f64(v)
+    ref = oracle.batched(oracle.noncausal, Q, K, V, phi_kind=phi, normalize=normalize)
+    assert oracle.max_row_rel_err(f64(out), ref) < TOL[DT[dt]]
+    S_ref, z_ref = oracle.kv_summary_batched(K, V, phi)
+    assert oracle.max_row_rel_err(f64(S), S_ref) < 1e-5
+    assert oracle.max_row_rel_err(f64(z)[..., None, :], z_ref[..., None, :]) < 1e-5
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("d", DS)
+@pytest.mark.parametrize("N", [1, 300, 777])
+def test_kv_summary(dt, d, N):
+    _, k, v = qkv(1, 2, N, d, dt, seed=7 * N + d)
+    S, z = la.la_kv_summary(k, v)
+    S_ref, z_ref = oracle.kv_summary_batched(f64(k), f64(v))
+    assert oracle.max_row_rel_err(f64(S), S_ref) < 1e-5
+    np.testing.assert_allclose(f64(z), z_ref, rtol=1e-5)
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("d", DS)
+@pytest.mark.parametrize("N", [1, 63, 130, 700])
+@pytest.mark.parametrize("chunk", [64, 128])
+@pytest.mark.parametrize("phi,normalize", [("relu1", True), ("identity", False)])
+def test_causal(dt, d, N, chunk, phi, normalize):
+    sigma = 1.0 if phi == "relu1" else d ** -0.5
+    q, k, v = qkv(1, 3, N, d, dt, seed=3 * N + d, sigma=sigma)
+    out = la.la_causal_chunked(q, k, v, chunk=chunk, phi=phi, normalize=normalize)
+    ref = oracle.batched(oracle.causal, f64(q), f64(k), f64(v), phi_kind=phi, normalize=normalize)
+    assert oracle.max_row_rel_err(f64(out), ref) < TOL[DT[dt]]
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("d", DS)
+@pytest.mark.parametrize("N", [1, 129, 640])
+@pytest.mark.parametrize("phi,normalize", [("relu1", True), ("identity", False)])
+def test_prefix_mask_uniform(dt, d, N, phi, normalize):
+    sigma = 1.0 if phi == "relu1" else d ** -0.5
+    B = 2
+    q, k, v = qkv(B, 2, N, d, dt, seed=5 * N + d, sigma=sigma)
+    m = workloads.prefix_mask_uniform(B, N, seed=N, device="cuda")
+    ws = la.workspace(la._desc_of(q, phi, normalize), "prefix", 64)
+    out = la.la_prefix_mask(q, k, v, m, phi=phi, normalize=normalize, ws=ws)
+    assert la.la_last_error(ws) == (0, 0)
+    ref = oracle.batched(oracle.prefix_mask, f64(q), f64(k), f64(v), phi_kind=phi,
+                         normalize=normalize, m=m.cpu().numpy())
+    assert oracle.max_row_rel_err(f64(out), ref) < TOL[DT[dt]]
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("kind", ["zeros", "last", "arange", "blocks"])
+def test_prefix_mask_degenerate(dt, kind):
+    B, H, N, d = 2, 2, 300, 64
+    q, k, v = qkv(B, H, N, d, dt, seed=11)
+    if kind == "zeros":
+        m = torch.zeros(B, N, dtype=torch.int32, device="cuda")
+    elif kind == "last":
+        m = torch.full((B, N), N - 1, dtype=torch.int32, device="cuda")
+    elif kind == "arange":
+        m = workloads.prefix_mask_arange(B, N, device="cuda")
+    else:  # every query's limit at a chunk edge, including -1 partial chunks
+        m = (torch.arange(N, device="cuda", dtype=torch.int32) // 64 * 64 + 63).clamp(max=N - 1)
+        m = m.repeat(B, 1).contiguous()
+    out = la.la_prefix_mask(q, k, v, m)
+    ref = oracle.batched(oracle.prefix_mask, f64(q), f64(k), f64(v), m=m.cpu().numpy())
+    assert oracle.max_row_rel_err(f64(out), ref) < TOL[DT[dt]]
+    if kind == "last":
+        nc = la.la_noncausal(q, k, v)
+        assert oracle.max_row_rel_err(f64(out), f64(nc)) < TOL[DT[dt]]
+    if kind == "arange":
+        c = la.la_causal_chunked(q, k, v)
+        assert oracle.max_row_rel_err(f64(out), f64(c)) < TOL[DT[dt]]
+
+
+def test_prefix_mask_out_of_range_is_clamped_and_flagged():
+    B, H, N, d = 1, 2, 200, 32
+    q, k, v = qkv(B, H, N, d, "f32", seed=12)
+    m = workloads.prefix_mask_uniform(B, N, seed=3, device="cuda")
+    m[0, 5] = -4
+    m[0, 9] = N + 10
+    ws = la.workspace(la._desc_of(q, "relu1", True), "prefix", 64)
+    out = la.la_prefix_mask(q, k, v, m, ws=ws)
+    status, flags = la.la_last_error(ws)
+    assert status == 6 and flags == 1
+    assert la.la_last_error(ws) == (0, 0)  # cleared by the read
+    mc = m.clamp(0, N - 1).cpu().numpy()
+    ref = oracle.batched(oracle.prefix_mask, f64(q), f64(k), f64(v), m=mc)
+    assert oracle.max_row_rel_err(f64(out), ref) < TOL[torch.float32]
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("d", DS)
+def test_decode_from_prefill(dt, d):
+    B, H, N0, T = 2, 3, 150, 20
+    q, k, v = qkv(B, H, N0 + T, d, dt, seed=d)
+    S, z = la.la_kv_summary(k[:, :, :N0].contiguous(), v[:, :, :N0].contiguous())
+    outs = []
+    for t in range(N0, N0 + T):
+        sl = lambda x: x[:, :, t:t + 1].contiguous()
+        outs.append(la.la_decode_step(sl(q), sl(k), sl(v), S, z))
+    got = torch.cat(outs, dim=2)
+    Q, K, V = f64(q), f64(k), f64(v)
+    ref = np.empty(got.shape)
+    for b in range(B):
+        for h in range(H):
+            S0, z0 = oracle.kv_summary(K[b, h, :N0], V[b, h, :N0])
+            ref[b, h] = oracle.causal(Q[b, h, N0:], K[b, h, N0:], V[b, h, N0:], S0=S0, z0=z0)[0]
+    assert oracle.max_row_rel_err(f64(got), ref) < TOL[DT[dt]]
+    S_ref, z_ref = oracle.kv_summary_batched(K, V)
+    assert oracle.max_row_rel_err(f64(S), S_ref) < 1e-5
+
+
+def test_decode_from_empty_cache_equals_causal():
+    B, H, N, d = 1, 2, 40, 64
+    q, k, v = qkv(B, H, N, d, "f32", seed=13)
+    S = torch.zeros(B, H, d, d, device="cuda")
+    z = torch.zeros(B, H, d, device="cuda")
+    got = torch.cat([la.la_decode_step(q[:, :, t:t + 1].contiguous(), k[:, :, t:t + 1].contiguous(),
+                                       v[:, :, t:t + 1].contiguous(), S, z) for t in range(N)], dim=2)
+    causal = la.la_causal_chunked(q, k, v)
+    ref = oracle.batched(oracle.causal, f64(q), f64(k), f64(v))
+    assert oracle.max_row_rel_err(f64(got), ref) < 1e-4
+    assert oracle.max_row_rel_err(f64(causal), ref) < 1e-4
+
+
+def test_results_are_deterministic():
+    q, k, v = qkv(2, 4, 1500, 64, "bf16", seed=21)
+    m = workloads.prefix_mask_uniform(2, 1500, seed=21, device="cuda")
+    for fn in (lambda: la.la_noncausal(q, k, v), lambda: la.la_causal_chunked(q, k, v),
+               lambda: la.la_prefix_mask(q, k, v, m)):
+        a, b = fn(), fn()
+        assert torch.equal(a, b)
+
+
+def test_chunk_size_does_not_change_the_result():
+    q, k, v = qkv(1, 2, 1000, 128, "bf16", seed=22)
+    a = la.la_causal_chunked(q, k, v, chunk=64)
+    b = la.la_causal_chunked(q, k, v, chunk=128)
+    ref = oracle.batched(oracle.causal, f64(q), f64(k), f64(v))
+    assert oracle.max_row_rel_err(f64(a), ref) < 2e-2
+    assert oracle.max_row_rel_err(f64(b), ref) < 2e-2
+
+
+def test_worked_example_on_gpu(golden_dir):
+    """The nx source's gate 2 (Q = K = I2, V = [[2,4],[6,8]]) padded to the
+    smallest supported head size: extra feature dimensions are 0 in Q and K
+    and add phi = 1 to every weight, so the padded case is checked against
+    the oracle rather than the printed numbers; the unpadded values are
+    pinned in the oracle tests."""
+    d = 16
+    Q = torch.zeros(1, 1, 2, d)
+    Q[0, 0, 0, 0] = 1
+    Q[0, 0, 1, 1] = 1
+    V = torch.zeros(1, 1, 2, d)
+    V[0, 0, :, :2] = torch.tensor([[2.0, 4.0], [6.0, 8.0]])
+    q, k, v = Q.cuda(), Q.cuda(), V.cuda()
+    out = la.la_noncausal(q, k, v)
+    ref = oracle.batched(oracle.noncausal, f64(q), f64(k), f64(v))
+    assert oracle.max_row_rel_err(f64(out), ref) < 1e-6
