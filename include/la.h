@@ -62,7 +62,9 @@ typedef enum {
     LA_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
     LA_ERR_WORKSPACE = 4,    /* ws is NULL or smaller than la_workspace_size() */
     LA_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */
-    LA_ERR_MASK_RANGE = 6    /* (la_last_error) some m_i was outside [0, N-1] */
+    LA_ERR_MASK_RANGE = 6,   /* (la_last_error) some m_i was outside [0, N-1] */
+    LA_ERR_TIMEOUT = 7       /* (la_last_error) a kernel's bounded internal wait expired;
+                                the outputs of that call are undefined (internal error) */
 } la_status;
 
 typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
@@ -145,10 +147,13 @@ LA_API la_status la_decode_step(const la_desc* desc, const void* q, const void* 
                          void* stream);
 
 /* Waits for `stream`, then reads and clears the error word of workspace `ws`
- * (written by la_prefix_mask). *flags_out (may be NULL) receives the raw
- * bits: bit 0 = a mask value was out of range. Returns LA_ERR_MASK_RANGE
- * when bit 0 was set, LA_OK when no bit was set, LA_ERR_CUDA on a CUDA
- * failure. */
+ * (written by the calls that used it). *flags_out (may be NULL) receives the
+ * raw bits: bit 0 = a mask value was out of range (la_prefix_mask); bit 1 =
+ * a kernel's bounded wait on its own asynchronous copies or tensor-core
+ * operations expired and the kernel returned early. Returns LA_ERR_TIMEOUT
+ * when bit 1 was set, else LA_ERR_MASK_RANGE when bit 0 was set, LA_OK when
+ * no bit was set, LA_ERR_CUDA on a CUDA failure. Calls that use a workspace
+ * do not clear its error word; la_prefix_mask clears it when it starts. */
 LA_API la_status la_last_error(void* ws, void* stream, uint32_t* flags_out);
 
 /* Static string naming a status. */

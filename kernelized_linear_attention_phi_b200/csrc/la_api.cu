@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "tc.h"
+#include "tc_common.cuh"
 
 namespace la {
 namespace {
@@ -158,7 +159,7 @@ la_status kv_summary_impl(const Problem& p, const void* k, const void* v, float*
     const SplitPlan sp = kv_plan(p);
     float* part = at<float>(ws, ws_layout(p, LA_OP_KV_SUMMARY).part);
     if (tc_supported(p)) {
-        LA_TRY(cuda_status(tc_kv_partial(p, k, v, sp.tps, sp.nsplit, part, st)));
+        LA_TRY(cuda_status(tc_kv_partial(p, k, v, sp.tps, sp.nsplit, part, at<uint32_t>(ws, 0), st)));
     } else {
         LA_TRY(cuda_status(simt_kv_partial(p, k, v, sp.tps, sp.nsplit, part, st)));
     }
@@ -183,6 +184,7 @@ const char* la_status_string(la_status s) {
         case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE";
         case LA_ERR_CUDA: return "LA_ERR_CUDA";
         case LA_ERR_MASK_RANGE: return "LA_ERR_MASK_RANGE";
+        case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT";
     }
     return "LA_ERR_UNKNOWN";
 }
@@ -225,7 +227,7 @@ la_status la_noncausal(const la_desc* desc, const void* q, const void* k, const 
         z = S + (size_t)p.bh() * p.d * p.d;
     }
     LA_TRY(kv_summary_impl(p, k, v, S, z, ws, st));
-    if (tc_supported(p)) return cuda_status(tc_readout(p, q, S, z, out, st));
+    if (tc_supported(p)) return cuda_status(tc_readout(p, q, S, z, out, at<uint32_t>(ws, 0), st));
     return cuda_status(simt_readout(p, q, S, z, out, st));
 }
 
@@ -244,14 +246,16 @@ la_status la_causal_chunked(const la_desc* desc, int32_t chunk, const void* q, c
     float* part = at<float>(ws, L.part);
     // phase 1: per-block states; phase 2: exclusive prefix over blocks;
     // phase 3: each block's outputs from its prefix state.
+    uint32_t* flags = at<uint32_t>(ws, 0);
     if (tc_supported(p)) {
-        LA_TRY(cuda_status(tc_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
+        LA_TRY(cuda_status(tc_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
     } else {
         LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
     }
     LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
-    if (tc_supported(p))
-        return cuda_status(tc_causal(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, out, st));
+    if (tc_causal_supported(p))
+        return cuda_status(
+            tc_causal(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, out, flags, st));
     return cuda_status(simt_chunked(p, q, k, v, part, bp.block_tokens, bp.nblk, nullptr, nullptr,
                                     nullptr, 0, out, st));
 }
@@ -279,7 +283,11 @@ la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, cons
     float* part = at<float>(ws, L.part);
     LA_TRY(cuda_status(cudaMemsetAsync(flags, 0, sizeof(uint32_t), st)));
     LA_TRY(cuda_status(bin_queries(p, m, kSimtChunk, nbins, perm, bins, mcl, flags, st)));
-    LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
+    if (tc_supported(p)) {
+        LA_TRY(cuda_status(tc_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
+    } else {
+        LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
+    }
     LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
     return cuda_status(simt_chunked(p, q, k, v, part, bp.block_tokens, bp.nblk, perm, bins, mcl,
                                     nbins, out, st));
@@ -308,6 +316,7 @@ la_status la_last_error(void* ws, void* stream, uint32_t* flags_out) {
     LA_TRY(cuda_status(cudaMemsetAsync(ws, 0, sizeof(uint32_t), st)));
     LA_TRY(cuda_status(cudaStreamSynchronize(st)));
     if (flags_out) *flags_out = host;
+    if (host & tc::FLAG_TIMEOUT) return LA_ERR_TIMEOUT;
     if (host & FLAG_MASK_RANGE) return LA_ERR_MASK_RANGE;
     return LA_OK;
 }
