@@ -8,14 +8,18 @@ workload: non-causal (KV summary + readout), causal (chunked), prefix mask
 (queries binned by m_i) and one decode step on the state the non-causal pass
 produced. The default workload is multi-head attention with B=2, H=8,
 N=4096, d=64 (the lineartile quick-start shape), phi = relu+1, normalized,
-bf16, chunk 64, m_i uniform in [0, N-1].
+bf16, chunk 64, m_i uniform in [0, N-1]. Other workloads (--workload) run
+only the forms they are defined for.
 
-Tokens counted per step: B*N for each of the three full-sequence forms plus
-B for the decode step. ``value`` is tokens/s over all ranks (weak scaling:
-each rank runs its own batch; the path has no exchange step, so there is no
-data-path collective). Timing: CUDA events around every step on the
-launching stream, L2 flushed (a 256 MiB write) between steps outside the
-events, W untimed warm-up steps, max over ranks.
+Tokens counted per step: B*N for each full-sequence form plus B for a decode
+step. ``value`` is tokens/s over all ranks (weak scaling: each rank runs its
+own batch; the path has no exchange step, so there is no data-path
+collective). Each library call is captured once into a CUDA graph and the
+graphs are replayed. Timing: CUDA events between the calls of every step on
+the launching stream, L2 flushed (a 256 MiB write) between steps outside the
+events, W untimed warm-up steps, max over ranks. ``e2e`` repeats the step
+through the plain API calls with pinned host inputs copied in and the
+outputs copied back inside the timed region.
 """
 
 from __future__ import annotations
@@ -125,9 +129,12 @@ class ClockSampler:
 class Step:
     """Device buffers and the four library calls of one step."""
 
-    def __init__(self, wl, dtype, seed, device):
+    ALL_FORMS = ("noncausal", "causal", "prefix", "decode")
+
+    def __init__(self, wl, dtype, seed, device, forms):
         from kernelized_linear_attention_phi_b200 import binding as la
         self.la = la
+        self.forms = forms
         B, H, N, d = wl.B, wl.H, wl.N, wl.d
         self.wl, self.B, self.H, self.N, self.d = wl, B, H, N, d
         self.phi, self.normalize, self.chunk = wl.phi, wl.normalize, wl.chunk
@@ -143,21 +150,25 @@ class Step:
         self.z = torch.empty(B, H, d, dtype=torch.float32, device=device)
         desc = la._desc_of(self.q, self.phi, self.normalize)
         self.ws = {op: la.workspace(desc, op, self.chunk, device) for op in ("noncausal", "causal", "prefix")}
-        self.tokens = 3 * B * N + B
+        self.tokens = sum(B if f == "decode" else B * N for f in forms)
         self.elem = self.q.element_size()
+        if "decode" in forms and "noncausal" not in forms:
+            # the cached state the decode steps continue from: a prefill of N tokens
+            la.la_kv_summary(self.k, self.v, self.S, self.z, self.phi)
 
     def calls(self):
         la = self.la
-        return [
-            ("noncausal", lambda: la.la_noncausal(self.q, self.k, self.v, self.out_nc, self.S, self.z,
-                                                  self.phi, self.normalize, self.ws["noncausal"])),
-            ("causal", lambda: la.la_causal_chunked(self.q, self.k, self.v, self.out_c, self.chunk,
-                                                    self.phi, self.normalize, self.ws["causal"])),
-            ("prefix", lambda: la.la_prefix_mask(self.q, self.k, self.v, self.m, self.out_m, self.chunk,
-                                                 self.phi, self.normalize, self.ws["prefix"])),
-            ("decode", lambda: la.la_decode_step(self.q1, self.k1, self.v1, self.S, self.z, self.out_d,
-                                                 self.phi, self.normalize)),
-        ]
+        table = {
+            "noncausal": lambda: la.la_noncausal(self.q, self.k, self.v, self.out_nc, self.S, self.z,
+                                                 self.phi, self.normalize, self.ws["noncausal"]),
+            "causal": lambda: la.la_causal_chunked(self.q, self.k, self.v, self.out_c, self.chunk,
+                                                   self.phi, self.normalize, self.ws["causal"]),
+            "prefix": lambda: la.la_prefix_mask(self.q, self.k, self.v, self.m, self.out_m, self.chunk,
+                                                self.phi, self.normalize, self.ws["prefix"]),
+            "decode": lambda: la.la_decode_step(self.q1, self.k1, self.v1, self.S, self.z, self.out_d,
+                                                self.phi, self.normalize),
+        }
+        return [(f, table[f]) for f in self.forms]
 
     def algorithmic_bytes(self):
         """Bytes each call must move at least: its inputs once and outputs once."""
@@ -168,8 +179,11 @@ class Step:
                 "decode": 2 * st + 4 * one}
 
     def host_io(self):
-        ins = [self.q, self.k, self.v, self.m, self.q1, self.k1, self.v1]
-        outs = [self.out_nc, self.out_c, self.out_m, self.out_d]
+        full = [f for f in self.forms if f != "decode"]
+        ins = ([self.q, self.k, self.v] if full else []) + ([self.m] if "prefix" in self.forms else []) \
+            + ([self.q1, self.k1, self.v1] if "decode" in self.forms else [])
+        outs = [{"noncausal": self.out_nc, "causal": self.out_c, "prefix": self.out_m,
+                 "decode": self.out_d}[f] for f in self.forms]
         return ins, outs
 
 
@@ -189,16 +203,27 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     wl = W.WORKLOADS[args.workload]
-    dtype = args.dtype
-    step = Step(wl, dtype, wl.seed + 1000 * rank, device)
+    dtype = args.dtype if args.dtype in wl.dtypes else wl.dtypes[0]
+    forms = Step.ALL_FORMS if args.workload == "multi_head" else wl.forms
+    step = Step(wl, dtype, wl.seed + 1000 * rank, device, forms)
     calls = step.calls()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
-    stream = torch.cuda.current_stream(device)
 
     for _ in range(max(args.warmup, 3)):
         for _, fn in calls:
             fn()
     torch.cuda.synchronize()
+    graphs = []
+    for _, fn in calls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        graphs.append(g)
+    for _ in range(max(args.warmup, 3)):
+        for g in graphs:
+            g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(device)
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(K)]
@@ -210,8 +235,8 @@ def run_ours(args, rank, world, local_rank):
         for i in range(K):
             flush_l2(flush)
             ev[i][0].record(stream)
-            for j, (_, fn) in enumerate(calls):
-                fn()
+            for j, g in enumerate(graphs):
+                g.replay()
                 ev[i][j + 1].record(stream)
         torch.cuda.synchronize()
     if world > 1:
@@ -284,10 +309,12 @@ def run_ours(args, rank, world, local_rank):
         "dtype": dtype,
         "data": "synthetic",
         "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} N={wl.N} d={wl.d} {dtype} phi={wl.phi} "
-                               f"normalize={int(wl.normalize)} chunk={wl.chunk}; step = noncausal + "
-                               f"causal + prefix mask (m uniform) + 1 decode step",
+                               f"normalize={int(wl.normalize)} chunk={wl.chunk}; step = "
+                               + " + ".join({"noncausal": "noncausal", "causal": "causal",
+                                             "prefix": "prefix mask (m uniform)",
+                                             "decode": "1 decode step"}[f] for f in forms),
                    "global_batch": wl.B * world, "seq_len": wl.N, "parallelism": f"dp{world}",
-                   "l2": "flushed between steps (256 MiB write)",
+                   "l2": "flushed between steps (256 MiB write)", "launch": "one CUDA graph per call",
                    "tokens_per_step_per_gpu": step.tokens},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -330,56 +357,72 @@ def _blas_threads():
         return 1
 
 
-def oracle_sample(q, k, v, m, q1, k1, v1, phi, normalize, heads):
-    """Runs the oracle's four forms on the first `heads` heads of sequence 0.
-    Returns (tokens processed, seconds)."""
+def oracle_sample(q, k, v, m, q1, k1, v1, phi, normalize, heads, forms):
+    """Runs the oracle's forms on the first `heads` heads of sequence 0.
+    Returns (seconds, tokens processed), tokens counted like the GPU step
+    (B*N per full-sequence form, B per decode step) scaled by heads/H."""
     import oracle
     f = lambda t: t.detach().to(torch.float64).cpu().numpy()
+    H = q.shape[1]
     Q, K, V = f(q[0, :heads]), f(k[0, :heads]), f(v[0, :heads])
     M = m[0].cpu().numpy()
     q1_, k1_, v1_ = f(q1[0, :heads, 0]), f(k1[0, :heads, 0]), f(v1[0, :heads, 0])
+    N = Q.shape[1]
     t0 = time.perf_counter()
     for h in range(heads):
-        _, S, z = oracle.noncausal(Q[h], K[h], V[h], phi, normalize)
-        oracle.causal(Q[h], K[h], V[h], phi, normalize)
-        oracle.prefix_mask(Q[h], K[h], V[h], M, phi, normalize)
-        oracle.decode_step(S, z, q1_[h], k1_[h], v1_[h], phi, normalize)
+        S = z = None
+        if "noncausal" in forms:
+            _, S, z = oracle.noncausal(Q[h], K[h], V[h], phi, normalize)
+        if "causal" in forms:
+            oracle.causal(Q[h], K[h], V[h], phi, normalize)
+        if "prefix" in forms:
+            oracle.prefix_mask(Q[h], K[h], V[h], M, phi, normalize)
+        if "decode" in forms:
+            if S is None:
+                S, z = oracle.kv_summary(K[h], V[h], phi)
+            oracle.decode_step(S, z, q1_[h], k1_[h], v1_[h], phi, normalize)
     dt = time.perf_counter() - t0
-    N = Q.shape[1]
-    # tokens are counted per sequence over all its heads, so a sample of
-    # `heads` heads of one sequence processes heads/H of each sequence's tokens
-    return dt, N, heads
+    per_seq = sum(1 if fm == "decode" else N for fm in forms)
+    return dt, per_seq * heads / H
 
 
-def cpu_baseline(step, heads=2):
-    dt, N, h = oracle_sample(step.q, step.k, step.v, step.m, step.q1, step.k1, step.v1,
-                             step.phi, step.normalize, heads)
-    tokens = (3 * N + 1) * h / step.H
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"oracle (numpy fp64) on {h} of {step.H} heads of sequence 0, all four forms, "
-                      f"N={N}; tokens scaled by heads/H; {dt:.2f} s"}
+def cpu_baseline(step, heads=2, min_seconds=10.0):
+    """The oracle, as it is, on the host cores: repeated passes over a
+    sample of heads until about `min_seconds` of CPU work."""
+    total_t, total_tok, passes = 0.0, 0.0, 0
+    while total_t < min_seconds:
+        dt, tok = oracle_sample(step.q, step.k, step.v, step.m, step.q1, step.k1, step.v1,
+                                step.phi, step.normalize, heads, step.forms)
+        total_t += dt
+        total_tok += tok
+        passes += 1
+    return {"value": total_tok / total_t, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"oracle (numpy fp64) on {heads} of {step.H} heads of sequence 0, forms "
+                      f"{'+'.join(step.forms)}, N={step.N}, {passes} passes, {total_t:.1f} s; tokens "
+                      f"scaled by heads/H; Python loops single-threaded, BLAS calls may use the cores"}
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
     wl = W.WORKLOADS[args.workload]
-    dtype = args.dtype
+    dtype = args.dtype if args.dtype in wl.dtypes else wl.dtypes[0]
+    forms = Step.ALL_FORMS if args.workload == "multi_head" else wl.forms
     q, k, v = W.qkv(1, wl.H, wl.N, wl.d, wl.sigma, wl.seed, dtype, "cpu")
     m = W.prefix_mask_uniform(1, wl.N, wl.seed, "cpu")
     q1, k1, v1 = (t[0] for t in W.decode_tokens(1, 1, wl.H, wl.d, wl.sigma, wl.seed, dtype, "cpu"))
     heads = 1
     for _ in range(args.warmup):
-        oracle_sample(q, k, v, m, q1, k1, v1, wl.phi, wl.normalize, heads)
-    total = 0.0
+        oracle_sample(q, k, v, m, q1, k1, v1, wl.phi, wl.normalize, heads, forms)
+    total, tokens = 0.0, 0.0
     for _ in range(args.steps):
-        dt, N, h = oracle_sample(q, k, v, m, q1, k1, v1, wl.phi, wl.normalize, heads)
+        dt, tok = oracle_sample(q, k, v, m, q1, k1, v1, wl.phi, wl.normalize, heads, forms)
         total += dt
-    tokens = (3 * wl.N + 1) * heads / wl.H * args.steps
+        tokens += tok
     value = tokens / total
     cores = _blas_threads()
-    sample = (f"oracle (numpy fp64) on {heads} of {wl.H} heads of one sequence per step, all four "
-              f"forms, N={wl.N}; tokens scaled by heads/H")
+    sample = (f"oracle (numpy fp64) on {heads} of {wl.H} heads of one sequence per step, forms "
+              f"{'+'.join(forms)}, N={wl.N}; tokens scaled by heads/H")
     print(json.dumps({
         "impl": "reference",
         "metric": "tokens/sec (fwd, 1xB200) and % of HBM / bf16 tensor-core roofline per kernel",

@@ -116,7 +116,7 @@ WsLayout ws_layout(const Problem& p, int op) {
         L.part = off;
         off = round_up(off + (size_t)p.bh() * bp.nblk * rec, kAlign);
         if (op == LA_OP_PREFIX) {
-            const int nbins = prefix_nbins(p, kSimtChunk);
+            const int nbins = prefix_nbins(p, 64);  // the most bins any kernel uses
             L.perm = off;
             off = round_up(off + sizeof(int32_t) * (size_t)p.B * p.N, kAlign);
             L.mcl = off;
@@ -253,9 +253,9 @@ la_status la_causal_chunked(const la_desc* desc, int32_t chunk, const void* q, c
         LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
     }
     LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
-    if (tc_causal_supported(p))
-        return cuda_status(
-            tc_causal(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, out, flags, st));
+    if (tc_supported(p))
+        return cuda_status(tc_chunked(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, nullptr,
+                                      nullptr, nullptr, 0, out, flags, st));
     return cuda_status(simt_chunked(p, q, k, v, part, bp.block_tokens, bp.nblk, nullptr, nullptr,
                                     nullptr, 0, out, st));
 }
@@ -275,20 +275,25 @@ la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, cons
     LA_TRY(check_device());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const BlockPlan bp = block_plan(p);
-    const int nbins = prefix_nbins(p, kSimtChunk);
+    const bool tc = tc_supported(p);
+    const int kchunk = tc ? tc_chunk(p, chunk) : kSimtChunk;  // chunk length of the kernel used
+    const int nbins = prefix_nbins(p, kchunk);
     uint32_t* flags = at<uint32_t>(ws, 0);
     int32_t* perm = at<int32_t>(ws, L.perm);
     int32_t* mcl = at<int32_t>(ws, L.mcl);
     int32_t* bins = at<int32_t>(ws, L.bins);
     float* part = at<float>(ws, L.part);
     LA_TRY(cuda_status(cudaMemsetAsync(flags, 0, sizeof(uint32_t), st)));
-    LA_TRY(cuda_status(bin_queries(p, m, kSimtChunk, nbins, perm, bins, mcl, flags, st)));
-    if (tc_supported(p)) {
+    LA_TRY(cuda_status(bin_queries(p, m, kchunk, nbins, perm, bins, mcl, flags, st)));
+    if (tc) {
         LA_TRY(cuda_status(tc_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
     } else {
         LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
     }
     LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
+    if (tc)
+        return cuda_status(tc_chunked(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, perm, bins,
+                                      mcl, nbins, out, flags, st));
     return cuda_status(simt_chunked(p, q, k, v, part, bp.block_tokens, bp.nblk, perm, bins, mcl,
                                     nbins, out, st));
 }

@@ -433,6 +433,435 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const float* __restric
 }
 
 // ---------------------------------------------------------------------------
+// Chunked causal / prefix-mask outputs of one block
+// ---------------------------------------------------------------------------
+// The block's chunks are swept in order with the running state (S, z) of all
+// earlier keys: S lives in TMEM (fp32, M = d_k rows), starting from the
+// block's prefix record. For each chunk of C keys and each tile of (up to)
+// C queries answered there:
+//   P  = phi(Q) phi(K_c)^T               (MMA, M = C queries, N = C keys)
+//   P~ = P masked to keys j <= lim_i, bf16 (CUDA cores; den_i += rowsum)
+//   O  = phi(Q) S_prev + P~ V_c          (MMAs; S_prev as a bf16 operand)
+//   Oz = phi(Q) [z_hi; z_lo]             (MMA, N = 16; den_i += Oz_0 + Oz_1)
+//   out_i = O_i / den_i
+// then S += phi(K_c)^T V_c (MMA, M = d_k) and z += column sums of phi(K_c).
+// Causal: the queries of chunk c are its own tokens, lim_i = i - cC.
+// Prefix mask: the queries of bin c (floor((m_i+1)/C) = c) are gathered
+// rows, lim_i = m_i - cC in [-1, C-2].
+template <int D, int C, bool GATHER>
+struct ChCfg {
+    static constexpr int NB = D / 64;
+    static constexpr int TILE = C * D * 2;           // one [C x D] bf16 tile
+    static constexpr int NT = GATHER ? 2 : 3;        // tiles per stage: (Q,) K, V
+    static constexpr int STAGES = (D == 64 && C == 64) ? 3 : 2;
+    static constexpr int STAGE = NT * TILE;
+    static constexpr int PT = C * C * 2;             // P~, K-major
+    static constexpr int B3 = D * D * 2;             // S_prev, MN-major
+    static constexpr int BZ = 16 * D * 2;            // z_hi, z_lo, 14 zero rows; K-major
+    static constexpr int QG = GATHER ? TILE : 0;     // gathered queries
+    static constexpr int ZRED = 128 * NB * 8 * 4;
+    static constexpr int COL_O = 0, COL_OZ = D, COL_P = D + 16, COL_S = D + 16 + C;
+    static constexpr uint32_t TMEM_COLS = (D + 16 + C + D) <= 256 ? 256u : 512u;
+    static constexpr int NBAR = 2 * STAGES + 6;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + PT + B3 + BZ + QG + ZRED +
+                                   D * 4 + 2 * C * 4 + 8 * NBAR + 16;
+    static_assert(C == 64 || C == 128, "chunk");
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+template <int D, int C, bool GATHER>
+__global__ void __launch_bounds__(kTcThreads, 1)
+tc_chunked_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                  const __grid_constant__ CUtensorMap mV, const __nv_bfloat16* __restrict__ Qg,
+                  const float* __restrict__ prefix, int H, int N, int block_tokens, int nblk,
+                  const int32_t* __restrict__ perm, const int32_t* __restrict__ bin_start,
+                  const int32_t* __restrict__ mcl, int nbins, int phi, int normalize,
+                  __nv_bfloat16* __restrict__ out, uint32_t* __restrict__ err) {
+    using CF = ChCfg<D, C, GATHER>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* stages = align1024(smem_raw);
+    uint8_t* pt = stages + CF::STAGES * CF::STAGE;
+    uint8_t* b3 = pt + CF::PT;
+    uint8_t* bz = b3 + CF::B3;
+    uint8_t* qg = bz + CF::BZ;
+    float* zred = reinterpret_cast<float*>(qg + CF::QG);
+    float* zprev = zred + 128 * CF::NB * 8;
+    int* srow = reinterpret_cast<int*>(zprev + D);
+    int* slim = srow + C;
+    uint64_t* full = reinterpret_cast<uint64_t*>(slim + C);
+    uint64_t* empty = full + CF::STAGES;
+    uint64_t* bkv = empty + CF::STAGES;
+    uint64_t* bq = bkv + 1;
+    uint64_t* bpt = bq + 1;
+    uint64_t* bp = bpt + 1;
+    uint64_t* bo = bp + 1;
+    uint64_t* bs = bo + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bs + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int blk = blockIdx.x;
+    const int bh = blockIdx.y;
+    const int b = bh / H;
+    const int nchunks = (N + C - 1) / C;
+    const int c_begin = blk * (block_tokens / C);
+    const int c_end = (GATHER && blk == nblk - 1) ? nbins : min(nchunks, c_begin + block_tokens / C);
+    const int nci = c_end - c_begin;
+    const bool relu = phi == PHI_RELU1;
+
+    auto q_tiles = [&](int c) -> int {
+        if (!GATHER) return c < nchunks ? 1 : 0;
+        const int cnt = bin_start[(size_t)b * (nbins + 1) + c + 1] - bin_start[(size_t)b * (nbins + 1) + c];
+        return (cnt + C - 1) / C;
+    };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < CF::STAGES; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        mbar_init(bkv, 128);
+        mbar_init(bq, 128);
+        mbar_init(bpt, 128);
+        mbar_init(bp, 1);
+        mbar_init(bo, 1);
+        mbar_init(bs, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, CF::TMEM_COLS);
+    if (threadIdx.x == 0) {
+        if (!GATHER) tma_prefetch_map(&mQ);
+        tma_prefetch_map(&mK);
+        tma_prefetch_map(&mV);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int issued[CF::STAGES] = {};
+            for (int ci = 0; ci < nci; ++ci) {
+                const int s = ci % CF::STAGES, u = ci / CF::STAGES;
+                if (u > 0 && !mbar_wait(empty + s, (u - 1) & 1, err)) break;
+                mbar_arrive_expect_tx(full + s, CF::STAGE);
+                uint8_t* st = stages + s * CF::STAGE;
+                const int row = (c_begin + ci) * C;
+#pragma unroll
+                for (int bx = 0; bx < CF::NB; ++bx) {
+                    int t = 0;
+                    if (!GATHER) tma_load_3d(st + (t++) * CF::TILE + bx * C * 128, &mQ, full + s, bx * 64, row, bh);
+                    tma_load_3d(st + (t++) * CF::TILE + bx * C * 128, &mK, full + s, bx * 64, row, bh);
+                    tma_load_3d(st + t * CF::TILE + bx * C * 128, &mV, full + s, bx * 64, row, bh);
+                }
+                issued[s] = u + 1;
+            }
+            for (int s = 0; s < CF::STAGES; ++s)
+                if (issued[s] > 0) mbar_wait(full + s, (issued[s] - 1) & 1, err);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t id1 = idesc_bf16(C, C, false, false);   // P = Q K^T
+            constexpr uint32_t id3 = idesc_bf16(C, D, false, true);    // O = Q S
+            constexpr uint32_t idz = idesc_bf16(C, 16, false, false);  // Oz = Q [z]
+            constexpr uint32_t id2 = idesc_bf16(C, D, false, true);    // O += P~ V
+            constexpr uint32_t id4 = idesc_bf16(D, D, true, true);     // S += K^T V
+            const uint32_t b3a = smem_u32(b3), bza = smem_u32(bz), pta = smem_u32(pt);
+            int tq = 0;
+            bool ok = true;
+            for (int ci = 0; ci < nci && ok; ++ci) {
+                const int s = ci % CF::STAGES;
+                const uint32_t st = smem_u32(stages + s * CF::STAGE);
+                const uint32_t kt = st + (GATHER ? 0 : CF::TILE);
+                const uint32_t vt = kt + CF::TILE;
+                const uint32_t qt = GATHER ? smem_u32(qg) : st;
+                ok = mbar_wait(bkv, ci & 1, err);
+                if (!ok) break;
+                tc_fence_after();
+                const int ntq = q_tiles(c_begin + ci);
+                for (int t = 0; t < ntq && ok; ++t, ++tq) {
+                    if (GATHER) {
+                        ok = mbar_wait(bq, tq & 1, err);
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t ko = (kk / 4) * (C * 128) + (kk % 4) * 32;
+                        mma_bf16(tmem + CF::COL_P, sdesc(qt + ko, 16, 1024), sdesc(kt + ko, 16, 1024), id1,
+                                 kk > 0);
+                    }
+                    mma_commit(bp);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t a = sdesc(qt + (kk / 4) * (C * 128) + (kk % 4) * 32, 16, 1024);
+                        mma_bf16(tmem + CF::COL_O, a, sdesc(b3a + kk * 2048, D * 128, 1024), id3, kk > 0);
+                        if (normalize)
+                            mma_bf16(tmem + CF::COL_OZ, a,
+                                     sdesc(bza + (kk / 4) * (16 * 128) + (kk % 4) * 32, 16, 1024), idz, kk > 0);
+                    }
+                    ok = mbar_wait(bpt, tq & 1, err);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        mma_bf16(tmem + CF::COL_O, sdesc(pta + (kk / 4) * (C * 128) + (kk % 4) * 32, 16, 1024),
+                                 sdesc(vt + kk * 2048, C * 128, 1024), id2, 1u);
+                    mma_commit(bo);
+                }
+                if (!ok) break;
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_bf16(tmem + CF::COL_S, sdesc(kt + kk * 2048, C * 128, 1024),
+                             sdesc(vt + kk * 2048, C * 128, 1024), id4, 1u);
+                mma_commit(bs);
+                mma_commit(empty + s);
+            }
+        }
+    } else {
+        const int et = threadIdx.x - 64;
+        const int sp = warp & 3;
+        const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
+        // rows owned in M = C and M = D accumulators (M = 64: lanes 0..15 of each sub-partition)
+        constexpr int RQ = C == 128 ? 32 : 16;
+        constexpr int RS = D == 128 ? 32 : 16;
+        const int qrow = sp * RQ + lane;
+        const bool qown = lane < RQ;
+        const int srow_a = sp * RS + lane;
+        const bool sown = lane < RS;
+        const float* pre = prefix + ((size_t)bh * nblk + blk) * (size_t)(D * D + D);
+        const size_t hoff = (size_t)bh * N * D;
+
+        for (int c = et; c < 16 * D / 8; c += 128) {  // Bz rows 2..15 stay zero
+            const int n = c / (D / 8), col = (c % (D / 8)) * 8;
+            if (n >= 2)
+                *reinterpret_cast<uint4*>(bz + (col / 64) * (16 * 128) + sw128_off(n, col % 64)) =
+                    make_uint4(0, 0, 0, 0);
+        }
+        for (int a = et; a < D; a += 128) zprev[a] = pre[D * D + a];
+        named_bar(1, 128);
+
+        bool ok = true;
+        int tq = 0;
+        for (int ci = 0; ci < nci && ok; ++ci) {
+            const int c = c_begin + ci;
+            const int s = ci % CF::STAGES, u = ci / CF::STAGES;
+            const int kvalid = c < nchunks ? min(C, N - c * C) : 0;
+            uint8_t* st = stages + s * CF::STAGE;
+            uint4* kt = reinterpret_cast<uint4*>(st + (GATHER ? 0 : CF::TILE));
+            ok = mbar_wait(full + s, u & 1, err);
+            if (!ok) break;
+            // phi on the K tile (rows >= kvalid -> 0) and on the Q tile
+            float zacc[CF::NB][8];
+#pragma unroll
+            for (int bx = 0; bx < CF::NB; ++bx)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) zacc[bx][e] = 0.f;
+#pragma unroll
+            for (int i = 0; i < CF::NB * C / 16; ++i) {
+                const int p = et + 128 * i;
+                const int bx = p / (C * 8);
+                const int r = (p % (C * 8)) >> 3;
+                float f[8];
+                unpack8(kt[p], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    f[e] = r < kvalid ? phi_apply(f[e], phi) : 0.f;
+                    zacc[bx][e] += f[e];
+                }
+                kt[p] = pack8(f);
+                if (!GATHER && relu) {
+                    uint4* qt = reinterpret_cast<uint4*>(st);
+                    unpack8(qt[p], f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = phi_relu1(f[e]);
+                    qt[p] = pack8(f);
+                }
+            }
+            // S_prev -> bf16 operand (and, for the first chunk, the prefix -> TMEM)
+            if (ci > 0) {
+                ok = mbar_wait(bs, (ci - 1) & 1, err);
+                tc_fence_after();
+            }
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                uint32_t r[16];
+                if (ci == 0) {
+                    if (sown) {
+                        const float4* src = reinterpret_cast<const float4*>(pre + (size_t)srow_a * D + c0);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const float4 x = src[q4];
+                            r[4 * q4] = __float_as_uint(x.x);
+                            r[4 * q4 + 1] = __float_as_uint(x.y);
+                            r[4 * q4 + 2] = __float_as_uint(x.z);
+                            r[4 * q4 + 3] = __float_as_uint(x.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) r[e] = 0u;
+                    }
+                    tmem_st16(tmem + CF::COL_S + lane_base + c0, r);
+                } else {
+                    tmem_ld16(tmem + CF::COL_S + lane_base + c0, r);
+                    tmem_ld_wait();
+                }
+                if (sown) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int col = c0 + 8 * h;
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * h + e]);
+                        *reinterpret_cast<uint4*>(b3 + (col / 64) * (D * 128) + sw128_off(srow_a, col % 64)) =
+                            pack8(f);
+                    }
+                }
+            }
+            if (ci == 0) tmem_st_wait();
+            // z_prev -> rows 0 (hi) and 1 (lo) of the z operand
+            if (et < D / 8) {
+                const int col = et * 8;
+                float hi[8], lo[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float zv = zprev[col + e];
+                    hi[e] = __bfloat162float(__float2bfloat16_rn(zv));
+                    lo[e] = zv - hi[e];
+                }
+                uint8_t* base = bz + (col / 64) * (16 * 128);
+                *reinterpret_cast<uint4*>(base + sw128_off(0, col % 64)) = pack8(hi);
+                *reinterpret_cast<uint4*>(base + sw128_off(1, col % 64)) = pack8(lo);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(bkv);
+
+            // z += column sums of phi(K_c)
+#pragma unroll
+            for (int bx = 0; bx < CF::NB; ++bx)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) zred[et * CF::NB * 8 + bx * 8 + e] = zacc[bx][e];
+            named_bar(1, 128);
+            if (et < D) {
+                const int bx = et / 64, g = (et % 64) / 8, e = et % 8;
+                float zs = 0.f;
+                for (int t = 0; t < 128; ++t)
+                    if ((((t & 7) ^ ((t >> 3) & 7))) == g) zs += zred[t * CF::NB * 8 + bx * 8 + e];
+                zprev[et] += zs;
+            }
+            named_bar(1, 128);
+
+            const int ntq = q_tiles(c);
+            const int qbase = GATHER ? bin_start[(size_t)b * (nbins + 1) + c] : 0;
+            const int qend = GATHER ? bin_start[(size_t)b * (nbins + 1) + c + 1] : 0;
+            for (int t = 0; t < ntq && ok; ++t, ++tq) {
+                if (GATHER) {
+                    if (et < C) {
+                        const int idx = qbase + t * C + et;
+                        if (idx < qend) {
+                            const int i = perm[(size_t)b * N + idx];
+                            srow[et] = i;
+                            slim[et] = mcl[(size_t)b * N + i] - c * C;
+                        } else {
+                            srow[et] = -1;
+                            slim[et] = -1;
+                        }
+                    }
+                    named_bar(1, 128);
+                    for (int p = et; p < C * D / 8; p += 128) {
+                        const int r = p / (D / 8), col = (p % (D / 8)) * 8;
+                        float f[8];
+                        const int i = srow[r];
+                        if (i >= 0) {
+                            unpack8(ldg_stream(Qg + hoff + (size_t)i * D + col), f);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) f[e] = phi_apply(f[e], phi);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) f[e] = 0.f;
+                        }
+                        *reinterpret_cast<uint4*>(qg + (col / 64) * (C * 128) + sw128_off(r, col % 64)) = pack8(f);
+                    }
+                    fence_async_smem();
+                    tc_fence_before();
+                    mbar_arrive(bq);
+                }
+                // mask P and write P~ (this thread's query row)
+                const int lim = GATHER ? (qown ? slim[qrow] : -1) : qrow;
+                ok = mbar_wait(bp, tq & 1, err);
+                tc_fence_after();
+                float rowsum = 0.f;
+#pragma unroll
+                for (int c0 = 0; c0 < C; c0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tmem + CF::COL_P + lane_base + c0, r);
+                    tmem_ld_wait();
+                    float f[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        f[e] = (c0 + e <= lim) ? __uint_as_float(r[e]) : 0.f;
+                        rowsum += f[e];
+                    }
+                    if (qown) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int col = c0 + 8 * h;
+                            *reinterpret_cast<uint4*>(pt + (col / 64) * (C * 128) + sw128_off(qrow, col % 64)) =
+                                pack8(f + 8 * h);
+                        }
+                    }
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(bpt);
+                // epilogue
+                ok = ok && mbar_wait(bo, tq & 1, err);
+                tc_fence_after();
+                uint32_t o[D];
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tmem + CF::COL_O + lane_base + c0, r);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[c0 + e] = r[e];
+                }
+                uint32_t zr[16];
+                tmem_ld16(tmem + CF::COL_OZ + lane_base, zr);
+                tmem_ld_wait();
+                tc_fence_before();
+                int tok = -1;
+                if (qown) {
+                    if (GATHER) tok = srow[qrow];
+                    else if (qrow < kvalid) tok = c * C + qrow;
+                }
+                if (ok && tok >= 0) {
+                    const float den = rowsum + __uint_as_float(zr[0]) + __uint_as_float(zr[1]);
+                    uint4* dst = reinterpret_cast<uint4*>(out + hoff + (size_t)tok * D);
+#pragma unroll
+                    for (int c0 = 0; c0 < D; c0 += 8) {
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float num = __uint_as_float(o[c0 + e]);
+                            f[e] = normalize ? num / den : num;
+                        }
+                        dst[c0 / 8] = pack8(f);
+                    }
+                }
+                if (GATHER) named_bar(1, 128);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, CF::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -496,9 +925,32 @@ cudaError_t launch_readout(const Problem& p, const void* q, const float* S, cons
     return cudaGetLastError();
 }
 
+template <int D, int C, bool GATHER>
+cudaError_t launch_chunked(const Problem& p, const void* q, const void* k, const void* v,
+                           const float* prefix, int block_tokens, int nblk, const int32_t* perm,
+                           const int32_t* bins, const int32_t* mcl, int nbins, void* out, uint32_t* err,
+                           cudaStream_t st) {
+    if (block_tokens % C != 0) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv;
+    cudaError_t e = make_map(&mq, q, D, p.N, p.bh(), C);
+    if (e == cudaSuccess) e = make_map(&mk, k, D, p.N, p.bh(), C);
+    if (e == cudaSuccess) e = make_map(&mv, v, D, p.N, p.bh(), C);
+    if (e != cudaSuccess) return e;
+    constexpr size_t smem = ChCfg<D, C, GATHER>::SMEM;
+    e = ensure_smem<tc_chunked_kernel<D, C, GATHER>>(smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(nblk, (unsigned)p.bh());
+    tc_chunked_kernel<D, C, GATHER><<<grid, kTcThreads, smem, st>>>(
+        mq, mk, mv, static_cast<const __nv_bfloat16*>(q), prefix, p.H, p.N, block_tokens, nblk, perm, bins,
+        mcl, nbins, p.phi, p.normalize, static_cast<__nv_bfloat16*>(out), err);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool tc_supported(const Problem& p) { return p.dtype == DT_BF16 && (p.d == 64 || p.d == 128); }
+
+int tc_chunk(const Problem& p, int chunk) { return p.d == 128 ? 64 : chunk; }
 
 cudaError_t tc_kv_partial(const Problem& p, const void* k, const void* v, int tps, int nsplit, float* part,
                           uint32_t* err, cudaStream_t st) {
@@ -513,11 +965,25 @@ cudaError_t tc_readout(const Problem& p, const void* q, const float* S, const fl
                      : launch_readout<128>(p, q, S, z, out, err, st);
 }
 
-bool tc_causal_supported(const Problem&) { return false; }
-
-cudaError_t tc_causal(const Problem&, int, const void*, const void*, const void*, const float*, int, int,
-                      void*, uint32_t*, cudaStream_t) {
-    return cudaErrorNotSupported;
+cudaError_t tc_chunked(const Problem& p, int chunk, const void* q, const void* k, const void* v,
+                       const float* prefix, int block_tokens, int nblk, const int32_t* perm,
+                       const int32_t* bins, const int32_t* mcl, int nbins, void* out, uint32_t* err,
+                       cudaStream_t st) {
+    const int C = tc_chunk(p, chunk);
+    const bool g = perm != nullptr;
+#define LA_CH(D_, C_, G_) \
+    return launch_chunked<D_, C_, G_>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, mcl, nbins, out, err, st)
+    if (p.d == 128) {
+        if (g) LA_CH(128, 64, true);
+        LA_CH(128, 64, false);
+    }
+    if (C == 64) {
+        if (g) LA_CH(64, 64, true);
+        LA_CH(64, 64, false);
+    }
+    if (g) LA_CH(64, 128, true);
+    LA_CH(64, 128, false);
+#undef LA_CH
 }
 
 }  // namespace la

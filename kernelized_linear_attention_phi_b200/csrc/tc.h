@@ -17,11 +17,14 @@ cudaError_t tc_kv_partial(const Problem& p, const void* k, const void* v, int to
 // Same contract as simt_readout.
 cudaError_t tc_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,
                        uint32_t* err, cudaStream_t st);
-// True when tc_causal handles this problem.
-bool tc_causal_supported(const Problem& p);
-// Causal outputs of every block from its prefix state.
-cudaError_t tc_causal(const Problem& p, int chunk, const void* q, const void* k, const void* v,
-                      const float* prefix, int block_tokens, int nblk, void* out, uint32_t* err,
-                      cudaStream_t st);
+// Chunk length the tensor-core chunked kernel runs at for a requested chunk
+// (d = 128 always runs 64-token chunks: the shared-memory budget).
+int tc_chunk(const Problem& p, int chunk);
+// Same contract as simt_chunked, at chunk length tc_chunk(p, chunk); the
+// prefix-mask inputs (perm, bins, mcl, nbins) must be binned at that length.
+cudaError_t tc_chunked(const Problem& p, int chunk, const void* q, const void* k, const void* v,
+                       const float* prefix, int block_tokens, int nblk, const int32_t* perm,
+                       const int32_t* bins, const int32_t* mcl, int nbins, void* out, uint32_t* err,
+                       cudaStream_t st);
 
 }  // namespace la
