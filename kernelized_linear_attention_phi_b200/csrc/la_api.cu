@@ -86,8 +86,12 @@ SplitPlan kv_plan(const Problem& p) {
 struct BlockPlan {
     int block_tokens, nblk;
 };
+// Blocks of the chunked forms: every (block, head) is one CTA of the chunk
+// sweep, so the block count per head is chosen to fill one wave (CTAs that
+// fit on an SM at once x 148 SMs) without spilling into a second.
 BlockPlan block_plan(const Problem& p) {
-    const long long target = std::max(1LL, cdiv(2 * kNumSMs, p.bh()));
+    const int per_sm = (p.dtype == LA_BF16 && p.d == 128) ? 1 : 2;
+    const long long target = std::max(1LL, (long long)(per_sm * kNumSMs) / p.bh());
     long long bt = (long long)round_up((size_t)cdiv(p.N, target), 128);
     bt = std::max(bt, 256LL);
     return BlockPlan{(int)bt, (int)cdiv(p.N, bt)};

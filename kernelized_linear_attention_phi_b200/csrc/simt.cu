@@ -110,22 +110,40 @@ __global__ void state_reduce_kernel(const float* __restrict__ part, int nsplit, 
     else z[(size_t)bh * D + (e - D * D)] = s;
 }
 
+// One thread per float4 of a record; loads are issued eight blocks at a time
+// so that several are in flight, the running sum stays in registers.
 __global__ void state_scan_kernel(float* __restrict__ part, int nblk, int D,
                                   float* __restrict__ S_total, float* __restrict__ z_total) {
-    const int rec = D * D + D;
+    const int rec4 = (D * D + D) / 4;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     const long long bh = blockIdx.y;
-    if (e >= rec) return;
-    float* p = part + (size_t)bh * nblk * rec + e;
-    float run = 0.f;
-    for (int i = 0; i < nblk; ++i) {
-        const float t = p[(size_t)i * rec];
-        p[(size_t)i * rec] = run;
-        run += t;
+    if (e >= rec4) return;
+    float4* p = reinterpret_cast<float4*>(part + (size_t)bh * nblk * (rec4 * 4)) + e;
+    float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int b0 = 0; b0 < nblk; b0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (b0 + j < nblk) v[j] = p[(size_t)(b0 + j) * rec4];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (b0 + j < nblk) {
+                p[(size_t)(b0 + j) * rec4] = run;
+                run.x += v[j].x;
+                run.y += v[j].y;
+                run.z += v[j].z;
+                run.w += v[j].w;
+            }
+        }
     }
     if (S_total != nullptr) {
-        if (e < D * D) S_total[(size_t)bh * D * D + e] = run;
-        else z_total[(size_t)bh * D + (e - D * D)] = run;
+        const float r[4] = {run.x, run.y, run.z, run.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int idx = 4 * e + q;
+            if (idx < D * D) S_total[(size_t)bh * D * D + idx] = r[q];
+            else z_total[(size_t)bh * D + (idx - D * D)] = r[q];
+        }
     }
 }
 
@@ -491,9 +509,9 @@ cudaError_t state_reduce(const Problem& p, const float* part, int nsplit, float*
 
 cudaError_t state_exclusive_scan(const Problem& p, float* part, int nblk, float* S_total,
                                  float* z_total, cudaStream_t st) {
-    const int rec = p.d * p.d + p.d;
-    dim3 grid((rec + 255) / 256, (unsigned)p.bh());
-    state_scan_kernel<<<grid, 256, 0, st>>>(part, nblk, p.d, S_total, z_total);
+    const int rec4 = (p.d * p.d + p.d) / 4;
+    dim3 grid((rec4 + 127) / 128, (unsigned)p.bh());
+    state_scan_kernel<<<grid, 128, 0, st>>>(part, nblk, p.d, S_total, z_total);
     return cudaGetLastError();
 }
 

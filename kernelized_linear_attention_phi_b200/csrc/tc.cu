@@ -435,68 +435,76 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const float* __restric
 // ---------------------------------------------------------------------------
 // Chunked causal / prefix-mask outputs of one block
 // ---------------------------------------------------------------------------
-// The block's chunks are swept in order with the running state (S, z) of all
-// earlier keys: S lives in TMEM (fp32, M = d_k rows), starting from the
-// block's prefix record. For each chunk of C keys and each tile of (up to)
-// C queries answered there:
-//   P  = phi(Q) phi(K_c)^T               (MMA, M = C queries, N = C keys)
-//   P~ = P masked to keys j <= lim_i, bf16 (CUDA cores; den_i += rowsum)
-//   O  = phi(Q) S_prev + P~ V_c          (MMAs; S_prev as a bf16 operand)
-//   Oz = phi(Q) [z_hi; z_lo]             (MMA, N = 16; den_i += Oz_0 + Oz_1)
-//   out_i = O_i / den_i
-// then S += phi(K_c)^T V_c (MMA, M = d_k) and z += column sums of phi(K_c).
+// The block's chunks are swept in order with the running state of all
+// earlier keys kept in TMEM: S (fp32, M = d_k rows) and z (fp32, every column
+// of a 16-column block equal to z), both seeded from the block's prefix
+// record. For chunk c (C keys) and each tile of up to C queries answered
+// there:
+//   S_prev, z_prev -> bf16 operands (z as hi + lo rows)      [prep warps]
+//   S += phi(K_c)^T V_c ;  z += phi(K_c)^T 1                   [MMA]
+//   P  = phi(Q) phi(K_c)^T                                     [MMA, M = C]
+//   P~ = P with keys j > lim_i zeroed, bf16; den_i = rowsum   [mask warps]
+//   O  = phi(Q) S_prev + P~ V_c ; den_i += phi(Q) z_prev       [MMA]
+//   out_i = O_i / den_i                                        [mask warps]
 // Causal: the queries of chunk c are its own tokens, lim_i = i - cC.
 // Prefix mask: the queries of bin c (floor((m_i+1)/C) = c) are gathered
 // rows, lim_i = m_i - cC in [-1, C-2].
+//
+// Warp roles (320 threads): warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 "prep"
+// (phi on the K / Q tiles, state -> operands, query gather), warps 6-9 "mask"
+// (P~, epilogue). Prep runs one chunk ahead of mask; the S / z operands are
+// double-buffered, the gathered query tiles too.
 template <int D, int C, bool GATHER>
-struct ChCfg {
+struct SwCfg {
     static constexpr int NB = D / 64;
     static constexpr int TILE = C * D * 2;           // one [C x D] bf16 tile
     static constexpr int NT = GATHER ? 2 : 3;        // tiles per stage: (Q,) K, V
     static constexpr int STAGES = (D == 64 && C == 64) ? 3 : 2;
     static constexpr int STAGE = NT * TILE;
     static constexpr int PT = C * C * 2;             // P~, K-major
-    static constexpr int B3 = D * D * 2;             // S_prev, MN-major
-    static constexpr int BZ = 16 * D * 2;            // z_hi, z_lo, 14 zero rows; K-major
-    static constexpr int QG = GATHER ? TILE : 0;     // gathered queries
-    static constexpr int ZRED = 128 * NB * 8 * 4;
-    static constexpr int COL_O = 0, COL_OZ = D, COL_P = D + 16, COL_S = D + 16 + C;
-    static constexpr uint32_t TMEM_COLS = (D + 16 + C + D) <= 256 ? 256u : 512u;
-    static constexpr int NBAR = 2 * STAGES + 6;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + PT + B3 + BZ + QG + ZRED +
-                                   D * 4 + 2 * C * 4 + 8 * NBAR + 16;
+    static constexpr int B3 = D * D * 2;             // S_prev, MN-major (x2)
+    static constexpr int BZ = 16 * D * 2;            // z_hi, z_lo, 14 zero rows; K-major (x2)
+    static constexpr int ONES = 16 * C * 2;          // all-ones B operand, 16 x C, K-major
+    static constexpr int QG = GATHER ? 2 * TILE : 0; // gathered queries (x2)
+    static constexpr int ROWS = GATHER ? 2 * 2 * C * 4 : 0;  // token / limit per row (x2)
+    static constexpr int COL_S = 0, COL_Z = D, COL_P = D + 16, COL_O = D + 16 + C, COL_OZ = 2 * D + 16 + C;
+    static constexpr uint32_t TMEM_COLS = (2 * D + 32 + C) <= 256 ? 256u : 512u;
+    static constexpr int NBAR = 2 * STAGES + 8;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + PT + 2 * B3 + 2 * BZ + ONES + QG +
+                                   ROWS + 8 * NBAR + 16;
+    static constexpr int THREADS = 320;
+    static constexpr int MIN_BLOCKS = (D == 64 && C == 64) ? 2 : 1;
     static_assert(C == 64 || C == 128, "chunk");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
 template <int D, int C, bool GATHER>
-__global__ void __launch_bounds__(kTcThreads, 1)
-tc_chunked_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
-                  const __grid_constant__ CUtensorMap mV, const __nv_bfloat16* __restrict__ Qg,
-                  const float* __restrict__ prefix, int H, int N, int block_tokens, int nblk,
-                  const int32_t* __restrict__ perm, const int32_t* __restrict__ bin_start,
-                  const int32_t* __restrict__ mcl, int nbins, int phi, int normalize,
-                  __nv_bfloat16* __restrict__ out, uint32_t* __restrict__ err) {
-    using CF = ChCfg<D, C, GATHER>;
+__global__ void __launch_bounds__(SwCfg<D, C, GATHER>::THREADS, SwCfg<D, C, GATHER>::MIN_BLOCKS)
+tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                const __grid_constant__ CUtensorMap mV, const __nv_bfloat16* __restrict__ Qg,
+                const float* __restrict__ prefix, int H, int N, int block_tokens, int nblk,
+                const int32_t* __restrict__ perm, const int32_t* __restrict__ bin_start,
+                const int32_t* __restrict__ mcl, int nbins, int phi, int normalize,
+                __nv_bfloat16* __restrict__ out, uint32_t* __restrict__ err) {
+    using CF = SwCfg<D, C, GATHER>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* stages = align1024(smem_raw);
     uint8_t* pt = stages + CF::STAGES * CF::STAGE;
     uint8_t* b3 = pt + CF::PT;
-    uint8_t* bz = b3 + CF::B3;
-    uint8_t* qg = bz + CF::BZ;
-    float* zred = reinterpret_cast<float*>(qg + CF::QG);
-    float* zprev = zred + 128 * CF::NB * 8;
-    int* srow = reinterpret_cast<int*>(zprev + D);
-    int* slim = srow + C;
-    uint64_t* full = reinterpret_cast<uint64_t*>(slim + C);
+    uint8_t* bz = b3 + 2 * CF::B3;
+    uint8_t* ones = bz + 2 * CF::BZ;
+    uint8_t* qg = ones + CF::ONES;
+    int* rows = reinterpret_cast<int*>(qg + CF::QG);  // [slot][srow C | slim C]
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(rows) + CF::ROWS);
     uint64_t* empty = full + CF::STAGES;
-    uint64_t* bkv = empty + CF::STAGES;
-    uint64_t* bq = bkv + 1;
-    uint64_t* bpt = bq + 1;
-    uint64_t* bp = bpt + 1;
-    uint64_t* bo = bp + 1;
-    uint64_t* bs = bo + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bs + 1);
+    uint64_t* bprep = empty + CF::STAGES;
+    uint64_t* bsdone = bprep + 1;
+    uint64_t* bpfull = bsdone + 1;
+    uint64_t* bptready = bpfull + 1;
+    uint64_t* bofull = bptready + 1;
+    uint64_t* bofree = bofull + 1;  // [2], one per query-tile slot
+    uint64_t* bqready = bofree + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bqready + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int blk = blockIdx.x;
@@ -507,6 +515,7 @@ tc_chunked_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
     const int c_end = (GATHER && blk == nblk - 1) ? nbins : min(nchunks, c_begin + block_tokens / C);
     const int nci = c_end - c_begin;
     const bool relu = phi == PHI_RELU1;
+    const size_t hoff = (size_t)bh * N * D;
 
     auto q_tiles = [&](int c) -> int {
         if (!GATHER) return c < nchunks ? 1 : 0;
@@ -519,12 +528,14 @@ tc_chunked_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
             mbar_init(full + s, 1);
             mbar_init(empty + s, 1);
         }
-        mbar_init(bkv, 128);
-        mbar_init(bq, 128);
-        mbar_init(bpt, 128);
-        mbar_init(bp, 1);
-        mbar_init(bo, 1);
-        mbar_init(bs, 1);
+        mbar_init(bprep, 128);
+        mbar_init(bsdone, 1);
+        mbar_init(bpfull, 1);
+        mbar_init(bptready, 128);
+        mbar_init(bofull, 1);
+        mbar_init(bofree, 128);
+        mbar_init(bofree + 1, 128);
+        mbar_init(bqready, 128);
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, CF::TMEM_COLS);
@@ -539,6 +550,7 @@ tc_chunked_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
+        // ---------------- TMA producer ----------------
         if (lane == 0) {
             int issued[CF::STAGES] = {};
             for (int ci = 0; ci < nci; ++ci) {
@@ -560,13 +572,15 @@ tc_chunked_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                 if (issued[s] > 0) mbar_wait(full + s, (issued[s] - 1) & 1, err);
         }
     } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
         if (lane == 0) {
             constexpr uint32_t id1 = idesc_bf16(C, C, false, false);   // P = Q K^T
             constexpr uint32_t id3 = idesc_bf16(C, D, false, true);    // O = Q S
             constexpr uint32_t idz = idesc_bf16(C, 16, false, false);  // Oz = Q [z]
             constexpr uint32_t id2 = idesc_bf16(C, D, false, true);    // O += P~ V
             constexpr uint32_t id4 = idesc_bf16(D, D, true, true);     // S += K^T V
-            const uint32_t b3a = smem_u32(b3), bza = smem_u32(bz), pta = smem_u32(pt);
+            constexpr uint32_t id5 = idesc_bf16(D, 16, true, false);   // Z += K^T 1
+            const uint32_t pta = smem_u32(pt), onesa = smem_u32(ones);
             int tq = 0;
             bool ok = true;
             for (int ci = 0; ci < nci && ok; ++ci) {
@@ -574,73 +588,99 @@ tc_chunked_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                 const uint32_t st = smem_u32(stages + s * CF::STAGE);
                 const uint32_t kt = st + (GATHER ? 0 : CF::TILE);
                 const uint32_t vt = kt + CF::TILE;
-                const uint32_t qt = GATHER ? smem_u32(qg) : st;
-                ok = mbar_wait(bkv, ci & 1, err);
+                ok = mbar_wait(bprep, ci & 1, err);
                 if (!ok) break;
                 tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk) {
+                    const uint64_t a = sdesc(kt + kk * 2048, C * 128, 1024);
+                    mma_bf16(tmem + CF::COL_S, a, sdesc(vt + kk * 2048, C * 128, 1024), id4, 1u);
+                    if (normalize)
+                        mma_bf16(tmem + CF::COL_Z, a, sdesc(onesa + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024),
+                                 id5, 1u);
+                }
+                mma_commit(bsdone);
+                const uint32_t b3a = smem_u32(b3 + (ci & 1) * CF::B3);
+                const uint32_t bza = smem_u32(bz + (ci & 1) * CF::BZ);
                 const int ntq = q_tiles(c_begin + ci);
                 for (int t = 0; t < ntq && ok; ++t, ++tq) {
-                    if (GATHER) {
-                        ok = mbar_wait(bq, tq & 1, err);
-                        if (!ok) break;
-                        tc_fence_after();
-                    }
+                    const uint32_t qt = GATHER ? smem_u32(qg + (tq & 1) * CF::TILE) : st;
+                    if (GATHER) ok = mbar_wait(bqready, tq & 1, err);
+                    if (ok && tq > 0) ok = mbar_wait(bptready, (tq - 1) & 1, err);  // P read by the mask warps
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t ko = (kk / 4) * (C * 128) + (kk % 4) * 32;
-                        mma_bf16(tmem + CF::COL_P, sdesc(qt + ko, 16, 1024), sdesc(kt + ko, 16, 1024), id1,
-                                 kk > 0);
+                        mma_bf16(tmem + CF::COL_P, sdesc(qt + ko, 16, 1024), sdesc(kt + ko, 16, 1024), id1, kk > 0);
                     }
-                    mma_commit(bp);
+                    mma_commit(bpfull);
+                    if (tq > 0) ok = mbar_wait(bofree + ((tq - 1) & 1), ((tq - 1) >> 1) & 1, err);  // O read
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t a = sdesc(qt + (kk / 4) * (C * 128) + (kk % 4) * 32, 16, 1024);
                         mma_bf16(tmem + CF::COL_O, a, sdesc(b3a + kk * 2048, D * 128, 1024), id3, kk > 0);
                         if (normalize)
-                            mma_bf16(tmem + CF::COL_OZ, a,
-                                     sdesc(bza + (kk / 4) * (16 * 128) + (kk % 4) * 32, 16, 1024), idz, kk > 0);
+                            mma_bf16(tmem + CF::COL_OZ, a, sdesc(bza + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024),
+                                     idz, kk > 0);
                     }
-                    ok = mbar_wait(bpt, tq & 1, err);
+                    ok = mbar_wait(bptready, tq & 1, err);
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk)
                         mma_bf16(tmem + CF::COL_O, sdesc(pta + (kk / 4) * (C * 128) + (kk % 4) * 32, 16, 1024),
                                  sdesc(vt + kk * 2048, C * 128, 1024), id2, 1u);
-                    mma_commit(bo);
+                    mma_commit(bofull);
                 }
-                if (!ok) break;
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    mma_bf16(tmem + CF::COL_S, sdesc(kt + kk * 2048, C * 128, 1024),
-                             sdesc(vt + kk * 2048, C * 128, 1024), id4, 1u);
-                mma_commit(bs);
                 mma_commit(empty + s);
             }
         }
-    } else {
+    } else if (warp < 6) {
+        // ---------------- prep warps ----------------
         const int et = threadIdx.x - 64;
         const int sp = warp & 3;
         const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
-        // rows owned in M = C and M = D accumulators (M = 64: lanes 0..15 of each sub-partition)
-        constexpr int RQ = C == 128 ? 32 : 16;
-        constexpr int RS = D == 128 ? 32 : 16;
-        const int qrow = sp * RQ + lane;
-        const bool qown = lane < RQ;
-        const int srow_a = sp * RS + lane;
-        const bool sown = lane < RS;
+        constexpr int RS = D == 128 ? 32 : 16;  // S rows per sub-partition
         const float* pre = prefix + ((size_t)bh * nblk + blk) * (size_t)(D * D + D);
-        const size_t hoff = (size_t)bh * N * D;
-
-        for (int c = et; c < 16 * D / 8; c += 128) {  // Bz rows 2..15 stay zero
-            const int n = c / (D / 8), col = (c % (D / 8)) * 8;
-            if (n >= 2)
-                *reinterpret_cast<uint4*>(bz + (col / 64) * (16 * 128) + sw128_off(n, col % 64)) =
-                    make_uint4(0, 0, 0, 0);
+        {
+            const uint4 one8 = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+            for (int c = et; c < CF::ONES / 16; c += 128) reinterpret_cast<uint4*>(ones)[c] = one8;
+            for (int c = et; c < 2 * 16 * D / 8; c += 128) {  // z operand rows 2..15 stay zero
+                const int buf = c / (16 * D / 8), cc = c % (16 * D / 8);
+                const int n = cc / (D / 8), col = (cc % (D / 8)) * 8;
+                if (n >= 2)
+                    *reinterpret_cast<uint4*>(bz + buf * CF::BZ + (col / 64) * 2048 + sw128_off(n, col % 64)) =
+                        make_uint4(0, 0, 0, 0);
+            }
+            // seed the TMEM state with the block's prefix
+            const int a = sp * RS + lane;
+            const bool own = lane < RS;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                uint32_t r[16];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 x = own ? reinterpret_cast<const float4*>(pre + (size_t)a * D + c0)[q4]
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                    r[4 * q4] = __float_as_uint(x.x);
+                    r[4 * q4 + 1] = __float_as_uint(x.y);
+                    r[4 * q4 + 2] = __float_as_uint(x.z);
+                    r[4 * q4 + 3] = __float_as_uint(x.w);
+                }
+                tmem_st16(tmem + CF::COL_S + lane_base + c0, r);
+            }
+            if (normalize) {
+                uint32_t r[16];
+                const uint32_t zv = own ? __float_as_uint(pre[(size_t)D * D + a]) : 0u;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) r[e] = zv;
+                tmem_st16(tmem + CF::COL_Z + lane_base, r);
+            }
+            tmem_st_wait();
         }
-        for (int a = et; a < D; a += 128) zprev[a] = pre[D * D + a];
-        named_bar(1, 128);
-
         bool ok = true;
         int tq = 0;
         for (int ci = 0; ci < nci && ok; ++ci) {
@@ -651,24 +691,14 @@ tc_chunked_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
             uint4* kt = reinterpret_cast<uint4*>(st + (GATHER ? 0 : CF::TILE));
             ok = mbar_wait(full + s, u & 1, err);
             if (!ok) break;
-            // phi on the K tile (rows >= kvalid -> 0) and on the Q tile
-            float zacc[CF::NB][8];
-#pragma unroll
-            for (int bx = 0; bx < CF::NB; ++bx)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) zacc[bx][e] = 0.f;
-#pragma unroll
+#pragma unroll 4
             for (int i = 0; i < CF::NB * C / 16; ++i) {
                 const int p = et + 128 * i;
-                const int bx = p / (C * 8);
                 const int r = (p % (C * 8)) >> 3;
                 float f[8];
                 unpack8(kt[p], f);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    f[e] = r < kvalid ? phi_apply(f[e], phi) : 0.f;
-                    zacc[bx][e] += f[e];
-                }
+                for (int e = 0; e < 8; ++e) f[e] = r < kvalid ? phi_apply(f[e], phi) : 0.f;
                 kt[p] = pack8(f);
                 if (!GATHER && relu) {
                     uint4* qt = reinterpret_cast<uint4*>(st);
@@ -678,85 +708,73 @@ tc_chunked_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                     qt[p] = pack8(f);
                 }
             }
-            // S_prev -> bf16 operand (and, for the first chunk, the prefix -> TMEM)
             if (ci > 0) {
-                ok = mbar_wait(bs, (ci - 1) & 1, err);
+                ok = mbar_wait(bsdone, (ci - 1) & 1, err);
                 tc_fence_after();
             }
+            // S_prev -> bf16 MN-major operand (rows = d_k index)
+            uint8_t* b3b = b3 + (ci & 1) * CF::B3;
+            if (D == 128) {
+                const int a = sp * 32 + lane;
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                uint32_t r[16];
-                if (ci == 0) {
-                    if (sown) {
-                        const float4* src = reinterpret_cast<const float4*>(pre + (size_t)srow_a * D + c0);
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t r[64];
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const float4 x = src[q4];
-                            r[4 * q4] = __float_as_uint(x.x);
-                            r[4 * q4 + 1] = __float_as_uint(x.y);
-                            r[4 * q4 + 2] = __float_as_uint(x.z);
-                            r[4 * q4 + 3] = __float_as_uint(x.w);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) r[e] = 0u;
-                    }
-                    tmem_st16(tmem + CF::COL_S + lane_base + c0, r);
-                } else {
-                    tmem_ld16(tmem + CF::COL_S + lane_base + c0, r);
+                    for (int j = 0; j < 4; ++j)
+                        tmem_ld16(tmem + CF::COL_S + lane_base + 64 * h + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(r + 16 * j));
                     tmem_ld_wait();
-                }
-                if (sown) {
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int col = c0 + 8 * h;
+                    for (int g = 0; g < 8; ++g) {
                         float f[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * h + e]);
-                        *reinterpret_cast<uint4*>(b3 + (col / 64) * (D * 128) + sw128_off(srow_a, col % 64)) =
-                            pack8(f);
+                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * g + e]);
+                        *reinterpret_cast<uint4*>(b3b + h * (D * 128) + sw128_off(a, 8 * g)) = pack8(f);
                     }
                 }
-            }
-            if (ci == 0) tmem_st_wait();
-            // z_prev -> rows 0 (hi) and 1 (lo) of the z operand
-            if (et < D / 8) {
-                const int col = et * 8;
-                float hi[8], lo[8];
+            } else {
+                const int a = sp * 16 + (lane & 15);
+                const int cb = lane < 16 ? 0 : 32;
+                uint32_t r[32];
+                tmem_ld16x2<32>(tmem + CF::COL_S + lane_base, *reinterpret_cast<uint32_t(*)[16]>(r));
+                tmem_ld16x2<32>(tmem + CF::COL_S + lane_base + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+                tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float zv = zprev[col + e];
-                    hi[e] = __bfloat162float(__float2bfloat16_rn(zv));
-                    lo[e] = zv - hi[e];
+                for (int g = 0; g < 4; ++g) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * g + e]);
+                    *reinterpret_cast<uint4*>(b3b + sw128_off(a, cb + 8 * g)) = pack8(f);
                 }
-                uint8_t* base = bz + (col / 64) * (16 * 128);
-                *reinterpret_cast<uint4*>(base + sw128_off(0, col % 64)) = pack8(hi);
-                *reinterpret_cast<uint4*>(base + sw128_off(1, col % 64)) = pack8(lo);
+            }
+            // z_prev -> rows 0 (hi) and 1 (lo) of the z operand
+            if (normalize) {
+                uint32_t r[16];
+                tmem_ld16(tmem + CF::COL_Z + lane_base, r);
+                tmem_ld_wait();
+                if (lane < RS) {
+                    const int a = sp * RS + lane;
+                    const float zv = __uint_as_float(r[0]);
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
+                    uint8_t* base = bz + (ci & 1) * CF::BZ + (a / 64) * 2048;
+                    *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(0, a % 64)) = hi;
+                    *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(1, a % 64)) = lo;
+                }
             }
             fence_async_smem();
             tc_fence_before();
-            mbar_arrive(bkv);
+            mbar_arrive(bprep);
 
-            // z += column sums of phi(K_c)
-#pragma unroll
-            for (int bx = 0; bx < CF::NB; ++bx)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) zred[et * CF::NB * 8 + bx * 8 + e] = zacc[bx][e];
-            named_bar(1, 128);
-            if (et < D) {
-                const int bx = et / 64, g = (et % 64) / 8, e = et % 8;
-                float zs = 0.f;
-                for (int t = 0; t < 128; ++t)
-                    if ((((t & 7) ^ ((t >> 3) & 7))) == g) zs += zred[t * CF::NB * 8 + bx * 8 + e];
-                zprev[et] += zs;
-            }
-            named_bar(1, 128);
-
-            const int ntq = q_tiles(c);
-            const int qbase = GATHER ? bin_start[(size_t)b * (nbins + 1) + c] : 0;
-            const int qend = GATHER ? bin_start[(size_t)b * (nbins + 1) + c + 1] : 0;
-            for (int t = 0; t < ntq && ok; ++t, ++tq) {
-                if (GATHER) {
+            if (GATHER) {
+                const int ntq = q_tiles(c);
+                const int qbase = bin_start[(size_t)b * (nbins + 1) + c];
+                const int qend = bin_start[(size_t)b * (nbins + 1) + c + 1];
+                for (int t = 0; t < ntq && ok; ++t, ++tq) {
+                    const int slot = tq & 1;
+                    if (tq >= 2) ok = mbar_wait(bofree + slot, ((tq >> 1) - 1) & 1, err);
+                    if (!ok) break;
+                    int* srow = rows + slot * 2 * C;
+                    int* slim = srow + C;
                     if (et < C) {
                         const int idx = qbase + t * C + et;
                         if (idx < qend) {
@@ -769,6 +787,7 @@ tc_chunked_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                         }
                     }
                     named_bar(1, 128);
+                    uint8_t* q = qg + slot * CF::TILE;
                     for (int p = et; p < C * D / 8; p += 128) {
                         const int r = p / (D / 8), col = (p % (D / 8)) * 8;
                         float f[8];
@@ -781,75 +800,110 @@ tc_chunked_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
 #pragma unroll
                             for (int e = 0; e < 8; ++e) f[e] = 0.f;
                         }
-                        *reinterpret_cast<uint4*>(qg + (col / 64) * (C * 128) + sw128_off(r, col % 64)) = pack8(f);
+                        *reinterpret_cast<uint4*>(q + (col / 64) * (C * 128) + sw128_off(r, col % 64)) = pack8(f);
                     }
                     fence_async_smem();
-                    tc_fence_before();
-                    mbar_arrive(bq);
+                    mbar_arrive(bqready);
                 }
-                // mask P and write P~ (this thread's query row)
-                const int lim = GATHER ? (qown ? slim[qrow] : -1) : qrow;
-                ok = mbar_wait(bp, tq & 1, err);
+            }
+        }
+    } else {
+        // ---------------- mask + epilogue warps ----------------
+        const int sp = warp & 3;
+        const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
+        // M = C accumulators: C = 128 -> lane = row; C = 64 -> rows in lanes
+        // 0..15, the two halves of the warp take the two column halves.
+        const int i = C == 128 ? sp * 32 + lane : sp * 16 + (lane & 15);
+        const int half = (C == 64 && lane >= 16) ? 1 : 0;
+        bool ok = true;
+        int tq = 0;
+        for (int ci = 0; ci < nci && ok; ++ci) {
+            const int c = c_begin + ci;
+            const int kvalid = c < nchunks ? min(C, N - c * C) : 0;
+            const int ntq = q_tiles(c);
+            for (int t = 0; t < ntq && ok; ++t, ++tq) {
+                const int slot = tq & 1;
+                ok = mbar_wait(bpfull, tq & 1, err);
                 tc_fence_after();
-                float rowsum = 0.f;
+                // the row table of a gathered tile is written before its MMAs are issued
+                const int* srow = rows + slot * 2 * C;
+                const int lim = GATHER ? srow[C + i] : i;
+                const int tok = GATHER ? srow[i] : (i < kvalid ? c * C + i : -1);
+                float rs = 0.f;
+                if (C == 128) {
 #pragma unroll
-                for (int c0 = 0; c0 < C; c0 += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(tmem + CF::COL_P + lane_base + c0, r);
-                    tmem_ld_wait();
-                    float f[16];
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t r[64];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        f[e] = (c0 + e <= lim) ? __uint_as_float(r[e]) : 0.f;
-                        rowsum += f[e];
-                    }
-                    if (qown) {
+                        for (int j = 0; j < 4; ++j)
+                            tmem_ld16(tmem + CF::COL_P + lane_base + 64 * h + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(r + 16 * j));
+                        tmem_ld_wait();
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int col = c0 + 8 * h;
-                            *reinterpret_cast<uint4*>(pt + (col / 64) * (C * 128) + sw128_off(qrow, col % 64)) =
-                                pack8(f + 8 * h);
+                        for (int g = 0; g < 8; ++g) {
+                            float f[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const int j = 64 * h + 8 * g + e;
+                                f[e] = j <= lim ? __uint_as_float(r[8 * g + e]) : 0.f;
+                                rs += f[e];
+                            }
+                            *reinterpret_cast<uint4*>(pt + h * (C * 128) + sw128_off(i, 8 * g)) = pack8(f);
                         }
                     }
-                }
-                fence_async_smem();
-                tc_fence_before();
-                mbar_arrive(bpt);
-                // epilogue
-                ok = ok && mbar_wait(bo, tq & 1, err);
-                tc_fence_after();
-                uint32_t o[D];
+                } else {
+                    uint32_t r[32];
+                    tmem_ld16x2<32>(tmem + CF::COL_P + lane_base, *reinterpret_cast<uint32_t(*)[16]>(r));
+                    tmem_ld16x2<32>(tmem + CF::COL_P + lane_base + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+                    tmem_ld_wait();
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(tmem + CF::COL_O + lane_base + c0, r);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) o[c0 + e] = r[e];
-                }
-                uint32_t zr[16];
-                tmem_ld16(tmem + CF::COL_OZ + lane_base, zr);
-                tmem_ld_wait();
-                tc_fence_before();
-                int tok = -1;
-                if (qown) {
-                    if (GATHER) tok = srow[qrow];
-                    else if (qrow < kvalid) tok = c * C + qrow;
-                }
-                if (ok && tok >= 0) {
-                    const float den = rowsum + __uint_as_float(zr[0]) + __uint_as_float(zr[1]);
-                    uint4* dst = reinterpret_cast<uint4*>(out + hoff + (size_t)tok * D);
-#pragma unroll
-                    for (int c0 = 0; c0 < D; c0 += 8) {
+                    for (int g = 0; g < 4; ++g) {
                         float f[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            const float num = __uint_as_float(o[c0 + e]);
+                            const int j = 32 * half + 8 * g + e;
+                            f[e] = j <= lim ? __uint_as_float(r[8 * g + e]) : 0.f;
+                            rs += f[e];
+                        }
+                        *reinterpret_cast<uint4*>(pt + sw128_off(i, 32 * half + 8 * g)) = pack8(f);
+                    }
+                    rs += __shfl_xor_sync(0xffffffffu, rs, 16);
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(bptready);
+                // epilogue: this thread's segment of output row i
+                ok = ok && mbar_wait(bofull, tq & 1, err);
+                tc_fence_after();
+                constexpr int SEG = C == 128 ? D : D / 2;
+                uint32_t o[SEG];
+#pragma unroll
+                for (int j = 0; j < SEG / 16; ++j) {
+                    if (C == 128)
+                        tmem_ld16(tmem + CF::COL_O + lane_base + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(o + 16 * j));
+                    else
+                        tmem_ld16x2<D / 2>(tmem + CF::COL_O + lane_base + 16 * j,
+                                           *reinterpret_cast<uint32_t(*)[16]>(o + 16 * j));
+                }
+                uint32_t oz[2];
+                tmem_ld2(tmem + CF::COL_OZ + lane_base, oz);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(bofree + slot);
+                float den = rs + __uint_as_float(oz[0]) + __uint_as_float(oz[1]);
+                if (C == 64) den = __shfl_sync(0xffffffffu, den, lane & 15);
+                if (ok && tok >= 0) {
+                    uint4* dst = reinterpret_cast<uint4*>(out + hoff + (size_t)tok * D + half * SEG);
+#pragma unroll
+                    for (int g = 0; g < SEG / 8; ++g) {
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float num = __uint_as_float(o[8 * g + e]);
                             f[e] = normalize ? num / den : num;
                         }
-                        dst[c0 / 8] = pack8(f);
+                        dst[g] = pack8(f);
                     }
                 }
-                if (GATHER) named_bar(1, 128);
             }
         }
     }
@@ -936,11 +990,12 @@ cudaError_t launch_chunked(const Problem& p, const void* q, const void* k, const
     if (e == cudaSuccess) e = make_map(&mk, k, D, p.N, p.bh(), C);
     if (e == cudaSuccess) e = make_map(&mv, v, D, p.N, p.bh(), C);
     if (e != cudaSuccess) return e;
-    constexpr size_t smem = ChCfg<D, C, GATHER>::SMEM;
-    e = ensure_smem<tc_chunked_kernel<D, C, GATHER>>(smem);
+    using CF = SwCfg<D, C, GATHER>;
+    constexpr size_t smem = CF::SMEM;
+    e = ensure_smem<tc_sweep_kernel<D, C, GATHER>>(smem);
     if (e != cudaSuccess) return e;
     dim3 grid(nblk, (unsigned)p.bh());
-    tc_chunked_kernel<D, C, GATHER><<<grid, kTcThreads, smem, st>>>(
+    tc_sweep_kernel<D, C, GATHER><<<grid, CF::THREADS, smem, st>>>(
         mq, mk, mv, static_cast<const __nv_bfloat16*>(q), prefix, p.H, p.N, block_tokens, nblk, perm, bins,
         mcl, nbins, p.phi, p.normalize, static_cast<__nv_bfloat16*>(out), err);
     return cudaGetLastError();
