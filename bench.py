@@ -271,6 +271,10 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_s = sum(a.elapsed_time(b) for a, b in e_ev) / 1e3
 
+    # every call reports expired bounded waits in its workspace error word
+    flags = {op: step.la.la_last_error(ws)[1] for op, ws in step.ws.items()}
+    bad_flags = {op: f for op, f in flags.items() if f}
+
     if world > 1:
         import torch.distributed as dist
         tt = torch.tensor([t_s, e2e_s], dtype=torch.float64, device=device)
@@ -327,10 +331,14 @@ def run_ours(args, rank, world, local_rank):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(step, heads=2)
+    if bad_flags:
+        result["error_flags"] = bad_flags
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
+    if bad_flags:
+        raise SystemExit(f"library error flags set during the run: {bad_flags}")
 
 
 def load_peaks():

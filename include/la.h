@@ -25,7 +25,10 @@
  *   - All pointers are device pointers owned by the caller, 16-byte aligned.
  *     The library never allocates device memory and keeps no pointer after
  *     a call returns; scratch space is the caller's workspace (ws), sized by
- *     la_workspace_size().
+ *     la_workspace_size(). A workspace starts with an error word that must
+ *     be zero when the workspace is first used (see la_last_error); the rest
+ *     needs no initialization. Calls that overlap on the GPU need distinct
+ *     workspaces.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream). Buffers must stay valid until the stream
  *     reaches the call's work.
@@ -146,14 +149,16 @@ LA_API la_status la_decode_step(const la_desc* desc, const void* q, const void* 
                          const void* v, float* S, float* z, void* out,
                          void* stream);
 
-/* Waits for `stream`, then reads and clears the error word of workspace `ws`
- * (written by the calls that used it). *flags_out (may be NULL) receives the
- * raw bits: bit 0 = a mask value was out of range (la_prefix_mask); bit 1 =
- * a kernel's bounded wait on its own asynchronous copies or tensor-core
+/* Waits for `stream`, then reads and clears the error word of workspace `ws`.
+ * The error word is the first 4 bytes of a workspace; it is sticky: the
+ * calls that use the workspace only set bits in it, so the caller zeroes it
+ * once when allocating the workspace, and la_last_error reports everything
+ * since the previous read. *flags_out (may be NULL) receives the raw bits:
+ * bit 0 = a mask value was out of range (la_prefix_mask); bit 1 = a
+ * kernel's bounded wait on its own asynchronous copies or tensor-core
  * operations expired and the kernel returned early. Returns LA_ERR_TIMEOUT
  * when bit 1 was set, else LA_ERR_MASK_RANGE when bit 0 was set, LA_OK when
- * no bit was set, LA_ERR_CUDA on a CUDA failure. Calls that use a workspace
- * do not clear its error word; la_prefix_mask clears it when it starts. */
+ * no bit was set, LA_ERR_CUDA on a CUDA failure. */
 LA_API la_status la_last_error(void* ws, void* stream, uint32_t* flags_out);
 
 /* Static string naming a status. */

@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_PKG, "_lib", "libla_b200.so")
 LA_OK = 0
 STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED",
                 3: "LA_ERR_MISALIGNED", 4: "LA_ERR_WORKSPACE", 5: "LA_ERR_CUDA",
-                6: "LA_ERR_MASK_RANGE"}
+                6: "LA_ERR_MASK_RANGE", 7: "LA_ERR_TIMEOUT"}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 PHIS = {"relu1": 0, "identity": 1}
 OPS = {"kv_summary": 0, "noncausal": 1, "causal": 2, "prefix": 3, "decode": 4}
@@ -131,9 +131,11 @@ def la_workspace_size(desc: la_desc, op, chunk: int = 64) -> int:
 
 
 def workspace(desc: la_desc, op, chunk: int = 64, device="cuda") -> torch.Tensor:
-    """A device buffer big enough for ``op`` on ``desc``."""
+    """A device buffer big enough for ``op`` on ``desc``, with its error word
+    zeroed (the library only sets bits in it; la_last_error reads and
+    clears)."""
     n = la_workspace_size(desc, op, chunk)
-    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
 
 
 def la_kv_summary(k, v, S_out=None, z_out=None, phi="relu1", ws=None, stream=None):

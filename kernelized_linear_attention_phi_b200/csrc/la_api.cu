@@ -108,9 +108,15 @@ WsLayout ws_layout(const Problem& p, int op) {
     size_t off = WS_HEADER;
     const size_t rec = p.state_floats() * sizeof(float);
     if (op == LA_OP_KV_SUMMARY || op == LA_OP_NONCAUSAL) {
-        const SplitPlan sp = kv_plan(p);
+        size_t nrec;
+        if (tc_supported(p)) {
+            const KvBalanced w = kv_balanced_plan(p);
+            nrec = (size_t)w.G * w.K;
+        } else {
+            nrec = (size_t)p.bh() * kv_plan(p).nsplit;
+        }
         L.part = off;
-        off = round_up(off + (size_t)p.bh() * sp.nsplit * rec, kAlign);
+        off = round_up(off + nrec * rec, kAlign);
         if (op == LA_OP_NONCAUSAL) {
             L.sz = off;
             off = round_up(off + (size_t)p.bh() * rec, kAlign);
@@ -160,13 +166,10 @@ la_status check_ws(const WsLayout& L, void* ws, size_t ws_bytes) {
 
 la_status kv_summary_impl(const Problem& p, const void* k, const void* v, float* S, float* z,
                           void* ws, cudaStream_t st) {
-    const SplitPlan sp = kv_plan(p);
     float* part = at<float>(ws, ws_layout(p, LA_OP_KV_SUMMARY).part);
-    if (tc_supported(p)) {
-        LA_TRY(cuda_status(tc_kv_partial(p, k, v, sp.tps, sp.nsplit, part, at<uint32_t>(ws, 0), st)));
-    } else {
-        LA_TRY(cuda_status(simt_kv_partial(p, k, v, sp.tps, sp.nsplit, part, st)));
-    }
+    if (tc_supported(p)) return cuda_status(tc_kv_summary(p, k, v, part, S, z, at<uint32_t>(ws, 0), st));
+    const SplitPlan sp = kv_plan(p);
+    LA_TRY(cuda_status(simt_kv_partial(p, k, v, sp.tps, sp.nsplit, part, st)));
     return cuda_status(state_reduce(p, part, sp.nsplit, S, z, st));
 }
 
@@ -252,7 +255,7 @@ la_status la_causal_chunked(const la_desc* desc, int32_t chunk, const void* q, c
     // phase 3: each block's outputs from its prefix state.
     uint32_t* flags = at<uint32_t>(ws, 0);
     if (tc_supported(p)) {
-        LA_TRY(cuda_status(tc_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
+        LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
     } else {
         LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
     }
@@ -287,10 +290,9 @@ la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, cons
     int32_t* mcl = at<int32_t>(ws, L.mcl);
     int32_t* bins = at<int32_t>(ws, L.bins);
     float* part = at<float>(ws, L.part);
-    LA_TRY(cuda_status(cudaMemsetAsync(flags, 0, sizeof(uint32_t), st)));
     LA_TRY(cuda_status(bin_queries(p, m, kchunk, nbins, perm, bins, mcl, flags, st)));
     if (tc) {
-        LA_TRY(cuda_status(tc_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
+        LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
     } else {
         LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
     }

@@ -1,6 +1,8 @@
 // Tensor-core (tcgen05 / TMEM / TMA) kernels for bf16 inputs, d in {64, 128}.
 #pragma once
 
+#include <cuda.h>
+
 #include "internal.h"
 
 namespace la {
@@ -8,15 +10,32 @@ namespace la {
 // True when the tcgen05 path handles this problem (bf16, d = 64 or 128).
 bool tc_supported(const Problem& p);
 
-// The kernels below bound every wait; an expired wait sets
+// Every kernel below bounds its waits; an expired wait sets
 // tc::FLAG_TIMEOUT in *err (the workspace error word) and the kernel returns.
 
-// Same contract as simt_kv_partial; tokens_per_split must be a multiple of 128.
-cudaError_t tc_kv_partial(const Problem& p, const void* k, const void* v, int tokens_per_split,
-                          int nsplit, float* part, uint32_t* err, cudaStream_t st);
+// Balanced split of the KV summary: a 1-D grid of G CTAs (one per SM) cuts
+// the flattened sequence of (head, 128-token tile) pairs into G contiguous
+// ranges of equal length. A range that touches several heads writes one
+// partial record per head; slot (cta * K + j) holds the record of the
+// j-th head the CTA touches.
+struct KvBalanced {
+    int G, K, tph;     // CTAs, record slots per CTA, tiles per head
+    long long total;   // bh * tph
+};
+KvBalanced kv_balanced_plan(const Problem& p);
+
+// KV summary in balanced mode: partial records into `part` (G*K slots of
+// d*d + d floats), then a fixed-order reduction into S [bh][d*d], z [bh][d].
+cudaError_t tc_kv_summary(const Problem& p, const void* k, const void* v, float* part, float* S,
+                          float* z, uint32_t* err, cudaStream_t st);
+// KV summary per block: CTA (block, head) writes record (head*nblk + block)
+// over tokens [block*block_tokens, ...); block_tokens must be a multiple of 128.
+cudaError_t tc_kv_blocks(const Problem& p, const void* k, const void* v, int block_tokens, int nblk,
+                         float* part, uint32_t* err, cudaStream_t st);
 // Same contract as simt_readout.
 cudaError_t tc_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,
                        uint32_t* err, cudaStream_t st);
+
 // Chunk length the tensor-core chunked kernel runs at for a requested chunk
 // (d = 128 always runs 64-token chunks: the shared-memory budget).
 int tc_chunk(const Problem& p, int chunk);
@@ -26,5 +45,9 @@ cudaError_t tc_chunked(const Problem& p, int chunk, const void* q, const void* k
                        const float* prefix, int block_tokens, int nblk, const int32_t* perm,
                        const int32_t* bins, const int32_t* mcl, int nbins, void* out, uint32_t* err,
                        cudaStream_t st);
+
+// [BH, N, d] bf16 viewed as 3-D for TMA: 64-column x `rows` boxes, 128-byte
+// swizzle, zero fill outside the tensor.
+cudaError_t make_map(CUtensorMap* map, const void* base, int d, int N, long long bh, int rows);
 
 }  // namespace la

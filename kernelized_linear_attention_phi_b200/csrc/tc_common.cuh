@@ -210,10 +210,45 @@ __device__ __forceinline__ void named_bar(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+constexpr int kTile = 128;  // tokens per TMA tile of the KV-summary and readout kernels
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+__device__ __forceinline__ void unpack8(const uint4& w, float* f) { Vec16<__nv_bfloat16>::unpack(w, f); }
+__device__ __forceinline__ uint4 pack8(const float* f) { return Vec16<__nv_bfloat16>::pack(f); }
+
 // Byte offset of element (row, col) in a 128-byte-swizzled tile of bf16
 // rows, 64 elements per row (col < 64).
 __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t col) {
     return row * 128u + ((((col >> 3) ^ (row & 7u)) << 4) | ((col & 7u) << 1));
+}
+
+// phi = relu(x) + 1 on eight packed bf16 values: max(x, 0) then + 1 in
+// bf16x2 arithmetic (each result rounded once, as fp32 followed by a round to
+// bf16 would give; -0.0 maps to 1 like +0.0).
+__device__ __forceinline__ uint4 phi_relu1_x8(uint4 w) {
+    const __nv_bfloat162 zero = __float2bfloat162_rn(0.0f), one = __float2bfloat162_rn(1.0f);
+    uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&v[i]);
+        h = __hadd2(__hmax2(h, zero), one);
+        v[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    return make_uint4(v[0], v[1], v[2], v[3]);
+}
+// relu on eight packed bf16 values (exact).
+__device__ __forceinline__ uint4 relu_x8(uint4 w) {
+    const __nv_bfloat162 zero = __float2bfloat162_rn(0.0f);
+    uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&v[i]);
+        h = __hmax2(h, zero);
+        v[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    return make_uint4(v[0], v[1], v[2], v[3]);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

@@ -1,26 +1,5 @@
-// Tensor-core kernels (tcgen05 + TMEM + TMA) for bf16 inputs, d = 64 or 128.
-//
-// KV summary ("nx_f32_linear_attention.nx source", KV-summary loop):
-//   S = phi(K)^T V over a token range, as MMAs with M = d_k, N = d_v and the
-//   tokens as the contraction dimension. TMA stages 128-token K and V tiles;
-//   four warps prepare K in shared memory (and sum z = sum phi(K) in fp32 on
-//   the way); one thread issues tcgen05.mma with S accumulating in TMEM.
-//   For phi = relu+1 the operand is relu(K), which is exact in bf16, and the
-//   "+1" part is added as 1 (x) colsum(V): a second MMA against an all-ones
-//   operand gives colsum(V). So S carries no rounding of phi(K) to bf16.
-// Readout (nx source, per-query loop):
-//   out = phi(Q) S / (phi(Q) . z) for 128-token tiles: MMA with M = tokens,
-//   N = d_v, K = d_k against S in shared memory (bf16), and a second
-//   N = 16 MMA against z for the denominator; the division and the bf16
-//   store run in the TMEM epilogue.
-//
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
-// issues MMAs, warps 2-5 transform tiles (phi) and run epilogues.
-
-#include <cudaTypedefs.h>
-
-#include <algorithm>
-#include <mutex>
+// Chunked causal / prefix-mask attention on tcgen05 tensor cores (bf16).
+// See the comment above the kernel for the algorithm and the warp roles.
 
 #include "launch_util.h"
 #include "tc.h"
@@ -30,407 +9,6 @@ namespace la {
 namespace {
 
 using namespace tc;
-
-constexpr int kTcThreads = 192;
-constexpr int kTile = 128;  // tokens per TMA tile
-
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-__device__ __forceinline__ void unpack8(const uint4& w, float* f) { Vec16<__nv_bfloat16>::unpack(w, f); }
-__device__ __forceinline__ uint4 pack8(const float* f) { return Vec16<__nv_bfloat16>::pack(f); }
-
-// ---------------------------------------------------------------------------
-// Partial KV summaries
-// ---------------------------------------------------------------------------
-template <int D>
-struct KvCfg {
-    static constexpr int NB = D / 64;                 // 64-column boxes per tile
-    static constexpr int TILE = kTile * D * 2;        // bytes of a K or V tile
-    static constexpr int STAGES = D == 64 ? 4 : 3;
-    static constexpr int ONES = kTile * 128;           // all-ones MN-major operand (M = 64)
-    static constexpr int ZRED = 128 * NB * 8 * 4;     // z partial sums
-    static constexpr int BARS = 3 * STAGES + 1;
-    static constexpr uint32_t TMEM_COLS = D == 64 ? 128 : 256;  // S, then the colsum block
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * 2 * TILE + ONES + ZRED + 8 * BARS + 16;
-};
-
-template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1)
-tc_kv_partial_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
-                     int N, int tps, int nsplit, int phi, float* __restrict__ part,
-                     uint32_t* __restrict__ err) {
-    using C = KvCfg<D>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* tiles = align1024(smem_raw);
-    uint8_t* ones = tiles + C::STAGES * 2 * C::TILE;
-    float* zred = reinterpret_cast<float*>(ones + C::ONES);
-    uint64_t* full = reinterpret_cast<uint64_t*>(zred + 128 * C::NB * 8);
-    uint64_t* tdone = full + C::STAGES;
-    uint64_t* empty = tdone + C::STAGES;
-    uint64_t* done = empty + C::STAGES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int split = blockIdx.x;
-    const int bh = blockIdx.y;
-    const int t0 = split * tps;
-    const int t1 = min(N, t0 + tps);
-    const int ntiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(full + s, 1);
-            mbar_init(tdone + s, 128);
-            mbar_init(empty + s, 1);
-        }
-        mbar_init(done, 1);
-        fence_mbar_init();
-    }
-    if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
-    if (threadIdx.x == 0) {
-        tma_prefetch_map(&mK);
-        tma_prefetch_map(&mV);
-    }
-    const bool relu = phi == PHI_RELU1;
-    if (relu) {
-        const uint4 one8 = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-        for (int c = threadIdx.x; c < C::ONES / 16; c += kTcThreads) reinterpret_cast<uint4*>(ones)[c] = one8;
-        fence_async_smem();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            int issued[C::STAGES] = {};
-            for (int it = 0; it < ntiles; ++it) {
-                const int s = it % C::STAGES, u = it / C::STAGES;
-                if (u > 0 && !mbar_wait(empty + s, (u - 1) & 1, err)) break;
-                mbar_arrive_expect_tx(full + s, 2 * C::TILE);
-                uint8_t* kt = tiles + s * 2 * C::TILE;
-                const int row = t0 + it * kTile;
-#pragma unroll
-                for (int b = 0; b < C::NB; ++b) {
-                    tma_load_3d(kt + b * kTile * 128, &mK, full + s, b * 64, row, bh);
-                    tma_load_3d(kt + C::TILE + b * kTile * 128, &mV, full + s, b * 64, row, bh);
-                }
-                issued[s] = u + 1;
-            }
-            // no copy may still be landing when the CTA exits
-            for (int s = 0; s < C::STAGES; ++s)
-                if (issued[s] > 0) mbar_wait(full + s, (issued[s] - 1) & 1, err);
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(D, D, true, true);
-            constexpr uint32_t idesc_ones = idesc_bf16(64, D, true, true);
-            const uint32_t ob = smem_u32(ones);
-            for (int it = 0; it < ntiles; ++it) {
-                const int s = it % C::STAGES, u = it / C::STAGES;
-                if (!mbar_wait(tdone + s, u & 1, err)) break;
-                tc_fence_after();
-                const uint32_t kt = smem_u32(tiles + s * 2 * C::TILE);
-                const uint32_t vt = kt + C::TILE;
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
-                    const uint64_t a = sdesc(kt + kk * 2048, kTile * 128, 1024);
-                    const uint64_t b = sdesc(vt + kk * 2048, kTile * 128, 1024);
-                    mma_bf16(tmem, a, b, idesc, (it > 0 || kk > 0) ? 1u : 0u);
-                    if (relu)  // every row of this block is colsum(V)
-                        mma_bf16(tmem + D, sdesc(ob + kk * 2048, kTile * 128, 1024), b, idesc_ones,
-                                 (it > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(empty + s);
-            }
-            mma_commit(done);
-        }
-    } else {
-        const int et = threadIdx.x - 64;  // 0..127
-        float zacc[C::NB][8];
-#pragma unroll
-        for (int b = 0; b < C::NB; ++b)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) zacc[b][e] = 0.f;
-        bool ok = true;
-        for (int it = 0; it < ntiles && ok; ++it) {
-            const int s = it % C::STAGES, u = it / C::STAGES;
-            ok = mbar_wait(full + s, u & 1, err);
-            if (!ok) break;
-            const int valid = min(kTile, t1 - (t0 + it * kTile));
-            uint4* kt = reinterpret_cast<uint4*>(tiles + s * 2 * C::TILE);
-#pragma unroll
-            for (int i = 0; i < C::NB * 8; ++i) {
-                const int p = et + 128 * i;   // 16-byte chunk index
-                const int b = i / 8;          // box
-                const int r = (p & 1023) >> 3;  // token row within the tile
-                float f[8];
-                unpack8(kt[p], f);
-                if (r < valid) {
-                    // operand: relu(k) for phi = relu+1 (exact in bf16), k for identity
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float ph = phi_apply(f[e], phi);
-                        zacc[b][e] += ph;
-                        f[e] = relu ? ph - 1.0f : ph;
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = 0.f;
-                }
-                kt[p] = pack8(f);
-            }
-            fence_async_smem();
-            mbar_arrive(tdone + s);
-        }
-        // z: the 16 threads sharing a column group hold its partial sums
-#pragma unroll
-        for (int b = 0; b < C::NB; ++b)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) zred[et * C::NB * 8 + b * 8 + e] = zacc[b][e];
-        named_bar(1, 128);
-        float* rec = part + ((size_t)bh * nsplit + split) * (size_t)(D * D + D);
-        if (et < D) {
-            const int b = et / 64, g = (et % 64) / 8, e = et % 8;
-            float zs = 0.f;
-            for (int t = 0; t < 128; ++t)
-                if ((((t & 7) ^ ((t >> 3) & 7))) == g) zs += zred[t * C::NB * 8 + b * 8 + e];
-            rec[D * D + et] = zs;
-        }
-        // S from TMEM: lane = row of S (d_k index), columns = d_v
-        const int sp = warp & 3;
-        const bool have = ntiles > 0 && ok && mbar_wait(done, 0, err);
-        tc_fence_after();
-        constexpr int ROWS_PER_WARP = D == 128 ? 32 : 16;
-        const int a = sp * ROWS_PER_WARP + lane;
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 16) {
-            uint32_t r[16];
-            tmem_ld16(tmem + (static_cast<uint32_t>(sp * 32) << 16) + c0, r);
-            if (relu) {
-                // lanes 0..15 of each sub-partition hold a row of the M = 64
-                // colsum block; every such row equals colsum(V)
-                uint32_t c[16];
-                tmem_ld16(tmem + (static_cast<uint32_t>(sp * 32) << 16) + D + c0, c);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    r[e] = __float_as_uint(__uint_as_float(r[e]) +
-                                           __uint_as_float(__shfl_sync(0xffffffffu, c[e], lane & 15)));
-            }
-            tmem_ld_wait();
-            if (lane < ROWS_PER_WARP) {
-                float4* o = reinterpret_cast<float4*>(rec + (size_t)a * D + c0);
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    o[q] = have ? make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                              __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, C::TMEM_COLS);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Readout
-// ---------------------------------------------------------------------------
-template <int D>
-struct RoCfg {
-    static constexpr int NB = D / 64;
-    static constexpr int TILE = kTile * D * 2;         // Q tile bytes
-    static constexpr int STAGES = D == 64 ? 4 : 3;
-    static constexpr int BS = D * D * 2;               // S, MN-major bf16
-    static constexpr int BZ = 16 * D * 2;              // z row + 15 zero rows, K-major
-    static constexpr int ACC = D + 16;                 // accumulator columns per buffer
-    static constexpr uint32_t TMEM_COLS = D == 64 ? 256 : 512;
-    static constexpr int BARS = 3 * STAGES + 4;
-    // d = 64 pads shared memory so that at most two CTAs share an SM (their
-    // TMEM allocations then always fit side by side).
-    static constexpr size_t SMEM_USED = 1024 + (size_t)STAGES * TILE + BS + BZ + 8 * BARS + 16;
-    static constexpr size_t SMEM = D == 64 ? (SMEM_USED > 80 * 1024 ? SMEM_USED : 80 * 1024) : SMEM_USED;
-};
-
-template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1)
-tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const float* __restrict__ S,
-                  const float* __restrict__ z, __nv_bfloat16* __restrict__ out, int N, int phi,
-                  int normalize, uint32_t* __restrict__ err) {
-    using C = RoCfg<D>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* tiles = align1024(smem_raw);
-    uint8_t* bS = tiles + C::STAGES * C::TILE;
-    uint8_t* bZ = bS + C::BS;
-    uint64_t* full = reinterpret_cast<uint64_t*>(bZ + C::BZ);
-    uint64_t* tdone = full + C::STAGES;
-    uint64_t* empty = tdone + C::STAGES;
-    uint64_t* acc_full = empty + C::STAGES;   // [2]
-    uint64_t* acc_empty = acc_full + 2;       // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int bh = blockIdx.y;
-    const int ntiles_head = (N + kTile - 1) / kTile;
-    const int my_tiles = blockIdx.x < ntiles_head ? (ntiles_head - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(full + s, 1);
-            mbar_init(tdone + s, 128);
-            mbar_init(empty + s, 1);
-        }
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(acc_full + a, 1);
-            mbar_init(acc_empty + a, 128);
-        }
-        fence_mbar_init();
-    }
-    if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
-    if (threadIdx.x == 0) tma_prefetch_map(&mQ);
-
-    // S -> bf16, MN-major (rows = d_k index a, 64-wide d_v atoms LBO = D*128 apart)
-    const float* Sh = S + (size_t)bh * D * D;
-    for (int c = threadIdx.x; c < D * D / 8; c += kTcThreads) {
-        const int a = c / (D / 8), col = (c % (D / 8)) * 8;
-        const float4 x0 = reinterpret_cast<const float4*>(Sh + (size_t)a * D + col)[0];
-        const float4 x1 = reinterpret_cast<const float4*>(Sh + (size_t)a * D + col)[1];
-        const float f[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-        *reinterpret_cast<uint4*>(bS + (col / 64) * (D * 128) + sw128_off(a, col % 64)) = pack8(f);
-    }
-    // z -> row 0 of a 16-row K-major operand (rows 1..15 zero)
-    for (int c = threadIdx.x; c < 16 * D / 8; c += kTcThreads) {
-        const int n = c / (D / 8), col = (c % (D / 8)) * 8;
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = n == 0 ? z[(size_t)bh * D + col + e] : 0.f;
-        *reinterpret_cast<uint4*>(bZ + (col / 64) * (16 * 128) + sw128_off(n, col % 64)) = pack8(f);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            int issued[C::STAGES] = {};
-            for (int it = 0; it < my_tiles; ++it) {
-                const int s = it % C::STAGES, u = it / C::STAGES;
-                if (u > 0 && !mbar_wait(empty + s, (u - 1) & 1, err)) break;
-                mbar_arrive_expect_tx(full + s, C::TILE);
-                const int tile = blockIdx.x + it * gridDim.x;
-#pragma unroll
-                for (int b = 0; b < C::NB; ++b)
-                    tma_load_3d(tiles + s * C::TILE + b * kTile * 128, &mQ, full + s, b * 64,
-                                tile * kTile, bh);
-                issued[s] = u + 1;
-            }
-            for (int s = 0; s < C::STAGES; ++s)
-                if (issued[s] > 0) mbar_wait(full + s, (issued[s] - 1) & 1, err);
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t id_s = idesc_bf16(128, D, false, true);
-            constexpr uint32_t id_z = idesc_bf16(128, 16, false, false);
-            const uint32_t sb = smem_u32(bS), zb = smem_u32(bZ);
-            for (int it = 0; it < my_tiles; ++it) {
-                const int s = it % C::STAGES, u = it / C::STAGES;
-                const int ab = it & 1, ua = it >> 1;
-                if (!mbar_wait(tdone + s, u & 1, err)) break;
-                if (ua > 0 && !mbar_wait(acc_empty + ab, (ua - 1) & 1, err)) break;
-                tc_fence_after();
-                const uint32_t qt = smem_u32(tiles + s * C::TILE);
-                const uint32_t acc = tmem + ab * C::ACC;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t a = sdesc(qt + (kk / 4) * (kTile * 128) + (kk % 4) * 32, 16, 1024);
-                    mma_bf16(acc, a, sdesc(sb + kk * 2048, D * 128, 1024), id_s, kk > 0 ? 1u : 0u);
-                    if (normalize)
-                        mma_bf16(acc + D, a, sdesc(zb + (kk / 4) * (16 * 128) + (kk % 4) * 32, 16, 1024),
-                                 id_z, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(empty + s);
-                mma_commit(acc_full + ab);
-            }
-        }
-    } else {
-        const int et = threadIdx.x - 64;
-        const int sp = warp & 3;
-        const bool relu = phi == PHI_RELU1;
-        bool ok = true;
-        auto transform = [&](int it) {
-            const int s = it % C::STAGES, u = it / C::STAGES;
-            ok = ok && mbar_wait(full + s, u & 1, err);
-            if (!ok) return;
-            if (relu) {
-                uint4* qt = reinterpret_cast<uint4*>(tiles + s * C::TILE);
-#pragma unroll
-                for (int i = 0; i < C::NB * 8; ++i) {
-                    float f[8];
-                    unpack8(qt[et + 128 * i], f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = phi_relu1(f[e]);
-                    qt[et + 128 * i] = pack8(f);
-                }
-                fence_async_smem();
-            }
-            mbar_arrive(tdone + s);
-        };
-        auto epilogue = [&](int it) {
-            const int ab = it & 1;
-            ok = ok && mbar_wait(acc_full + ab, (it >> 1) & 1, err);
-            tc_fence_after();
-            const uint32_t acc = tmem + ab * C::ACC + (static_cast<uint32_t>(sp * 32) << 16);
-            uint32_t v[D];
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                uint32_t r[16];
-                tmem_ld16(acc + c0, r);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[c0 + e] = r[e];
-            }
-            uint32_t zr[16];
-            tmem_ld16(acc + D, zr);
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(acc_empty + ab);
-            const int tile = blockIdx.x + it * gridDim.x;
-            const int tok = tile * kTile + sp * 32 + lane;
-            if (!ok || tok >= N) return;
-            const float den = __uint_as_float(zr[0]);
-            uint4* o = reinterpret_cast<uint4*>(out + ((size_t)bh * N + tok) * D);
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 8) {
-                float f[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float num = __uint_as_float(v[c0 + e]);
-                    f[e] = normalize ? num / den : num;
-                }
-                o[c0 / 8] = pack8(f);
-            }
-        };
-        if (my_tiles > 0) transform(0);
-        for (int it = 0; it < my_tiles; ++it) {
-            if (it + 1 < my_tiles) transform(it + 1);
-            epilogue(it);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, C::TMEM_COLS);
-    }
-}
 
 // ---------------------------------------------------------------------------
 // Chunked causal / prefix-mask outputs of one block
@@ -469,7 +47,7 @@ struct SwCfg {
     static constexpr int ROWS = GATHER ? 2 * 2 * C * 4 : 0;  // token / limit per row (x2)
     static constexpr int COL_S = 0, COL_Z = D, COL_P = D + 16, COL_O = D + 16 + C, COL_OZ = 2 * D + 16 + C;
     static constexpr uint32_t TMEM_COLS = (2 * D + 32 + C) <= 256 ? 256u : 512u;
-    static constexpr int NBAR = 2 * STAGES + 8;
+    static constexpr int NBAR = 2 * STAGES + 9;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + PT + 2 * B3 + 2 * BZ + ONES + QG +
                                    ROWS + 8 * NBAR + 16;
     static constexpr int THREADS = 320;
@@ -502,9 +80,12 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     uint64_t* bpfull = bsdone + 1;
     uint64_t* bptready = bpfull + 1;
     uint64_t* bofull = bptready + 1;
-    uint64_t* bofree = bofull + 1;  // [2], one per query-tile slot
-    uint64_t* bqready = bofree + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bqready + 1);
+    // Barriers with one phase per query tile whose producer can run two
+    // tiles ahead of a waiter are kept per slot (tile t uses slot t % 2), so
+    // that no waiter is ever two phases behind (parity waits would alias).
+    uint64_t* bofree = bofull + 1;   // [2]
+    uint64_t* bqready = bofree + 2;  // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bqready + 2);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int blk = blockIdx.x;
@@ -536,6 +117,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         mbar_init(bofree, 128);
         mbar_init(bofree + 1, 128);
         mbar_init(bqready, 128);
+        mbar_init(bqready + 1, 128);
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, CF::TMEM_COLS);
@@ -605,7 +187,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 const int ntq = q_tiles(c_begin + ci);
                 for (int t = 0; t < ntq && ok; ++t, ++tq) {
                     const uint32_t qt = GATHER ? smem_u32(qg + (tq & 1) * CF::TILE) : st;
-                    if (GATHER) ok = mbar_wait(bqready, tq & 1, err);
+                    if (GATHER) ok = mbar_wait(bqready + (tq & 1), (tq >> 1) & 1, err);
                     if (ok && tq > 0) ok = mbar_wait(bptready, (tq - 1) & 1, err);  // P read by the mask warps
                     if (!ok) break;
                     tc_fence_after();
@@ -695,17 +277,14 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             for (int i = 0; i < CF::NB * C / 16; ++i) {
                 const int p = et + 128 * i;
                 const int r = (p % (C * 8)) >> 3;
-                float f[8];
-                unpack8(kt[p], f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = r < kvalid ? phi_apply(f[e], phi) : 0.f;
-                kt[p] = pack8(f);
+                if (r < kvalid) {
+                    if (relu) kt[p] = phi_relu1_x8(kt[p]);
+                } else {
+                    kt[p] = make_uint4(0, 0, 0, 0);
+                }
                 if (!GATHER && relu) {
                     uint4* qt = reinterpret_cast<uint4*>(st);
-                    unpack8(qt[p], f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = phi_relu1(f[e]);
-                    qt[p] = pack8(f);
+                    qt[p] = phi_relu1_x8(qt[p]);
                 }
             }
             if (ci > 0) {
@@ -790,20 +369,16 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                     uint8_t* q = qg + slot * CF::TILE;
                     for (int p = et; p < C * D / 8; p += 128) {
                         const int r = p / (D / 8), col = (p % (D / 8)) * 8;
-                        float f[8];
                         const int i = srow[r];
+                        uint4 w = make_uint4(0, 0, 0, 0);
                         if (i >= 0) {
-                            unpack8(ldg_stream(Qg + hoff + (size_t)i * D + col), f);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) f[e] = phi_apply(f[e], phi);
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) f[e] = 0.f;
+                            w = ldg_stream(Qg + hoff + (size_t)i * D + col);
+                            if (relu) w = phi_relu1_x8(w);
                         }
-                        *reinterpret_cast<uint4*>(q + (col / 64) * (C * 128) + sw128_off(r, col % 64)) = pack8(f);
+                        *reinterpret_cast<uint4*>(q + (col / 64) * (C * 128) + sw128_off(r, col % 64)) = w;
                     }
                     fence_async_smem();
-                    mbar_arrive(bqready);
+                    mbar_arrive(bqready + slot);
                 }
             }
         }
@@ -892,15 +467,13 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 float den = rs + __uint_as_float(oz[0]) + __uint_as_float(oz[1]);
                 if (C == 64) den = __shfl_sync(0xffffffffu, den, lane & 15);
                 if (ok && tok >= 0) {
+                    const float inv = normalize ? __frcp_rn(den) : 1.0f;
                     uint4* dst = reinterpret_cast<uint4*>(out + hoff + (size_t)tok * D + half * SEG);
 #pragma unroll
                     for (int g = 0; g < SEG / 8; ++g) {
                         float f[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float num = __uint_as_float(o[8 * g + e]);
-                            f[e] = normalize ? num / den : num;
-                        }
+                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[8 * g + e]) * inv;
                         dst[g] = pack8(f);
                     }
                 }
@@ -913,70 +486,6 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         tc_fence_after();
         tmem_dealloc(tmem, CF::TMEM_COLS);
     }
-}
-
-// ---------------------------------------------------------------------------
-// Host side
-// ---------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// [BH, N, d] bf16 viewed as 3-D; 64-column x `rows` boxes, 128-byte swizzle,
-// zero fill outside the tensor.
-cudaError_t make_map(CUtensorMap* map, const void* base, int d, int N, long long bh, int rows) {
-    auto fn = encode_fn();
-    if (fn == nullptr) return cudaErrorNotSupported;
-    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)bh};
-    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                          box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
-template <int D>
-cudaError_t launch_kv(const Problem& p, const void* k, const void* v, int tps, int nsplit, float* part,
-                      uint32_t* err, cudaStream_t st) {
-    CUtensorMap mk, mv;
-    cudaError_t e = make_map(&mk, k, D, p.N, p.bh(), kTile);
-    if (e == cudaSuccess) e = make_map(&mv, v, D, p.N, p.bh(), kTile);
-    if (e != cudaSuccess) return e;
-    constexpr size_t smem = KvCfg<D>::SMEM;
-    e = ensure_smem<tc_kv_partial_kernel<D>>(smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid(nsplit, (unsigned)p.bh());
-    tc_kv_partial_kernel<D><<<grid, kTcThreads, smem, st>>>(mk, mv, p.N, tps, nsplit, p.phi, part, err);
-    return cudaGetLastError();
-}
-
-template <int D>
-cudaError_t launch_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,
-                           uint32_t* err, cudaStream_t st) {
-    CUtensorMap mq;
-    cudaError_t e = make_map(&mq, q, D, p.N, p.bh(), kTile);
-    if (e != cudaSuccess) return e;
-    constexpr size_t smem = RoCfg<D>::SMEM;
-    e = ensure_smem<tc_readout_kernel<D>>(smem);
-    if (e != cudaSuccess) return e;
-    const int ntiles = (p.N + kTile - 1) / kTile;
-    const long long want = std::max(1LL, (2LL * 148 + p.bh() - 1) / p.bh());
-    const int gx = (int)std::min<long long>(ntiles, want);
-    dim3 grid(gx, (unsigned)p.bh());
-    tc_readout_kernel<D><<<grid, kTcThreads, smem, st>>>(mq, S, z, static_cast<__nv_bfloat16*>(out), p.N,
-                                                         p.phi, p.normalize, err);
-    return cudaGetLastError();
 }
 
 template <int D, int C, bool GATHER>
@@ -1002,23 +511,6 @@ cudaError_t launch_chunked(const Problem& p, const void* q, const void* k, const
 }
 
 }  // namespace
-
-bool tc_supported(const Problem& p) { return p.dtype == DT_BF16 && (p.d == 64 || p.d == 128); }
-
-int tc_chunk(const Problem& p, int chunk) { return p.d == 128 ? 64 : chunk; }
-
-cudaError_t tc_kv_partial(const Problem& p, const void* k, const void* v, int tps, int nsplit, float* part,
-                          uint32_t* err, cudaStream_t st) {
-    if (tps % kTile != 0) return cudaErrorInvalidValue;
-    return p.d == 64 ? launch_kv<64>(p, k, v, tps, nsplit, part, err, st)
-                     : launch_kv<128>(p, k, v, tps, nsplit, part, err, st);
-}
-
-cudaError_t tc_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,
-                       uint32_t* err, cudaStream_t st) {
-    return p.d == 64 ? launch_readout<64>(p, q, S, z, out, err, st)
-                     : launch_readout<128>(p, q, S, z, out, err, st);
-}
 
 cudaError_t tc_chunked(const Problem& p, int chunk, const void* q, const void* k, const void* v,
                        const float* prefix, int block_tokens, int nblk, const int32_t* perm,

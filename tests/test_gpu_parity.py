@@ -198,3 +198,40 @@ def test_worked_example_on_gpu(golden_dir):
     out = la.la_noncausal(q, k, v)
     ref = oracle.batched(oracle.noncausal, f64(q), f64(k), f64(v))
     assert oracle.max_row_rel_err(f64(out), ref) < 1e-6
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("chunk", [64, 128])
+def test_prefix_mask_many_query_tiles_per_bin(d, chunk):
+    """Masks whose values cluster on a few positions put hundreds of queries
+    into one bin, so a chunk answers many query tiles back to back; repeated
+    calls exercise the pipelining of those tiles."""
+    B, H, N = 2, 3, 1500
+    q, k, v = qkv(B, H, N, d, "bf16", seed=31 + d)
+    gen = torch.Generator().manual_seed(5)
+    choices = torch.tensor([0, 63, 64, 127, 128, 700, N - 1], dtype=torch.int32)
+    m = choices[torch.randint(0, len(choices), (B, N), generator=gen)].contiguous().cuda()
+    ref = oracle.batched(oracle.prefix_mask, f64(q), f64(k), f64(v), m=m.cpu().numpy())
+    ws = la.workspace(la._desc_of(q, "relu1", True), "prefix", chunk)
+    for _ in range(10):
+        out = la.la_prefix_mask(q, k, v, m, chunk=chunk, ws=ws)
+        assert oracle.max_row_rel_err(f64(out), ref) < 2e-2
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("B,H,N", [(4, 40, 300), (8, 50, 1), (2, 100, 129), (1, 3, 20000)])
+def test_balanced_split_ranges_cross_heads(d, B, H, N):
+    """The KV summary and readout split the flattened (head, 128-token tile)
+    sequence evenly over the SMs, so one CTA's range can cover the end of
+    one head and the start of the next, or several whole heads."""
+    q, k, v = qkv(B, H, N, d, "bf16", seed=B * H + N)
+    S = torch.empty(B, H, d, d, device="cuda")
+    z = torch.empty(B, H, d, device="cuda")
+    out = la.la_noncausal(q, k, v, S_out=S, z_out=z)
+    Q, K, V = f64(q), f64(k), f64(v)
+    S_ref, z_ref = oracle.kv_summary_batched(K, V)
+    assert oracle.max_row_rel_err(f64(S), S_ref) < 1e-5
+    np.testing.assert_allclose(f64(z), z_ref, rtol=1e-5)
+    ref = np.einsum("bhna,bhac->bhnc", oracle.phi(Q), S_ref) / \
+        np.einsum("bhna,bha->bhn", oracle.phi(Q), z_ref)[..., None]
+    assert oracle.max_row_rel_err(f64(out), ref) < 2e-2
