@@ -53,25 +53,47 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  "r"(bytes)
                  : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// One try_wait: the thread may be suspended in hardware until the phase
+// completes or about `hint_ns` pass, whichever is first.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
         : "memory");
     return ok != 0;
 }
-// Waits for the phase with the given parity to complete. Gives up after
-// kWaitTimeoutNs, sets FLAG_TIMEOUT in *err and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Per-CTA abort flag: set by the first wait that expires. From then on every
+// abortable wait of the CTA returns at once, so the warps run through the
+// rest of their schedule without waiting and reach every named barrier and
+// the final __syncthreads together. Kernels clear it with cta_abort_reset()
+// before their first __syncthreads.
+__device__ __forceinline__ volatile int* cta_abort() {
+    __shared__ int flag;
+    return &flag;
+}
+__device__ __forceinline__ void cta_abort_reset() { *cta_abort() = 0; }
+
+// Waits for the phase with the given parity to complete. The waiting thread
+// sleeps in try_wait (no polling); the clock is read only between sleeps.
+// Gives up after kWaitTimeoutNs: sets FLAG_TIMEOUT in *err and the CTA's
+// abort flag, returns false. An abortable wait also returns false at once
+// when the abort flag is set; the end-of-kernel waits for a CTA's own copies
+// in flight are not abortable (but still bounded).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                          bool abortable = true) {
+    constexpr uint32_t kHintNs = 100000;
+    if (mbar_try_wait(bar, parity, kHintNs)) return true;
+    volatile int* ab = cta_abort();
     const uint64_t t0 = globaltimer();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait(bar, parity, kHintNs)) {
+        if (abortable && *ab) return false;
         if (globaltimer() - t0 > kWaitTimeoutNs) {
             atomicOr(err, FLAG_TIMEOUT);
+            *ab = 1;
             return false;
         }
     }
@@ -93,6 +115,23 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
+// 3-D tiled store from shared memory (bulk group). Parts of the box outside
+// the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+        "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until the shared-memory sources of this thread's bulk stores may be
+// reused (the stores may still be in flight to global memory).
+__device__ __forceinline__ void bulk_wait_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Waits until this thread's bulk stores have completed.
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Orders this thread's generic-proxy shared-memory accesses before later
 // async-proxy (TMA / tcgen05) accesses.
 __device__ __forceinline__ void fence_async_smem() {

@@ -1,13 +1,14 @@
 // KV summary and readout on tcgen05 tensor cores (bf16, d = 64 or 128).
 //
 // KV summary ("nx_f32_linear_attention.nx source", KV-summary loop):
-//   S = phi(K)^T V and z = phi(K)^T 1 over a token range, as MMAs with the
-//   tokens as the contraction dimension; TMA stages 128-token K and V tiles
-//   in shared memory (128-byte swizzle). For phi = relu+1 the K operand is
-//   relu(K), which is exact in bf16, and the "+1" is added exactly:
-//   S = relu(K)^T V + 1 (x) colsum(V) and z = relu(K)^T 1 + count, where
-//   colsum(V) comes from an MMA with an all-ones A operand. Accumulation is
-//   fp32 in TMEM throughout, so S and z carry no bf16 rounding of phi(K).
+//   S = phi(K)^T V over a token range as MMAs with the tokens as the
+//   contraction dimension; TMA stages 128-token K and V tiles in shared
+//   memory (128-byte swizzle). For phi = relu+1 the K operand is relu(K),
+//   which is exact in bf16, and the "+1" is added exactly:
+//   S = relu(K)^T V + 1 (x) colsum(V) and z = sum relu(K) + count. The
+//   column sums of relu(K) and V are fp32 sums taken by the warps that
+//   prepare each tile; S accumulates in fp32 in TMEM. So S and z carry no
+//   bf16 rounding of phi(K).
 // Readout (nx source, per-query loop):
 //   out = phi(Q) S / (phi(Q) . z): MMA with M = 128 tokens, N = d_v,
 //   K = d_k against S (bf16, MN-major) plus an N = 16 MMA against
@@ -109,11 +110,10 @@ struct KvCfg {
     static constexpr int NB = D / 64;                 // 64-column boxes per tile
     static constexpr int TILE = kTile * D * 2;        // bytes of a K or V tile
     static constexpr int STAGES = D == 64 ? 4 : 3;
-    static constexpr int ONES = kTile * 128;          // all-ones operand
-    static constexpr int COL_S = 0, COL_CS = D, COL_Z = 2 * D;
-    static constexpr uint32_t TMEM_COLS = (2 * D + 16) <= 256 ? 256u : 512u;
+    static constexpr int RED = 128 * 2 * NB * 8 * 4 + D * 4;  // per-thread column sums, colsum(V)
+    static constexpr uint32_t TMEM_COLS = D <= 64 ? 64u : 128u;
     static constexpr int BARS = 3 * STAGES + 1;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * 2 * TILE + ONES + 8 * BARS + 16;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * 2 * TILE + RED + 8 * BARS + 16;
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -125,8 +125,9 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
     constexpr size_t REC = (size_t)D * D + D;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles = align1024(smem_raw);
-    uint8_t* ones = tiles + C::STAGES * 2 * C::TILE;
-    uint64_t* full = reinterpret_cast<uint64_t*>(ones + C::ONES);
+    float* red = reinterpret_cast<float*>(tiles + C::STAGES * 2 * C::TILE);
+    float* csum = red + 128 * 2 * C::NB * 8;
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + C::RED);
     uint64_t* tdone = full + C::STAGES;
     uint64_t* empty = tdone + C::STAGES;
     uint64_t* segdone = empty + C::STAGES;
@@ -137,6 +138,7 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
     const bool relu = phi == PHI_RELU1;
 
     if (threadIdx.x == 0) {
+        cta_abort_reset();
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(full + s, 1);
             mbar_init(tdone + s, 128);
@@ -148,11 +150,6 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
         tma_prefetch_map(&mV);
     }
     if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
-    {
-        const uint4 one8 = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-        for (int c = threadIdx.x; c < C::ONES / 16; c += kThreads) reinterpret_cast<uint4*>(ones)[c] = one8;
-        fence_async_smem();
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -182,14 +179,11 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
             }
             // no copy may still be landing when the CTA exits
             for (int s = 0; s < C::STAGES; ++s)
-                if (issued[s] > 0) mbar_wait(full + s, (issued[s] - 1) & 1, err);
+                if (issued[s] > 0) mbar_wait(full + s, (issued[s] - 1) & 1, err, false);
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t id_s = idesc_bf16(D, D, true, true);     // S += K^T V
-            constexpr uint32_t id_cs = idesc_bf16(64, D, true, true);   // rows = colsum(V)
-            constexpr uint32_t id_z = idesc_bf16(D, 16, true, false);   // z += K^T 1
-            const uint32_t ob = smem_u32(ones);
+            constexpr uint32_t id_s = idesc_bf16(D, D, true, true);  // S += K^T V
             int it = 0;
             bool ok = true;
             for (int j = 0; j < nseg && ok; ++j) {
@@ -202,15 +196,9 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
                     const uint32_t kt = smem_u32(tiles + s * 2 * C::TILE);
                     const uint32_t vt = kt + C::TILE;
 #pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk) {
-                        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-                        const uint64_t a = sdesc(kt + kk * 2048, kTile * 128, 1024);
-                        const uint64_t b = sdesc(vt + kk * 2048, kTile * 128, 1024);
-                        mma_bf16(tmem + C::COL_S, a, b, id_s, acc);
-                        if (relu) mma_bf16(tmem + C::COL_CS, sdesc(ob + kk * 2048, kTile * 128, 1024), b, id_cs, acc);
-                        mma_bf16(tmem + C::COL_Z, a, sdesc(ob + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024), id_z,
-                                 acc);
-                    }
+                    for (int kk = 0; kk < kTile / 16; ++kk)
+                        mma_bf16(tmem, sdesc(kt + kk * 2048, kTile * 128, 1024),
+                                 sdesc(vt + kk * 2048, kTile * 128, 1024), id_s, (i > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(empty + s);
                 }
                 mma_commit(segdone);
@@ -220,86 +208,115 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
         const int et = threadIdx.x - 64;  // 0..127
         const int sp = warp & 3;
         const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
+        // The thread always touches the same 16-byte chunk position of each
+        // 128-byte row, so within a 64-column box it owns one group of 8
+        // columns, (et % 8) xor ((et / 8) % 8); the column sums below rely
+        // on that.
+        // No early exit here: after a failed wait the loop runs on without
+        // waiting (see cta_abort), so the named barriers stay matched.
         int it = 0;
-        bool ok = true;
-        for (int j = 0; j < nseg && ok; ++j) {
+        for (int j = 0; j < nseg; ++j) {
             const Seg sg = kv_seg(w, N, j);
             const int nt = (sg.t1 - sg.t0 + kTile - 1) / kTile;
+            float zk[C::NB][8], cv[C::NB][8];  // column sums of relu(K) (or K) and of V
+#pragma unroll
+            for (int b = 0; b < C::NB; ++b)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) zk[b][e] = cv[b][e] = 0.f;
             for (int i = 0; i < nt; ++i, ++it) {
                 const int s = it % C::STAGES, u = it / C::STAGES;
-                if (!(ok = mbar_wait(full + s, u & 1, err))) break;
+                mbar_wait(full + s, u & 1, err);
                 const int valid = min(kTile, sg.t1 - (sg.t0 + i * kTile));
-                if (relu || valid < kTile) {
-                    uint4* kt = reinterpret_cast<uint4*>(tiles + s * 2 * C::TILE);
+                uint4* kt = reinterpret_cast<uint4*>(tiles + s * 2 * C::TILE);
+                const uint4* vt = reinterpret_cast<const uint4*>(tiles + s * 2 * C::TILE + C::TILE);
 #pragma unroll
-                    for (int q = 0; q < C::NB * 8; ++q) {
-                        const int p = et + 128 * q;       // 16-byte chunk index
-                        const int r = (p & 1023) >> 3;    // token row in the tile
-                        if (r < valid) {
-                            if (relu) kt[p] = relu_x8(kt[p]);
-                        } else {
-                            kt[p] = make_uint4(0, 0, 0, 0);
+                for (int q = 0; q < C::NB * 8; ++q) {
+                    const int p = et + 128 * q;      // 16-byte chunk index
+                    const int b = q / 8;             // 64-column box
+                    const int r = (p & 1023) >> 3;   // token row in the tile
+                    uint4 wk = kt[p];
+                    if (r < valid) {
+                        if (relu) {
+                            wk = relu_x8(wk);
+                            kt[p] = wk;
                         }
+                    } else {
+                        wk = make_uint4(0, 0, 0, 0);
+                        kt[p] = wk;
                     }
-                    fence_async_smem();
+                    float f[8];
+                    unpack8(wk, f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) zk[b][e] += f[e];
+                    if (relu) {  // rows past the end of the head are zero in V (TMA fill)
+                        unpack8(vt[p], f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) cv[b][e] += f[e];
+                    }
                 }
+                fence_async_smem();
                 mbar_arrive(tdone + s);
             }
-            if (!ok) break;
-            // epilogue of segment j: TMEM -> record (S rows, then z)
-            ok = mbar_wait(segdone, j & 1, err);
-            tc_fence_after();
+            // column sums: the 16 threads of a column group add up their parts
+#pragma unroll
+            for (int b = 0; b < C::NB; ++b)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    red[(et * 2 + 0) * C::NB * 8 + b * 8 + e] = zk[b][e];
+                    red[(et * 2 + 1) * C::NB * 8 + b * 8 + e] = cv[b][e];
+                }
+            named_bar(1, 128);
             float* rec = part + (size_t)sg.slot * REC;
-            const float cnt = relu ? (float)(sg.t1 - sg.t0) : 0.0f;
+            if (et < D) {
+                const int b = et / 64, g = (et % 64) / 8, e = et % 8;
+                float zs = relu ? (float)(sg.t1 - sg.t0) : 0.f;
+                float cs = 0.f;
+                for (int t = 0; t < 128; ++t) {
+                    if ((((t & 7) ^ ((t >> 3) & 7))) == g) {
+                        zs += red[(t * 2 + 0) * C::NB * 8 + b * 8 + e];
+                        cs += red[(t * 2 + 1) * C::NB * 8 + b * 8 + e];
+                    }
+                }
+                rec[(size_t)D * D + et] = zs;
+                csum[et] = relu ? cs : 0.f;
+            }
+            named_bar(1, 128);
+            // epilogue of segment j: S rows from TMEM (+ colsum(V) for phi = relu+1)
+            mbar_wait(segdone, j & 1, err);
+            tc_fence_after();
             if (D == 128) {
                 const int a = sp * 32 + lane;
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += 16) {
-                    uint32_t r[16], cs[16];
-                    tmem_ld16(tmem + C::COL_S + lane_base + c0, r);
-                    if (relu) tmem_ld16(tmem + C::COL_CS + lane_base + c0, cs);
+                    uint32_t r[16];
+                    tmem_ld16(tmem + lane_base + c0, r);
                     tmem_ld_wait();
-                    float f[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        // lanes 0..15 of the M = 64 colsum block each hold colsum(V)
-                        const float c = relu ? __uint_as_float(__shfl_sync(0xffffffffu, cs[e], lane & 15)) : 0.0f;
-                        f[e] = __uint_as_float(r[e]) + c;
-                    }
                     float4* o = reinterpret_cast<float4*>(rec + (size_t)a * D + c0);
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) o[q4] = make_float4(f[4 * q4], f[4 * q4 + 1], f[4 * q4 + 2], f[4 * q4 + 3]);
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        o[q4] = make_float4(__uint_as_float(r[4 * q4]) + csum[c0 + 4 * q4],
+                                            __uint_as_float(r[4 * q4 + 1]) + csum[c0 + 4 * q4 + 1],
+                                            __uint_as_float(r[4 * q4 + 2]) + csum[c0 + 4 * q4 + 2],
+                                            __uint_as_float(r[4 * q4 + 3]) + csum[c0 + 4 * q4 + 3]);
                 }
-                uint32_t zr[16];
-                tmem_ld16(tmem + C::COL_Z + lane_base, zr);
-                tmem_ld_wait();
-                rec[(size_t)D * D + a] = __uint_as_float(zr[0]) + cnt;
             } else {
-                // M = 64 accumulators: rows in lanes 0..15; the warp halves take column halves
+                // M = 64 accumulator: rows in lanes 0..15; the warp halves take column halves
                 const int a = sp * 16 + (lane & 15);
-                const int half = lane >> 4;
-                uint32_t r[32], cs[32];
-                tmem_ld16x2<32>(tmem + C::COL_S + lane_base, *reinterpret_cast<uint32_t(*)[16]>(r));
-                tmem_ld16x2<32>(tmem + C::COL_S + lane_base + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
-                if (relu) {
-                    tmem_ld16x2<32>(tmem + C::COL_CS + lane_base, *reinterpret_cast<uint32_t(*)[16]>(cs));
-                    tmem_ld16x2<32>(tmem + C::COL_CS + lane_base + 16, *reinterpret_cast<uint32_t(*)[16]>(cs + 16));
-                }
-                uint32_t zr[2];
-                tmem_ld2(tmem + C::COL_Z + lane_base, zr);
+                const int c0 = 32 * (lane >> 4);
+                uint32_t r[32];
+                tmem_ld16x2<32>(tmem + lane_base, *reinterpret_cast<uint32_t(*)[16]>(r));
+                tmem_ld16x2<32>(tmem + lane_base + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
                 tmem_ld_wait();
-                float4* o = reinterpret_cast<float4*>(rec + (size_t)a * D + 32 * half);
+                float4* o = reinterpret_cast<float4*>(rec + (size_t)a * D + c0);
 #pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                    float f[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        f[e] = __uint_as_float(r[4 * q4 + e]) + (relu ? __uint_as_float(cs[4 * q4 + e]) : 0.0f);
-                    o[q4] = make_float4(f[0], f[1], f[2], f[3]);
-                }
-                if (lane < 16) rec[(size_t)D * D + a] = __uint_as_float(zr[0]) + cnt;
+                for (int q4 = 0; q4 < 8; ++q4)
+                    o[q4] = make_float4(__uint_as_float(r[4 * q4]) + csum[c0 + 4 * q4],
+                                        __uint_as_float(r[4 * q4 + 1]) + csum[c0 + 4 * q4 + 1],
+                                        __uint_as_float(r[4 * q4 + 2]) + csum[c0 + 4 * q4 + 2],
+                                        __uint_as_float(r[4 * q4 + 3]) + csum[c0 + 4 * q4 + 3]);
             }
             tc_fence_before();
+            named_bar(1, 128);  // `red` is reused by the next segment
         }
     }
     tc_fence_before();
@@ -350,22 +367,24 @@ struct RoCfg {
     static constexpr int ACC = D + 16;                 // accumulator columns per buffer
     static constexpr uint32_t TMEM_COLS = D == 64 ? 256 : 512;
     static constexpr int BARS = 3 * STAGES + 4;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * TILE + 2 * BS + 2 * BZ + 8 * BARS + 16;
+    // Q stages, S and z operands (x2), the output staging tile
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * TILE + 2 * BS + 2 * BZ + TILE + 8 * BARS + 16;
     static constexpr int PER_SM = D == 64 ? 2 : 1;     // CTAs an SM holds (TMEM and smem)
     static_assert(SMEM * PER_SM <= 227 * 1024, "shared memory");
 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const float* __restrict__ S,
-                  const float* __restrict__ z, __nv_bfloat16* __restrict__ out, int N, long long total,
+tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mOut,
+                  const float* __restrict__ S, const float* __restrict__ z, int N, long long total,
                   int tph, int phi, int normalize, uint32_t* __restrict__ err) {
     using C = RoCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles = align1024(smem_raw);
     uint8_t* bS = tiles + C::STAGES * C::TILE;
     uint8_t* bZ = bS + 2 * C::BS;
-    uint64_t* full = reinterpret_cast<uint64_t*>(bZ + 2 * C::BZ);
+    uint8_t* stg = bZ + 2 * C::BZ;  // output tile, same layout as a Q tile
+    uint64_t* full = reinterpret_cast<uint64_t*>(stg + C::TILE);
     uint64_t* tdone = full + C::STAGES;
     uint64_t* empty = tdone + C::STAGES;
     uint64_t* acc_full = empty + C::STAGES;  // [2]
@@ -379,6 +398,7 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const float* __restric
     const long long h0 = lo / tph;
 
     if (threadIdx.x == 0) {
+        cta_abort_reset();
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(full + s, 1);
             mbar_init(tdone + s, 128);
@@ -390,6 +410,7 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const float* __restric
         }
         fence_mbar_init();
         tma_prefetch_map(&mQ);
+        tma_prefetch_map(&mOut);
     }
     if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
     for (int c = threadIdx.x; c < 2 * 16 * D / 8; c += kThreads) {  // z operand rows 2..15 stay zero
@@ -420,7 +441,7 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const float* __restric
                 issued[s] = u + 1;
             }
             for (int s = 0; s < C::STAGES; ++s)
-                if (issued[s] > 0) mbar_wait(full + s, (issued[s] - 1) & 1, err);
+                if (issued[s] > 0) mbar_wait(full + s, (issued[s] - 1) & 1, err, false);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -506,16 +527,25 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const float* __restric
             tc_fence_before();
             mbar_arrive(acc_empty + ab);
             const long long g = lo + it;
-            const int tok = (int)(g % tph) * kTile + sp * 32 + lane;
-            if (!ok || tok >= N) return;
+            // the staging tile is free once the previous tile's store has read it
+            if (et == 0) bulk_wait_read0();
+            named_bar(2, 128);
+            const int r = sp * 32 + lane;  // row of the tile
             const float inv = normalize ? __frcp_rn(__uint_as_float(zr[0]) + __uint_as_float(zr[1])) : 1.0f;
-            uint4* o = reinterpret_cast<uint4*>(out + ((size_t)(g / tph) * N + tok) * D);
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 8) {
                 float f[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[c0 + e]) * inv;
-                o[c0 / 8] = pack8(f);
+                *reinterpret_cast<uint4*>(stg + (c0 / 64) * (kTile * 128) + sw128_off(r, c0 % 64)) = pack8(f);
+            }
+            fence_async_smem();
+            named_bar(2, 128);
+            if (et == 0 && ok) {
+#pragma unroll
+                for (int b = 0; b < C::NB; ++b)
+                    tma_store_3d(&mOut, stg + b * (kTile * 128), b * 64, (int)(g % tph) * kTile, (int)(g / tph));
+                bulk_commit();
             }
         };
         if (ntile > 0) transform(0);
@@ -523,6 +553,7 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const float* __restric
             if (it + 1 < ntile) transform(it + 1);
             epilogue(it);
         }
+        if (et == 0) bulk_wait0();
     }
     tc_fence_before();
     __syncthreads();
@@ -549,8 +580,9 @@ cudaError_t launch_kv(const Problem& p, const void* k, const void* v, const KvWo
 template <int D>
 cudaError_t launch_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,
                            uint32_t* err, cudaStream_t st) {
-    CUtensorMap mq;
+    CUtensorMap mq, mo;
     cudaError_t e = make_map(&mq, q, D, p.N, p.bh(), kTile);
+    if (e == cudaSuccess) e = make_map(&mo, out, D, p.N, p.bh(), kTile);
     if (e != cudaSuccess) return e;
     constexpr size_t smem = RoCfg<D>::SMEM;
     e = ensure_smem<tc_readout_kernel<D>>(smem);
@@ -558,8 +590,7 @@ cudaError_t launch_readout(const Problem& p, const void* q, const float* S, cons
     const int tph = (p.N + kTile - 1) / kTile;
     const long long total = p.bh() * tph;
     const int G = (int)std::min<long long>(total, 148LL * RoCfg<D>::PER_SM);
-    tc_readout_kernel<D><<<G, kThreads, smem, st>>>(mq, S, z, static_cast<__nv_bfloat16*>(out), p.N, total, tph,
-                                                    p.phi, p.normalize, err);
+    tc_readout_kernel<D><<<G, kThreads, smem, st>>>(mq, mo, S, z, p.N, total, tph, p.phi, p.normalize, err);
     return cudaGetLastError();
 }
 

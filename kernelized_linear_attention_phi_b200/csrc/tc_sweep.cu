@@ -45,11 +45,12 @@ struct SwCfg {
     static constexpr int ONES = 16 * C * 2;          // all-ones B operand, 16 x C, K-major
     static constexpr int QG = GATHER ? 2 * TILE : 0; // gathered queries (x2)
     static constexpr int ROWS = GATHER ? 2 * 2 * C * 4 : 0;  // token / limit per row (x2)
+    static constexpr int STG = GATHER ? 0 : TILE;    // output staging tile (causal: one TMA store)
     static constexpr int COL_S = 0, COL_Z = D, COL_P = D + 16, COL_O = D + 16 + C, COL_OZ = 2 * D + 16 + C;
     static constexpr uint32_t TMEM_COLS = (2 * D + 32 + C) <= 256 ? 256u : 512u;
     static constexpr int NBAR = 2 * STAGES + 9;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + PT + 2 * B3 + 2 * BZ + ONES + QG +
-                                   ROWS + 8 * NBAR + 16;
+                                   STG + ROWS + 8 * NBAR + 16;
     static constexpr int THREADS = 320;
     static constexpr int MIN_BLOCKS = (D == 64 && C == 64) ? 2 : 1;
     static_assert(C == 64 || C == 128, "chunk");
@@ -59,7 +60,8 @@ struct SwCfg {
 template <int D, int C, bool GATHER>
 __global__ void __launch_bounds__(SwCfg<D, C, GATHER>::THREADS, SwCfg<D, C, GATHER>::MIN_BLOCKS)
 tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
-                const __grid_constant__ CUtensorMap mV, const __nv_bfloat16* __restrict__ Qg,
+                const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mOut,
+                const __nv_bfloat16* __restrict__ Qg,
                 const float* __restrict__ prefix, int H, int N, int block_tokens, int nblk,
                 const int32_t* __restrict__ perm, const int32_t* __restrict__ bin_start,
                 const int32_t* __restrict__ mcl, int nbins, int phi, int normalize,
@@ -72,7 +74,8 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     uint8_t* bz = b3 + 2 * CF::B3;
     uint8_t* ones = bz + 2 * CF::BZ;
     uint8_t* qg = ones + CF::ONES;
-    int* rows = reinterpret_cast<int*>(qg + CF::QG);  // [slot][srow C | slim C]
+    uint8_t* stg = qg + CF::QG;
+    int* rows = reinterpret_cast<int*>(stg + CF::STG);  // [slot][srow C | slim C]
     uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(rows) + CF::ROWS);
     uint64_t* empty = full + CF::STAGES;
     uint64_t* bprep = empty + CF::STAGES;
@@ -105,6 +108,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     };
 
     if (threadIdx.x == 0) {
+        cta_abort_reset();
         for (int s = 0; s < CF::STAGES; ++s) {
             mbar_init(full + s, 1);
             mbar_init(empty + s, 1);
@@ -122,7 +126,10 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     }
     if (warp == 1) tmem_alloc(tmem_slot, CF::TMEM_COLS);
     if (threadIdx.x == 0) {
-        if (!GATHER) tma_prefetch_map(&mQ);
+        if (!GATHER) {
+            tma_prefetch_map(&mQ);
+            tma_prefetch_map(&mOut);
+        }
         tma_prefetch_map(&mK);
         tma_prefetch_map(&mV);
     }
@@ -151,7 +158,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 issued[s] = u + 1;
             }
             for (int s = 0; s < CF::STAGES; ++s)
-                if (issued[s] > 0) mbar_wait(full + s, (issued[s] - 1) & 1, err);
+                if (issued[s] > 0) mbar_wait(full + s, (issued[s] - 1) & 1, err, false);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -263,16 +270,16 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             }
             tmem_st_wait();
         }
-        bool ok = true;
+        // No early exit in this warpgroup: after a failed wait the loops run on
+        // without waiting (see cta_abort), so the named barriers stay matched.
         int tq = 0;
-        for (int ci = 0; ci < nci && ok; ++ci) {
+        for (int ci = 0; ci < nci; ++ci) {
             const int c = c_begin + ci;
             const int s = ci % CF::STAGES, u = ci / CF::STAGES;
             const int kvalid = c < nchunks ? min(C, N - c * C) : 0;
             uint8_t* st = stages + s * CF::STAGE;
             uint4* kt = reinterpret_cast<uint4*>(st + (GATHER ? 0 : CF::TILE));
-            ok = mbar_wait(full + s, u & 1, err);
-            if (!ok) break;
+            mbar_wait(full + s, u & 1, err);
 #pragma unroll 4
             for (int i = 0; i < CF::NB * C / 16; ++i) {
                 const int p = et + 128 * i;
@@ -288,7 +295,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 }
             }
             if (ci > 0) {
-                ok = mbar_wait(bsdone, (ci - 1) & 1, err);
+                mbar_wait(bsdone, (ci - 1) & 1, err);
                 tc_fence_after();
             }
             // S_prev -> bf16 MN-major operand (rows = d_k index)
@@ -348,10 +355,9 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 const int ntq = q_tiles(c);
                 const int qbase = bin_start[(size_t)b * (nbins + 1) + c];
                 const int qend = bin_start[(size_t)b * (nbins + 1) + c + 1];
-                for (int t = 0; t < ntq && ok; ++t, ++tq) {
+                for (int t = 0; t < ntq; ++t, ++tq) {
                     const int slot = tq & 1;
-                    if (tq >= 2) ok = mbar_wait(bofree + slot, ((tq >> 1) - 1) & 1, err);
-                    if (!ok) break;
+                    if (tq >= 2) mbar_wait(bofree + slot, ((tq >> 1) - 1) & 1, err);
                     int* srow = rows + slot * 2 * C;
                     int* slim = srow + C;
                     if (et < C) {
@@ -390,15 +396,17 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         // 0..15, the two halves of the warp take the two column halves.
         const int i = C == 128 ? sp * 32 + lane : sp * 16 + (lane & 15);
         const int half = (C == 64 && lane >= 16) ? 1 : 0;
+        // No early exit in this warpgroup either (named barrier 3 in the
+        // causal epilogue); a failed wait only suppresses the output stores.
         bool ok = true;
         int tq = 0;
-        for (int ci = 0; ci < nci && ok; ++ci) {
+        for (int ci = 0; ci < nci; ++ci) {
             const int c = c_begin + ci;
             const int kvalid = c < nchunks ? min(C, N - c * C) : 0;
             const int ntq = q_tiles(c);
-            for (int t = 0; t < ntq && ok; ++t, ++tq) {
+            for (int t = 0; t < ntq; ++t, ++tq) {
                 const int slot = tq & 1;
-                ok = mbar_wait(bpfull, tq & 1, err);
+                ok = mbar_wait(bpfull, tq & 1, err) && ok;
                 tc_fence_after();
                 // the row table of a gathered tile is written before its MMAs are issued
                 const int* srow = rows + slot * 2 * C;
@@ -466,8 +474,30 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 mbar_arrive(bofree + slot);
                 float den = rs + __uint_as_float(oz[0]) + __uint_as_float(oz[1]);
                 if (C == 64) den = __shfl_sync(0xffffffffu, den, lane & 15);
-                if (ok && tok >= 0) {
-                    const float inv = normalize ? __frcp_rn(den) : 1.0f;
+                const float inv = normalize ? __frcp_rn(den) : 1.0f;
+                if (!GATHER) {
+                    // causal: the chunk's rows are contiguous; stage them and
+                    // write the tile with one TMA store (rows past N are clipped)
+                    const int et2 = threadIdx.x - 192;
+                    if (et2 == 0) bulk_wait_read0();
+                    named_bar(3, 128);
+#pragma unroll
+                    for (int g = 0; g < SEG / 8; ++g) {
+                        const int col = half * SEG + 8 * g;
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[8 * g + e]) * inv;
+                        *reinterpret_cast<uint4*>(stg + (col / 64) * (C * 128) + sw128_off(i, col % 64)) = pack8(f);
+                    }
+                    fence_async_smem();
+                    named_bar(3, 128);
+                    if (et2 == 0 && ok) {
+#pragma unroll
+                        for (int bx = 0; bx < CF::NB; ++bx)
+                            tma_store_3d(&mOut, stg + bx * (C * 128), bx * 64, c * C, bh);
+                        bulk_commit();
+                    }
+                } else if (ok && tok >= 0) {
                     uint4* dst = reinterpret_cast<uint4*>(out + hoff + (size_t)tok * D + half * SEG);
 #pragma unroll
                     for (int g = 0; g < SEG / 8; ++g) {
@@ -480,6 +510,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             }
         }
     }
+    if (!GATHER && threadIdx.x == 192) bulk_wait0();  // the output stores have landed
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -494,10 +525,11 @@ cudaError_t launch_chunked(const Problem& p, const void* q, const void* k, const
                            const int32_t* bins, const int32_t* mcl, int nbins, void* out, uint32_t* err,
                            cudaStream_t st) {
     if (block_tokens % C != 0) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     cudaError_t e = make_map(&mq, q, D, p.N, p.bh(), C);
     if (e == cudaSuccess) e = make_map(&mk, k, D, p.N, p.bh(), C);
     if (e == cudaSuccess) e = make_map(&mv, v, D, p.N, p.bh(), C);
+    if (e == cudaSuccess) e = make_map(&mo, out, D, p.N, p.bh(), C);
     if (e != cudaSuccess) return e;
     using CF = SwCfg<D, C, GATHER>;
     constexpr size_t smem = CF::SMEM;
@@ -505,7 +537,7 @@ cudaError_t launch_chunked(const Problem& p, const void* q, const void* k, const
     if (e != cudaSuccess) return e;
     dim3 grid(nblk, (unsigned)p.bh());
     tc_sweep_kernel<D, C, GATHER><<<grid, CF::THREADS, smem, st>>>(
-        mq, mk, mv, static_cast<const __nv_bfloat16*>(q), prefix, p.H, p.N, block_tokens, nblk, perm, bins,
+        mq, mk, mv, mo, static_cast<const __nv_bfloat16*>(q), prefix, p.H, p.N, block_tokens, nblk, perm, bins,
         mcl, nbins, p.phi, p.normalize, static_cast<__nv_bfloat16*>(out), err);
     return cudaGetLastError();
 }
