@@ -191,6 +191,27 @@ def flush_l2(buf):
     buf.add_(1)
 
 
+def rank_seed(wl, rank):
+    """Each rank runs its own batch (weak scaling): the workload's seed
+    shifted by the rank."""
+    return wl.seed + 1000 * rank
+
+
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def aggregate_tokens_per_s(tokens_per_step, steps, world, seconds):
+    """Whole-job throughput: the tokens every rank processed over the slowest
+    rank's time."""
+    return tokens_per_step * steps * world / seconds
+
+
 def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
@@ -205,7 +226,7 @@ def run_ours(args, rank, world, local_rank):
     wl = W.WORKLOADS[args.workload]
     dtype = args.dtype if args.dtype in wl.dtypes else wl.dtypes[0]
     forms = Step.ALL_FORMS if args.workload == "multi_head" else wl.forms
-    step = Step(wl, dtype, wl.seed + 1000 * rank, device, forms)
+    step = Step(wl, dtype, rank_seed(wl, rank), device, forms)
     calls = step.calls()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
 
@@ -275,15 +296,9 @@ def run_ours(args, rank, world, local_rank):
     flags = {op: step.la.la_last_error(ws)[1] for op, ws in step.ws.items()}
     bad_flags = {op: f for op, f in flags.items() if f}
 
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([t_s, e2e_s], dtype=torch.float64, device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_s, e2e_s = float(tt[0]), float(tt[1])
-
-    tokens_all = step.tokens * K * world
-    value = tokens_all / t_s
-    e2e_value = step.tokens * Ke * world / e2e_s
+    t_s, e2e_s = max_over_ranks([t_s, e2e_s], device)
+    value = aggregate_tokens_per_s(step.tokens, K, world, t_s)
+    e2e_value = aggregate_tokens_per_s(step.tokens, Ke, world, e2e_s)
 
     # roofline of the dominant call (its kernels together), bytes per launch
     alg = step.algorithmic_bytes()
