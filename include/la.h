@@ -149,6 +149,31 @@ LA_API la_status la_decode_step(const la_desc* desc, const void* q, const void* 
                          const void* v, float* S, float* z, void* out,
                          void* stream);
 
+/* la_kv_summary without a caller workspace, for callers that cannot allocate
+ * device memory: code that runs where cudaMalloc is off limits (inside a
+ * stream capture, in a real-time path that must not allocate, or behind a
+ * host framework that owns every device allocation and hands the caller only
+ * its tensors). The pages describe no such variant; it exists for these
+ * callers only.
+ *
+ * Same inputs, outputs and result as la_kv_summary. The scratch the KV
+ * summary needs lives in a device array of 32 MiB inside the library, which
+ * every GPU that loads the library holds until the process exits; a problem
+ * whose la_workspace_size(desc, LA_OP_KV_SUMMARY, 0) exceeds 32 MiB is
+ * rejected with LA_ERR_WORKSPACE before anything is launched. The call
+ * allocates nothing: it issues a 4-byte cudaMemsetAsync (clearing the
+ * array's error word) and the kernels.
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, once per device, with that device current); make
+ *   that first call before any stream capture.
+ * - All calls share the one array, which keeps the last call's contents:
+ *   calls that may overlap on the GPU (different streams, or different host
+ *   threads) race and give undefined results; serialize them.
+ * - An expired bounded wait leaves S_out and z_out undefined and is recorded
+ *   only in the array's error word, which no entry point reads. */
+LA_API la_status la_kv_summary_static(const la_desc* desc, const void* k, const void* v,
+                                      float* S_out, float* z_out, void* stream);
+
 /* Waits for `stream`, then reads and clears the error word of workspace `ws`.
  * The error word is the first 4 bytes of a workspace; it is sticky: the
  * calls that use the workspace only set bits in it, so the caller zeroes it

@@ -55,6 +55,7 @@ _SIGS = {
     "la_prefix_mask": (ctypes.c_int, [ctypes.POINTER(la_desc), ctypes.c_int32, _P, _P, _P, _P, _P,
                                       _P, ctypes.c_size_t, _P]),
     "la_decode_step": (ctypes.c_int, [ctypes.POINTER(la_desc), _P, _P, _P, _P, _P, _P, _P]),
+    "la_kv_summary_static": (ctypes.c_int, [ctypes.POINTER(la_desc), _P, _P, _P, _P, _P]),
     "la_last_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "la_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "la_version": (ctypes.c_int32, []),
@@ -152,6 +153,18 @@ def la_kv_summary(k, v, S_out=None, z_out=None, phi="relu1", ws=None, stream=Non
     _check("la_kv_summary", lib().la_kv_summary(
         ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(S_out), _ptr(z_out), _ptr(ws), ws.numel(),
         _stream(k, stream)))
+    return S_out, z_out
+
+
+def la_kv_summary_static(k, v, S_out, z_out, phi="relu1", stream=None):
+    """la_kv_summary with the library's own device scratch instead of a
+    workspace: for callers that cannot allocate device memory. Allocates
+    nothing; S_out [B,H,d,d] and z_out [B,H,d] float32 are the caller's.
+    Calls that overlap on the GPU race (they share the scratch)."""
+    _same(k, v)
+    desc = _desc_of(k, phi, True)
+    _check("la_kv_summary_static", lib().la_kv_summary_static(
+        ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(S_out), _ptr(z_out), _stream(k, stream)))
     return S_out, z_out
 
 

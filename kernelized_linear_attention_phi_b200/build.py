@@ -23,7 +23,8 @@ LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libla_b200.so")
 INCLUDE = os.path.join(ROOT, "include")
 
-SOURCES = ["la_api.cu", "simt.cu", "bin.cu", "decode.cu", "tc_host.cu", "tc_kv.cu", "tc_sweep.cu"]
+SOURCES = ["la_api.cu", "simt.cu", "bin.cu", "decode.cu", "tc_host.cu", "tc_kv.cu", "tc_sweep.cu",
+           "static_scratch.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

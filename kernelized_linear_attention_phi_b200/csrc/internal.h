@@ -2,10 +2,16 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <la.h>
 #include <stddef.h>
 #include <stdint.h>
 
 namespace la {
+
+// la_kv_summary after its argument checks: validation, then the KV summary
+// with `ws` as workspace (la_api.cu).
+la_status kv_summary_checked(const la_desc* desc, const void* k, const void* v, float* S_out,
+                             float* z_out, void* ws, size_t ws_bytes, cudaStream_t st);
 
 struct Problem {
     int B, H, N, d;

@@ -174,6 +174,19 @@ la_status kv_summary_impl(const Problem& p, const void* k, const void* v, float*
 }
 
 }  // namespace
+
+la_status kv_summary_checked(const la_desc* desc, const void* k, const void* v, float* S_out,
+                             float* z_out, void* ws, size_t ws_bytes, cudaStream_t st) {
+    LA_TRY(check_desc(desc));
+    if (!k || !v || !S_out || !z_out) return LA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(S_out) || !aligned16(z_out))
+        return LA_ERR_MISALIGNED;
+    const Problem p = to_problem(desc);
+    LA_TRY(check_ws(ws_layout(p, LA_OP_KV_SUMMARY), ws, ws_bytes));
+    LA_TRY(check_device());
+    return kv_summary_impl(p, k, v, S_out, z_out, ws, st);
+}
+
 }  // namespace la
 
 using namespace la;
@@ -205,14 +218,8 @@ size_t la_workspace_size(const la_desc* desc, int32_t op, int32_t chunk) {
 
 la_status la_kv_summary(const la_desc* desc, const void* k, const void* v, float* S_out,
                         float* z_out, void* ws, size_t ws_bytes, void* stream) {
-    LA_TRY(check_desc(desc));
-    if (!k || !v || !S_out || !z_out) return LA_ERR_INVALID_ARG;
-    if (!aligned16(k) || !aligned16(v) || !aligned16(S_out) || !aligned16(z_out))
-        return LA_ERR_MISALIGNED;
-    const Problem p = to_problem(desc);
-    LA_TRY(check_ws(ws_layout(p, LA_OP_KV_SUMMARY), ws, ws_bytes));
-    LA_TRY(check_device());
-    return kv_summary_impl(p, k, v, S_out, z_out, ws, static_cast<cudaStream_t>(stream));
+    return la::kv_summary_checked(desc, k, v, S_out, z_out, ws, ws_bytes,
+                                  static_cast<cudaStream_t>(stream));
 }
 
 la_status la_noncausal(const la_desc* desc, const void* q, const void* k, const void* v, void* out,
