@@ -43,9 +43,16 @@ from kernelized_linear_attention_phi_b200 import workloads as W  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20
 
-# Kernels each library call launches (memsets excluded); kept in step with
-# la_api.cu's dispatch and checked against the ncu launch list.
-LAUNCHES = {"noncausal": 3, "causal": 3, "prefix": 4, "decode": 1}
+# Kernels each library call launches on the bf16 tensor-core path, in launch
+# order; kept in step with la_api.cu's dispatch and checked against the ncu
+# launch list (--record-traffic matches them there).
+CALL_KERNELS = {
+    "noncausal": ["tc_kv_kernel", "kv_reduce_balanced_kernel", "tc_readout_kernel"],
+    "causal": ["tc_kv_kernel", "state_scan_kernel", "tc_sweep_kernel"],
+    "prefix": ["bin_kernel", "tc_kv_kernel", "state_scan_kernel", "tc_sweep_kernel"],
+    "decode": ["decode_kernel"],
+}
+LAUNCHES = {k: len(v) for k, v in CALL_KERNELS.items()}
 
 
 def parse():
@@ -57,6 +64,10 @@ def parse():
     ap.add_argument("--workload", default="multi_head")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f32"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--record-traffic", metavar="NCU_CSV",
+                    help="read an ncu launch list with dram__bytes_read.sum and "
+                         "dram__bytes_write.sum of this workload's bench run and store "
+                         "each call's DRAM bytes in profiles/traffic.json")
     return ap.parse_args()
 
 
@@ -247,27 +258,32 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(device)
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(K)]
     sampler = ClockSampler(device)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    # Every call starts with a cold L2 (a 256 MiB write between calls, outside
+    # the events), so each call reads its inputs from HBM; a step's time is
+    # the sum of its calls' times.
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(len(calls))] for _ in range(K)]
     with sampler:
         for i in range(K):
-            flush_l2(flush)
-            ev[i][0].record(stream)
             for j, g in enumerate(graphs):
+                flush_l2(flush)
+                ev[i][j][0].record(stream)
                 g.replay()
-                ev[i][j + 1].record(stream)
+                ev[i][j][1].record(stream)
         torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     per_call = {name: 0.0 for name, _ in calls}
     total_ms = 0.0
     for i in range(K):
-        total_ms += ev[i][0].elapsed_time(ev[i][-1])
         for j, (name, _) in enumerate(calls):
-            per_call[name] += ev[i][j].elapsed_time(ev[i][j + 1])
+            ms = ev[i][j][0].elapsed_time(ev[i][j][1])
+            per_call[name] += ms
+            total_ms += ms
     t_s = total_ms / 1e3
 
     # end to end through the public API: pinned host inputs in, outputs back
@@ -339,8 +355,10 @@ def run_ours(args, rank, world, local_rank):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": sum(LAUNCHES[n] for n, _ in calls) * K,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
-                     "kernel": f"la_{dom} (all its kernels)", "peak_source": peaks.get("_src")},
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": recorded_traffic(wl.name, dtype, dom),
+                     "kernel": f"la_{dom} (all its kernels)", "peak_source": peaks.get("_src"),
+                     "algorithmic_bytes": alg[dom]},
         "per_call": per_kernel,
         "clocks": sampler.summary(),
     }
@@ -354,6 +372,32 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.destroy_process_group()
     if bad_flags:
         raise SystemExit(f"library error flags set during the run: {bad_flags}")
+
+
+def library_source_hash():
+    """Hash of the library's CUDA sources: recorded DRAM traffic counts only
+    for the kernels it was measured on."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kernelized_linear_attention_phi_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, dtype, call):
+    """DRAM bytes (read + write) per call, summed over the call's kernels, from
+    the ncu capture in profiles/traffic.json; None when none was taken for
+    this workload and call, or the kernels changed since."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("source_hash") != library_source_hash():
+        return None
+    return rec.get("bytes", {}).get(f"{workload}/{dtype}/{call}")
 
 
 def load_peaks():
@@ -460,8 +504,57 @@ def run_reference(args, rank, world):
     }), flush=True)
 
 
+def record_traffic(csv_path, workload, dtype):
+    """Per call of the last complete step in an ncu launch list: the sum of
+    dram__bytes_read.sum + dram__bytes_write.sum over the call's kernels."""
+    import csv
+    with open(csv_path) as f:
+        rows = [r for r in csv.reader(f)]
+    head = next(i for i, r in enumerate(rows) if r and r[0] == "ID")
+    h = rows[head]
+    ik, im, iv, iu = (h.index(c) for c in ("Kernel Name", "Metric Name", "Metric Value", "Metric Unit"))
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    launches = {}
+    for r in rows[head + 1:]:
+        if len(r) <= iv or "la::" not in r[ik]:
+            continue
+        rec = launches.setdefault(int(r[0]), {"name": r[ik], "bytes": 0.0})
+        if r[im] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            rec["bytes"] += float(r[iv].replace(",", "")) * scale.get(r[iu], 1)
+    seq = [launches[i] for i in sorted(launches)]
+    forms = Step.ALL_FORMS if workload == "multi_head" else W.WORKLOADS[workload].forms
+    want = [(f, k) for f in forms for k in CALL_KERNELS[f]]
+    for start in range(len(seq) - len(want), -1, -1):
+        if all(k in seq[start + n]["name"] for n, (_, k) in enumerate(want)):
+            break
+    else:
+        raise SystemExit("the launch list holds no complete step of this workload")
+    per_call = {}
+    for n, (f, _) in enumerate(want):
+        per_call[f] = per_call.get(f, 0.0) + seq[start + n]["bytes"]
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            out = json.load(f)
+    except Exception:
+        out = {}
+    if out.get("source_hash") != library_source_hash():
+        out = {"source_hash": library_source_hash(), "bytes": {}}
+    out["note"] = ("DRAM bytes read + written per library call, summed over the call's kernels, "
+                   "from an ncu launch list (cold cache per kernel); valid for the CUDA sources "
+                   "with this hash")
+    for f, b in per_call.items():
+        out["bytes"][f"{workload}/{dtype}/{f}"] = int(b)
+    with open(path, "w") as f:
+        json.dump(out, f, indent=1, sort_keys=True)
+    print(json.dumps(per_call))
+
+
 def main():
     args = parse()
+    if args.record_traffic:
+        record_traffic(args.record_traffic, args.workload, args.dtype)
+        return
     rank, world, local_rank = dist_env()
     if args.impl == "reference":
         run_reference(args, rank, world)
