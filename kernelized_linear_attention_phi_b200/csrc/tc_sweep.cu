@@ -45,7 +45,7 @@ struct SwCfg {
     static constexpr int ONES = 16 * C * 2;          // all-ones B operand, 16 x C, K-major
     static constexpr int QG = GATHER ? 2 * TILE : 0; // gathered queries (x2)
     static constexpr int ROWS = GATHER ? 2 * 2 * C * 4 : 0;  // token / limit per row (x2)
-    static constexpr int STG = GATHER ? 0 : TILE;    // output staging tile (causal: one TMA store)
+    static constexpr int STG = TILE;                 // output staging tile
     static constexpr int COL_S = 0, COL_Z = D, COL_P = D + 16, COL_O = D + 16 + C, COL_OZ = 2 * D + 16 + C;
     static constexpr uint32_t TMEM_COLS = (2 * D + 32 + C) <= 256 ? 256u : 512u;
     static constexpr int NBAR = 2 * STAGES + 9;
@@ -372,16 +372,23 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                         }
                     }
                     named_bar(1, 128);
+                    // all of this thread's row loads are issued before any is used
+                    constexpr int NL = C * D / 8 / 128;
                     uint8_t* q = qg + slot * CF::TILE;
-                    for (int p = et; p < C * D / 8; p += 128) {
+                    uint4 w[NL];
+#pragma unroll
+                    for (int j = 0; j < NL; ++j) {
+                        const int p = et + 128 * j;
                         const int r = p / (D / 8), col = (p % (D / 8)) * 8;
                         const int i = srow[r];
-                        uint4 w = make_uint4(0, 0, 0, 0);
-                        if (i >= 0) {
-                            w = ldg_stream(Qg + hoff + (size_t)i * D + col);
-                            if (relu) w = phi_relu1_x8(w);
-                        }
-                        *reinterpret_cast<uint4*>(q + (col / 64) * (C * 128) + sw128_off(r, col % 64)) = w;
+                        w[j] = i >= 0 ? ldg_stream(Qg + hoff + (size_t)i * D + col) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int j = 0; j < NL; ++j) {
+                        const int p = et + 128 * j;
+                        const int r = p / (D / 8), col = (p % (D / 8)) * 8;
+                        *reinterpret_cast<uint4*>(q + (col / 64) * (C * 128) + sw128_off(r, col % 64)) =
+                            relu ? phi_relu1_x8(w[j]) : w[j];
                     }
                     fence_async_smem();
                     mbar_arrive(bqready + slot);
@@ -471,6 +478,14 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 tmem_ld2(tmem + CF::COL_OZ + lane_base, oz);
                 tmem_ld_wait();
                 tc_fence_before();
+                // gathered rows: this thread's copy-out rows, read before the
+                // slot (and its row table) is handed back
+                constexpr int NC = C * D / 8 / 128;
+                int dst_row[GATHER ? NC : 1];
+                if (GATHER) {
+#pragma unroll
+                    for (int j = 0; j < NC; ++j) dst_row[j] = srow[(threadIdx.x - 192 + 128 * j) / (D / 8)];
+                }
                 mbar_arrive(bofree + slot);
                 float den = rs + __uint_as_float(oz[0]) + __uint_as_float(oz[1]);
                 if (C == 64) den = __shfl_sync(0xffffffffu, den, lane & 15);
@@ -497,15 +512,29 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                             tma_store_3d(&mOut, stg + bx * (C * 128), bx * 64, c * C, bh);
                         bulk_commit();
                     }
-                } else if (ok && tok >= 0) {
-                    uint4* dst = reinterpret_cast<uint4*>(out + hoff + (size_t)tok * D + half * SEG);
+                } else {
+                    // gathered rows: stage the tile, then copy it out a full row
+                    // per 8 (d = 64) or 16 (d = 128) consecutive threads
+                    const int et2 = threadIdx.x - 192;
+                    named_bar(3, 128);  // the previous tile's copy-out has read the staging tile
 #pragma unroll
                     for (int g = 0; g < SEG / 8; ++g) {
+                        const int col = half * SEG + 8 * g;
                         float f[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[8 * g + e]) * inv;
-                        dst[g] = pack8(f);
+                        *reinterpret_cast<uint4*>(stg + (col / 64) * (C * 128) + sw128_off(i, col % 64)) = pack8(f);
                     }
+                    named_bar(3, 128);
+#pragma unroll
+                    for (int j = 0; j < NC; ++j) {
+                        const int p = et2 + 128 * j;
+                        const int r = p / (D / 8), col = (p % (D / 8)) * 8;
+                        if (ok && dst_row[j] >= 0)
+                            *reinterpret_cast<uint4*>(out + hoff + (size_t)dst_row[j] * D + col) =
+                                *reinterpret_cast<const uint4*>(stg + (col / 64) * (C * 128) + sw128_off(r, col % 64));
+                    }
+                    (void)tok;
                 }
             }
         }
