@@ -18,6 +18,7 @@ bin_kernel(const int32_t* __restrict__ m, int N, int chunk, int nbins, int32_t* 
            int32_t* __restrict__ bin_start, int32_t* __restrict__ mcl, uint32_t* __restrict__ flags) {
     extern __shared__ int32_t cnt[];  // nbins + 1
     __shared__ int32_t warp_tot[kBinThreads / 32];
+    pdl_wait();
     const int b = blockIdx.x;
     const int32_t* mb = m + (size_t)b * N;
     for (int c = threadIdx.x; c <= nbins; c += kBinThreads) cnt[c] = 0;
@@ -73,6 +74,7 @@ bin_kernel(const int32_t* __restrict__ m, int N, int chunk, int nbins, int32_t* 
         const int pos = atomicAdd(&cnt[(mi + 1) / chunk], 1);
         perm[(size_t)b * N + pos] = i;
     }
+    pdl_trigger();
 }
 
 }  // namespace
@@ -82,9 +84,8 @@ cudaError_t bin_queries(const Problem& p, const int32_t* m, int chunk, int nbins
     const size_t smem = sizeof(int32_t) * (size_t)(nbins + 1);
     cudaError_t e = ensure_smem<bin_kernel>(smem);
     if (e != cudaSuccess) return e;
-    bin_kernel<<<p.B, kBinThreads, smem, st>>>(m, p.N, chunk, nbins, perm, bin_start, mclamped,
-                                               flags);
-    return cudaGetLastError();
+    return launch_pdl(bin_kernel, dim3(p.B), dim3(kBinThreads), smem, st, m, p.N, chunk, nbins, perm,
+                      bin_start, mclamped, flags);
 }
 
 }  // namespace la

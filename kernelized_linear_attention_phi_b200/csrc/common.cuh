@@ -71,6 +71,16 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// Programmatic dependent launch. Every kernel of the library is launched
+// with programmatic stream serialization: it may start while the previous
+// kernel on the stream finishes, runs its prologue (shared memory, barriers,
+// TMEM), and waits in pdl_wait() before it touches global memory. Each kernel
+// lets its dependents launch only at its very end (pdl_trigger() after all
+// its work and its TMEM release), so a waiting dependent never holds resources
+// that a CTA of the running kernel still needs.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Streaming 16-byte global load (read once: do not keep in L1).
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
     uint4 r;

@@ -10,6 +10,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "launch_util.h"
 
 namespace la {
 namespace {
@@ -41,6 +42,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     __shared__ float sden[kThreads / 32];
     const long long bh = blockIdx.x;
     const int tid = threadIdx.x;
+    pdl_wait();
     if (tid < D) {
         spk[tid] = phi_apply(to_f32<T>(k[bh * D + tid]), phi);
         spq[tid] = phi_apply(to_f32<T>(q[bh * D + tid]), phi);
@@ -94,15 +96,15 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         for (int w = 0; w < kThreads / 32; ++w) den += sden[w];
         out[bh * D + tid] = from_f32<T>(normalize ? acc / den : acc);
     }
+    pdl_trigger();
 }
 
 template <typename T, int D>
 cudaError_t launch_decode(const Problem& p, const void* q, const void* k, const void* v, float* S,
                           float* z, void* out, cudaStream_t st) {
-    decode_kernel<T, D><<<(unsigned)p.bh(), kThreads, 0, st>>>(
-        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), S, z,
-        static_cast<T*>(out), p.phi, p.normalize);
-    return cudaGetLastError();
+    return launch_pdl(decode_kernel<T, D>, dim3((unsigned)p.bh()), dim3(kThreads), 0, st,
+                      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), S, z,
+                      static_cast<T*>(out), p.phi, p.normalize);
 }
 
 }  // namespace

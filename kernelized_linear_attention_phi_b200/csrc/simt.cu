@@ -54,6 +54,7 @@ kv_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int N, int t
     const long long bh = blockIdx.y;
     const int t0 = s * tps;
     const int t1 = min(N, t0 + tps);
+    pdl_wait();
     const T* Kh = K + bh * (long long)N * D;
     const T* Vh = V + bh * (long long)N * D;
     const int ta = threadIdx.x / 16, tb = threadIdx.x % 16;
@@ -92,6 +93,7 @@ kv_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int N, int t
         for (int c = 0; c < R; ++c) o[(ta * R + r) * D + tb * R + c] = acc[r][c];
         if (tb == 0) o[D * D + ta * R + r] = zacc[r];
     }
+    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -102,12 +104,15 @@ __global__ void state_reduce_kernel(const float* __restrict__ part, int nsplit, 
     const int rec = D * D + D;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     const long long bh = blockIdx.y;
-    if (e >= rec) return;
-    const float* p = part + (size_t)bh * nsplit * rec + e;
-    float s = 0.f;
-    for (int i = 0; i < nsplit; ++i) s += p[(size_t)i * rec];
-    if (e < D * D) S[(size_t)bh * D * D + e] = s;
-    else z[(size_t)bh * D + (e - D * D)] = s;
+    pdl_wait();
+    if (e < rec) {
+        const float* p = part + (size_t)bh * nsplit * rec + e;
+        float s = 0.f;
+        for (int i = 0; i < nsplit; ++i) s += p[(size_t)i * rec];
+        if (e < D * D) S[(size_t)bh * D * D + e] = s;
+        else z[(size_t)bh * D + (e - D * D)] = s;
+    }
+    pdl_trigger();
 }
 
 // One thread per float4 of a record; loads are issued eight blocks at a time
@@ -117,7 +122,11 @@ __global__ void state_scan_kernel(float* __restrict__ part, int nblk, int D,
     const int rec4 = (D * D + D) / 4;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     const long long bh = blockIdx.y;
-    if (e >= rec4) return;
+    pdl_wait();
+    if (e >= rec4) {
+        pdl_trigger();
+        return;
+    }
     float4* p = reinterpret_cast<float4*>(part + (size_t)bh * nblk * (rec4 * 4)) + e;
     float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int b0 = 0; b0 < nblk; b0 += 8) {
@@ -145,6 +154,7 @@ __global__ void state_scan_kernel(float* __restrict__ part, int nblk, int D,
             else z_total[(size_t)bh * D + (idx - D * D)] = r[q];
         }
     }
+    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -167,6 +177,7 @@ readout_kernel(const T* __restrict__ Q, const float* __restrict__ S, const float
     float* sDen = sQ + TQ * LDQ;
     const int tile = blockIdx.x;
     const long long bh = blockIdx.y;
+    pdl_wait();
     const float4* S4 = reinterpret_cast<const float4*>(S + (size_t)bh * D * D);
     for (int e = threadIdx.x; e < D * D / 4; e += kThreads) reinterpret_cast<float4*>(sS)[e] = S4[e];
     for (int e = threadIdx.x; e < D; e += kThreads) sz[e] = z[(size_t)bh * D + e];
@@ -207,6 +218,7 @@ readout_kernel(const T* __restrict__ Q, const float* __restrict__ S, const float
         for (int c = 0; c < RC; ++c)
             Oh[(long long)row * D + tc * RC + c] = from_f32<T>(normalize ? acc[i][c] / den : acc[i][c]);
     }
+    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -248,6 +260,7 @@ chunked_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __rest
     const T* Vh = V + hoff;
     T* Oh = out + hoff;
 
+    pdl_wait();
     const float* pre = prefix + ((size_t)bh * nblk + blk) * (size_t)(D * D + D);
     for (int e = threadIdx.x; e < D * D + D; e += kThreads) {
         if (e < D * D) sS[e] = pre[e];
@@ -409,16 +422,15 @@ chunked_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __rest
             }
         }
     }
+    pdl_trigger();
 }
 
 template <typename T, int D>
 cudaError_t launch_kv_partial(const Problem& p, const void* k, const void* v, int tps, int nsplit,
                               float* part, cudaStream_t st) {
     dim3 grid(nsplit, (unsigned)p.bh());
-    kv_partial_kernel<T, D><<<grid, kThreads, 0, st>>>(static_cast<const T*>(k),
-                                                       static_cast<const T*>(v), p.N, tps, nsplit,
-                                                       p.phi, part);
-    return cudaGetLastError();
+    return launch_pdl(kv_partial_kernel<T, D>, grid, dim3(kThreads), 0, st, static_cast<const T*>(k),
+                      static_cast<const T*>(v), p.N, tps, nsplit, p.phi, part);
 }
 
 template <typename T, int D>
@@ -428,10 +440,8 @@ cudaError_t launch_readout(const Problem& p, const void* q, const float* S, cons
     cudaError_t e = ensure_smem<readout_kernel<T, D>>(smem);
     if (e != cudaSuccess) return e;
     dim3 grid((p.N + 63) / 64, (unsigned)p.bh());
-    readout_kernel<T, D><<<grid, kThreads, smem, st>>>(static_cast<const T*>(q), S, z,
-                                                       static_cast<T*>(out), p.N, p.phi,
-                                                       p.normalize);
-    return cudaGetLastError();
+    return launch_pdl(readout_kernel<T, D>, grid, dim3(kThreads), smem, st, static_cast<const T*>(q), S, z,
+                      static_cast<T*>(out), p.N, p.phi, p.normalize);
 }
 
 template <typename T, int D>
@@ -444,19 +454,19 @@ cudaError_t launch_chunked(const Problem& p, const void* q, const void* k, const
     if (perm == nullptr) {
         cudaError_t e = ensure_smem<chunked_kernel<T, D, false>>(smem);
         if (e != cudaSuccess) return e;
-        chunked_kernel<T, D, false><<<grid, kThreads, smem, st>>>(
-            static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), prefix,
-            p.H, p.N, block_tokens, nblk, nullptr, nullptr, nullptr, 0, p.phi, p.normalize,
-            static_cast<T*>(out));
+        return launch_pdl(chunked_kernel<T, D, false>, grid, dim3(kThreads), smem, st,
+                          static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+                          prefix, p.H, p.N, block_tokens, nblk, (const int32_t*)nullptr,
+                          (const int32_t*)nullptr, (const int32_t*)nullptr, 0, p.phi, p.normalize,
+                          static_cast<T*>(out));
     } else {
         cudaError_t e = ensure_smem<chunked_kernel<T, D, true>>(smem);
         if (e != cudaSuccess) return e;
-        chunked_kernel<T, D, true><<<grid, kThreads, smem, st>>>(
-            static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), prefix,
-            p.H, p.N, block_tokens, nblk, perm, bin_start, m, nbins, p.phi, p.normalize,
-            static_cast<T*>(out));
+        return launch_pdl(chunked_kernel<T, D, true>, grid, dim3(kThreads), smem, st,
+                          static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+                          prefix, p.H, p.N, block_tokens, nblk, perm, bin_start, m, nbins, p.phi,
+                          p.normalize, static_cast<T*>(out));
     }
-    return cudaGetLastError();
 }
 
 }  // namespace
@@ -503,16 +513,14 @@ cudaError_t state_reduce(const Problem& p, const float* part, int nsplit, float*
                          cudaStream_t st) {
     const int rec = p.d * p.d + p.d;
     dim3 grid((rec + 255) / 256, (unsigned)p.bh());
-    state_reduce_kernel<<<grid, 256, 0, st>>>(part, nsplit, p.d, S, z);
-    return cudaGetLastError();
+    return launch_pdl(state_reduce_kernel, grid, dim3(256), 0, st, part, nsplit, p.d, S, z);
 }
 
 cudaError_t state_exclusive_scan(const Problem& p, float* part, int nblk, float* S_total,
                                  float* z_total, cudaStream_t st) {
     const int rec4 = (p.d * p.d + p.d) / 4;
     dim3 grid((rec4 + 127) / 128, (unsigned)p.bh());
-    state_scan_kernel<<<grid, 128, 0, st>>>(part, nblk, p.d, S_total, z_total);
-    return cudaGetLastError();
+    return launch_pdl(state_scan_kernel, grid, dim3(128), 0, st, part, nblk, p.d, S_total, z_total);
 }
 
 }  // namespace la

@@ -154,6 +154,7 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -325,6 +326,7 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
+    pdl_trigger();
 }
 
 // Sums the partial records of each head in CTA order (deterministic).
@@ -333,17 +335,35 @@ __global__ void kv_reduce_balanced_kernel(const float* __restrict__ part, KvBala
     const int rec4 = (D * D + D) / 4;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     const long long h = blockIdx.y;
-    if (e >= rec4) return;
+    if (e >= rec4) {
+        pdl_wait();
+        pdl_trigger();
+        return;
+    }
+    pdl_wait();
     const int c0 = cta_of(w, h * w.tph);
     const int c1 = cta_of(w, (h + 1) * w.tph - 1);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = c0; c <= c1; ++c) {
-        const long long j = h - range_lo(w.total, w.G, c) / w.tph;
-        const float4 v = reinterpret_cast<const float4*>(part + ((size_t)c * w.K + j) * (size_t)(rec4 * 4))[e];
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+    // eight record loads in flight at a time; the sum stays in CTA order
+    for (int cb = c0; cb <= c1; cb += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int c = cb + u;
+            if (c <= c1) {
+                const long long j = h - range_lo(w.total, w.G, c) / w.tph;
+                v[u] = reinterpret_cast<const float4*>(part + ((size_t)c * w.K + j) * (size_t)(rec4 * 4))[e];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (cb + u <= c1) {
+                acc.x += v[u].x;
+                acc.y += v[u].y;
+                acc.z += v[u].z;
+                acc.w += v[u].w;
+            }
+        }
     }
     const float r[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
@@ -352,6 +372,7 @@ __global__ void kv_reduce_balanced_kernel(const float* __restrict__ part, KvBala
         if (idx < D * D) S[(size_t)h * D * D + idx] = r[q];
         else z[(size_t)h * D + (idx - D * D)] = r[q];
     }
+    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -425,6 +446,7 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -561,6 +583,7 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
+    pdl_trigger();
 }
 
 template <int D>
@@ -573,8 +596,7 @@ cudaError_t launch_kv(const Problem& p, const void* k, const void* v, const KvWo
     constexpr size_t smem = KvCfg<D>::SMEM;
     e = ensure_smem<tc_kv_kernel<D>>(smem);
     if (e != cudaSuccess) return e;
-    tc_kv_kernel<D><<<grid, kThreads, smem, st>>>(mk, mv, p.N, w, p.phi, part, err);
-    return cudaGetLastError();
+    return launch_pdl(tc_kv_kernel<D>, grid, dim3(kThreads), smem, st, mk, mv, p.N, w, p.phi, part, err);
 }
 
 template <int D>
@@ -590,8 +612,8 @@ cudaError_t launch_readout(const Problem& p, const void* q, const float* S, cons
     const int tph = (p.N + kTile - 1) / kTile;
     const long long total = p.bh() * tph;
     const int G = (int)std::min<long long>(total, 148LL * RoCfg<D>::PER_SM);
-    tc_readout_kernel<D><<<G, kThreads, smem, st>>>(mq, mo, S, z, p.N, total, tph, p.phi, p.normalize, err);
-    return cudaGetLastError();
+    return launch_pdl(tc_readout_kernel<D>, dim3(G), dim3(kThreads), smem, st, mq, mo, S, z, p.N, total, tph,
+                      p.phi, p.normalize, err);
 }
 
 }  // namespace
@@ -606,8 +628,8 @@ cudaError_t tc_kv_summary(const Problem& p, const void* k, const void* v, float*
                               : launch_kv<128>(p, k, v, w, grid, part, err, st);
     if (e != cudaSuccess) return e;
     const int rec4 = (p.d * p.d + p.d) / 4;
-    kv_reduce_balanced_kernel<<<dim3((rec4 + 127) / 128, (unsigned)p.bh()), 128, 0, st>>>(part, w.b, p.d, S, z);
-    return cudaGetLastError();
+    return launch_pdl(kv_reduce_balanced_kernel, dim3((rec4 + 127) / 128, (unsigned)p.bh()), dim3(128), 0, st,
+                      part, w.b, p.d, S, z);
 }
 
 cudaError_t tc_kv_blocks(const Problem& p, const void* k, const void* v, int block_tokens, int nblk, float* part,

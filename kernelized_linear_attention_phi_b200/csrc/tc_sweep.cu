@@ -31,30 +31,45 @@ using namespace tc;
 // Warp roles (320 threads): warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 "prep"
 // (phi on the K / Q tiles, state -> operands, query gather), warps 6-9 "mask"
 // (P~, epilogue). Prep runs one chunk ahead of mask; the S / z operands are
-// double-buffered, the gathered query tiles too.
+// double-buffered, the gathered query tiles too. The per-tile accumulators
+// (P, O, Oz) and the P~ operand are double-buffered by tile parity ("slot"),
+// so the tensor core starts tile t+1 while the mask warps finish tile t: with
+// 64-row chunks (M = 64 accumulators, which use TMEM lanes 0..15 of each
+// sub-partition) slot 1 lives in lanes 16..31 of the same columns, with
+// 128-row chunks in separate columns.
 template <int D, int C, bool GATHER>
 struct SwCfg {
     static constexpr int NB = D / 64;
     static constexpr int TILE = C * D * 2;           // one [C x D] bf16 tile
     static constexpr int NT = GATHER ? 2 : 3;        // tiles per stage: (Q,) K, V
-    static constexpr int STAGES = (D == 64 && C == 64) ? 3 : 2;
+    static constexpr int STAGES = 2;
     static constexpr int STAGE = NT * TILE;
-    static constexpr int PT = C * C * 2;             // P~, K-major
+    static constexpr int PT = C * C * 2;             // P~, K-major (x2)
     static constexpr int B3 = D * D * 2;             // S_prev, MN-major (x2)
     static constexpr int BZ = 16 * D * 2;            // z_hi, z_lo, 14 zero rows; K-major (x2)
     static constexpr int ONES = 16 * C * 2;          // all-ones B operand, 16 x C, K-major
     static constexpr int QG = GATHER ? 2 * TILE : 0; // gathered queries (x2)
     static constexpr int ROWS = GATHER ? 2 * 2 * C * 4 : 0;  // token / limit per row (x2)
     static constexpr int STG = TILE;                 // output staging tile
-    static constexpr int COL_S = 0, COL_Z = D, COL_P = D + 16, COL_O = D + 16 + C, COL_OZ = 2 * D + 16 + C;
-    static constexpr uint32_t TMEM_COLS = (2 * D + 32 + C) <= 256 ? 256u : 512u;
-    static constexpr int NBAR = 2 * STAGES + 9;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + PT + 2 * B3 + 2 * BZ + ONES + QG +
+    // TMEM columns: S, z, then P, O, Oz (two slots each; see above)
+    static constexpr int SLOTC = C == 64 ? 1 : 2;    // column copies per slot pair
+    static constexpr int COL_S = 0, COL_Z = D, COL_P = D + 16, COL_O = COL_P + SLOTC * C,
+                         COL_OZ = COL_O + SLOTC * D, COL_END = COL_OZ + SLOTC * 16;
+    static constexpr uint32_t TMEM_COLS = COL_END <= 256 ? 256u : 512u;
+    static_assert(COL_END <= 512, "TMEM");
+    static constexpr int NBAR = 2 * STAGES + 2 + 5 * 2;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 2 * PT + 2 * B3 + 2 * BZ + ONES + QG +
                                    STG + ROWS + 8 * NBAR + 16;
+    // TMEM address offsets of slot j for P, O and Oz
+    __device__ static constexpr uint32_t p_slot(int j) { return C == 64 ? (uint32_t)j * (16u << 16) : (uint32_t)j * C; }
+    __device__ static constexpr uint32_t o_slot(int j) { return C == 64 ? (uint32_t)j * (16u << 16) : (uint32_t)j * D; }
+    __device__ static constexpr uint32_t oz_slot(int j) { return C == 64 ? (uint32_t)j * (16u << 16) : (uint32_t)j * 16; }
     static constexpr int THREADS = 320;
     static constexpr int MIN_BLOCKS = (D == 64 && C == 64) ? 2 : 1;
     static_assert(C == 64 || C == 128, "chunk");
     static_assert(SMEM <= 227 * 1024, "shared memory");
+    // two resident CTAs per SM: 228 KiB per SM, 1 KiB reserved per CTA
+    static_assert(MIN_BLOCKS == 1 || MIN_BLOCKS * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
 template <int D, int C, bool GATHER>
@@ -70,7 +85,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* stages = align1024(smem_raw);
     uint8_t* pt = stages + CF::STAGES * CF::STAGE;
-    uint8_t* b3 = pt + CF::PT;
+    uint8_t* b3 = pt + 2 * CF::PT;
     uint8_t* bz = b3 + 2 * CF::B3;
     uint8_t* ones = bz + 2 * CF::BZ;
     uint8_t* qg = ones + CF::ONES;
@@ -80,14 +95,15 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     uint64_t* empty = full + CF::STAGES;
     uint64_t* bprep = empty + CF::STAGES;
     uint64_t* bsdone = bprep + 1;
-    uint64_t* bpfull = bsdone + 1;
-    uint64_t* bptready = bpfull + 1;
-    uint64_t* bofull = bptready + 1;
-    // Barriers with one phase per query tile whose producer can run two
-    // tiles ahead of a waiter are kept per slot (tile t uses slot t % 2), so
-    // that no waiter is ever two phases behind (parity waits would alias).
-    uint64_t* bofree = bofull + 1;   // [2]
-    uint64_t* bqready = bofree + 2;  // [2]
+    // Per-tile barriers are kept per slot (tile t uses slot t % 2, phase t / 2),
+    // so that no waiter is ever two phases behind its barrier (parity waits
+    // would alias): P ready, P~ written (P read), O ready, O read, queries
+    // gathered.
+    uint64_t* bpfull = bsdone + 1;     // [2]
+    uint64_t* bptready = bpfull + 2;   // [2]
+    uint64_t* bofull = bptready + 2;   // [2]
+    uint64_t* bofree = bofull + 2;     // [2]
+    uint64_t* bqready = bofree + 2;    // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bqready + 2);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -115,13 +131,13 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         }
         mbar_init(bprep, 128);
         mbar_init(bsdone, 1);
-        mbar_init(bpfull, 1);
-        mbar_init(bptready, 128);
-        mbar_init(bofull, 1);
-        mbar_init(bofree, 128);
-        mbar_init(bofree + 1, 128);
-        mbar_init(bqready, 128);
-        mbar_init(bqready + 1, 128);
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(bpfull + j, 1);
+            mbar_init(bptready + j, 128);
+            mbar_init(bofull + j, 1);
+            mbar_init(bofree + j, 128);
+            mbar_init(bqready + j, 128);
+        }
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, CF::TMEM_COLS);
@@ -137,6 +153,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -193,36 +210,40 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 const uint32_t bza = smem_u32(bz + (ci & 1) * CF::BZ);
                 const int ntq = q_tiles(c_begin + ci);
                 for (int t = 0; t < ntq && ok; ++t, ++tq) {
-                    const uint32_t qt = GATHER ? smem_u32(qg + (tq & 1) * CF::TILE) : st;
-                    if (GATHER) ok = mbar_wait(bqready + (tq & 1), (tq >> 1) & 1, err);
-                    if (ok && tq > 0) ok = mbar_wait(bptready, (tq - 1) & 1, err);  // P read by the mask warps
+                    const int j = tq & 1, k = tq >> 1;  // slot, use of the slot
+                    const uint32_t qt = GATHER ? smem_u32(qg + j * CF::TILE) : st;
+                    if (GATHER) ok = mbar_wait(bqready + j, k & 1, err);
+                    if (ok && k > 0) ok = mbar_wait(bptready + j, (k - 1) & 1, err);  // P[j] read two tiles ago
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t ko = (kk / 4) * (C * 128) + (kk % 4) * 32;
-                        mma_bf16(tmem + CF::COL_P, sdesc(qt + ko, 16, 1024), sdesc(kt + ko, 16, 1024), id1, kk > 0);
+                        mma_bf16(tmem + CF::COL_P + CF::p_slot(j), sdesc(qt + ko, 16, 1024), sdesc(kt + ko, 16, 1024),
+                                 id1, kk > 0);
                     }
-                    mma_commit(bpfull);
-                    if (tq > 0) ok = mbar_wait(bofree + ((tq - 1) & 1), ((tq - 1) >> 1) & 1, err);  // O read
+                    mma_commit(bpfull + j);
+                    if (k > 0) ok = mbar_wait(bofree + j, (k - 1) & 1, err);  // O[j] read two tiles ago
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t a = sdesc(qt + (kk / 4) * (C * 128) + (kk % 4) * 32, 16, 1024);
-                        mma_bf16(tmem + CF::COL_O, a, sdesc(b3a + kk * 2048, D * 128, 1024), id3, kk > 0);
+                        mma_bf16(tmem + CF::COL_O + CF::o_slot(j), a, sdesc(b3a + kk * 2048, D * 128, 1024), id3,
+                                 kk > 0);
                         if (normalize)
-                            mma_bf16(tmem + CF::COL_OZ, a, sdesc(bza + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024),
-                                     idz, kk > 0);
+                            mma_bf16(tmem + CF::COL_OZ + CF::oz_slot(j), a,
+                                     sdesc(bza + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024), idz, kk > 0);
                     }
-                    ok = mbar_wait(bptready, tq & 1, err);
+                    ok = mbar_wait(bptready + j, k & 1, err);
                     if (!ok) break;
                     tc_fence_after();
+                    const uint32_t ptj = pta + j * CF::PT;
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk)
-                        mma_bf16(tmem + CF::COL_O, sdesc(pta + (kk / 4) * (C * 128) + (kk % 4) * 32, 16, 1024),
+                        mma_bf16(tmem + CF::COL_O + CF::o_slot(j), sdesc(ptj + (kk / 4) * (C * 128) + (kk % 4) * 32, 16, 1024),
                                  sdesc(vt + kk * 2048, C * 128, 1024), id2, 1u);
-                    mma_commit(bofull);
+                    mma_commit(bofull + j);
                 }
                 mma_commit(empty + s);
             }
@@ -412,8 +433,10 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             const int kvalid = c < nchunks ? min(C, N - c * C) : 0;
             const int ntq = q_tiles(c);
             for (int t = 0; t < ntq; ++t, ++tq) {
-                const int slot = tq & 1;
-                ok = mbar_wait(bpfull, tq & 1, err) && ok;
+                const int slot = tq & 1, use = tq >> 1;
+                const uint32_t lane_s = C == 64 ? lane_base + CF::p_slot(slot) : lane_base;
+                uint8_t* pts = pt + slot * CF::PT;
+                ok = mbar_wait(bpfull + slot, use & 1, err) && ok;
                 tc_fence_after();
                 // the row table of a gathered tile is written before its MMAs are issued
                 const int* srow = rows + slot * 2 * C;
@@ -426,7 +449,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                         uint32_t r[64];
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
-                            tmem_ld16(tmem + CF::COL_P + lane_base + 64 * h + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(r + 16 * j));
+                            tmem_ld16(tmem + CF::COL_P + CF::p_slot(slot) + lane_base + 64 * h + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(r + 16 * j));
                         tmem_ld_wait();
 #pragma unroll
                         for (int g = 0; g < 8; ++g) {
@@ -437,13 +460,13 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                                 f[e] = j <= lim ? __uint_as_float(r[8 * g + e]) : 0.f;
                                 rs += f[e];
                             }
-                            *reinterpret_cast<uint4*>(pt + h * (C * 128) + sw128_off(i, 8 * g)) = pack8(f);
+                            *reinterpret_cast<uint4*>(pts + h * (C * 128) + sw128_off(i, 8 * g)) = pack8(f);
                         }
                     }
                 } else {
                     uint32_t r[32];
-                    tmem_ld16x2<32>(tmem + CF::COL_P + lane_base, *reinterpret_cast<uint32_t(*)[16]>(r));
-                    tmem_ld16x2<32>(tmem + CF::COL_P + lane_base + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+                    tmem_ld16x2<32>(tmem + CF::COL_P + lane_s, *reinterpret_cast<uint32_t(*)[16]>(r));
+                    tmem_ld16x2<32>(tmem + CF::COL_P + lane_s + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
                     tmem_ld_wait();
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
@@ -454,28 +477,32 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                             f[e] = j <= lim ? __uint_as_float(r[8 * g + e]) : 0.f;
                             rs += f[e];
                         }
-                        *reinterpret_cast<uint4*>(pt + sw128_off(i, 32 * half + 8 * g)) = pack8(f);
+                        *reinterpret_cast<uint4*>(pts + sw128_off(i, 32 * half + 8 * g)) = pack8(f);
                     }
                     rs += __shfl_xor_sync(0xffffffffu, rs, 16);
                 }
                 fence_async_smem();
                 tc_fence_before();
-                mbar_arrive(bptready);
+                mbar_arrive(bptready + slot);
                 // epilogue: this thread's segment of output row i
-                ok = ok && mbar_wait(bofull, tq & 1, err);
+                ok = ok && mbar_wait(bofull + slot, use & 1, err);
                 tc_fence_after();
                 constexpr int SEG = C == 128 ? D : D / 2;
                 uint32_t o[SEG];
 #pragma unroll
                 for (int j = 0; j < SEG / 16; ++j) {
                     if (C == 128)
-                        tmem_ld16(tmem + CF::COL_O + lane_base + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(o + 16 * j));
+                        tmem_ld16(tmem + CF::COL_O + CF::o_slot(slot) + lane_base + 16 * j,
+                                  *reinterpret_cast<uint32_t(*)[16]>(o + 16 * j));
                     else
-                        tmem_ld16x2<D / 2>(tmem + CF::COL_O + lane_base + 16 * j,
+                        tmem_ld16x2<D / 2>(tmem + CF::COL_O + lane_s + 16 * j,
                                            *reinterpret_cast<uint32_t(*)[16]>(o + 16 * j));
                 }
+                // Oz: a 32x32b load must start at the warp's sub-partition
+                // base; with 64-row chunks slot 1 sits in lanes 16..31 and is
+                // picked out below with a shuffle
                 uint32_t oz[2];
-                tmem_ld2(tmem + CF::COL_OZ + lane_base, oz);
+                tmem_ld2(tmem + CF::COL_OZ + lane_base + (C == 64 ? 0u : CF::oz_slot(slot)), oz);
                 tmem_ld_wait();
                 tc_fence_before();
                 // gathered rows: this thread's copy-out rows, read before the
@@ -488,7 +515,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 }
                 mbar_arrive(bofree + slot);
                 float den = rs + __uint_as_float(oz[0]) + __uint_as_float(oz[1]);
-                if (C == 64) den = __shfl_sync(0xffffffffu, den, lane & 15);
+                if (C == 64) den = __shfl_sync(0xffffffffu, den, (lane & 15) + 16 * slot);
                 const float inv = normalize ? __frcp_rn(den) : 1.0f;
                 if (!GATHER) {
                     // causal: the chunk's rows are contiguous; stage them and
@@ -546,6 +573,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         tc_fence_after();
         tmem_dealloc(tmem, CF::TMEM_COLS);
     }
+    pdl_trigger();
 }
 
 template <int D, int C, bool GATHER>
@@ -565,10 +593,9 @@ cudaError_t launch_chunked(const Problem& p, const void* q, const void* k, const
     e = ensure_smem<tc_sweep_kernel<D, C, GATHER>>(smem);
     if (e != cudaSuccess) return e;
     dim3 grid(nblk, (unsigned)p.bh());
-    tc_sweep_kernel<D, C, GATHER><<<grid, CF::THREADS, smem, st>>>(
-        mq, mk, mv, mo, static_cast<const __nv_bfloat16*>(q), prefix, p.H, p.N, block_tokens, nblk, perm, bins,
-        mcl, nbins, p.phi, p.normalize, static_cast<__nv_bfloat16*>(out), err);
-    return cudaGetLastError();
+    return launch_pdl(tc_sweep_kernel<D, C, GATHER>, grid, dim3(CF::THREADS), smem, st, mq, mk, mv, mo,
+                      static_cast<const __nv_bfloat16*>(q), prefix, p.H, p.N, block_tokens, nblk, perm, bins,
+                      mcl, nbins, p.phi, p.normalize, static_cast<__nv_bfloat16*>(out), err);
 }
 
 }  // namespace
