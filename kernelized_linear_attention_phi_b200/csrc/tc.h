@@ -46,6 +46,11 @@ cudaError_t tc_chunked(const Problem& p, int chunk, const void* q, const void* k
                        const int32_t* bins, const int32_t* mcl, int nbins, void* out, uint32_t* err,
                        cudaStream_t st);
 
+// The d = 128 kernel behind tc_chunked (64-token chunks, state kept as S^T).
+cudaError_t tc_chunked_t(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
+                         int block_tokens, int nblk, const int32_t* perm, const int32_t* bins,
+                         const int32_t* mcl, int nbins, void* out, uint32_t* err, cudaStream_t st);
+
 // [BH, N, d] bf16 viewed as 3-D for TMA: 64-column x `rows` boxes, 128-byte
 // swizzle, zero fill outside the tensor.
 cudaError_t make_map(CUtensorMap* map, const void* base, int d, int N, long long bh, int rows);

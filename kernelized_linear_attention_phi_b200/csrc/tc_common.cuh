@@ -192,6 +192,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b
         : "memory");
 }
 // Arrives on `bar` once every MMA this thread issued before has completed.
+// Same, with the A operand read from TMEM instead of shared memory: M lanes
+// from the address's lane, K-major, two 16-bit elements per 32-bit column
+// (the lower k in the low half), K / 2 columns per instruction.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      smem_u32(bar))
@@ -222,6 +234,13 @@ __device__ __forceinline__ void tmem_ld16x2(uint32_t taddr, uint32_t (&r)[16]) {
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
           "=r"(r[14]), "=r"(r[15])
         : "r"(taddr), "n"(SPLIT));
+}
+// Warp-wide, one column of an M = 64 accumulator: lanes 0..15 receive TMEM
+// lane (base + i) at the address's column, lanes 16..31 TMEM lane
+// (base + i - 16) at column + SPLIT.
+template <int SPLIT>
+__device__ __forceinline__ void tmem_ld1x2(uint32_t taddr, uint32_t& r) {
+    asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x1.b32 {%0}, [%1], %2;" : "=r"(r) : "r"(taddr), "n"(SPLIT));
 }
 // Warp-wide: lane i receives TMEM lane (base + i), 2 columns.
 __device__ __forceinline__ void tmem_ld2(uint32_t taddr, uint32_t (&r)[2]) {

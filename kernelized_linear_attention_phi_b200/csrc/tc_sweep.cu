@@ -608,10 +608,7 @@ cudaError_t tc_chunked(const Problem& p, int chunk, const void* q, const void* k
     const bool g = perm != nullptr;
 #define LA_CH(D_, C_, G_) \
     return launch_chunked<D_, C_, G_>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, mcl, nbins, out, err, st)
-    if (p.d == 128) {
-        if (g) LA_CH(128, 64, true);
-        LA_CH(128, 64, false);
-    }
+    if (p.d == 128) return tc_chunked_t(p, q, k, v, prefix, block_tokens, nblk, perm, bins, mcl, nbins, out, err, st);
     if (C == 64) {
         if (g) LA_CH(64, 64, true);
         LA_CH(64, 64, false);
