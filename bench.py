@@ -19,7 +19,11 @@ graphs are replayed. Timing: CUDA events between the calls of every step on
 the launching stream, L2 flushed (a 256 MiB write) between steps outside the
 events, W untimed warm-up steps, max over ranks. ``e2e`` repeats the step
 through the plain API calls with pinned host inputs copied in and the
-outputs copied back inside the timed region.
+outputs copied back inside the timed region. ``roofline`` is the dominant
+kernel's: after the timed steps every call is replayed again from a graph
+captured with the library's per-kernel timing events (la_timing_enable), L2
+flushed before each replay, and the kernel with the largest mean time has its
+algorithmic bytes divided by that time.
 """
 
 from __future__ import annotations
@@ -48,11 +52,23 @@ L2_FLUSH_BYTES = 256 << 20
 # launch list (--record-traffic matches them there).
 CALL_KERNELS = {
     "noncausal": ["tc_kv_kernel", "kv_reduce_balanced_kernel", "tc_readout_kernel"],
-    "causal": ["tc_kv_kernel", "state_scan_kernel", "tc_sweep_kernel"],
-    "prefix": ["bin_kernel", "tc_kv_kernel", "state_scan_kernel", "tc_sweep_kernel"],
+    "causal": ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"],
+    "prefix": ["bin_kernel", "tc_kv_kernel", "state_scan_kernel", "tc_sweep"],
+    "decode": ["decode_kernel"],
+}
+# The same on the fp32 (CUDA-core) path.
+CALL_KERNELS_F32 = {
+    "noncausal": ["kv_partial_kernel", "state_reduce_kernel", "readout_kernel"],
+    "causal": ["kv_partial_kernel", "state_scan_kernel", "chunked_kernel"],
+    "prefix": ["bin_kernel", "kv_partial_kernel", "state_scan_kernel", "chunked_kernel"],
     "decode": ["decode_kernel"],
 }
 LAUNCHES = {k: len(v) for k, v in CALL_KERNELS.items()}
+# What each kernel does, for its algorithmic bytes (Step.kernel_bytes).
+KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balanced_kernel": "reduce",
+               "state_reduce_kernel": "reduce", "tc_readout_kernel": "readout", "readout_kernel": "readout",
+               "state_scan_kernel": "scan", "tc_sweep": "sweep", "chunked_kernel": "sweep",
+               "bin_kernel": "bin", "decode_kernel": "decode"}
 
 
 def parse():
@@ -189,6 +205,19 @@ class Step:
         return {"noncausal": 4 * t + st, "causal": 4 * t, "prefix": 4 * t + self.B * self.N * 4,
                 "decode": 2 * st + 4 * one}
 
+    def kernel_bytes(self, call, kernel):
+        """Algorithmic bytes of one kernel of a call: the method's tensors it
+        must read or write once (Q, K, V, out, S, z, m). Scratch the library
+        keeps between its kernels (partial and block-state records, the
+        binning tables) is not counted, so a kernel that only moves scratch
+        (the prefix scan over block states) has none."""
+        t = self.B * self.H * self.N * self.d * self.elem
+        st = self.B * self.H * (self.d * self.d + self.d) * 4
+        one = self.B * self.H * self.d * self.elem
+        role = KERNEL_ROLE.get(kernel)
+        return {"kv": 2 * t, "reduce": st, "readout": 2 * t + st, "scan": 0, "sweep": 4 * t,
+                "bin": self.B * self.N * 4, "decode": 2 * st + 4 * one}.get(role, 0)
+
     def host_io(self):
         full = [f for f in self.forms if f != "decode"]
         ins = ([self.q, self.k, self.v] if full else []) + ([self.m] if "prefix" in self.forms else []) \
@@ -196,6 +225,33 @@ class Step:
         outs = [{"noncausal": self.out_nc, "causal": self.out_c, "prefix": self.out_m,
                  "decode": self.out_d}[f] for f in self.forms]
         return ins, outs
+
+
+def kernel_times(step, calls, flush, reps):
+    """Per call: the mean duration (ms) of each kernel it launches, from the
+    library's timing events over `reps` replays of a graph of the call."""
+    la = step.la
+    la.la_timing_enable(True)
+    out = {}
+    try:
+        for name, fn in calls:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            acc = None
+            for _ in range(reps):
+                flush_l2(flush)
+                g.replay()
+                ms = la.la_timing_read()
+                acc = ms if acc is None else [a + b for a, b in zip(acc, ms)]
+            out[name] = [a / reps for a in acc]
+            del g
+    finally:
+        la.la_timing_enable(False)
+    return out
 
 
 def flush_l2(buf):
@@ -308,6 +364,12 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_s = sum(a.elapsed_time(b) for a, b in e_ev) / 1e3
 
+    # each kernel's own duration: the calls replayed again from graphs
+    # captured with the library's per-kernel timing events (an event node
+    # between two kernels; the call-level numbers above come from graphs
+    # without them), L2 flushed before every replay, averaged over the replays
+    kt = kernel_times(step, calls, flush, max(3, min(K, 20)))
+
     # every call reports expired bounded waits in its workspace error word
     flags = {op: step.la.la_last_error(ws)[1] for op, ws in step.ws.items()}
     bad_flags = {op: f for op, f in flags.items() if f}
@@ -316,20 +378,32 @@ def run_ours(args, rank, world, local_rank):
     value = aggregate_tokens_per_s(step.tokens, K, world, t_s)
     e2e_value = aggregate_tokens_per_s(step.tokens, Ke, world, e2e_s)
 
-    # roofline of the dominant call (its kernels together), bytes per launch
-    alg = step.algorithmic_bytes()
-    dom = max(per_call, key=per_call.get)
-    dom_s = per_call[dom] / 1e3 / K
-    achieved = alg[dom] / dom_s / 1e9
     peaks = load_peaks()
     peak = peaks.get("hbm_gbs", 6650.0)
+    names = CALL_KERNELS if dtype == "bf16" else CALL_KERNELS_F32
     per_kernel = {}
     for name in per_call:
-        s = per_call[name] / 1e3 / K
-        per_kernel[name] = {"us": round(s * 1e6, 2), "GB_s": round(alg[name] / s / 1e9, 1),
-                            "frac_hbm": round(alg[name] / s / 1e9 / peak, 3),
-                            "share": round(per_call[name] / sum(per_call.values()), 3)}
+        s_call = per_call[name] / 1e3 / K
+        a = step.algorithmic_bytes()[name]
+        entry = {"us": round(s_call * 1e6, 2), "GB_s": round(a / s_call / 1e9, 1),
+                 "frac_hbm": round(a / s_call / 1e9 / peak, 3),
+                 "share": round(per_call[name] / sum(per_call.values()), 3), "kernels": []}
+        for i, ms in enumerate(kt.get(name, [])):
+            kn = names[name][i] if i < len(names[name]) else f"kernel{i}"
+            kb = step.kernel_bytes(name, kn)
+            entry["kernels"].append({"kernel": kn, "us": round(ms * 1e3, 2),
+                                     "GB_s": round(kb / (ms / 1e3) / 1e9, 1) if kb else None,
+                                     "frac_hbm": round(kb / (ms / 1e3) / 1e9 / peak, 3) if kb else None})
+        per_kernel[name] = entry
 
+    # roofline of the dominant kernel: the (call, kernel) with the largest
+    # time in the step, its algorithmic bytes over its own timed duration
+    cands = [(ms, name, i) for name, lst in kt.items() for i, ms in enumerate(lst)
+             if step.kernel_bytes(name, names[name][i] if i < len(names[name]) else "") > 0]
+    dom_ms, dom, di = max(cands)
+    dom_kernel = names[dom][di]
+    dom_bytes = step.kernel_bytes(dom, dom_kernel)
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
     result = {
         "metric": "tokens/sec (fwd, 1xB200) and % of HBM / bf16 tensor-core roofline per kernel",
         "value": value,
@@ -356,9 +430,10 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": sum(LAUNCHES[n] for n, _ in calls) * K,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": recorded_traffic(wl.name, dtype, dom),
-                     "kernel": f"la_{dom} (all its kernels)", "peak_source": peaks.get("_src"),
-                     "algorithmic_bytes": alg[dom]},
+                     "traffic": recorded_traffic(wl.name, dtype, f"{dom}/{di}"),
+                     "kernel": f"{dom_kernel} (kernel {di} of la_{dom})",
+                     "kernel_us": round(dom_ms * 1e3, 2), "peak_source": peaks.get("_src"),
+                     "algorithmic_bytes": dom_bytes},
         "per_call": per_kernel,
         "clocks": sampler.summary(),
     }
@@ -386,10 +461,11 @@ def library_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload, dtype, call):
-    """DRAM bytes (read + write) per call, summed over the call's kernels, from
-    the ncu capture in profiles/traffic.json; None when none was taken for
-    this workload and call, or the kernels changed since."""
+def recorded_traffic(workload, dtype, key):
+    """DRAM bytes (read + write) of one call ("causal") or one of its kernels
+    ("causal/2", by launch index) from the ncu capture in
+    profiles/traffic.json; None when none was taken for this workload and
+    key, or the kernels changed since."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)
@@ -397,7 +473,7 @@ def recorded_traffic(workload, dtype, call):
         return None
     if rec.get("source_hash") != library_source_hash():
         return None
-    return rec.get("bytes", {}).get(f"{workload}/{dtype}/{call}")
+    return rec.get("bytes", {}).get(f"{workload}/{dtype}/{key}")
 
 
 def load_peaks():
@@ -529,9 +605,11 @@ def record_traffic(csv_path, workload, dtype):
             break
     else:
         raise SystemExit("the launch list holds no complete step of this workload")
-    per_call = {}
+    per_call, per_kernel = {}, {}
     for n, (f, _) in enumerate(want):
         per_call[f] = per_call.get(f, 0.0) + seq[start + n]["bytes"]
+        i = sum(1 for g, _ in want[:n] if g == f)  # the kernel's index within its call
+        per_kernel[f"{f}/{i}"] = seq[start + n]["bytes"]
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -540,11 +618,14 @@ def record_traffic(csv_path, workload, dtype):
         out = {}
     if out.get("source_hash") != library_source_hash():
         out = {"source_hash": library_source_hash(), "bytes": {}}
-    out["note"] = ("DRAM bytes read + written per library call, summed over the call's kernels, "
+    out["note"] = ("DRAM bytes read + written per library call (workload/dtype/call, summed over "
+                   "the call's kernels) and per kernel (workload/dtype/call/index in launch order), "
                    "from an ncu launch list (cold cache per kernel); valid for the CUDA sources "
                    "with this hash")
     for f, b in per_call.items():
         out["bytes"][f"{workload}/{dtype}/{f}"] = int(b)
+    for key, b in per_kernel.items():
+        out["bytes"][f"{workload}/{dtype}/{key}"] = int(b)
     with open(path, "w") as f:
         json.dump(out, f, indent=1, sort_keys=True)
     print(json.dumps(per_call))

@@ -186,6 +186,26 @@ LA_API la_status la_kv_summary_static(const la_desc* desc, const void* k, const 
  * no bit was set, LA_ERR_CUDA on a CUDA failure. */
 LA_API la_status la_last_error(void* ws, void* stream, uint32_t* flags_out);
 
+/* Per-kernel timing, a measurement aid with no counterpart in the method.
+ * While enabled, every entry point records a CUDA event on its stream before
+ * its first kernel and one after each kernel it launches (16 at most per
+ * call). The events are the library's own, created by la_timing_enable(1) on
+ * the current device (LA_ERR_CUDA if that fails); la_timing_enable(0) stops
+ * the recording. Under stream capture the records become event nodes of the
+ * graph and are taken again at each replay; an event node between two kernels
+ * ends the overlap of the second kernel's start with the first one's end, so
+ * timed calls can run slightly slower than untimed ones. The state is global
+ * to the process: only one call at a time may run while timing is on.
+ *
+ * la_timing_read waits for the last call's (or the last replay's) final
+ * event, then writes the duration in milliseconds of its kernel i (from the
+ * event before it to the event after it) to ms[i] for i < capacity, and the
+ * number of kernels that call launched to *count (0 if no call was recorded).
+ * Returns LA_ERR_INVALID_ARG for a NULL count, a negative capacity or a NULL
+ * ms with capacity > 0, LA_ERR_CUDA on a CUDA failure. */
+LA_API la_status la_timing_enable(int32_t enable);
+LA_API la_status la_timing_read(float* ms, int32_t capacity, int32_t* count);
+
 /* Static string naming a status. */
 LA_API const char* la_status_string(la_status status);
 

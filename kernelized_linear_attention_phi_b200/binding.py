@@ -57,6 +57,9 @@ _SIGS = {
     "la_decode_step": (ctypes.c_int, [ctypes.POINTER(la_desc), _P, _P, _P, _P, _P, _P, _P]),
     "la_kv_summary_static": (ctypes.c_int, [ctypes.POINTER(la_desc), _P, _P, _P, _P, _P]),
     "la_last_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
+    "la_timing_enable": (ctypes.c_int, [ctypes.c_int32]),
+    "la_timing_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.c_int32,
+                                      ctypes.POINTER(ctypes.c_int32)]),
     "la_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "la_version": (ctypes.c_int32, []),
 }
@@ -239,3 +242,18 @@ def la_last_error(ws, stream=None):
     flags = ctypes.c_uint32(0)
     st = lib().la_last_error(_ptr(ws), _stream(ws, stream), ctypes.byref(flags))
     return int(st), int(flags.value)
+
+
+def la_timing_enable(enable=True):
+    """Turns the library's per-kernel timing events on or off (on: creates
+    them on the current device)."""
+    _check("la_timing_enable", lib().la_timing_enable(1 if enable else 0))
+
+
+def la_timing_read(capacity=16):
+    """Durations in ms of the kernels of the last timed call (or graph
+    replay), in launch order; waits for that call to finish."""
+    buf = (ctypes.c_float * capacity)()
+    n = ctypes.c_int32(0)
+    _check("la_timing_read", lib().la_timing_read(buf, capacity, ctypes.byref(n)))
+    return [float(buf[i]) for i in range(min(n.value, capacity))]

@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "launch_util.h"
 #include "tc.h"
 #include "tc_common.cuh"
 
@@ -184,6 +185,7 @@ la_status kv_summary_checked(const la_desc* desc, const void* k, const void* v, 
     const Problem p = to_problem(desc);
     LA_TRY(check_ws(ws_layout(p, LA_OP_KV_SUMMARY), ws, ws_bytes));
     LA_TRY(check_device());
+    timing_begin(st);
     return kv_summary_impl(p, k, v, S_out, z_out, ws, st);
 }
 
@@ -234,6 +236,7 @@ la_status la_noncausal(const la_desc* desc, const void* q, const void* k, const 
     LA_TRY(check_ws(L, ws, ws_bytes));
     LA_TRY(check_device());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    timing_begin(st);
     float* S = S_out;
     float* z = z_out;
     if (S == nullptr) {
@@ -256,6 +259,7 @@ la_status la_causal_chunked(const la_desc* desc, int32_t chunk, const void* q, c
     LA_TRY(check_ws(L, ws, ws_bytes));
     LA_TRY(check_device());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    timing_begin(st);
     const BlockPlan bp = block_plan(p);
     float* part = at<float>(ws, L.part);
     // phase 1: per-block states; phase 2: exclusive prefix over blocks;
@@ -288,6 +292,7 @@ la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, cons
     LA_TRY(check_ws(L, ws, ws_bytes));
     LA_TRY(check_device());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    timing_begin(st);
     const BlockPlan bp = block_plan(p);
     const bool tc = tc_supported(p);
     const int kchunk = tc ? tc_chunk(p, chunk) : kSimtChunk;  // chunk length of the kernel used
@@ -322,6 +327,7 @@ la_status la_decode_step(const la_desc* desc, const void* q, const void* k, cons
         !aligned16(out))
         return LA_ERR_MISALIGNED;
     LA_TRY(check_device());
+    timing_begin(static_cast<cudaStream_t>(stream));
     return cuda_status(decode_step(to_problem(&d1), q, k, v, S, z, out,
                                    static_cast<cudaStream_t>(stream)));
 }

@@ -9,6 +9,11 @@
 
 namespace la {
 
+// Per-launch timing hook (timing.cu): an event before a call's first kernel
+// and one after each launch, while la_timing_enable is on.
+void timing_begin(cudaStream_t st);
+void timing_mark(cudaStream_t st);
+
 // Launches `kernel` with programmatic stream serialization (see pdl_wait /
 // pdl_trigger in common.cuh).
 template <typename... KArgs, typename... Args>
@@ -24,7 +29,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    if (e == cudaSuccess) timing_mark(st);
+    return e;
 }
 
 // Raises a kernel's dynamic shared-memory limit once per device (the

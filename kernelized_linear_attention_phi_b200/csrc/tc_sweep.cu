@@ -301,18 +301,24 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             uint8_t* st = stages + s * CF::STAGE;
             uint4* kt = reinterpret_cast<uint4*>(st + (GATHER ? 0 : CF::TILE));
             mbar_wait(full + s, u & 1, err);
-#pragma unroll 4
-            for (int i = 0; i < CF::NB * C / 16; ++i) {
-                const int p = et + 128 * i;
-                const int r = (p % (C * 8)) >> 3;
-                if (r < kvalid) {
-                    if (relu) kt[p] = phi_relu1_x8(kt[p]);
-                } else {
-                    kt[p] = make_uint4(0, 0, 0, 0);
+            // in groups of 4 chunks, all loads of a group first: a load placed
+            // after a shared store could not be moved ahead of it (aliasing)
+#pragma unroll
+            for (int i0 = 0; i0 < CF::NB * C / 16; i0 += 4) {
+                uint4* qt = reinterpret_cast<uint4*>(st);
+                uint4 kx[4], qx[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int p = et + 128 * (i0 + i);
+                    kx[i] = kt[p];
+                    if (!GATHER && relu) qx[i] = qt[p];
                 }
-                if (!GATHER && relu) {
-                    uint4* qt = reinterpret_cast<uint4*>(st);
-                    qt[p] = phi_relu1_x8(qt[p]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int p = et + 128 * (i0 + i);
+                    const int r = (p % (C * 8)) >> 3;
+                    kt[p] = r < kvalid ? (relu ? phi_relu1_x8(kx[i]) : kx[i]) : make_uint4(0, 0, 0, 0);
+                    if (!GATHER && relu) qt[p] = phi_relu1_x8(qx[i]);
                 }
             }
             if (ci > 0) {

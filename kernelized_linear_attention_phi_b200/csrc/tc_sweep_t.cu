@@ -200,6 +200,8 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                 const int s = ci % CF::STAGES;
                 const uint32_t st = smem_u32(stages + s * CF::STAGE);
                 const uint32_t kt = st + CF::OFF_K, vt = st + CF::OFF_V;
+                flush();
+                if (!ok) break;
                 ok = mbar_wait(bprep, ci & 1, err);
                 if (!ok) break;
                 tc_fence_after();
@@ -230,7 +232,7 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                     for (int kk = 0; kk < D / 16; ++kk)
                         mma_bf16_ts(tmem + CF::COL_O + j * C, sb + kk * 8,
                                     sdesc(qt + (kk / 4) * CF::BOX + (kk % 4) * 32, 16, 1024), idO, kk > 0);
-                    flush();
+                    if (t > 0) flush();
                     pend = tq;
                     pend_vt = vt;
                     pend_stage = t == ntq - 1 ? s : -1;

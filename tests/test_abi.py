@@ -109,3 +109,21 @@ def test_valid_request_without_gpu_reports_cuda_error(lib):
     """A request that passes validation reaches the device check, which fails
     cleanly with LA_ERR_CUDA when no GPU is present (nothing is launched)."""
     assert call_noncausal(lib, desc()) == 5
+
+
+def test_timing_read_validation(lib):
+    """la_timing_read rejects a NULL count, a negative capacity and a NULL
+    buffer with room asked for; with nothing recorded it reports 0 kernels."""
+    n = ctypes.c_int32(-1)
+    buf = (ctypes.c_float * 4)()
+    assert lib.la_timing_read(buf, 4, None) == 1
+    assert lib.la_timing_read(buf, -1, ctypes.byref(n)) == 1
+    assert lib.la_timing_read(None, 4, ctypes.byref(n)) == 1
+    assert lib.la_timing_enable(0) == 0
+    assert lib.la_timing_read(None, 0, ctypes.byref(n)) == 0 and n.value == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful on a machine with no GPU")
+def test_timing_enable_without_gpu_reports_cuda_error(lib):
+    assert lib.la_timing_enable(1) == 5
+    assert lib.la_timing_enable(0) == 0
