@@ -74,7 +74,6 @@ bin_kernel(const int32_t* __restrict__ m, int N, int chunk, int nbins, int32_t* 
         const int pos = atomicAdd(&cnt[(mi + 1) / chunk], 1);
         perm[(size_t)b * N + pos] = i;
     }
-    pdl_trigger();
 }
 
 }  // namespace

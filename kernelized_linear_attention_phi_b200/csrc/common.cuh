@@ -72,14 +72,20 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 }
 
 // Programmatic dependent launch. Every kernel of the library is launched
-// with programmatic stream serialization: it may start while the previous
-// kernel on the stream finishes, runs its prologue (shared memory, barriers,
-// TMEM), and waits in pdl_wait() before it touches global memory. Each kernel
-// lets its dependents launch only at its very end (pdl_trigger() after all
-// its work and its TMEM release), so a waiting dependent never holds resources
-// that a CTA of the running kernel still needs.
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// with programmatic stream serialization and calls pdl_wait() after its
+// prologue (shared memory, barriers, TMEM), before it touches global memory.
+// pdl_wait() waits for the previous kernel on the stream to complete with its
+// memory visible, then lets this kernel's own dependents launch: the hardware
+// starts them once every CTA of this grid has got that far, so their launch
+// and prologue overlap this kernel's work, and their own pdl_wait() still
+// waits for this whole grid to complete. (No CTA of this grid is left to
+// start by then, so an early dependent never takes an SM from this grid;
+// one that is resident on an SM where this grid still holds TMEM waits in its
+// allocation until that CTA releases it.)
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // Streaming 16-byte global load (read once: do not keep in L1).
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {

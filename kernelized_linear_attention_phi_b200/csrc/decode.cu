@@ -96,7 +96,6 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         for (int w = 0; w < kThreads / 32; ++w) den += sden[w];
         out[bh * D + tid] = from_f32<T>(normalize ? acc / den : acc);
     }
-    pdl_trigger();
 }
 
 template <typename T, int D>

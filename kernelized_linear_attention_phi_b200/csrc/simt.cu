@@ -93,7 +93,6 @@ kv_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int N, int t
         for (int c = 0; c < R; ++c) o[(ta * R + r) * D + tb * R + c] = acc[r][c];
         if (tb == 0) o[D * D + ta * R + r] = zacc[r];
     }
-    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -112,7 +111,6 @@ __global__ void state_reduce_kernel(const float* __restrict__ part, int nsplit, 
         if (e < D * D) S[(size_t)bh * D * D + e] = s;
         else z[(size_t)bh * D + (e - D * D)] = s;
     }
-    pdl_trigger();
 }
 
 // One thread per float4 of a record; loads are issued eight blocks at a time
@@ -124,7 +122,6 @@ __global__ void state_scan_kernel(float* __restrict__ part, int nblk, int D,
     const long long bh = blockIdx.y;
     pdl_wait();
     if (e >= rec4) {
-        pdl_trigger();
         return;
     }
     float4* p = reinterpret_cast<float4*>(part + (size_t)bh * nblk * (rec4 * 4)) + e;
@@ -154,7 +151,6 @@ __global__ void state_scan_kernel(float* __restrict__ part, int nblk, int D,
             else z_total[(size_t)bh * D + (idx - D * D)] = r[q];
         }
     }
-    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -218,7 +214,6 @@ readout_kernel(const T* __restrict__ Q, const float* __restrict__ S, const float
         for (int c = 0; c < RC; ++c)
             Oh[(long long)row * D + tc * RC + c] = from_f32<T>(normalize ? acc[i][c] / den : acc[i][c]);
     }
-    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -422,7 +417,6 @@ chunked_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __rest
             }
         }
     }
-    pdl_trigger();
 }
 
 template <typename T, int D>

@@ -326,7 +326,6 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
-    pdl_trigger();
 }
 
 // Sums the partial records of each head in CTA order (deterministic).
@@ -337,7 +336,6 @@ __global__ void kv_reduce_balanced_kernel(const float* __restrict__ part, KvBala
     const long long h = blockIdx.y;
     if (e >= rec4) {
         pdl_wait();
-        pdl_trigger();
         return;
     }
     pdl_wait();
@@ -372,7 +370,6 @@ __global__ void kv_reduce_balanced_kernel(const float* __restrict__ part, KvBala
         if (idx < D * D) S[(size_t)h * D * D + idx] = r[q];
         else z[(size_t)h * D + (idx - D * D)] = r[q];
     }
-    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -583,7 +580,6 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
-    pdl_trigger();
 }
 
 template <int D>

@@ -579,7 +579,6 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         tc_fence_after();
         tmem_dealloc(tmem, CF::TMEM_COLS);
     }
-    pdl_trigger();
 }
 
 template <int D, int C, bool GATHER>

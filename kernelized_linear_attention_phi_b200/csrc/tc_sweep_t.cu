@@ -508,7 +508,6 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
         tc_fence_after();
         tmem_dealloc(tmem, CF::TMEM_COLS);
     }
-    pdl_trigger();
 }
 
 template <bool GATHER>
