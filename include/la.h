@@ -35,9 +35,10 @@
  *   - Validation is fail-closed: on any status other than LA_OK nothing was
  *     launched, except LA_ERR_CUDA, which reports a failed launch.
  *   - Supported: d in {16, 32, 64, 128}; dtype LA_F32 or LA_BF16;
- *     phi LA_PHI_RELU1 or LA_PHI_IDENTITY; normalize in {0, 1}, with
- *     normalize = 1 only for LA_PHI_RELU1 (with the identity map the
- *     denominator phi(q).z can be zero or negative). Device: compute
+ *     phi LA_PHI_RELU1, LA_PHI_IDENTITY or LA_PHI_ELU1; normalize in
+ *     {0, 1}, with normalize = 1 only for the positive maps LA_PHI_RELU1 and
+ *     LA_PHI_ELU1 (with the identity map the denominator phi(q).z can be
+ *     zero or negative). Device: compute
  *     capability 10.x (B200).
  *   - Results are deterministic: every reduction runs in a fixed order, so
  *     repeated calls on the same inputs give bit-identical outputs.
@@ -74,7 +75,9 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
 
 typedef enum {
     LA_PHI_RELU1 = 0,    /* phi(x) = relu(x) + 1, relu by the sign bit (-0.0 -> 1) */
-    LA_PHI_IDENTITY = 1  /* phi(x) = x (unnormalized Q K^T V form) */
+    LA_PHI_IDENTITY = 1, /* phi(x) = x (unnormalized Q K^T V form) */
+    LA_PHI_ELU1 = 2      /* phi(x) = elu(x) + 1: x + 1 for x > 0, exp(x) otherwise
+                            (lineartile 1.0.1, "How It Works"; elu with alpha = 1) */
 } la_phi;
 
 typedef enum {
@@ -126,6 +129,18 @@ LA_API la_status la_noncausal(const la_desc* desc, const void* q, const void* k,
 LA_API la_status la_causal_chunked(const la_desc* desc, int32_t chunk, const void* q,
                             const void* k, const void* v, void* out,
                             void* ws, size_t ws_bytes, void* stream);
+
+/* Causal prefill (trim-transformer 0.1.0, "Key-value caching": the cache
+ * built over a prompt is what the one-token steps continue from): the same
+ * outputs as la_causal_chunked, and in the same pass the state after the last
+ * token, S_out = sum_j phi(k_j)^T v_j and z_out = sum_j phi(k_j) over all N
+ * keys, float32 [B,H,d,d] and [B,H,d], overwritten, ready for
+ * la_decode_step. Same arguments, workspace (op LA_OP_CAUSAL) and errors as
+ * la_causal_chunked, plus LA_ERR_INVALID_ARG for a NULL S_out or z_out and
+ * LA_ERR_MISALIGNED when either is not 16-byte aligned. */
+LA_API la_status la_causal_prefill(const la_desc* desc, int32_t chunk, const void* q,
+                                   const void* k, const void* v, void* out, float* S_out,
+                                   float* z_out, void* ws, size_t ws_bytes, void* stream);
 
 /* Prefix-mask attention (trim-transformer 0.1.0, "Masking"): query i of
  * sequence b sees keys 0..m[b*N + i], inclusive. m: int32 [B, N] device

@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED",
                 3: "LA_ERR_MISALIGNED", 4: "LA_ERR_WORKSPACE", 5: "LA_ERR_CUDA",
                 6: "LA_ERR_MASK_RANGE", 7: "LA_ERR_TIMEOUT"}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
-PHIS = {"relu1": 0, "identity": 1}
+PHIS = {"relu1": 0, "identity": 1, "elu1": 2}
 OPS = {"kv_summary": 0, "noncausal": 1, "causal": 2, "prefix": 3, "decode": 4}
 
 
@@ -51,6 +51,8 @@ _SIGS = {
     "la_noncausal": (ctypes.c_int, [ctypes.POINTER(la_desc), _P, _P, _P, _P, _P, _P, _P,
                                     ctypes.c_size_t, _P]),
     "la_causal_chunked": (ctypes.c_int, [ctypes.POINTER(la_desc), ctypes.c_int32, _P, _P, _P, _P,
+                                         _P, ctypes.c_size_t, _P]),
+    "la_causal_prefill": (ctypes.c_int, [ctypes.POINTER(la_desc), ctypes.c_int32, _P, _P, _P, _P, _P, _P,
                                          _P, ctypes.c_size_t, _P]),
     "la_prefix_mask": (ctypes.c_int, [ctypes.POINTER(la_desc), ctypes.c_int32, _P, _P, _P, _P, _P,
                                       _P, ctypes.c_size_t, _P]),
@@ -199,6 +201,31 @@ def la_causal_chunked(q, k, v, out=None, chunk=64, phi="relu1", normalize=True, 
         ctypes.byref(desc), int(chunk), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(ws),
         ws.numel(), _stream(q, stream)))
     return out
+
+
+def la_causal_prefill(q, k, v, out=None, S_out=None, z_out=None, chunk=64, phi="relu1", normalize=True,
+                      ws=None, stream=None):
+    """Causal attention plus the state after the last token (the cache a
+    decode continues from). Returns (out, S, z)."""
+    if out is None:
+        out = torch.empty_like(q)
+    _same(q, k, v, out)
+    B, H, _, d = q.shape
+    if S_out is None:
+        S_out = torch.empty(B, H, d, d, dtype=torch.float32, device=q.device)
+    if z_out is None:
+        z_out = torch.empty(B, H, d, dtype=torch.float32, device=q.device)
+    if S_out.dtype != torch.float32 or tuple(S_out.shape) != (B, H, d, d) or not S_out.is_contiguous():
+        raise ValueError("S_out must be contiguous float32 [B, H, d, d]")
+    if z_out.dtype != torch.float32 or tuple(z_out.shape) != (B, H, d) or not z_out.is_contiguous():
+        raise ValueError("z_out must be contiguous float32 [B, H, d]")
+    desc = _desc_of(q, phi, normalize)
+    if ws is None:
+        ws = workspace(desc, "causal", chunk, device=q.device)
+    _check("la_causal_prefill", lib().la_causal_prefill(
+        ctypes.byref(desc), int(chunk), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(S_out), _ptr(z_out),
+        _ptr(ws), ws.numel(), _stream(q, stream)))
+    return out, S_out, z_out
 
 
 def la_prefix_mask(q, k, v, m, out=None, chunk=64, phi="relu1", normalize=True, ws=None,

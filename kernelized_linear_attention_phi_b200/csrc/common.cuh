@@ -7,7 +7,7 @@
 
 namespace la {
 
-enum { PHI_RELU1 = 0, PHI_IDENTITY = 1 };
+enum { PHI_RELU1 = 0, PHI_IDENTITY = 1, PHI_ELU1 = 2 };
 enum { DT_F32 = 0, DT_BF16 = 1 };
 
 // Error-word bits written into the workspace header.
@@ -22,8 +22,11 @@ constexpr size_t WS_HEADER = 256;
 __device__ __forceinline__ float phi_relu1(float x) {
     return ((__float_as_uint(x) & 0x80000000u) ? 0.0f : x) + 1.0f;
 }
+// elu1: elu(x) + 1 with alpha = 1, i.e. x + 1 for x > 0 and exp(x)
+// otherwise (lineartile 1.0.1, "How It Works"); -0.0 and +0.0 both map to 1.
+__device__ __forceinline__ float phi_elu1(float x) { return x > 0.0f ? x + 1.0f : expf(x); }
 __device__ __forceinline__ float phi_apply(float x, int phi) {
-    return phi == PHI_RELU1 ? phi_relu1(x) : x;
+    return phi == PHI_RELU1 ? phi_relu1(x) : phi == PHI_ELU1 ? phi_elu1(x) : x;
 }
 
 // 16-byte vector <-> floats.

@@ -31,7 +31,7 @@ la_status check_desc(const la_desc* d) {
     if (d == nullptr) return LA_ERR_INVALID_ARG;
     if (d->B <= 0 || d->H <= 0 || d->N <= 0 || d->d <= 0) return LA_ERR_INVALID_ARG;
     if (d->dtype != LA_F32 && d->dtype != LA_BF16) return LA_ERR_INVALID_ARG;
-    if (d->phi != LA_PHI_RELU1 && d->phi != LA_PHI_IDENTITY) return LA_ERR_INVALID_ARG;
+    if (d->phi != LA_PHI_RELU1 && d->phi != LA_PHI_IDENTITY && d->phi != LA_PHI_ELU1) return LA_ERR_INVALID_ARG;
     if (d->normalize != 0 && d->normalize != 1) return LA_ERR_INVALID_ARG;
     if (d->d != 16 && d->d != 32 && d->d != 64 && d->d != 128) return LA_ERR_UNSUPPORTED;
     if (d->normalize == 1 && d->phi == LA_PHI_IDENTITY) return LA_ERR_UNSUPPORTED;
@@ -248,34 +248,61 @@ la_status la_noncausal(const la_desc* desc, const void* q, const void* k, const 
     return cuda_status(simt_readout(p, q, S, z, out, st));
 }
 
-la_status la_causal_chunked(const la_desc* desc, int32_t chunk, const void* q, const void* k,
-                            const void* v, void* out, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace la {
+namespace {
+
+// Causal outputs; with S_total/z_total (both or neither) also the state after
+// the last token, written by the block-state scan.
+la_status causal_impl(const la_desc* desc, int32_t chunk, const void* q, const void* k, const void* v,
+                      void* out, float* S_total, float* z_total, void* ws, size_t ws_bytes,
+                      cudaStream_t st) {
     LA_TRY(check_desc(desc));
     LA_TRY(check_chunk(chunk));
     if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_MISALIGNED;
+    if (S_total && (!aligned16(S_total) || !aligned16(z_total))) return LA_ERR_MISALIGNED;
     const Problem p = to_problem(desc);
     const WsLayout L = ws_layout(p, LA_OP_CAUSAL);
     LA_TRY(check_ws(L, ws, ws_bytes));
     LA_TRY(check_device());
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     timing_begin(st);
     const BlockPlan bp = block_plan(p);
     float* part = at<float>(ws, L.part);
-    // phase 1: per-block states; phase 2: exclusive prefix over blocks;
-    // phase 3: each block's outputs from its prefix state.
+    // phase 1: per-block states; phase 2: exclusive prefix over blocks (and
+    // the total); phase 3: each block's outputs from its prefix state.
     uint32_t* flags = at<uint32_t>(ws, 0);
     if (tc_supported(p)) {
         LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
     } else {
         LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
     }
-    LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
+    LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, S_total, z_total, st)));
     if (tc_supported(p))
         return cuda_status(tc_chunked(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, nullptr,
                                       nullptr, nullptr, 0, out, flags, st));
     return cuda_status(simt_chunked(p, q, k, v, part, bp.block_tokens, bp.nblk, nullptr, nullptr,
                                     nullptr, 0, out, st));
+}
+
+}  // namespace
+}  // namespace la
+
+extern "C" {
+
+la_status la_causal_chunked(const la_desc* desc, int32_t chunk, const void* q, const void* k,
+                            const void* v, void* out, void* ws, size_t ws_bytes, void* stream) {
+    return causal_impl(desc, chunk, q, k, v, out, nullptr, nullptr, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream));
+}
+
+la_status la_causal_prefill(const la_desc* desc, int32_t chunk, const void* q, const void* k,
+                            const void* v, void* out, float* S_out, float* z_out, void* ws,
+                            size_t ws_bytes, void* stream) {
+    if (S_out == nullptr || z_out == nullptr) return LA_ERR_INVALID_ARG;
+    return causal_impl(desc, chunk, q, k, v, out, S_out, z_out, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream));
 }
 
 la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, const void* k,

@@ -296,6 +296,19 @@ __device__ __forceinline__ uint4 phi_relu1_x8(uint4 w) {
     }
     return make_uint4(v[0], v[1], v[2], v[3]);
 }
+// phi = elu(x) + 1 (alpha = 1) on eight packed bf16 values: x + 1 for x > 0,
+// exp(x) otherwise, in fp32, each result rounded to bf16 once.
+__device__ __forceinline__ uint4 phi_elu1_x8(uint4 w) {
+    float f[8];
+    unpack8(w, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = f[e] > 0.0f ? f[e] + 1.0f : __expf(f[e]);
+    return pack8(f);
+}
+// A feature map other than the identity on eight packed bf16 values.
+__device__ __forceinline__ uint4 phi_x8(uint4 w, int phi) {
+    return phi == PHI_ELU1 ? phi_elu1_x8(w) : phi_relu1_x8(w);
+}
 // relu on eight packed bf16 values (exact).
 __device__ __forceinline__ uint4 relu_x8(uint4 w) {
     const __nv_bfloat162 zero = __float2bfloat162_rn(0.0f);

@@ -8,7 +8,8 @@
 //   S = relu(K)^T V + 1 (x) colsum(V) and z = sum relu(K) + count. The
 //   column sums of relu(K) and V are fp32 sums taken by the warps that
 //   prepare each tile; S accumulates in fp32 in TMEM. So S and z carry no
-//   bf16 rounding of phi(K).
+//   bf16 rounding of phi(K). For phi = elu+1 (no such split) the K operand
+//   is phi(K) rounded to bf16 and z sums those values.
 // Readout (nx source, per-query loop):
 //   out = phi(Q) S / (phi(Q) . z): MMA with M = 128 tokens, N = d_v,
 //   K = d_k against S (bf16, MN-major) plus an N = 16 MMA against
@@ -136,6 +137,7 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int nseg = kv_nseg(w);
     const bool relu = phi == PHI_RELU1;
+    const bool elu = phi == PHI_ELU1;
 
     if (threadIdx.x == 0) {
         cta_abort_reset();
@@ -219,7 +221,7 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
         for (int j = 0; j < nseg; ++j) {
             const Seg sg = kv_seg(w, N, j);
             const int nt = (sg.t1 - sg.t0 + kTile - 1) / kTile;
-            float zk[C::NB][8], cv[C::NB][8];  // column sums of relu(K) (or K) and of V
+            float zk[C::NB][8], cv[C::NB][8];  // column sums of the K operand and of V
 #pragma unroll
             for (int b = 0; b < C::NB; ++b)
 #pragma unroll
@@ -239,6 +241,9 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
                     if (r < valid) {
                         if (relu) {
                             wk = relu_x8(wk);
+                            kt[p] = wk;
+                        } else if (elu) {  // no exact split: phi(K) itself, rounded to bf16
+                            wk = phi_elu1_x8(wk);
                             kt[p] = wk;
                         }
                     } else {
@@ -491,7 +496,6 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
     } else {
         const int et = threadIdx.x - 64;
         const int sp = warp & 3;
-        const bool relu = phi == PHI_RELU1;
         bool ok = true;
         auto transform = [&](int it) {
             const long long g = lo + it;
@@ -524,10 +528,10 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
             }
             const int s = it % C::STAGES, u = it / C::STAGES;
             ok = ok && mbar_wait(full + s, u & 1, err);
-            if (ok && relu) {
+            if (ok && phi != PHI_IDENTITY) {
                 uint4* qt = reinterpret_cast<uint4*>(tiles + s * C::TILE);
 #pragma unroll
-                for (int i = 0; i < C::NB * 8; ++i) qt[et + 128 * i] = phi_relu1_x8(qt[et + 128 * i]);
+                for (int i = 0; i < C::NB * 8; ++i) qt[et + 128 * i] = phi_x8(qt[et + 128 * i], phi);
             }
             fence_async_smem();
             mbar_arrive(tdone + s);

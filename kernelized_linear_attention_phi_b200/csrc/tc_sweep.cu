@@ -114,7 +114,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     const int c_begin = blk * (block_tokens / C);
     const int c_end = (GATHER && blk == nblk - 1) ? nbins : min(nchunks, c_begin + block_tokens / C);
     const int nci = c_end - c_begin;
-    const bool relu = phi == PHI_RELU1;
+    const bool mapped = phi != PHI_IDENTITY;  // phi applied to Q and K tiles
     const size_t hoff = (size_t)bh * N * D;
 
     auto q_tiles = [&](int c) -> int {
@@ -311,14 +311,14 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 for (int i = 0; i < 4; ++i) {
                     const int p = et + 128 * (i0 + i);
                     kx[i] = kt[p];
-                    if (!GATHER && relu) qx[i] = qt[p];
+                    if (!GATHER && mapped) qx[i] = qt[p];
                 }
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int p = et + 128 * (i0 + i);
                     const int r = (p % (C * 8)) >> 3;
-                    kt[p] = r < kvalid ? (relu ? phi_relu1_x8(kx[i]) : kx[i]) : make_uint4(0, 0, 0, 0);
-                    if (!GATHER && relu) qt[p] = phi_relu1_x8(qx[i]);
+                    kt[p] = r < kvalid ? (mapped ? phi_x8(kx[i], phi) : kx[i]) : make_uint4(0, 0, 0, 0);
+                    if (!GATHER && mapped) qt[p] = phi_x8(qx[i], phi);
                 }
             }
             if (ci > 0) {
@@ -415,7 +415,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                         const int p = et + 128 * j;
                         const int r = p / (D / 8), col = (p % (D / 8)) * 8;
                         *reinterpret_cast<uint4*>(q + (col / 64) * (C * 128) + sw128_off(r, col % 64)) =
-                            relu ? phi_relu1_x8(w[j]) : w[j];
+                            mapped ? phi_x8(w[j], phi) : w[j];
                     }
                     fence_async_smem();
                     mbar_arrive(bqready + slot);

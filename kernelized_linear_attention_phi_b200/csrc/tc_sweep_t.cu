@@ -105,7 +105,7 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
     const int c_begin = blk * (block_tokens / C);
     const int c_end = (GATHER && blk == nblk - 1) ? nbins : min(nchunks, c_begin + block_tokens / C);
     const int nci = c_end - c_begin;
-    const bool relu = phi == PHI_RELU1;
+    const bool mapped = phi != PHI_IDENTITY;  // phi applied to Q and K tiles
     const size_t hoff = (size_t)bh * N * D;
 
     auto q_tiles = [&](int c) -> int {
@@ -297,7 +297,7 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                     uint4* kp = reinterpret_cast<uint4*>(kt + bx * CF::KBOX + w * 16);
                     uint4 x = *kp;
                     if (r < kvalid) {
-                        if (relu) x = phi_relu1_x8(x);
+                        if (mapped) x = phi_x8(x, phi);
                     } else {
                         x = make_uint4(0, 0, 0, 0);
                     }
@@ -308,9 +308,9 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
 #pragma unroll
                         for (int e = 0; e < 8; ++e) cs[e] += f[e];
                     }
-                    if (!GATHER && relu) {
+                    if (!GATHER && mapped) {
                         uint4* qp = reinterpret_cast<uint4*>(st + bx * CF::BOX + w * 16);
-                        *qp = phi_relu1_x8(*qp);
+                        *qp = phi_x8(*qp, phi);
                     }
                 }
                 if (normalize) {
@@ -389,7 +389,7 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                         const int p = et + 128 * j;
                         const int r = p / (D / 8), col = (p % (D / 8)) * 8;
                         *reinterpret_cast<uint4*>(q + (col / 64) * CF::BOX + sw128_off(r, col % 64)) =
-                            relu ? phi_relu1_x8(w[j]) : w[j];
+                            mapped ? phi_x8(w[j], phi) : w[j];
                     }
                     fence_async_smem();
                     mbar_arrive(bqready + slot);

@@ -15,7 +15,9 @@ What is computed, and where it is stated:
 * feature map ``phi``: relu(x)+1 -- "nx_f32_linear_attention.nx source",
   function ``la_phi`` (a value whose sign bit is set becomes 0, then 1 is
   added); identity -- "trim-transformer 0.1.0", introduction
-  (Attn(Q,K,V) = Q K^T V).
+  (Attn(Q,K,V) = Q K^T V); elu(x)+1 -- "lineartile 1.0.1", "How It Works"
+  (the page names ELU without its parameter; read as the usual alpha = 1:
+  x + 1 for x > 0, exp(x) otherwise).
 * KV summary ``S = sum_j phi(K_j) (x) V_j`` (d_k x d_v, row-major ``S[a, b]``)
   and ``z = sum_j phi(K_j)`` -- nx source, header comment and the
   "accumulate KV-summary" loop.
@@ -55,7 +57,8 @@ import numpy as np
 
 PHI_RELU1 = "relu1"
 PHI_IDENTITY = "identity"
-PHI_KINDS = (PHI_RELU1, PHI_IDENTITY)
+PHI_ELU1 = "elu1"
+PHI_KINDS = (PHI_RELU1, PHI_IDENTITY, PHI_ELU1)
 
 FORM_NONCAUSAL = "noncausal"
 FORM_CAUSAL = "causal"
@@ -78,12 +81,16 @@ def phi(x, kind=PHI_RELU1):
     -0.0 maps to 0 + 1 = 1, like +0.0.
     identity: trim-transformer 0.1.0 introduction, where the attention kernel
     is Q K^T V with no feature map.
+    elu1: lineartile 1.0.1, "How It Works": elu(x) + 1 with alpha = 1, that
+    is x + 1 where x > 0 and exp(x) - 1 + 1 = exp(x) elsewhere.
     """
     x = _f64(x)
     if kind == PHI_RELU1:
         return np.where(np.signbit(x), 0.0, x) + 1.0
     if kind == PHI_IDENTITY:
         return x.copy()
+    if kind == PHI_ELU1:
+        return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
     raise ValueError(f"unknown feature map {kind!r}")
 
 

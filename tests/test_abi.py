@@ -127,3 +127,14 @@ def test_timing_read_validation(lib):
 def test_timing_enable_without_gpu_reports_cuda_error(lib):
     assert lib.la_timing_enable(1) == 5
     assert lib.la_timing_enable(0) == 0
+
+
+def test_causal_prefill_validation(lib):
+    """la_causal_prefill: the causal checks plus non-NULL, aligned S_out and
+    z_out (nothing is launched)."""
+    dsc = desc()
+    NULL = None
+    assert lib.la_causal_prefill(ctypes.byref(dsc), 64, P16, P16, P16, P16, NULL, P16, P16, 1 << 30, NULL) == 1
+    assert lib.la_causal_prefill(ctypes.byref(dsc), 64, P16, P16, P16, P16, P16, NULL, P16, 1 << 30, NULL) == 1
+    assert lib.la_causal_prefill(ctypes.byref(dsc), 64, P16, P16, P16, P16, P_MIS, P16, P16, 1 << 30, NULL) == 3
+    assert lib.la_causal_prefill(ctypes.byref(dsc), 96, P16, P16, P16, P16, P16, P16, P16, 1 << 30, NULL) == 2

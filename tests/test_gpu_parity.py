@@ -26,7 +26,7 @@ def _built():
 
 
 def _modes():
-    return [("relu1", True), ("relu1", False), ("identity", False)]
+    return [("relu1", True), ("relu1", False), ("identity", False), ("elu1", True)]
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
@@ -43,8 +43,17 @@ def test_noncausal(dt, d, N, phi, normalize):
     ref = oracle.batched(oracle.noncausal, Q, K, V, phi_kind=phi, normalize=normalize)
     assert oracle.max_row_rel_err(f64(out), ref) < TOL[DT[dt]]
     S_ref, z_ref = oracle.kv_summary_batched(K, V, phi)
-    assert oracle.max_row_rel_err(f64(S), S_ref) < 1e-5
-    assert oracle.max_row_rel_err(f64(z)[..., None, :], z_ref[..., None, :]) < 1e-5
+    assert oracle.max_row_rel_err(f64(S), S_ref) < _state_tol(dt, phi)
+    assert oracle.max_row_rel_err(f64(z)[..., None, :], z_ref[..., None, :]) < _state_tol(dt, phi)
+
+
+def _state_tol(dt, phi):
+    """Tolerance on a KV summary. relu+1 and the identity are exact in bf16
+    (relu(K) and K are bf16 values; the +1 is added exactly in fp32), so S
+    and z carry only fp32 accumulation error. elu+1 has no such split: the
+    bf16 path multiplies phi(K) rounded to bf16, and its state is held to the
+    bf16 tolerance of the outputs."""
+    return TOL[DT[dt]] if (phi == "elu1" and dt == "bf16") else 1e-5
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
@@ -235,3 +244,30 @@ def test_balanced_split_ranges_cross_heads(d, B, H, N):
     ref = np.einsum("bhna,bhac->bhnc", oracle.phi(Q), S_ref) / \
         np.einsum("bhna,bha->bhn", oracle.phi(Q), z_ref)[..., None]
     assert oracle.max_row_rel_err(f64(out), ref) < 2e-2
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("phi", ["relu1", "elu1"])
+def test_causal_prefill_then_decode(dt, d, phi):
+    """la_causal_prefill: the causal outputs (bit for bit those of
+    la_causal_chunked) and the state after the last token, from which decode
+    steps continue the sequence as the oracle's causal recurrence does."""
+    B, H, N0, T = 2, 3, 1100, 12
+    q, k, v = qkv(B, H, N0 + T, d, dt, seed=40 + d)
+    pre = lambda x: x[:, :, :N0].contiguous()
+    out, S, z = la.la_causal_prefill(pre(q), pre(k), pre(v), phi=phi)
+    assert torch.equal(out, la.la_causal_chunked(pre(q), pre(k), pre(v), phi=phi))
+    Q, K, V = f64(q), f64(k), f64(v)
+    S_ref, z_ref = oracle.kv_summary_batched(K[:, :, :N0], V[:, :, :N0], phi)
+    assert oracle.max_row_rel_err(f64(S), S_ref) < _state_tol(dt, phi)
+    assert oracle.max_row_rel_err(f64(z)[..., None, :], z_ref[..., None, :]) < _state_tol(dt, phi)
+    steps = []
+    for t in range(N0, N0 + T):
+        sl = lambda x: x[:, :, t:t + 1].contiguous()
+        steps.append(la.la_decode_step(sl(q), sl(k), sl(v), S, z, phi=phi))
+    got = torch.cat(steps, dim=2)
+    ref = oracle.batched(oracle.causal, Q, K, V, phi_kind=phi)[:, :, N0:]
+    assert oracle.max_row_rel_err(f64(got), ref) < TOL[DT[dt]]
+    ref_pre = oracle.batched(oracle.causal, Q[:, :, :N0], K[:, :, :N0], V[:, :, :N0], phi_kind=phi)
+    assert oracle.max_row_rel_err(f64(out), ref_pre) < TOL[DT[dt]]

@@ -30,6 +30,20 @@ def test_phi_relu1_sign_bit():
     np.testing.assert_array_equal(got, [1.0, 1.0, 1.0, 3.5, 1.0, 1.0 + 1e-30])
 
 
+def test_phi_elu1_matches_torch_elu():
+    """lineartile's map elu(x) + 1 (alpha = 1), against torch's own elu in
+    float64: x + 1 above zero, exp(x) at and below zero (so -0.0 and +0.0 map
+    to 1), strictly positive everywhere."""
+    import torch
+    x = np.array([-30.0, -3.5, -1.0, -1e-3, -0.0, 0.0, 1e-3, 0.5, 1.0, 7.25])
+    want = torch.nn.functional.elu(torch.tensor(x, dtype=torch.float64), alpha=1.0).numpy() + 1.0
+    got = la.phi(x, la.PHI_ELU1)
+    # torch forms expm1(x) + 1, which cancels far below zero: an absolute
+    # tolerance there (a wrong map misses by orders of magnitude more)
+    np.testing.assert_allclose(got, want, rtol=1e-15, atol=1e-16)
+    assert got[4] == 1.0 and got[5] == 1.0 and np.all(got > 0)
+
+
 def test_phi_identity_is_identity():
     x = np.array([-2.0, -0.0, 0.0, 3.25])
     np.testing.assert_array_equal(la.phi(x, la.PHI_IDENTITY), x)
