@@ -1,0 +1,85 @@
+"""Plain fp64 CPU oracle for the gradients of kernelized linear attention.
+
+TEST INFRASTRUCTURE, like the rest of ``oracle/``: only the tests,
+``__graft_entry__.smoke()`` and the CPU legs of ``bench.py`` may use it.
+
+The pages list a backward pass ("lineartile 1.0.1", "Project Structure":
+``core/kernels/backward.py`` and the ``test_backward`` suite) without giving
+its formulas. It is the derivative of the forward definition, written out
+here from that definition and nothing else:
+
+    a_i = phi(q_i), b_j = phi(k_j), w_ij = a_i . b_j for visible j (else 0),
+    num_i = sum_j w_ij v_j, den_i = sum_j w_ij, out_i = num_i / den_i
+    (out_i = num_i when unnormalized).
+
+With g_i = dL/dout_i:
+
+    dnum_i = g_i / den_i,   dden_i = -(g_i . out_i) / den_i     (normalized)
+    dnum_i = g_i,           dden_i = 0                          (unnormalized)
+    dw_ij  = dnum_i . v_j + dden_i          for visible j, else 0
+    dV     = W^T dnum
+    da_i   = sum_j dw_ij b_j,   db_j = sum_i dw_ij a_i
+    dQ = phi'(Q) * dA,  dK = phi'(K) * dB   (elementwise)
+
+phi' is 1 where x > 0 and 0 elsewhere for relu+1 (the derivative of relu is
+taken as 0 at 0, the usual convention), 1 for the identity, and 1 where
+x > 0, exp(x) elsewhere for elu+1. Everything is O(N^2 d) and float64; it is
+pinned by tests against finite differences of the forward definition and
+against torch's automatic differentiation of the same definition.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .linear_attention import (FORM_NONCAUSAL, PHI_ELU1, PHI_IDENTITY, PHI_RELU1, phi,
+                               visible)
+
+
+def phi_grad(x, kind=PHI_RELU1):
+    """d phi / dx, elementwise (see the module docstring for the value at 0)."""
+    x = np.asarray(x, dtype=np.float64)
+    if kind == PHI_RELU1:
+        return np.where(x > 0, 1.0, 0.0)
+    if kind == PHI_IDENTITY:
+        return np.ones_like(x)
+    if kind == PHI_ELU1:
+        return np.where(x > 0, 1.0, np.exp(np.minimum(x, 0.0)))
+    raise ValueError(f"unknown feature map {kind!r}")
+
+
+def backward_dense(Q, K, V, dO, form=FORM_NONCAUSAL, m=None, phi_kind=PHI_RELU1,
+                   normalize=True):
+    """(dQ, dK, dV) of one head by the definition above."""
+    Q, K, V, dO = (np.asarray(t, dtype=np.float64) for t in (Q, K, V, dO))
+    n = Q.shape[0]
+    A, Bk = phi(Q, phi_kind), phi(K, phi_kind)
+    W = np.where(visible(n, form, m), A @ Bk.T, 0.0)
+    num = W @ V
+    if normalize:
+        den = W.sum(axis=1)
+        out = num / den[:, None]
+        dnum = dO / den[:, None]
+        dden = -(dO * out).sum(axis=1) / den
+    else:
+        dnum = dO
+        dden = np.zeros(n)
+    dW = np.where(visible(n, form, m), dnum @ V.T + dden[:, None], 0.0)
+    dV = W.T @ dnum
+    dA = dW @ Bk
+    dB = dW.T @ A
+    return phi_grad(Q, phi_kind) * dA, phi_grad(K, phi_kind) * dB, dV
+
+
+def backward_batched(Q, K, V, dO, form=FORM_NONCAUSAL, m=None, **kw):
+    """backward_dense over every (b, h) of [B, H, N, d] arrays; m is [B, N]
+    (one mask per sequence) or None. Returns (dQ, dK, dV) as [B, H, N, d]."""
+    Q, K, V, dO = (np.asarray(t, dtype=np.float64) for t in (Q, K, V, dO))
+    out = [np.empty_like(Q), np.empty_like(K), np.empty_like(V)]
+    for b in range(Q.shape[0]):
+        for h in range(Q.shape[1]):
+            res = backward_dense(Q[b, h], K[b, h], V[b, h], dO[b, h], form,
+                                 None if m is None else m[b], **kw)
+            for o, r in zip(out, res):
+                o[b, h] = r
+    return tuple(out)
