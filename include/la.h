@@ -85,7 +85,9 @@ typedef enum {
     LA_OP_NONCAUSAL = 1,
     LA_OP_CAUSAL = 2,
     LA_OP_PREFIX = 3,
-    LA_OP_DECODE = 4
+    LA_OP_DECODE = 4,
+    LA_OP_NONCAUSAL_BWD = 5,  /* la_noncausal_backward */
+    LA_OP_CAUSAL_BWD = 6      /* la_causal_backward */
 } la_op;
 
 /* Problem description. d is both d_k and d_v. */
@@ -97,7 +99,7 @@ typedef struct {
 } la_desc;
 
 /* Bytes of workspace `op` needs for `desc` (chunk is used by LA_OP_CAUSAL and
- * LA_OP_PREFIX only). Returns 0 when the request is invalid or unsupported,
+ * LA_OP_PREFIX only; it must be 64 or 128 for those and is ignored otherwise). Returns 0 when the request is invalid or unsupported,
  * and for ops that need none (LA_OP_DECODE). A valid request that needs a
  * workspace always gets a non-zero size. Pure host function. */
 LA_API size_t la_workspace_size(const la_desc* desc, int32_t op, int32_t chunk);
@@ -141,6 +143,33 @@ LA_API la_status la_causal_chunked(const la_desc* desc, int32_t chunk, const voi
 LA_API la_status la_causal_prefill(const la_desc* desc, int32_t chunk, const void* q,
                                    const void* k, const void* v, void* out, float* S_out,
                                    float* z_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Gradients of the non-causal and causal forms (the training path; the
+ * pages list a backward pass, lineartile 1.0.1 "Project Structure":
+ * core/kernels/backward.py, without its formulas, so these are the
+ * derivatives of the forward definition above). Given dout = dL/dout
+ * ([B,H,N,d], input dtype), writes dq, dk, dv ([B,H,N,d], input dtype,
+ * overwritten) for the same desc (phi and normalize) and q, k, v as the
+ * forward call. With a = phi(q), b = phi(k), g = dout:
+ *   gn_i = g_i / den_i, gden_i = -(g_i . out_i) / den_i   (normalize = 1;
+ *   else gn_i = g_i, gden_i = 0)
+ *   dq_i = phi'(q_i) * (S_i gn_i + z_i gden_i)
+ *   dk_j = phi'(k_j) * (G_j v_j + h_j),  dv_j = G_j^T b_j
+ * where S_i, z_i are the state of the keys query i sees and G_j =
+ * sum a_i gn_i^T, h_j = sum a_i gden_i over the queries that see key j
+ * (non-causal: every query; causal: i >= j). phi' is 1 for x > 0 and 0
+ * otherwise for relu+1 (relu's derivative taken as 0 at 0), 1 for the
+ * identity, 1 for x > 0 and exp(x) otherwise for elu+1. Products and sums
+ * are fp32. Workspace: op LA_OP_NONCAUSAL_BWD / LA_OP_CAUSAL_BWD (it holds,
+ * among others, gn and gden in fp32: (d + 1) * 4 bytes per token and head).
+ * Errors as for the forward calls (NULL or misaligned dout, dq, dk, dv
+ * included). */
+LA_API la_status la_noncausal_backward(const la_desc* desc, const void* q, const void* k,
+                                       const void* v, const void* dout, void* dq, void* dk,
+                                       void* dv, void* ws, size_t ws_bytes, void* stream);
+LA_API la_status la_causal_backward(const la_desc* desc, const void* q, const void* k,
+                                    const void* v, const void* dout, void* dq, void* dk,
+                                    void* dv, void* ws, size_t ws_bytes, void* stream);
 
 /* Prefix-mask attention (trim-transformer 0.1.0, "Masking"): query i of
  * sequence b sees keys 0..m[b*N + i], inclusive. m: int32 [B, N] device

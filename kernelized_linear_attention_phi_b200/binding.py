@@ -27,7 +27,8 @@ STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED",
                 6: "LA_ERR_MASK_RANGE", 7: "LA_ERR_TIMEOUT"}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 PHIS = {"relu1": 0, "identity": 1, "elu1": 2}
-OPS = {"kv_summary": 0, "noncausal": 1, "causal": 2, "prefix": 3, "decode": 4}
+OPS = {"kv_summary": 0, "noncausal": 1, "causal": 2, "prefix": 3, "decode": 4, "noncausal_bwd": 5,
+       "causal_bwd": 6}
 
 
 class LaError(RuntimeError):
@@ -54,6 +55,10 @@ _SIGS = {
                                          _P, ctypes.c_size_t, _P]),
     "la_causal_prefill": (ctypes.c_int, [ctypes.POINTER(la_desc), ctypes.c_int32, _P, _P, _P, _P, _P, _P,
                                          _P, ctypes.c_size_t, _P]),
+    "la_noncausal_backward": (ctypes.c_int, [ctypes.POINTER(la_desc), _P, _P, _P, _P, _P, _P, _P, _P,
+                                             ctypes.c_size_t, _P]),
+    "la_causal_backward": (ctypes.c_int, [ctypes.POINTER(la_desc), _P, _P, _P, _P, _P, _P, _P, _P,
+                                          ctypes.c_size_t, _P]),
     "la_prefix_mask": (ctypes.c_int, [ctypes.POINTER(la_desc), ctypes.c_int32, _P, _P, _P, _P, _P,
                                       _P, ctypes.c_size_t, _P]),
     "la_decode_step": (ctypes.c_int, [ctypes.POINTER(la_desc), _P, _P, _P, _P, _P, _P, _P]),
@@ -284,3 +289,30 @@ def la_timing_read(capacity=16):
     n = ctypes.c_int32(0)
     _check("la_timing_read", lib().la_timing_read(buf, capacity, ctypes.byref(n)))
     return [float(buf[i]) for i in range(min(n.value, capacity))]
+
+
+def _backward(name, op, q, k, v, dout, dq, dk, dv, phi, normalize, ws, stream):
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _same(q, k, v, dout, dq, dk, dv)
+    desc = _desc_of(q, phi, normalize)
+    if ws is None:
+        ws = workspace(desc, op, 64, device=q.device)
+    _check(name, getattr(lib(), name)(
+        ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+        ws.numel(), _stream(q, stream)))
+    return dq, dk, dv
+
+
+def la_noncausal_backward(q, k, v, dout, dq=None, dk=None, dv=None, phi="relu1", normalize=True, ws=None,
+                          stream=None):
+    """Gradients (dq, dk, dv) of non-causal attention for upstream dout."""
+    return _backward("la_noncausal_backward", "noncausal_bwd", q, k, v, dout, dq, dk, dv, phi, normalize, ws,
+                     stream)
+
+
+def la_causal_backward(q, k, v, dout, dq=None, dk=None, dv=None, phi="relu1", normalize=True, ws=None,
+                       stream=None):
+    """Gradients (dq, dk, dv) of causal attention for upstream dout."""
+    return _backward("la_causal_backward", "causal_bwd", q, k, v, dout, dq, dk, dv, phi, normalize, ws, stream)

@@ -28,6 +28,13 @@ __device__ __forceinline__ float phi_elu1(float x) { return x > 0.0f ? x + 1.0f 
 __device__ __forceinline__ float phi_apply(float x, int phi) {
     return phi == PHI_RELU1 ? phi_relu1(x) : phi == PHI_ELU1 ? phi_elu1(x) : x;
 }
+// d phi / dx: relu1 1 for x > 0, else 0 (relu's derivative taken as 0 at 0);
+// elu1 1 for x > 0, else exp(x); identity 1.
+__device__ __forceinline__ float phi_grad(float x, int phi) {
+    if (phi == PHI_RELU1) return x > 0.0f ? 1.0f : 0.0f;
+    if (phi == PHI_ELU1) return x > 0.0f ? 1.0f : expf(x);
+    return 1.0f;
+}
 
 // 16-byte vector <-> floats.
 template <typename T> struct Vec16;

@@ -35,9 +35,10 @@ cudaError_t simt_kv_partial(const Problem& p, const void* k, const void* v, int 
 cudaError_t state_reduce(const Problem& p, const float* part, int nsplit, float* S, float* z,
                          cudaStream_t st);
 // In place: record b of each head becomes the sum of records 0..b-1 (zero for
-// b = 0). If S_total/z_total are non-null they receive the sum of all records.
+// b = 0), or with `reverse` of records b+1..nblk-1. If S_total/z_total are
+// non-null they receive the sum of all records.
 cudaError_t state_exclusive_scan(const Problem& p, float* part, int nblk, float* S_total,
-                                 float* z_total, cudaStream_t st);
+                                 float* z_total, cudaStream_t st, bool reverse = false);
 // out = phi(q) S / (phi(q).z) (or numerator only) for every token.
 cudaError_t simt_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,
                          cudaStream_t st);
@@ -59,6 +60,24 @@ cudaError_t simt_chunked(const Problem& p, const void* q, const void* k, const v
 // clamped mask.
 cudaError_t bin_queries(const Problem& p, const int32_t* m, int chunk, int nbins, int32_t* perm,
                         int32_t* bin_start, int32_t* mclamped, uint32_t* flags, cudaStream_t st);
+
+// ---- gradients (bwd.cu) -------------------------------------------------------
+// Chunk length of the gradient kernels (block_tokens must be a multiple).
+int bwd_chunk(const Problem& p);
+// Forward sweep: per block of block_tokens tokens (causal: its state is the
+// exclusive prefix (S, z) at index bh*nblk + blk; non-causal: the head totals
+// at index bh; S at S + index*s_stride, z at z + index*z_stride), writes dq,
+// gn [bh][N][d] and gden [bh][N] (fp32) and the block's own (G, h) record
+// grec[(bh*nblk + blk)] (d*d + d floats).
+cudaError_t bwd_q(const Problem& p, bool causal, const void* q, const void* k, const void* v, const void* dout,
+                  const float* S, const float* z, long long s_stride, long long z_stride, int block_tokens,
+                  int nblk, void* dq, float* gn, float* gden, float* grec, cudaStream_t st);
+// Reverse sweep: per block, from (G, h) of all later queries (causal: suffix
+// state at index bh*nblk + blk; non-causal: totals at index bh), writes dk
+// and dv.
+cudaError_t bwd_kv(const Problem& p, bool causal, const void* q, const void* k, const void* v, const float* gn,
+                   const float* gden, const float* G, const float* h, long long g_stride, long long h_stride,
+                   int block_tokens, int nblk, void* dk, void* dv, cudaStream_t st);
 
 // ---- decode (decode.cu) -------------------------------------------------------
 cudaError_t decode_step(const Problem& p, const void* q, const void* k, const void* v, float* S,

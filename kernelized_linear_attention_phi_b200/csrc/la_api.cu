@@ -102,6 +102,7 @@ int prefix_nbins(const Problem& p, int kchunk) { return p.N / kchunk + 1; }
 
 struct WsLayout {
     size_t part = 0, sz = 0, perm = 0, mcl = 0, bins = 0, total = 0;
+    size_t grec = 0, gtot = 0, gn = 0, gden = 0;  // gradients
 };
 
 WsLayout ws_layout(const Problem& p, int op) {
@@ -135,6 +136,26 @@ WsLayout ws_layout(const Problem& p, int op) {
             L.bins = off;
             off = round_up(off + sizeof(int32_t) * (size_t)p.B * (nbins + 1), kAlign);
         }
+    } else if (op == LA_OP_NONCAUSAL_BWD || op == LA_OP_CAUSAL_BWD) {
+        const BlockPlan bp = block_plan(p);
+        L.part = off;
+        if (op == LA_OP_NONCAUSAL_BWD) {
+            // the KV summary's own scratch where kv_summary_impl expects it,
+            // then the totals (S, z) and (G, h)
+            off = ws_layout(p, LA_OP_KV_SUMMARY).total;
+            L.sz = off;
+            off = round_up(off + (size_t)p.bh() * rec, kAlign);
+            L.gtot = off;
+            off = round_up(off + (size_t)p.bh() * rec, kAlign);
+        } else {
+            off = round_up(off + (size_t)p.bh() * bp.nblk * rec, kAlign);  // block states (S, z)
+        }
+        L.grec = off;
+        off = round_up(off + (size_t)p.bh() * bp.nblk * rec, kAlign);      // block states (G, h)
+        L.gn = off;
+        off = round_up(off + sizeof(float) * (size_t)p.bh() * p.N * p.d, kAlign);
+        L.gden = off;
+        off = round_up(off + sizeof(float) * (size_t)p.bh() * p.N, kAlign);
     } else {
         return L;
     }
@@ -214,7 +235,7 @@ const char* la_status_string(la_status s) {
 size_t la_workspace_size(const la_desc* desc, int32_t op, int32_t chunk) {
     if (check_desc(desc) != LA_OK) return 0;
     if ((op == LA_OP_CAUSAL || op == LA_OP_PREFIX) && check_chunk(chunk) != LA_OK) return 0;
-    if (op < LA_OP_KV_SUMMARY || op > LA_OP_DECODE) return 0;
+    if (op < LA_OP_KV_SUMMARY || op > LA_OP_CAUSAL_BWD) return 0;
     return ws_layout(to_problem(desc), op).total;
 }
 
@@ -286,10 +307,71 @@ la_status causal_impl(const la_desc* desc, int32_t chunk, const void* q, const v
                                     nullptr, 0, out, st));
 }
 
+// Gradients of the non-causal or causal form (see la.h): states of the
+// forward, a forward sweep for dq, gn, gden and per-block (G, h), the
+// suffix (causal) or total (non-causal) of (G, h), a reverse sweep for dk, dv.
+la_status backward_impl(const la_desc* desc, bool causal, const void* q, const void* k, const void* v,
+                        const void* dout, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                        cudaStream_t st) {
+    LA_TRY(check_desc(desc));
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return LA_ERR_INVALID_ARG;
+    for (const void* ptr : {q, k, v, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                            static_cast<const void*>(dv)})
+        if (!aligned16(ptr)) return LA_ERR_MISALIGNED;
+    const Problem p = to_problem(desc);
+    const WsLayout L = ws_layout(p, causal ? LA_OP_CAUSAL_BWD : LA_OP_NONCAUSAL_BWD);
+    LA_TRY(check_ws(L, ws, ws_bytes));
+    LA_TRY(check_device());
+    timing_begin(st);
+    const BlockPlan bp = block_plan(p);
+    if (bp.block_tokens % bwd_chunk(p) != 0) return LA_ERR_UNSUPPORTED;
+    const long long rec = (long long)p.state_floats();
+    float* grec = at<float>(ws, L.grec);
+    float* gn = at<float>(ws, L.gn);
+    float* gden = at<float>(ws, L.gden);
+    if (causal) {
+        float* part = at<float>(ws, L.part);
+        uint32_t* flags = at<uint32_t>(ws, 0);
+        if (tc_supported(p)) {
+            LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
+        } else {
+            LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
+        }
+        LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
+        LA_TRY(cuda_status(bwd_q(p, true, q, k, v, dout, part, part + (size_t)p.d * p.d, rec, rec,
+                                 bp.block_tokens, bp.nblk, dq, gn, gden, grec, st)));
+        LA_TRY(cuda_status(state_exclusive_scan(p, grec, bp.nblk, nullptr, nullptr, st, true)));
+        return cuda_status(bwd_kv(p, true, q, k, v, gn, gden, grec, grec + (size_t)p.d * p.d, rec, rec,
+                                  bp.block_tokens, bp.nblk, dk, dv, st));
+    }
+    float* S = at<float>(ws, L.sz);
+    float* z = S + (size_t)p.bh() * p.d * p.d;
+    float* G = at<float>(ws, L.gtot);
+    float* h = G + (size_t)p.bh() * p.d * p.d;
+    LA_TRY(kv_summary_impl(p, k, v, S, z, ws, st));
+    LA_TRY(cuda_status(bwd_q(p, false, q, k, v, dout, S, z, (long long)p.d * p.d, p.d, bp.block_tokens,
+                             bp.nblk, dq, gn, gden, grec, st)));
+    LA_TRY(cuda_status(state_reduce(p, grec, bp.nblk, G, h, st)));
+    return cuda_status(bwd_kv(p, false, q, k, v, gn, gden, G, h, (long long)p.d * p.d, p.d, bp.block_tokens,
+                              bp.nblk, dk, dv, st));
+}
+
 }  // namespace
 }  // namespace la
 
 extern "C" {
+
+la_status la_noncausal_backward(const la_desc* desc, const void* q, const void* k, const void* v,
+                                const void* dout, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                                void* stream) {
+    return backward_impl(desc, false, q, k, v, dout, dq, dk, dv, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+la_status la_causal_backward(const la_desc* desc, const void* q, const void* k, const void* v,
+                             const void* dout, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                             void* stream) {
+    return backward_impl(desc, true, q, k, v, dout, dq, dk, dv, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
 
 la_status la_causal_chunked(const la_desc* desc, int32_t chunk, const void* q, const void* k,
                             const void* v, void* out, void* ws, size_t ws_bytes, void* stream) {

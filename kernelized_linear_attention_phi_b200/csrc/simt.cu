@@ -115,8 +115,9 @@ __global__ void state_reduce_kernel(const float* __restrict__ part, int nsplit, 
 
 // One thread per float4 of a record; loads are issued eight blocks at a time
 // so that several are in flight, the running sum stays in registers.
+// With `reverse` the blocks are taken last to first (suffix sums).
 __global__ void state_scan_kernel(float* __restrict__ part, int nblk, int D,
-                                  float* __restrict__ S_total, float* __restrict__ z_total) {
+                                  float* __restrict__ S_total, float* __restrict__ z_total, int reverse) {
     const int rec4 = (D * D + D) / 4;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     const long long bh = blockIdx.y;
@@ -130,11 +131,11 @@ __global__ void state_scan_kernel(float* __restrict__ part, int nblk, int D,
         float4 v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-            if (b0 + j < nblk) v[j] = p[(size_t)(b0 + j) * rec4];
+            if (b0 + j < nblk) v[j] = p[(size_t)(reverse ? nblk - 1 - (b0 + j) : b0 + j) * rec4];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             if (b0 + j < nblk) {
-                p[(size_t)(b0 + j) * rec4] = run;
+                p[(size_t)(reverse ? nblk - 1 - (b0 + j) : b0 + j) * rec4] = run;
                 run.x += v[j].x;
                 run.y += v[j].y;
                 run.z += v[j].z;
@@ -511,10 +512,11 @@ cudaError_t state_reduce(const Problem& p, const float* part, int nsplit, float*
 }
 
 cudaError_t state_exclusive_scan(const Problem& p, float* part, int nblk, float* S_total,
-                                 float* z_total, cudaStream_t st) {
+                                 float* z_total, cudaStream_t st, bool reverse) {
     const int rec4 = (p.d * p.d + p.d) / 4;
     dim3 grid((rec4 + 127) / 128, (unsigned)p.bh());
-    return launch_pdl(state_scan_kernel, grid, dim3(128), 0, st, part, nblk, p.d, S_total, z_total);
+    return launch_pdl(state_scan_kernel, grid, dim3(128), 0, st, part, nblk, p.d, S_total, z_total,
+                      reverse ? 1 : 0);
 }
 
 }  // namespace la

@@ -7,5 +7,5 @@ a GPU (tests/test_oracle_pins.py); no function here is "parity unpinned".
 """
 
 from .linear_attention import *  # noqa: F401,F403
-from .metrics import max_row_rel_err  # noqa: F401
+from .metrics import max_row_grad_err, max_row_rel_err  # noqa: F401
 from .backward import backward_batched, backward_dense, phi_grad  # noqa: F401

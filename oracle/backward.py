@@ -49,8 +49,12 @@ def phi_grad(x, kind=PHI_RELU1):
 
 
 def backward_dense(Q, K, V, dO, form=FORM_NONCAUSAL, m=None, phi_kind=PHI_RELU1,
-                   normalize=True):
-    """(dQ, dK, dV) of one head by the definition above."""
+                   normalize=True, scales=False):
+    """(dQ, dK, dV) of one head by the definition above. With scales=True
+    also (tq, tk, tv): per row, the sum of the norms of the terms that make up
+    that row of dQ (phi' times sum_j dnum_i.v_j b_j and times dden_i sum_j
+    b_j), of dK (the same two with the roles of queries and keys swapped) and
+    of dV (sum_i |w_ij| ||dnum_i||), the size of what rounding acts on."""
     Q, K, V, dO = (np.asarray(t, dtype=np.float64) for t in (Q, K, V, dO))
     n = Q.shape[0]
     A, Bk = phi(Q, phi_kind), phi(K, phi_kind)
@@ -68,14 +72,27 @@ def backward_dense(Q, K, V, dO, form=FORM_NONCAUSAL, m=None, phi_kind=PHI_RELU1,
     dV = W.T @ dnum
     dA = dW @ Bk
     dB = dW.T @ A
-    return phi_grad(Q, phi_kind) * dA, phi_grad(K, phi_kind) * dB, dV
+    grads = (phi_grad(Q, phi_kind) * dA, phi_grad(K, phi_kind) * dB, dV)
+    if not scales:
+        return grads
+    vis = visible(n, form, m)
+    dnv = np.where(vis, dnum @ V.T, 0.0)   # dnum_i . v_j on visible entries
+    dd = np.where(vis, dden[:, None], 0.0)
+    pq, pk = phi_grad(Q, phi_kind), phi_grad(K, phi_kind)
+    tq = np.linalg.norm(pq * (dnv @ Bk), axis=1) + np.linalg.norm(pq * (dd @ Bk), axis=1)
+    tk = np.linalg.norm(pk * (dnv.T @ A), axis=1) + np.linalg.norm(pk * (dd.T @ A), axis=1)
+    tv = np.abs(W).T @ np.linalg.norm(dnum, axis=1)
+    return grads + (tq, tk, tv)
 
 
 def backward_batched(Q, K, V, dO, form=FORM_NONCAUSAL, m=None, **kw):
     """backward_dense over every (b, h) of [B, H, N, d] arrays; m is [B, N]
-    (one mask per sequence) or None. Returns (dQ, dK, dV) as [B, H, N, d]."""
+    (one mask per sequence) or None. Returns (dQ, dK, dV) as [B, H, N, d]
+    (and with scales=True the per-row scales as [B, H, N])."""
     Q, K, V, dO = (np.asarray(t, dtype=np.float64) for t in (Q, K, V, dO))
     out = [np.empty_like(Q), np.empty_like(K), np.empty_like(V)]
+    if kw.get("scales"):
+        out += [np.empty(Q.shape[:3]) for _ in range(3)]
     for b in range(Q.shape[0]):
         for h in range(Q.shape[1]):
             res = backward_dense(Q[b, h], K[b, h], V[b, h], dO[b, h], form,

@@ -138,3 +138,19 @@ def test_causal_prefill_validation(lib):
     assert lib.la_causal_prefill(ctypes.byref(dsc), 64, P16, P16, P16, P16, P16, NULL, P16, 1 << 30, NULL) == 1
     assert lib.la_causal_prefill(ctypes.byref(dsc), 64, P16, P16, P16, P16, P_MIS, P16, P16, 1 << 30, NULL) == 3
     assert lib.la_causal_prefill(ctypes.byref(dsc), 96, P16, P16, P16, P16, P16, P16, P16, 1 << 30, NULL) == 2
+
+
+def test_backward_validation(lib):
+    """Gradient entry points: the forward checks plus non-NULL, aligned dout,
+    dq, dk, dv; their workspace ops have a size, an unknown op has none."""
+    dsc = desc()
+    NULL = None
+    for fn in (lib.la_noncausal_backward, lib.la_causal_backward):
+        assert fn(ctypes.byref(dsc), P16, P16, P16, NULL, P16, P16, P16, P16, 1 << 30, NULL) == 1
+        assert fn(ctypes.byref(dsc), P16, P16, P16, P16, P16, P16, NULL, P16, 1 << 30, NULL) == 1
+        assert fn(ctypes.byref(dsc), P16, P16, P16, P16, P_MIS, P16, P16, P16, 1 << 30, NULL) == 3
+        assert fn(ctypes.byref(desc(d=8)), P16, P16, P16, P16, P16, P16, P16, P16, 1 << 30, NULL) == 2
+        assert fn(ctypes.byref(dsc), P16, P16, P16, P16, P16, P16, P16, P16, 16, NULL) == 4
+    assert B.la_workspace_size(dsc, "noncausal_bwd") > 0
+    assert B.la_workspace_size(dsc, "causal_bwd") > 0
+    assert lib.la_workspace_size(ctypes.byref(dsc), 7, 64) == 0

@@ -1,0 +1,84 @@
+"""Gradients on the GPU (la_noncausal_backward, la_causal_backward) against
+the fp64 gradient oracle, which differentiates the forward definition
+(oracle/backward.py, pinned by finite differences and autograd)."""
+
+import pytest
+import torch
+
+import oracle
+from kernelized_linear_attention_phi_b200 import binding as la
+
+from gpu_util import DT, TOL, f64, qkv
+
+pytestmark = pytest.mark.gpu
+
+MODES = [("relu1", True), ("relu1", False), ("identity", False), ("elu1", True)]
+FN = {"noncausal": la.la_noncausal_backward, "causal": la.la_causal_backward}
+
+
+def _case(form, dt, d, N, phi, normalize, B=1, H=2, seed=0):
+    sigma = 1.0 if phi != "identity" else d ** -0.5
+    q, k, v = qkv(B, H, N, d, dt, seed=seed, sigma=sigma)
+    g = torch.Generator(device="cpu").manual_seed(seed + 1000)
+    dout = torch.randn(B, H, N, d, generator=g).to(device="cuda", dtype=q.dtype)
+    dq, dk, dv = FN[form](q, k, v, dout, phi=phi, normalize=normalize)
+    ref = oracle.backward_batched(f64(q), f64(k), f64(v), f64(dout), form, phi_kind=phi, normalize=normalize,
+                                  scales=True)
+    return (dq, dk, dv), ref
+
+
+@pytest.mark.parametrize("form", ["noncausal", "causal"])
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [16, 32, 64, 128])
+@pytest.mark.parametrize("N", [2, 100, 700])
+@pytest.mark.parametrize("phi,normalize", MODES)
+def test_gradients_match_oracle(form, dt, d, N, phi, normalize):
+    got, ref = _case(form, dt, d, N, phi, normalize, seed=N + d)
+    for name, gt, rf, sc in zip(("dq", "dk", "dv"), got, ref[:3], ref[3:]):
+        err = oracle.max_row_grad_err(f64(gt), rf, sc)
+        assert err < TOL[DT[dt]], (name, err)
+
+
+@pytest.mark.parametrize("form", ["noncausal", "causal"])
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("phi", ["relu1", "elu1"])
+def test_single_token_normalized(form, dt, phi):
+    """One key: the normalized output is v whatever q and k are, so dq and dk
+    vanish (the kernels form them as differences of ordinary-size terms and
+    return rounding noise) and dv equals dout."""
+    q, k, v = qkv(2, 3, 1, 64, dt, seed=3)
+    dout = torch.randn_like(q)
+    dq, dk, dv = FN[form](q, k, v, dout, phi=phi)
+    assert float(dq.abs().max()) < 1e-5 and float(dk.abs().max()) < 1e-5
+    assert oracle.max_row_rel_err(f64(dv), f64(dout)) < TOL[DT[dt]]
+
+
+def test_gradients_several_heads_and_sequences():
+    got, ref = _case("causal", "bf16", 64, 1500, "relu1", True, B=2, H=3, seed=5)
+    for gt, rf, sc in zip(got, ref[:3], ref[3:]):
+        assert oracle.max_row_grad_err(f64(gt), rf, sc) < TOL[torch.bfloat16]
+
+
+def test_gradients_are_deterministic():
+    q, k, v = qkv(1, 2, 900, 64, "bf16", seed=8)
+    dout = torch.randn_like(q)
+    for fn in FN.values():
+        a, b = fn(q, k, v, dout), fn(q, k, v, dout)
+        for x, y in zip(a, b):
+            assert torch.equal(x, y)
+
+
+def test_causal_gradient_of_last_row_touches_every_key():
+    """A loss on the last output row only: every key and value of the head
+    gets a gradient (the last query sees them all), and dq is zero except in
+    that row."""
+    B, H, N, d = 1, 1, 300, 32
+    q, k, v = qkv(B, H, N, d, "f32", seed=9)
+    dout = torch.zeros_like(q)
+    dout[0, 0, -1] = 1.0
+    dq, dk, dv = la.la_causal_backward(q, k, v, dout)
+    assert torch.count_nonzero(dq[0, 0, :-1]) == 0
+    assert bool((dv[0, 0].abs().sum(dim=1) > 0).all())
+    ref = oracle.backward_batched(f64(q), f64(k), f64(v), f64(dout), "causal", scales=True)
+    for gt, rf, sc in zip((dq, dk, dv), ref[:3], ref[3:]):
+        assert oracle.max_row_grad_err(f64(gt), rf, sc) < TOL[torch.float32]

@@ -100,3 +100,21 @@ def test_finite_difference_pin_catches_a_dropped_denominator_term():
     got = bw.backward_dense(Q, K, V, G, la.FORM_CAUSAL, None, la.PHI_RELU1, normalize=False)
     want = _fd_grads(Q, K, V, G, la.FORM_CAUSAL, None, la.PHI_RELU1, True)
     assert any(not np.allclose(g, w, rtol=1e-6, atol=1e-7) for g, w in zip(got, want))
+
+
+def test_gradient_metric_and_scales():
+    """max_row_grad_err judges a row against the larger of its own norm and
+    its term scale; the oracle's scale of a structurally zero row (one visible
+    key, normalized) is the size of its two cancelling terms, which are
+    equal."""
+    from oracle.metrics import max_row_grad_err
+    ref = np.array([[3.0, 4.0], [0.0, 0.0]])
+    got = ref + np.array([[0.05, 0.0], [0.0, 0.01]])
+    assert abs(max_row_grad_err(got, ref, [5.0, 0.02]) - 0.5) < 1e-12  # row 1: 0.01 / 0.02
+    assert abs(max_row_grad_err(got, ref, [5.0, 2.0]) - 0.01) < 1e-12  # row 0: 0.05 / 5
+    Q, K, V, G, _ = _inputs(4, 3, 11, la.PHI_RELU1)
+    dq, dk, dv, tq, tk, tv = bw.backward_dense(Q, K, V, G, la.FORM_CAUSAL, scales=True)
+    assert np.linalg.norm(dq[0]) < 1e-12 < tq[0]        # row 0 sees one key
+    assert np.all(tq >= np.linalg.norm(dq, axis=1) - 1e-12)
+    assert np.all(tk >= np.linalg.norm(dk, axis=1) - 1e-12)
+    assert np.all(tv >= np.linalg.norm(dv, axis=1) - 1e-12)
