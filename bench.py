@@ -55,6 +55,9 @@ CALL_KERNELS = {
     "causal": ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"],
     "prefix": ["bin_kernel", "tc_kv_kernel", "state_scan_kernel", "tc_sweep"],
     "decode": ["decode_kernel"],
+    "noncausal_bwd": ["tc_kv_kernel", "kv_reduce_balanced_kernel", "bwd_q_kernel", "state_reduce_kernel",
+                      "bwd_kv_kernel"],
+    "causal_bwd": ["tc_kv_kernel", "state_scan_kernel", "bwd_q_kernel", "state_scan_kernel", "bwd_kv_kernel"],
 }
 # The same on the fp32 (CUDA-core) path.
 CALL_KERNELS_F32 = {
@@ -62,13 +65,17 @@ CALL_KERNELS_F32 = {
     "causal": ["kv_partial_kernel", "state_scan_kernel", "chunked_kernel"],
     "prefix": ["bin_kernel", "kv_partial_kernel", "state_scan_kernel", "chunked_kernel"],
     "decode": ["decode_kernel"],
+    "noncausal_bwd": ["kv_partial_kernel", "state_reduce_kernel", "bwd_q_kernel", "state_reduce_kernel",
+                      "bwd_kv_kernel"],
+    "causal_bwd": ["kv_partial_kernel", "state_scan_kernel", "bwd_q_kernel", "state_scan_kernel", "bwd_kv_kernel"],
 }
 LAUNCHES = {k: len(v) for k, v in CALL_KERNELS.items()}
 # What each kernel does, for its algorithmic bytes (Step.kernel_bytes).
 KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balanced_kernel": "reduce",
                "state_reduce_kernel": "reduce", "tc_readout_kernel": "readout", "readout_kernel": "readout",
                "state_scan_kernel": "scan", "tc_sweep": "sweep", "chunked_kernel": "sweep",
-               "bin_kernel": "bin", "decode_kernel": "decode"}
+               "bin_kernel": "bin", "decode_kernel": "decode", "bwd_q_kernel": "bwd_q",
+               "bwd_kv_kernel": "bwd_kv"}
 
 
 def parse():
@@ -173,10 +180,14 @@ class Step:
         self.out_c = torch.empty_like(self.q)
         self.out_m = torch.empty_like(self.q)
         self.out_d = torch.empty_like(self.q1)
+        if any(f.endswith("_bwd") for f in forms):
+            self.dout = W.upstream_grad(B, H, N, d, seed, dtype, device)
+            self.grads = {f: tuple(torch.empty_like(self.q) for _ in range(3)) for f in forms}
         self.S = torch.empty(B, H, d, d, dtype=torch.float32, device=device)
         self.z = torch.empty(B, H, d, dtype=torch.float32, device=device)
         desc = la._desc_of(self.q, self.phi, self.normalize)
-        self.ws = {op: la.workspace(desc, op, self.chunk, device) for op in ("noncausal", "causal", "prefix")}
+        self.ws = {op: la.workspace(desc, op, self.chunk, device)
+                   for op in ("noncausal", "causal", "prefix") + tuple(f for f in forms if f.endswith("_bwd"))}
         self.tokens = sum(B if f == "decode" else B * N for f in forms)
         self.elem = self.q.element_size()
         if "decode" in forms and "noncausal" not in forms:
@@ -194,6 +205,12 @@ class Step:
                                                 self.phi, self.normalize, self.ws["prefix"]),
             "decode": lambda: la.la_decode_step(self.q1, self.k1, self.v1, self.S, self.z, self.out_d,
                                                 self.phi, self.normalize),
+            "noncausal_bwd": lambda: la.la_noncausal_backward(self.q, self.k, self.v, self.dout,
+                                                              *self.grads["noncausal_bwd"], self.phi,
+                                                              self.normalize, self.ws["noncausal_bwd"]),
+            "causal_bwd": lambda: la.la_causal_backward(self.q, self.k, self.v, self.dout,
+                                                        *self.grads["causal_bwd"], self.phi, self.normalize,
+                                                        self.ws["causal_bwd"]),
         }
         return [(f, table[f]) for f in self.forms]
 
@@ -203,7 +220,7 @@ class Step:
         st = self.B * self.H * (self.d * self.d + self.d) * 4  # fp32 (S, z)
         one = self.B * self.H * self.d * self.elem
         return {"noncausal": 4 * t + st, "causal": 4 * t, "prefix": 4 * t + self.B * self.N * 4,
-                "decode": 2 * st + 4 * one}
+                "decode": 2 * st + 4 * one, "noncausal_bwd": 7 * t, "causal_bwd": 7 * t}
 
     def kernel_bytes(self, call, kernel):
         """Algorithmic bytes of one kernel of a call: the method's tensors it
@@ -215,15 +232,29 @@ class Step:
         st = self.B * self.H * (self.d * self.d + self.d) * 4
         one = self.B * self.H * self.d * self.elem
         role = KERNEL_ROLE.get(kernel)
+        if call.endswith("_bwd"):
+            # gradients: q, k, v, dout read and dq, dk, dv written once over
+            # the sweeps (non-causal: q, dout -> dq; k, v -> dk, dv; causal:
+            # q, k, v, dout -> dq; q, k, v -> dk, dv); the reductions of
+            # (G, h) move scratch only
+            causal = call == "causal_bwd"
+            return {"kv": 2 * t, "bwd_q": (5 if causal else 3) * t,
+                    "bwd_kv": (5 if causal else 4) * t}.get(role, 0)
         return {"kv": 2 * t, "reduce": st, "readout": 2 * t + st, "scan": 0, "sweep": 4 * t,
                 "bin": self.B * self.N * 4, "decode": 2 * st + 4 * one}.get(role, 0)
 
     def host_io(self):
         full = [f for f in self.forms if f != "decode"]
+        bwd = [f for f in self.forms if f.endswith("_bwd")]
         ins = ([self.q, self.k, self.v] if full else []) + ([self.m] if "prefix" in self.forms else []) \
-            + ([self.q1, self.k1, self.v1] if "decode" in self.forms else [])
-        outs = [{"noncausal": self.out_nc, "causal": self.out_c, "prefix": self.out_m,
-                 "decode": self.out_d}[f] for f in self.forms]
+            + ([self.q1, self.k1, self.v1] if "decode" in self.forms else []) + ([self.dout] if bwd else [])
+        outs = []
+        for f in self.forms:
+            if f.endswith("_bwd"):
+                outs += list(self.grads[f])
+            else:
+                outs.append({"noncausal": self.out_nc, "causal": self.out_c, "prefix": self.out_m,
+                             "decode": self.out_d}[f])
         return ins, outs
 
 
@@ -421,7 +452,9 @@ def run_ours(args, rank, world, local_rank):
                                f"normalize={int(wl.normalize)} chunk={wl.chunk}; step = "
                                + " + ".join({"noncausal": "noncausal", "causal": "causal",
                                              "prefix": "prefix mask (m uniform)",
-                                             "decode": "1 decode step"}[f] for f in forms),
+                                             "decode": "1 decode step",
+                                             "noncausal_bwd": "noncausal gradients",
+                                             "causal_bwd": "causal gradients"}[f] for f in forms),
                    "global_batch": wl.B * world, "seq_len": wl.N, "parallelism": f"dp{world}",
                    "l2": "flushed between steps (256 MiB write)", "launch": "one CUDA graph per call",
                    "tokens_per_step_per_gpu": step.tokens},
@@ -500,7 +533,7 @@ def _blas_threads():
         return 1
 
 
-def oracle_sample(q, k, v, m, q1, k1, v1, phi, normalize, heads, forms):
+def oracle_sample(q, k, v, m, q1, k1, v1, phi, normalize, heads, forms, dout=None):
     """Runs the oracle's forms on the first `heads` heads of sequence 0.
     Returns (seconds, tokens processed), tokens counted like the GPU step
     (B*N per full-sequence form, B per decode step) scaled by heads/H."""
@@ -510,6 +543,7 @@ def oracle_sample(q, k, v, m, q1, k1, v1, phi, normalize, heads, forms):
     Q, K, V = f(q[0, :heads]), f(k[0, :heads]), f(v[0, :heads])
     M = m[0].cpu().numpy()
     q1_, k1_, v1_ = f(q1[0, :heads, 0]), f(k1[0, :heads, 0]), f(v1[0, :heads, 0])
+    G = f(dout[0, :heads]) if dout is not None else None
     N = Q.shape[1]
     t0 = time.perf_counter()
     for h in range(heads):
@@ -524,6 +558,9 @@ def oracle_sample(q, k, v, m, q1, k1, v1, phi, normalize, heads, forms):
             if S is None:
                 S, z = oracle.kv_summary(K[h], V[h], phi)
             oracle.decode_step(S, z, q1_[h], k1_[h], v1_[h], phi, normalize)
+        for fm in ("noncausal_bwd", "causal_bwd"):
+            if fm in forms:
+                oracle.backward_dense(Q[h], K[h], V[h], G[h], fm[:-4], None, phi, normalize)
     dt = time.perf_counter() - t0
     per_seq = sum(1 if fm == "decode" else N for fm in forms)
     return dt, per_seq * heads / H
@@ -535,7 +572,7 @@ def cpu_baseline(step, heads=2, min_seconds=10.0):
     total_t, total_tok, passes = 0.0, 0.0, 0
     while total_t < min_seconds:
         dt, tok = oracle_sample(step.q, step.k, step.v, step.m, step.q1, step.k1, step.v1,
-                                step.phi, step.normalize, heads, step.forms)
+                                step.phi, step.normalize, heads, step.forms, getattr(step, "dout", None))
         total_t += dt
         total_tok += tok
         passes += 1
@@ -554,12 +591,13 @@ def run_reference(args, rank, world):
     q, k, v = W.qkv(1, wl.H, wl.N, wl.d, wl.sigma, wl.seed, dtype, "cpu")
     m = W.prefix_mask_uniform(1, wl.N, wl.seed, "cpu")
     q1, k1, v1 = (t[0] for t in W.decode_tokens(1, 1, wl.H, wl.d, wl.sigma, wl.seed, dtype, "cpu"))
+    dout = W.upstream_grad(1, wl.H, wl.N, wl.d, wl.seed, dtype, "cpu")
     heads = 1
     for _ in range(args.warmup):
-        oracle_sample(q, k, v, m, q1, k1, v1, wl.phi, wl.normalize, heads, forms)
+        oracle_sample(q, k, v, m, q1, k1, v1, wl.phi, wl.normalize, heads, forms, dout)
     total, tokens = 0.0, 0.0
     for _ in range(args.steps):
-        dt, tok = oracle_sample(q, k, v, m, q1, k1, v1, wl.phi, wl.normalize, heads, forms)
+        dt, tok = oracle_sample(q, k, v, m, q1, k1, v1, wl.phi, wl.normalize, heads, forms, dout)
         total += dt
         tokens += tok
     value = tokens / total

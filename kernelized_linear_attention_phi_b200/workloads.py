@@ -37,7 +37,8 @@ class Workload:
     dtypes: tuple
     phi: str            # "relu1" or "identity"
     normalize: bool
-    forms: tuple        # subset of ("noncausal", "causal", "prefix", "decode")
+    forms: tuple        # subset of ("noncausal", "causal", "prefix", "decode",
+                        # "noncausal_bwd", "causal_bwd")
     sigma: float        # standard deviation of Q, K, V entries
     seed: int
     chunk: int = 64
@@ -58,6 +59,10 @@ WORKLOADS = {
                             ("causal",), 1.0, 5, chunk=128),
     "decode": Workload("decode", 64, 32, 2048, 128, ("bf16",), "relu1", True,
                        ("decode",), 1.0, 6, decode_steps=1024),
+    # the gradients of the multi-head forms, for an upstream gradient
+    # dout ~ N(0, 1) (upstream_grad)
+    "multi_head_bwd": Workload("multi_head_bwd", 2, 8, 4096, 64, ("bf16", "f32"), "relu1", True,
+                               ("noncausal_bwd", "causal_bwd"), 1.0, 2, chunk=64),
 }
 
 TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -99,3 +104,9 @@ def decode_tokens(steps, B, H, d, sigma=1.0, seed=0, dtype="bf16", device="cpu")
     """q, k, v for ``steps`` one-token steps: three [steps, B, H, 1, d] tensors."""
     return tuple(normal((steps, B, H, 1, d), sigma, 20_000 + 3 * seed + i, dtype, device)
                  for i in range(3))
+
+
+def upstream_grad(B, H, N, d, seed, dtype="bf16", device="cpu"):
+    """dL/dout for the gradient workloads: N(0, 1) entries, generator seed
+    30000 + seed."""
+    return normal((B, H, N, d), 1.0, 30_000 + seed, dtype, device)
