@@ -53,7 +53,7 @@ L2_FLUSH_BYTES = 256 << 20
 CALL_KERNELS = {
     "noncausal": ["tc_kv_kernel", "kv_reduce_balanced_kernel", "tc_readout_kernel"],
     "causal": ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"],
-    "prefix": ["bin_kernel", "tc_kv_kernel", "state_scan_kernel", "tc_sweep"],
+    "prefix": ["tc_kv_kernel", "bin_kernel", "state_scan_kernel", "tc_sweep"],
     "decode": ["decode_kernel"],
     "noncausal_bwd": ["tc_kv_kernel", "kv_reduce_balanced_kernel", "bwd_q_kernel", "state_reduce_kernel",
                       "bwd_kv_kernel"],
@@ -63,7 +63,7 @@ CALL_KERNELS = {
 CALL_KERNELS_F32 = {
     "noncausal": ["kv_partial_kernel", "state_reduce_kernel", "readout_kernel"],
     "causal": ["kv_partial_kernel", "state_scan_kernel", "chunked_kernel"],
-    "prefix": ["bin_kernel", "kv_partial_kernel", "state_scan_kernel", "chunked_kernel"],
+    "prefix": ["kv_partial_kernel", "bin_kernel", "state_scan_kernel", "chunked_kernel"],
     "decode": ["decode_kernel"],
     "noncausal_bwd": ["kv_partial_kernel", "state_reduce_kernel", "bwd_q_kernel", "state_reduce_kernel",
                       "bwd_kv_kernel"],

@@ -18,7 +18,10 @@ bin_kernel(const int32_t* __restrict__ m, int N, int chunk, int nbins, int32_t* 
            int32_t* __restrict__ bin_start, int32_t* __restrict__ mcl, uint32_t* __restrict__ flags) {
     extern __shared__ int32_t cnt[];  // nbins + 1
     __shared__ int32_t warp_tot[kBinThreads / 32];
-    pdl_wait();
+    // Reads only the caller's mask and writes tables that no kernel of the
+    // call reads before the block-state scan, which waits for this kernel:
+    // launched after the KV pass, it runs beside it without waiting.
+    pdl_launch_dependents();
     const int b = blockIdx.x;
     const int32_t* mb = m + (size_t)b * N;
     for (int c = threadIdx.x; c <= nbins; c += kBinThreads) cnt[c] = 0;

@@ -96,6 +96,14 @@ __device__ __forceinline__ void pdl_wait() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// For a kernel (or a warp) that reads nothing the previous kernel of the
+// call writes: lets dependents launch without waiting. Memory written by
+// kernels that completed before the previous kernel started waiting is
+// visible all the same, which covers the caller's inputs of a library call
+// (its first kernel waits for them).
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // Streaming 16-byte global load (read once: do not keep in L1).
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {

@@ -411,12 +411,14 @@ la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, cons
     int32_t* mcl = at<int32_t>(ws, L.mcl);
     int32_t* bins = at<int32_t>(ws, L.bins);
     float* part = at<float>(ws, L.part);
-    LA_TRY(cuda_status(bin_queries(p, m, kchunk, nbins, perm, bins, mcl, flags, st)));
+    // the binning reads only m: launched after the KV pass it runs beside it
+    // (bin_kernel does not wait for its predecessor); the scan waits for it
     if (tc) {
         LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
     } else {
         LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
     }
+    LA_TRY(cuda_status(bin_queries(p, m, kchunk, nbins, perm, bins, mcl, flags, st)));
     LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
     if (tc)
         return cuda_status(tc_chunked(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, perm, bins,

@@ -448,7 +448,10 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    pdl_wait();
+    // The TMA producer (warp 0) loads only the caller's Q, so it does not wait
+    // for the previous kernel (the reduction of S, z) and fills the pipeline
+    // while that kernel finishes; every other warp waits before it reads S, z.
+    if (warp != 0) pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {

@@ -153,7 +153,11 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    pdl_wait();
+    // The TMA producer (warp 0) loads only the caller's inputs, so it does
+    // not wait for the previous kernel of the call and fills the pipeline
+    // while that kernel finishes; every other warp waits before it reads
+    // what that kernel wrote.
+    if (warp != 0) pdl_wait();
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
