@@ -70,23 +70,50 @@ __device__ void load_state(const float* __restrict__ M, const float* __restrict_
     for (int e = threadIdx.x; e < D; e += kThreads) sv[e] = vec[e];
 }
 
-// Masked C x C product out[i][j] = (A_i . B_j) (+ add_i) for visible (i, j),
-// else 0; visible is j <= i (lower) or j >= i (upper).
+// Masked C x C product out[i][j] = (A_i . B_j) (+ add) for visible (i, j),
+// else 0; visible is j <= i (lower, add = add[i]) or j >= i (upper,
+// add = add[j]). Register-tiled: thread (ti, tj) = (tid / 16, tid % 16)
+// owns rows ti + 16 r and columns tj + 16 c and reads both operands as float4
+// along d (rows interleaved so that neighbouring lanes read rows LD floats
+// apart: LD / 4 = D / 4 + 1 is odd, so their 16-byte reads fall in distinct
+// bank groups).
 template <int D, bool LOWER>
 __device__ void chunk_products(const float* sA_, const float* sB_, const float* add, float* sOut) {
     using CF = BwCfg<D>;
-    for (int idx = threadIdx.x; idx < CF::C * CF::C; idx += kThreads) {
-        const int i = idx / CF::C, j = idx % CF::C;
-        float p = 0.f;
-        if (LOWER ? j <= i : j >= i) {
-            const float* x = sA_ + i * CF::LD;
-            const float* y = sB_ + j * CF::LD;
-#pragma unroll 8
-            for (int a = 0; a < D; ++a) p = fmaf(x[a], y[a], p);
-            if (add) p += add[LOWER ? i : j];
-        }
-        sOut[i * CF::LDP + j] = p;
+    constexpr int C = CF::C, LD = CF::LD, RB = C / 16;
+    static_assert((LD / 4) % 2 == 1, "odd row stride in 16-byte units");
+    const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
+    float acc[RB][RB];
+#pragma unroll
+    for (int r = 0; r < RB; ++r)
+#pragma unroll
+        for (int c = 0; c < RB; ++c) acc[r][c] = 0.f;
+#pragma unroll 4
+    for (int a = 0; a < D; a += 4) {
+        float4 x[RB], y[RB];
+#pragma unroll
+        for (int r = 0; r < RB; ++r) x[r] = *reinterpret_cast<const float4*>(sA_ + (ti + 16 * r) * LD + a);
+#pragma unroll
+        for (int c = 0; c < RB; ++c) y[c] = *reinterpret_cast<const float4*>(sB_ + (tj + 16 * c) * LD + a);
+#pragma unroll
+        for (int r = 0; r < RB; ++r)
+#pragma unroll
+            for (int c = 0; c < RB; ++c) {
+                acc[r][c] = fmaf(x[r].x, y[c].x, acc[r][c]);
+                acc[r][c] = fmaf(x[r].y, y[c].y, acc[r][c]);
+                acc[r][c] = fmaf(x[r].z, y[c].z, acc[r][c]);
+                acc[r][c] = fmaf(x[r].w, y[c].w, acc[r][c]);
+            }
     }
+#pragma unroll
+    for (int r = 0; r < RB; ++r)
+#pragma unroll
+        for (int c = 0; c < RB; ++c) {
+            const int i = ti + 16 * r, j = tj + 16 * c;
+            float p = 0.f;
+            if (LOWER ? j <= i : j >= i) p = acc[r][c] + (add ? add[LOWER ? i : j] : 0.f);
+            sOut[i * CF::LDP + j] = p;
+        }
 }
 
 // ---------------------------------------------------------------------------
