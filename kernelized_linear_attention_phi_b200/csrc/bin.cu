@@ -15,12 +15,13 @@ constexpr int kBinThreads = 1024;
 // One CTA per sequence: clamp, histogram, exclusive scan, scatter.
 __global__ void __launch_bounds__(kBinThreads)
 bin_kernel(const int32_t* __restrict__ m, int N, int chunk, int nbins, int32_t* __restrict__ perm,
-           int32_t* __restrict__ bin_start, int32_t* __restrict__ mcl, uint32_t* __restrict__ flags) {
+           int32_t* __restrict__ bin_start, int32_t* __restrict__ msort, uint32_t* __restrict__ flags) {
     extern __shared__ int32_t cnt[];  // nbins + 1
     __shared__ int32_t warp_tot[kBinThreads / 32];
     // Reads only the caller's mask and writes tables that no kernel of the
     // call reads before the block-state scan, which waits for this kernel:
-    // launched after the KV pass, it runs beside it without waiting.
+    // launched after the KV pass, it runs beside it and waits for it only at
+    // its end (below).
     pdl_launch_dependents();
     const int b = blockIdx.x;
     const int32_t* mb = m + (size_t)b * N;
@@ -33,7 +34,6 @@ bin_kernel(const int32_t* __restrict__ m, int N, int chunk, int nbins, int32_t* 
             bad = true;
             mi = mi < 0 ? 0 : N - 1;
         }
-        mcl[(size_t)b * N + i] = mi;
         atomicAdd(&cnt[(mi + 1) / chunk], 1);
     }
     if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(flags, FLAG_MASK_RANGE);
@@ -73,21 +73,25 @@ bin_kernel(const int32_t* __restrict__ m, int N, int chunk, int nbins, int32_t* 
     }
     __syncthreads();
     for (int i = threadIdx.x; i < N; i += kBinThreads) {
-        const int32_t mi = mcl[(size_t)b * N + i];
+        const int32_t mi = min(max(mb[i], 0), N - 1);
         const int pos = atomicAdd(&cnt[(mi + 1) / chunk], 1);
         perm[(size_t)b * N + pos] = i;
+        msort[(size_t)b * N + pos] = mi;
     }
+    // This grid does not complete before the KV pass it runs beside: a
+    // kernel that waits for this one then finds both complete.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace
 
 cudaError_t bin_queries(const Problem& p, const int32_t* m, int chunk, int nbins, int32_t* perm,
-                        int32_t* bin_start, int32_t* mclamped, uint32_t* flags, cudaStream_t st) {
+                        int32_t* bin_start, int32_t* msort, uint32_t* flags, cudaStream_t st) {
     const size_t smem = sizeof(int32_t) * (size_t)(nbins + 1);
     cudaError_t e = ensure_smem<bin_kernel>(smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(bin_kernel, dim3(p.B), dim3(kBinThreads), smem, st, m, p.N, chunk, nbins, perm,
-                      bin_start, mclamped, flags);
+                      bin_start, msort, flags);
 }
 
 }  // namespace la

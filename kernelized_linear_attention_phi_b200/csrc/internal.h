@@ -46,20 +46,21 @@ cudaError_t simt_readout(const Problem& p, const void* q, const float* S, const 
 // [blk*block_tokens, ...) and starts from record blk of `prefix` (the state of
 // all earlier keys). With perm == nullptr the queries of chunk c are the
 // tokens of chunk c (causal); otherwise the queries answered at chunk c are
-// perm[b*N + bin_start[b*(nbins+1) + c] ...] with key limits m.
+// perm[b*N + bin_start[b*(nbins+1) + c] ...] with key limits msort at the
+// same positions (bin_queries).
 cudaError_t simt_chunked(const Problem& p, const void* q, const void* k, const void* v,
                          const float* prefix, int block_tokens, int nblk, const int32_t* perm,
-                         const int32_t* bin_start, const int32_t* m, int nbins, void* out,
+                         const int32_t* bin_start, const int32_t* msort, int nbins, void* out,
                          cudaStream_t st);
 
 // ---- prefix-mask binning (bin.cu) -------------------------------------------
 // For each sequence b: clamp m into [0, N-1] (setting FLAG_MASK_RANGE in
 // *flags when it had to), bin query i by floor((m_i + 1) / chunk) and write a
 // counting-sort permutation perm[b*N ...] plus bin offsets
-// bin_start[b*(nbins+1) ...] (nbins = N / chunk + 1). mclamped receives the
-// clamped mask.
+// bin_start[b*(nbins+1) ...] (nbins = N / chunk + 1); msort[b*N + pos] is
+// the clamped m of query perm[b*N + pos] (the mask in sorted order).
 cudaError_t bin_queries(const Problem& p, const int32_t* m, int chunk, int nbins, int32_t* perm,
-                        int32_t* bin_start, int32_t* mclamped, uint32_t* flags, cudaStream_t st);
+                        int32_t* bin_start, int32_t* msort, uint32_t* flags, cudaStream_t st);
 
 // ---- gradients (bwd.cu) -------------------------------------------------------
 // Chunk length of the gradient kernels (block_tokens must be a multiple).

@@ -101,7 +101,7 @@ BlockPlan block_plan(const Problem& p) {
 int prefix_nbins(const Problem& p, int kchunk) { return p.N / kchunk + 1; }
 
 struct WsLayout {
-    size_t part = 0, sz = 0, perm = 0, mcl = 0, bins = 0, total = 0;
+    size_t part = 0, sz = 0, perm = 0, msort = 0, bins = 0, total = 0;
     size_t grec = 0, gtot = 0, gn = 0, gden = 0;  // gradients
 };
 
@@ -131,7 +131,7 @@ WsLayout ws_layout(const Problem& p, int op) {
             const int nbins = prefix_nbins(p, 64);  // the most bins any kernel uses
             L.perm = off;
             off = round_up(off + sizeof(int32_t) * (size_t)p.B * p.N, kAlign);
-            L.mcl = off;
+            L.msort = off;
             off = round_up(off + sizeof(int32_t) * (size_t)p.B * p.N, kAlign);
             L.bins = off;
             off = round_up(off + sizeof(int32_t) * (size_t)p.B * (nbins + 1), kAlign);
@@ -408,22 +408,23 @@ la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, cons
     const int nbins = prefix_nbins(p, kchunk);
     uint32_t* flags = at<uint32_t>(ws, 0);
     int32_t* perm = at<int32_t>(ws, L.perm);
-    int32_t* mcl = at<int32_t>(ws, L.mcl);
+    int32_t* msort = at<int32_t>(ws, L.msort);
     int32_t* bins = at<int32_t>(ws, L.bins);
     float* part = at<float>(ws, L.part);
     // the binning reads only m: launched after the KV pass it runs beside it
-    // (bin_kernel does not wait for its predecessor); the scan waits for it
+    // (bin_kernel waits for its predecessor only at its end); the scan waits
+    // for both
     if (tc) {
         LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
     } else {
         LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
     }
-    LA_TRY(cuda_status(bin_queries(p, m, kchunk, nbins, perm, bins, mcl, flags, st)));
+    LA_TRY(cuda_status(bin_queries(p, m, kchunk, nbins, perm, bins, msort, flags, st)));
     LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
     if (tc)
         return cuda_status(tc_chunked(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, perm, bins,
-                                      mcl, nbins, out, flags, st));
-    return cuda_status(simt_chunked(p, q, k, v, part, bp.block_tokens, bp.nblk, perm, bins, mcl,
+                                      msort, nbins, out, flags, st));
+    return cuda_status(simt_chunked(p, q, k, v, part, bp.block_tokens, bp.nblk, perm, bins, msort,
                                     nbins, out, st));
 }
 

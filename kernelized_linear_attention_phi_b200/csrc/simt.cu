@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kThreads)
 chunked_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V,
                const float* __restrict__ prefix, int H, int N, int block_tokens, int nblk,
                const int32_t* __restrict__ perm, const int32_t* __restrict__ bin_start,
-               const int32_t* __restrict__ m, int nbins, int phi, int normalize,
+               const int32_t* __restrict__ msort, int nbins, int phi, int normalize,
                T* __restrict__ out) {
     constexpr int LD = D + 4, LDP = kC + 4;
     constexpr int R = D / 16;               // state-update block per thread (R x R)
@@ -294,9 +294,8 @@ chunked_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __rest
                 const int r = threadIdx.x;
                 if (r < nq) {
                     if (GATHER) {
-                        const int i = perm[(size_t)b * N + qt + r];
-                        sRow[r] = i;
-                        sLim[r] = m[(size_t)b * N + i] - c * kC;  // in [-1, kvalid-1]
+                        sRow[r] = perm[(size_t)b * N + qt + r];
+                        sLim[r] = msort[(size_t)b * N + qt + r] - c * kC;  // in [-1, kvalid-1]
                     } else {
                         sRow[r] = c * kC + r;
                         sLim[r] = r;

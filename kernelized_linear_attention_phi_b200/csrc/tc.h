@@ -40,19 +40,22 @@ cudaError_t tc_readout(const Problem& p, const void* q, const float* S, const fl
 // (d = 128 always runs 64-token chunks: the shared-memory budget).
 int tc_chunk(const Problem& p, int chunk);
 // Same contract as simt_chunked, at chunk length tc_chunk(p, chunk); the
-// prefix-mask inputs (perm, bins, mcl, nbins) must be binned at that length.
+// prefix-mask inputs (perm, bins, msort, nbins) must be binned at that length.
 cudaError_t tc_chunked(const Problem& p, int chunk, const void* q, const void* k, const void* v,
                        const float* prefix, int block_tokens, int nblk, const int32_t* perm,
-                       const int32_t* bins, const int32_t* mcl, int nbins, void* out, uint32_t* err,
+                       const int32_t* bins, const int32_t* msort, int nbins, void* out, uint32_t* err,
                        cudaStream_t st);
 
 // The d = 128 kernel behind tc_chunked (64-token chunks, state kept as S^T).
 cudaError_t tc_chunked_t(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
                          int block_tokens, int nblk, const int32_t* perm, const int32_t* bins,
-                         const int32_t* mcl, int nbins, void* out, uint32_t* err, cudaStream_t st);
+                         const int32_t* msort, int nbins, void* out, uint32_t* err, cudaStream_t st);
 
 // [BH, N, d] bf16 viewed as 3-D for TMA: 64-column x `rows` boxes, 128-byte
 // swizzle, zero fill outside the tensor.
 cudaError_t make_map(CUtensorMap* map, const void* base, int d, int N, long long bh, int rows);
+// The same tensor viewed as 2-D [rows = BH * N, d] for row gathers
+// (tile::gather4): 64-column x 1-row boxes, 128-byte swizzle.
+cudaError_t make_row_map(CUtensorMap* map, const void* base, int d, long long rows);
 
 }  // namespace la

@@ -115,6 +115,40 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
+// Row gather (tile::gather4) through a 2-D map whose box is one row high:
+// rows r0..r3, columns c0 .. c0 + box width, land as four consecutive rows
+// of the destination (swizzled by address like any tiled load), completing
+// on `bar`. c0 obeys the tiled-load rule (c0 * element size a multiple of 16).
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int r0,
+                                            int r1, int r2, int r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+// One gathered query tile of C rows x 64*NB columns, issued by a whole warp:
+// lane l holds the token indices of rows (C/32)*l .. (C/32)*l + C/32 - 1 in
+// tok[] (-1 for a padding row, which fetches token 0 instead), and lanes
+// 0 .. NB*C/4 - 1 each issue one gather4 of four rows of one 64-column box.
+// `dst` is the 1024-byte aligned tile, one [C x 64] box after another;
+// `row0` is the map row of token 0 of the head. The caller posts the
+// expected bytes (C * 64 * NB * 2) on `bar` before calling.
+template <int C, int NB>
+__device__ __forceinline__ void gather_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row0,
+                                            const int (&tok)[C / 32], int lane) {
+    constexpr int R = C / 32, G = C / 4;  // rows per lane, gathers per box
+    static_assert(NB * G <= 32, "one gather per lane");
+    const int g = lane % G;
+    int r[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) r[e] = __shfl_sync(0xffffffffu, tok[e % R], (4 * g + e) / R);
+    if (lane < NB * G) {
+        const int bx = lane / G;
+        tma_gather4(dst + bx * (C * 128) + g * 512, map, bar, bx * 64, row0 + max(r[0], 0), row0 + max(r[1], 0),
+                    row0 + max(r[2], 0), row0 + max(r[3], 0));
+    }
+}
 // 3-D tiled store from shared memory (bulk group). Parts of the box outside
 // the tensor are not written.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
@@ -305,9 +339,15 @@ __device__ __forceinline__ uint4 phi_elu1_x8(uint4 w) {
     for (int e = 0; e < 8; ++e) f[e] = f[e] > 0.0f ? f[e] + 1.0f : __expf(f[e]);
     return pack8(f);
 }
-// A feature map other than the identity on eight packed bf16 values.
-__device__ __forceinline__ uint4 phi_x8(uint4 w, int phi) {
-    return phi == PHI_ELU1 ? phi_elu1_x8(w) : phi_relu1_x8(w);
+// The feature map PHI on eight packed bf16 values. The map is a template
+// parameter of every tensor-core kernel: with a run-time choice both bodies
+// sit inline at every (unrolled) call site, and the larger code ran the d =
+// 128 sweep at two thirds of the speed of a single-map build.
+template <int PHI>
+__device__ __forceinline__ uint4 phi8(uint4 w) {
+    if constexpr (PHI == PHI_ELU1) return phi_elu1_x8(w);
+    else if constexpr (PHI == PHI_RELU1) return phi_relu1_x8(w);
+    else return w;
 }
 // relu on eight packed bf16 values (exact).
 __device__ __forceinline__ uint4 relu_x8(uint4 w) {

@@ -118,10 +118,10 @@ struct KvCfg {
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-template <int D>
+template <int D, int PHI>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV, int N,
-             KvWork w, int phi, float* __restrict__ part, uint32_t* __restrict__ err) {
+             KvWork w, float* __restrict__ part, uint32_t* __restrict__ err) {
     using C = KvCfg<D>;
     constexpr size_t REC = (size_t)D * D + D;
     extern __shared__ uint8_t smem_raw[];
@@ -136,8 +136,8 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int nseg = kv_nseg(w);
-    const bool relu = phi == PHI_RELU1;
-    const bool elu = phi == PHI_ELU1;
+    constexpr bool relu = PHI == PHI_RELU1;
+    constexpr bool elu = PHI == PHI_ELU1;
 
     if (threadIdx.x == 0) {
         cta_abort_reset();
@@ -396,11 +396,11 @@ struct RoCfg {
     static_assert(SMEM * PER_SM <= 227 * 1024, "shared memory");
 };
 
-template <int D>
+template <int D, int PHI>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mOut,
                   const float* __restrict__ S, const float* __restrict__ z, int N, long long total,
-                  int tph, int phi, int normalize, uint32_t* __restrict__ err) {
+                  int tph, int normalize, uint32_t* __restrict__ err) {
     using C = RoCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles = align1024(smem_raw);
@@ -531,10 +531,10 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
             }
             const int s = it % C::STAGES, u = it / C::STAGES;
             ok = ok && mbar_wait(full + s, u & 1, err);
-            if (ok && phi != PHI_IDENTITY) {
+            if (ok && PHI != PHI_IDENTITY) {
                 uint4* qt = reinterpret_cast<uint4*>(tiles + s * C::TILE);
 #pragma unroll
-                for (int i = 0; i < C::NB * 8; ++i) qt[et + 128 * i] = phi_x8(qt[et + 128 * i], phi);
+                for (int i = 0; i < C::NB * 8; ++i) qt[et + 128 * i] = phi8<PHI>(qt[et + 128 * i]);
             }
             fence_async_smem();
             mbar_arrive(tdone + s);
@@ -589,6 +589,16 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
     }
 }
 
+template <int D, int PHI>
+cudaError_t launch_kv_phi(const Problem& p, const CUtensorMap& mk, const CUtensorMap& mv, const KvWork& w,
+                          dim3 grid, float* part, uint32_t* err, cudaStream_t st) {
+    constexpr size_t smem = KvCfg<D>::SMEM;
+    cudaError_t e = ensure_smem<tc_kv_kernel<D, PHI>>(smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(tc_kv_kernel<D, PHI>, grid, dim3(kThreads), smem, st, mk, mv, p.N, w, part, err);
+}
+
+// one kernel per feature map (see phi8)
 template <int D>
 cudaError_t launch_kv(const Problem& p, const void* k, const void* v, const KvWork& w, dim3 grid, float* part,
                       uint32_t* err, cudaStream_t st) {
@@ -596,10 +606,24 @@ cudaError_t launch_kv(const Problem& p, const void* k, const void* v, const KvWo
     cudaError_t e = make_map(&mk, k, D, p.N, p.bh(), kTile);
     if (e == cudaSuccess) e = make_map(&mv, v, D, p.N, p.bh(), kTile);
     if (e != cudaSuccess) return e;
-    constexpr size_t smem = KvCfg<D>::SMEM;
-    e = ensure_smem<tc_kv_kernel<D>>(smem);
+    switch (p.phi) {
+        case PHI_RELU1: return launch_kv_phi<D, PHI_RELU1>(p, mk, mv, w, grid, part, err, st);
+        case PHI_ELU1: return launch_kv_phi<D, PHI_ELU1>(p, mk, mv, w, grid, part, err, st);
+        default: return launch_kv_phi<D, PHI_IDENTITY>(p, mk, mv, w, grid, part, err, st);
+    }
+}
+
+template <int D, int PHI>
+cudaError_t launch_readout_phi(const Problem& p, const CUtensorMap& mq, const CUtensorMap& mo, const float* S,
+                               const float* z, uint32_t* err, cudaStream_t st) {
+    constexpr size_t smem = RoCfg<D>::SMEM;
+    cudaError_t e = ensure_smem<tc_readout_kernel<D, PHI>>(smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(tc_kv_kernel<D>, grid, dim3(kThreads), smem, st, mk, mv, p.N, w, p.phi, part, err);
+    const int tph = (p.N + kTile - 1) / kTile;
+    const long long total = p.bh() * tph;
+    const int G = (int)std::min<long long>(total, 148LL * RoCfg<D>::PER_SM);
+    return launch_pdl(tc_readout_kernel<D, PHI>, dim3(G), dim3(kThreads), smem, st, mq, mo, S, z, p.N, total, tph,
+                      p.normalize, err);
 }
 
 template <int D>
@@ -609,14 +633,11 @@ cudaError_t launch_readout(const Problem& p, const void* q, const float* S, cons
     cudaError_t e = make_map(&mq, q, D, p.N, p.bh(), kTile);
     if (e == cudaSuccess) e = make_map(&mo, out, D, p.N, p.bh(), kTile);
     if (e != cudaSuccess) return e;
-    constexpr size_t smem = RoCfg<D>::SMEM;
-    e = ensure_smem<tc_readout_kernel<D>>(smem);
-    if (e != cudaSuccess) return e;
-    const int tph = (p.N + kTile - 1) / kTile;
-    const long long total = p.bh() * tph;
-    const int G = (int)std::min<long long>(total, 148LL * RoCfg<D>::PER_SM);
-    return launch_pdl(tc_readout_kernel<D>, dim3(G), dim3(kThreads), smem, st, mq, mo, S, z, p.N, total, tph,
-                      p.phi, p.normalize, err);
+    switch (p.phi) {  // one kernel per feature map (see phi8)
+        case PHI_RELU1: return launch_readout_phi<D, PHI_RELU1>(p, mq, mo, S, z, err, st);
+        case PHI_ELU1: return launch_readout_phi<D, PHI_ELU1>(p, mq, mo, S, z, err, st);
+        default: return launch_readout_phi<D, PHI_IDENTITY>(p, mq, mo, S, z, err, st);
+    }
 }
 
 }  // namespace

@@ -28,9 +28,11 @@ using namespace tc;
 // Prefix mask: the queries of bin c (floor((m_i+1)/C) = c) are gathered
 // rows, lim_i = m_i - cC in [-1, C-2].
 //
-// Warp roles (320 threads): warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 "prep"
-// (phi on the K / Q tiles, state -> operands, query gather), warps 6-9 "mask"
-// (P~, epilogue). Prep runs one chunk ahead of mask; the S / z operands are
+// Warp roles (320 threads): warp 0 TMA (K / V (/ Q) chunks; for the prefix
+// mask also each tile of gathered query rows, by tile::gather4 through a 2-D
+// row map of Q, and the tile's row table), warp 1 MMA + TMEM, warps 2-5
+// "prep" (phi on the K / Q tiles, state -> operands), warps 6-9 "mask" (P~,
+// epilogue). Prep runs one chunk ahead of mask; the S / z operands are
 // double-buffered, the gathered query tiles too. The per-tile accumulators
 // (P, O, Oz) and the P~ operand are double-buffered by tile parity ("slot"),
 // so the tensor core starts tile t+1 while the mask warps finish tile t: with
@@ -57,7 +59,7 @@ struct SwCfg {
                          COL_OZ = COL_O + SLOTC * D, COL_END = COL_OZ + SLOTC * 16;
     static constexpr uint32_t TMEM_COLS = COL_END <= 256 ? 256u : 512u;
     static_assert(COL_END <= 512, "TMEM");
-    static constexpr int NBAR = 2 * STAGES + 2 + 5 * 2;
+    static constexpr int NBAR = 2 * STAGES + 2 + 6 * 2;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 2 * PT + 2 * B3 + 2 * BZ + ONES + QG +
                                    STG + ROWS + 8 * NBAR + 16;
     // TMEM address offsets of slot j for P, O and Oz
@@ -72,14 +74,13 @@ struct SwCfg {
     static_assert(MIN_BLOCKS == 1 || MIN_BLOCKS * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
-template <int D, int C, bool GATHER>
+template <int D, int C, bool GATHER, int PHI>
 __global__ void __launch_bounds__(SwCfg<D, C, GATHER>::THREADS, SwCfg<D, C, GATHER>::MIN_BLOCKS)
 tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                 const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mOut,
-                const __nv_bfloat16* __restrict__ Qg,
                 const float* __restrict__ prefix, int H, int N, int block_tokens, int nblk,
                 const int32_t* __restrict__ perm, const int32_t* __restrict__ bin_start,
-                const int32_t* __restrict__ mcl, int nbins, int phi, int normalize,
+                const int32_t* __restrict__ msort, int nbins, int normalize,
                 __nv_bfloat16* __restrict__ out, uint32_t* __restrict__ err) {
     using CF = SwCfg<D, C, GATHER>;
     extern __shared__ uint8_t smem_raw[];
@@ -98,13 +99,14 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     // Per-tile barriers are kept per slot (tile t uses slot t % 2, phase t / 2),
     // so that no waiter is ever two phases behind its barrier (parity waits
     // would alias): P ready, P~ written (P read), O ready, O read, queries
-    // gathered.
+    // transformed, and (prefix mask) query rows landed with their row table.
     uint64_t* bpfull = bsdone + 1;     // [2]
     uint64_t* bptready = bpfull + 2;   // [2]
     uint64_t* bofull = bptready + 2;   // [2]
     uint64_t* bofree = bofull + 2;     // [2]
     uint64_t* bqready = bofree + 2;    // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bqready + 2);
+    uint64_t* qfull = bqready + 2;     // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qfull + 2);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int blk = blockIdx.x;
@@ -114,7 +116,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     const int c_begin = blk * (block_tokens / C);
     const int c_end = (GATHER && blk == nblk - 1) ? nbins : min(nchunks, c_begin + block_tokens / C);
     const int nci = c_end - c_begin;
-    const bool mapped = phi != PHI_IDENTITY;  // phi applied to Q and K tiles
+    constexpr bool mapped = PHI != PHI_IDENTITY;  // phi applied to Q and K tiles
     const size_t hoff = (size_t)bh * N * D;
 
     auto q_tiles = [&](int c) -> int {
@@ -137,15 +139,14 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             mbar_init(bofull + j, 1);
             mbar_init(bofree + j, 128);
             mbar_init(bqready + j, 128);
+            mbar_init(qfull + j, 1);
         }
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, CF::TMEM_COLS);
     if (threadIdx.x == 0) {
-        if (!GATHER) {
-            tma_prefetch_map(&mQ);
-            tma_prefetch_map(&mOut);
-        }
+        tma_prefetch_map(&mQ);
+        if (!GATHER) tma_prefetch_map(&mOut);
         tma_prefetch_map(&mK);
         tma_prefetch_map(&mV);
     }
@@ -153,19 +154,16 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // The TMA producer (warp 0) loads only the caller's inputs, so it does
-    // not wait for the previous kernel of the call and fills the pipeline
-    // while that kernel finishes; every other warp waits before it reads
-    // what that kernel wrote.
+    // The TMA producer (warp 0) first loads only the caller's inputs, so it
+    // fills the pipeline without waiting for the previous kernel of the call;
+    // every other warp waits before it reads what that kernel wrote.
     if (warp != 0) pdl_wait();
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
-        if (lane == 0) {
-            int issued[CF::STAGES] = {};
-            for (int ci = 0; ci < nci; ++ci) {
-                const int s = ci % CF::STAGES, u = ci / CF::STAGES;
-                if (u > 0 && !mbar_wait(empty + s, (u - 1) & 1, err)) break;
+        // ---------------- TMA producer (whole warp) ----------------
+        auto load_chunk = [&](int ci) {
+            const int s = ci % CF::STAGES;
+            if (lane == 0) {
                 mbar_arrive_expect_tx(full + s, CF::STAGE);
                 uint8_t* st = stages + s * CF::STAGE;
                 const int row = (c_begin + ci) * C;
@@ -176,10 +174,57 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                     tma_load_3d(st + (t++) * CF::TILE + bx * C * 128, &mK, full + s, bx * 64, row, bh);
                     tma_load_3d(st + t * CF::TILE + bx * C * 128, &mV, full + s, bx * 64, row, bh);
                 }
-                issued[s] = u + 1;
             }
-            for (int s = 0; s < CF::STAGES; ++s)
-                if (issued[s] > 0) mbar_wait(full + s, (issued[s] - 1) & 1, err, false);
+        };
+        int nld = min(nci, CF::STAGES);
+        for (int ci = 0; ci < nld; ++ci) load_chunk(ci);
+        // the bin tables below come from an earlier kernel of the call
+        if (GATHER) pdl_wait();
+        bool ok = true;
+        int tq = 0;
+        for (int ci = 0; ci < nci && ok; ++ci) {
+            if (ci >= CF::STAGES) {
+                const int s = ci % CF::STAGES, u = ci / CF::STAGES;
+                ok = __all_sync(0xffffffffu, mbar_wait(empty + s, (u - 1) & 1, err));
+                if (!ok) break;
+                load_chunk(ci);
+                nld = ci + 1;
+            }
+            if (GATHER) {
+                const int c = c_begin + ci;
+                const int qbase = bin_start[(size_t)b * (nbins + 1) + c];
+                const int qend = bin_start[(size_t)b * (nbins + 1) + c + 1];
+                for (int t = 0; qbase + t * C < qend; ++t, ++tq) {
+                    constexpr int R = C / 32;  // rows of the tile per lane
+                    const int slot = tq & 1;
+                    int tok[R], lim[R];
+#pragma unroll
+                    for (int e = 0; e < R; ++e) {
+                        const int idx = qbase + t * C + R * lane + e;
+                        tok[e] = idx < qend ? perm[(size_t)b * N + idx] : -1;
+                        lim[e] = idx < qend ? msort[(size_t)b * N + idx] - c * C : -1;
+                    }
+                    // the slot's previous tile has been read out (and its row table with it)
+                    if (tq >= 2) ok = __all_sync(0xffffffffu, mbar_wait(bofree + slot, ((tq >> 1) - 1) & 1, err));
+                    if (!ok) break;
+                    int* srow = rows + slot * 2 * C;
+#pragma unroll
+                    for (int e = 0; e < R; ++e) {
+                        srow[R * lane + e] = tok[e];
+                        srow[C + R * lane + e] = lim[e];
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_expect_tx(qfull + slot, CF::TILE);
+                    __syncwarp();
+                    gather_tile<C, CF::NB>(qg + slot * CF::TILE, &mQ, qfull + slot, bh * N, tok, lane);
+                }
+            }
+        }
+        // drain: the loads still in flight land before the CTA exits
+        if (lane == 0) {
+            for (int c2 = max(0, nld - CF::STAGES); c2 < nld; ++c2)
+                mbar_wait(full + c2 % CF::STAGES, (c2 / CF::STAGES) & 1, err, false);
+            for (int t2 = max(0, tq - 2); t2 < tq; ++t2) mbar_wait(qfull + (t2 & 1), (t2 >> 1) & 1, err, false);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -321,8 +366,8 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 for (int i = 0; i < 4; ++i) {
                     const int p = et + 128 * (i0 + i);
                     const int r = (p % (C * 8)) >> 3;
-                    kt[p] = r < kvalid ? (mapped ? phi_x8(kx[i], phi) : kx[i]) : make_uint4(0, 0, 0, 0);
-                    if (!GATHER && mapped) qt[p] = phi_x8(qx[i], phi);
+                    kt[p] = r < kvalid ? (mapped ? phi8<PHI>(kx[i]) : kx[i]) : make_uint4(0, 0, 0, 0);
+                    if (!GATHER && mapped) qt[p] = phi8<PHI>(qx[i]);
                 }
             }
             if (ci > 0) {
@@ -383,45 +428,21 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             mbar_arrive(bprep);
 
             if (GATHER) {
+                // the gathered query rows of the chunk's tiles: phi in place
                 const int ntq = q_tiles(c);
-                const int qbase = bin_start[(size_t)b * (nbins + 1) + c];
-                const int qend = bin_start[(size_t)b * (nbins + 1) + c + 1];
                 for (int t = 0; t < ntq; ++t, ++tq) {
                     const int slot = tq & 1;
-                    if (tq >= 2) mbar_wait(bofree + slot, ((tq >> 1) - 1) & 1, err);
-                    int* srow = rows + slot * 2 * C;
-                    int* slim = srow + C;
-                    if (et < C) {
-                        const int idx = qbase + t * C + et;
-                        if (idx < qend) {
-                            const int i = perm[(size_t)b * N + idx];
-                            srow[et] = i;
-                            slim[et] = mcl[(size_t)b * N + i] - c * C;
-                        } else {
-                            srow[et] = -1;
-                            slim[et] = -1;
-                        }
-                    }
-                    named_bar(1, 128);
-                    // all of this thread's row loads are issued before any is used
-                    constexpr int NL = C * D / 8 / 128;
-                    uint8_t* q = qg + slot * CF::TILE;
-                    uint4 w[NL];
+                    mbar_wait(qfull + slot, (tq >> 1) & 1, err);
+                    if (mapped) {
+                        constexpr int NL = C * D / 8 / 128;
+                        uint4* q = reinterpret_cast<uint4*>(qg + slot * CF::TILE);
+                        uint4 w[NL];
 #pragma unroll
-                    for (int j = 0; j < NL; ++j) {
-                        const int p = et + 128 * j;
-                        const int r = p / (D / 8), col = (p % (D / 8)) * 8;
-                        const int i = srow[r];
-                        w[j] = i >= 0 ? ldg_stream(Qg + hoff + (size_t)i * D + col) : make_uint4(0, 0, 0, 0);
-                    }
+                        for (int j = 0; j < NL; ++j) w[j] = q[et + 128 * j];
 #pragma unroll
-                    for (int j = 0; j < NL; ++j) {
-                        const int p = et + 128 * j;
-                        const int r = p / (D / 8), col = (p % (D / 8)) * 8;
-                        *reinterpret_cast<uint4*>(q + (col / 64) * (C * 128) + sw128_off(r, col % 64)) =
-                            mapped ? phi_x8(w[j], phi) : w[j];
+                        for (int j = 0; j < NL; ++j) q[et + 128 * j] = phi8<PHI>(w[j]);
+                        fence_async_smem();
                     }
-                    fence_async_smem();
                     mbar_arrive(bqready + slot);
                 }
             }
@@ -447,8 +468,9 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 const uint32_t lane_s = C == 64 ? lane_base + CF::p_slot(slot) : lane_base;
                 uint8_t* pts = pt + slot * CF::PT;
                 ok = mbar_wait(bpfull + slot, use & 1, err) && ok;
+                // the row table of a gathered tile (written by the TMA warp)
+                if (GATHER) ok = mbar_wait(qfull + slot, use & 1, err) && ok;
                 tc_fence_after();
-                // the row table of a gathered tile is written before its MMAs are issued
                 const int* srow = rows + slot * 2 * C;
                 const int lim = GATHER ? srow[C + i] : i;
                 const int tok = GATHER ? srow[i] : (i < kvalid ? c * C + i : -1);
@@ -585,39 +607,58 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     }
 }
 
-template <int D, int C, bool GATHER>
+template <int D, int C, bool GATHER, int PHI>
 cudaError_t launch_chunked(const Problem& p, const void* q, const void* k, const void* v,
                            const float* prefix, int block_tokens, int nblk, const int32_t* perm,
-                           const int32_t* bins, const int32_t* mcl, int nbins, void* out, uint32_t* err,
+                           const int32_t* bins, const int32_t* msort, int nbins, void* out, uint32_t* err,
                            cudaStream_t st) {
     if (block_tokens % C != 0) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv, mo;
-    cudaError_t e = make_map(&mq, q, D, p.N, p.bh(), C);
+    // gathered queries: a 2-D row map for tile::gather4
+    cudaError_t e = GATHER ? make_row_map(&mq, q, D, p.bh() * p.N) : make_map(&mq, q, D, p.N, p.bh(), C);
     if (e == cudaSuccess) e = make_map(&mk, k, D, p.N, p.bh(), C);
     if (e == cudaSuccess) e = make_map(&mv, v, D, p.N, p.bh(), C);
     if (e == cudaSuccess) e = make_map(&mo, out, D, p.N, p.bh(), C);
     if (e != cudaSuccess) return e;
     using CF = SwCfg<D, C, GATHER>;
     constexpr size_t smem = CF::SMEM;
-    e = ensure_smem<tc_sweep_kernel<D, C, GATHER>>(smem);
+    e = ensure_smem<tc_sweep_kernel<D, C, GATHER, PHI>>(smem);
     if (e != cudaSuccess) return e;
     dim3 grid(nblk, (unsigned)p.bh());
-    return launch_pdl(tc_sweep_kernel<D, C, GATHER>, grid, dim3(CF::THREADS), smem, st, mq, mk, mv, mo,
-                      static_cast<const __nv_bfloat16*>(q), prefix, p.H, p.N, block_tokens, nblk, perm, bins,
-                      mcl, nbins, p.phi, p.normalize, static_cast<__nv_bfloat16*>(out), err);
+    return launch_pdl(tc_sweep_kernel<D, C, GATHER, PHI>, grid, dim3(CF::THREADS), smem, st, mq, mk, mv, mo,
+                      prefix, p.H, p.N, block_tokens, nblk, perm, bins, msort, nbins, p.normalize,
+                      static_cast<__nv_bfloat16*>(out), err);
+}
+
+// one kernel per feature map (see phi8)
+template <int D, int C, bool GATHER>
+cudaError_t launch_phi(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
+                       int block_tokens, int nblk, const int32_t* perm, const int32_t* bins, const int32_t* msort,
+                       int nbins, void* out, uint32_t* err, cudaStream_t st) {
+    switch (p.phi) {
+        case PHI_RELU1:
+            return launch_chunked<D, C, GATHER, PHI_RELU1>(p, q, k, v, prefix, block_tokens, nblk, perm, bins,
+                                                           msort, nbins, out, err, st);
+        case PHI_ELU1:
+            return launch_chunked<D, C, GATHER, PHI_ELU1>(p, q, k, v, prefix, block_tokens, nblk, perm, bins,
+                                                          msort, nbins, out, err, st);
+        default:
+            return launch_chunked<D, C, GATHER, PHI_IDENTITY>(p, q, k, v, prefix, block_tokens, nblk, perm, bins,
+                                                              msort, nbins, out, err, st);
+    }
 }
 
 }  // namespace
 
 cudaError_t tc_chunked(const Problem& p, int chunk, const void* q, const void* k, const void* v,
                        const float* prefix, int block_tokens, int nblk, const int32_t* perm,
-                       const int32_t* bins, const int32_t* mcl, int nbins, void* out, uint32_t* err,
+                       const int32_t* bins, const int32_t* msort, int nbins, void* out, uint32_t* err,
                        cudaStream_t st) {
     const int C = tc_chunk(p, chunk);
     const bool g = perm != nullptr;
 #define LA_CH(D_, C_, G_) \
-    return launch_chunked<D_, C_, G_>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, mcl, nbins, out, err, st)
-    if (p.d == 128) return tc_chunked_t(p, q, k, v, prefix, block_tokens, nblk, perm, bins, mcl, nbins, out, err, st);
+    return launch_phi<D_, C_, G_>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort, nbins, out, err, st)
+    if (p.d == 128) return tc_chunked_t(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort, nbins, out, err, st);
     if (C == 64) {
         if (g) LA_CH(64, 64, true);
         LA_CH(64, 64, false);

@@ -17,9 +17,10 @@
 // in its columns 64 and 65. z itself is summed on the CUDA cores from the
 // transformed K tiles.
 //
-// Warp roles (320 threads) as in the d = 64 kernel: warp 0 TMA, warp 1 MMA +
-// TMEM, warps 2-5 "prep" (phi on K / Q, z, S^T -> bf16, query gather), warps
-// 6-9 "mask" (P~, denominators, epilogue). Three pipeline stages; P, O^T and
+// Warp roles (320 threads) as in the d = 64 kernel: warp 0 TMA (with the
+// gathered query rows and their row table for the prefix mask), warp 1 MMA +
+// TMEM, warps 2-5 "prep" (phi on K / Q, z, S^T -> bf16), warps 6-9 "mask"
+// (P~, denominators, epilogue). Three pipeline stages; P, O^T and
 // P~ are double-buffered by tile parity, and the MMA warp issues a tile's
 // O^T += V^T P~^T only after the next tile's P and O^T, so the tensor core
 // has work while the mask warps turn P into P~.
@@ -51,7 +52,7 @@ struct StCfg {
     static constexpr int OROWS = GATHER ? 2 * C * 4 : 0;  // output rows of a gathered tile (x2)
     static constexpr int RED = 2 * 4 * D * 4;         // column-sum partials [parity][warp][d_k]
     static constexpr int INV = C * 4;                 // 1 / den per query row
-    static constexpr int NBAR = 2 * STAGES + 2 + 5 * 2;
+    static constexpr int NBAR = 2 * STAGES + 2 + 6 * 2;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 2 * PT + STG + QG + ROWS + OROWS + RED + INV +
                                    8 * NBAR + 16;
     // TMEM columns
@@ -65,14 +66,14 @@ struct StCfg {
     static_assert(STAGE % 1024 == 0 && KBOX % 1024 == 0, "1024-byte aligned operand tiles");
 };
 
-template <bool GATHER>
+template <bool GATHER, int PHI>
 __global__ void __launch_bounds__(StCfg<GATHER>::THREADS, 1)
 tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                   const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mOut,
-                  const __nv_bfloat16* __restrict__ Qg, const float* __restrict__ prefix, int H, int N,
+                  const float* __restrict__ prefix, int H, int N,
                   int block_tokens, int nblk, const int32_t* __restrict__ perm,
-                  const int32_t* __restrict__ bin_start, const int32_t* __restrict__ mcl, int nbins,
-                  int phi, int normalize, __nv_bfloat16* __restrict__ out, uint32_t* __restrict__ err) {
+                  const int32_t* __restrict__ bin_start, const int32_t* __restrict__ msort, int nbins,
+                  int normalize, __nv_bfloat16* __restrict__ out, uint32_t* __restrict__ err) {
     using CF = StCfg<GATHER>;
     constexpr int D = CF::D, C = CF::C;
     extern __shared__ uint8_t smem_raw[];
@@ -89,13 +90,15 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
     uint64_t* bprep = empty + CF::STAGES;  // K', Q transformed and S_prev^T in TMEM
     uint64_t* bsdone = bprep + 1;          // S^T update of the chunk done
     // Per-tile barriers, per slot (tile t uses slot t % 2, phase t / 2): P
-    // ready, P~ written (P read), O^T ready, O^T read, queries gathered.
+    // ready, P~ written (P read), O^T ready, O^T read, queries transformed,
+    // and (prefix mask) query rows landed with their row table.
     uint64_t* bpfull = bsdone + 1;
     uint64_t* bptready = bpfull + 2;
     uint64_t* bofull = bptready + 2;
     uint64_t* bofree = bofull + 2;
     uint64_t* bqready = bofree + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bqready + 2);
+    uint64_t* qfull = bqready + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qfull + 2);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int blk = blockIdx.x;
@@ -105,7 +108,7 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
     const int c_begin = blk * (block_tokens / C);
     const int c_end = (GATHER && blk == nblk - 1) ? nbins : min(nchunks, c_begin + block_tokens / C);
     const int nci = c_end - c_begin;
-    const bool mapped = phi != PHI_IDENTITY;  // phi applied to Q and K tiles
+    constexpr bool mapped = PHI != PHI_IDENTITY;  // phi applied to Q and K tiles
     const size_t hoff = (size_t)bh * N * D;
 
     auto q_tiles = [&](int c) -> int {
@@ -128,15 +131,14 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
             mbar_init(bofull + j, 1);
             mbar_init(bofree + j, 128);
             mbar_init(bqready + j, 128);
+            mbar_init(qfull + j, 1);
         }
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, CF::TMEM_COLS);
     if (threadIdx.x == 0) {
-        if (!GATHER) {
-            tma_prefetch_map(&mQ);
-            tma_prefetch_map(&mOut);
-        }
+        tma_prefetch_map(&mQ);
+        if (!GATHER) tma_prefetch_map(&mOut);
         tma_prefetch_map(&mK);
         tma_prefetch_map(&mV);
     }
@@ -144,19 +146,16 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // The TMA producer (warp 0) loads only the caller's inputs, so it does
-    // not wait for the previous kernel of the call and fills the pipeline
-    // while that kernel finishes; every other warp waits before it reads
-    // what that kernel wrote.
+    // The TMA producer (warp 0) first loads only the caller's inputs, so it
+    // fills the pipeline without waiting for the previous kernel of the call;
+    // every other warp waits before it reads what that kernel wrote.
     if (warp != 0) pdl_wait();
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
-        if (lane == 0) {
-            int ci = 0;
-            for (; ci < nci; ++ci) {
-                const int s = ci % CF::STAGES, u = ci / CF::STAGES;
-                if (u > 0 && !mbar_wait(empty + s, (u - 1) & 1, err)) break;
+        // ---------------- TMA producer (whole warp) ----------------
+        auto load_chunk = [&](int ci) {
+            const int s = ci % CF::STAGES;
+            if (lane == 0) {
                 mbar_arrive_expect_tx(full + s, CF::TX);
                 uint8_t* st = stages + s * CF::STAGE;
                 const int row = (c_begin + ci) * C;
@@ -167,9 +166,56 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                     tma_load_3d(st + CF::OFF_V + bx * CF::BOX, &mV, full + s, bx * 64, row, bh);
                 }
             }
-            // drain: the last loads issued have landed before the CTA exits
-            for (int c2 = max(0, ci - CF::STAGES); c2 < ci; ++c2)
+        };
+        int nld = min(nci, CF::STAGES);
+        for (int ci = 0; ci < nld; ++ci) load_chunk(ci);
+        // the bin tables below come from an earlier kernel of the call
+        if (GATHER) pdl_wait();
+        bool ok = true;
+        int tq = 0;
+        for (int ci = 0; ci < nci && ok; ++ci) {
+            if (ci >= CF::STAGES) {
+                const int s = ci % CF::STAGES, u = ci / CF::STAGES;
+                ok = __all_sync(0xffffffffu, mbar_wait(empty + s, (u - 1) & 1, err));
+                if (!ok) break;
+                load_chunk(ci);
+                nld = ci + 1;
+            }
+            if (GATHER) {
+                const int c = c_begin + ci;
+                const int qbase = bin_start[(size_t)b * (nbins + 1) + c];
+                const int qend = bin_start[(size_t)b * (nbins + 1) + c + 1];
+                for (int t = 0; qbase + t * C < qend; ++t, ++tq) {
+                    constexpr int R = C / 32;  // rows of the tile per lane
+                    const int slot = tq & 1;
+                    int tok[R], lim[R];
+#pragma unroll
+                    for (int e = 0; e < R; ++e) {
+                        const int idx = qbase + t * C + R * lane + e;
+                        tok[e] = idx < qend ? perm[(size_t)b * N + idx] : -1;
+                        lim[e] = idx < qend ? msort[(size_t)b * N + idx] - c * C : -1;
+                    }
+                    // the slot's previous tile has been read out (and its row table with it)
+                    if (tq >= 2) ok = __all_sync(0xffffffffu, mbar_wait(bofree + slot, ((tq >> 1) - 1) & 1, err));
+                    if (!ok) break;
+                    int* srow = rows + slot * 2 * C;
+#pragma unroll
+                    for (int e = 0; e < R; ++e) {
+                        srow[R * lane + e] = tok[e];
+                        srow[C + R * lane + e] = lim[e];
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_expect_tx(qfull + slot, CF::TILE);
+                    __syncwarp();
+                    gather_tile<C, CF::NB>(qg + slot * CF::TILE, &mQ, qfull + slot, bh * N, tok, lane);
+                }
+            }
+        }
+        // drain: the loads still in flight land before the CTA exits
+        if (lane == 0) {
+            for (int c2 = max(0, nld - CF::STAGES); c2 < nld; ++c2)
                 mbar_wait(full + c2 % CF::STAGES, (c2 / CF::STAGES) & 1, err, false);
+            for (int t2 = max(0, tq - 2); t2 < tq; ++t2) mbar_wait(qfull + (t2 & 1), (t2 >> 1) & 1, err, false);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -301,7 +347,7 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                     uint4* kp = reinterpret_cast<uint4*>(kt + bx * CF::KBOX + w * 16);
                     uint4 x = *kp;
                     if (r < kvalid) {
-                        if (mapped) x = phi_x8(x, phi);
+                        if (mapped) x = phi8<PHI>(x);
                     } else {
                         x = make_uint4(0, 0, 0, 0);
                     }
@@ -314,7 +360,7 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                     }
                     if (!GATHER && mapped) {
                         uint4* qp = reinterpret_cast<uint4*>(st + bx * CF::BOX + w * 16);
-                        *qp = phi_x8(*qp, phi);
+                        *qp = phi8<PHI>(*qp);
                     }
                 }
                 if (normalize) {
@@ -358,44 +404,21 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
             mbar_arrive(bprep);
 
             if (GATHER) {
+                // the gathered query rows of the chunk's tiles: phi in place
                 const int ntq = q_tiles(c);
-                const int qbase = bin_start[(size_t)b * (nbins + 1) + c];
-                const int qend = bin_start[(size_t)b * (nbins + 1) + c + 1];
                 for (int t = 0; t < ntq; ++t, ++tq) {
                     const int slot = tq & 1;
-                    if (tq >= 2) mbar_wait(bofree + slot, ((tq >> 1) - 1) & 1, err);
-                    int* srow = rows + slot * 2 * C;
-                    int* slim = srow + C;
-                    if (et < C) {
-                        const int idx = qbase + t * C + et;
-                        if (idx < qend) {
-                            const int i = perm[(size_t)b * N + idx];
-                            srow[et] = i;
-                            slim[et] = mcl[(size_t)b * N + i] - c * C;
-                        } else {
-                            srow[et] = -1;
-                            slim[et] = -1;
-                        }
-                    }
-                    named_bar(1, 128);
-                    constexpr int NL = C * D / 8 / 128;
-                    uint8_t* q = qg + slot * CF::TILE;
-                    uint4 w[NL];
+                    mbar_wait(qfull + slot, (tq >> 1) & 1, err);
+                    if (mapped) {
+                        constexpr int NL = C * D / 8 / 128;
+                        uint4* q = reinterpret_cast<uint4*>(qg + slot * CF::TILE);
+                        uint4 w[NL];
 #pragma unroll
-                    for (int j = 0; j < NL; ++j) {
-                        const int p = et + 128 * j;
-                        const int r = p / (D / 8), col = (p % (D / 8)) * 8;
-                        const int i = srow[r];
-                        w[j] = i >= 0 ? ldg_stream(Qg + hoff + (size_t)i * D + col) : make_uint4(0, 0, 0, 0);
-                    }
+                        for (int j = 0; j < NL; ++j) w[j] = q[et + 128 * j];
 #pragma unroll
-                    for (int j = 0; j < NL; ++j) {
-                        const int p = et + 128 * j;
-                        const int r = p / (D / 8), col = (p % (D / 8)) * 8;
-                        *reinterpret_cast<uint4*>(q + (col / 64) * CF::BOX + sw128_off(r, col % 64)) =
-                            mapped ? phi_x8(w[j], phi) : w[j];
+                        for (int j = 0; j < NL; ++j) q[et + 128 * j] = phi8<PHI>(w[j]);
+                        fence_async_smem();
                     }
-                    fence_async_smem();
                     mbar_arrive(bqready + slot);
                 }
             }
@@ -420,6 +443,8 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                 const uint32_t lane_s = lane_base + static_cast<uint32_t>(slot) * (16u << 16);
                 uint8_t* pts = pt + slot * CF::PT;
                 ok = mbar_wait(bpfull + slot, use & 1, err) && ok;
+                // the row table of a gathered tile (written by the TMA warp)
+                if (GATHER) ok = mbar_wait(qfull + slot, use & 1, err) && ok;
                 tc_fence_after();
                 const int* srow = rows + slot * 2 * C;
                 const int lim = GATHER ? srow[C + i] : i;
@@ -514,34 +539,53 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
     }
 }
 
-template <bool GATHER>
+template <bool GATHER, int PHI>
 cudaError_t launch_t(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
-                     int block_tokens, int nblk, const int32_t* perm, const int32_t* bins, const int32_t* mcl,
+                     int block_tokens, int nblk, const int32_t* perm, const int32_t* bins, const int32_t* msort,
                      int nbins, void* out, uint32_t* err, cudaStream_t st) {
     using CF = StCfg<GATHER>;
     if (p.d != CF::D || block_tokens % CF::C != 0) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv, mo;
-    cudaError_t e = make_map(&mq, q, CF::D, p.N, p.bh(), CF::C);
+    // gathered queries: a 2-D row map for tile::gather4
+    cudaError_t e = GATHER ? make_row_map(&mq, q, CF::D, p.bh() * p.N) : make_map(&mq, q, CF::D, p.N, p.bh(), CF::C);
     if (e == cudaSuccess) e = make_map(&mk, k, CF::D, p.N, p.bh(), CF::C);
     if (e == cudaSuccess) e = make_map(&mv, v, CF::D, p.N, p.bh(), CF::C);
     if (e == cudaSuccess) e = make_map(&mo, out, CF::D, p.N, p.bh(), CF::C);
     if (e != cudaSuccess) return e;
-    e = ensure_smem<tc_sweep_t_kernel<GATHER>>(CF::SMEM);
+    e = ensure_smem<tc_sweep_t_kernel<GATHER, PHI>>(CF::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(nblk, (unsigned)p.bh());
-    return launch_pdl(tc_sweep_t_kernel<GATHER>, grid, dim3(CF::THREADS), CF::SMEM, st, mq, mk, mv, mo,
-                      static_cast<const __nv_bfloat16*>(q), prefix, p.H, p.N, block_tokens, nblk, perm, bins,
-                      mcl, nbins, p.phi, p.normalize, static_cast<__nv_bfloat16*>(out), err);
+    return launch_pdl(tc_sweep_t_kernel<GATHER, PHI>, grid, dim3(CF::THREADS), CF::SMEM, st, mq, mk, mv, mo,
+                      prefix, p.H, p.N, block_tokens, nblk, perm, bins, msort, nbins, p.normalize,
+                      static_cast<__nv_bfloat16*>(out), err);
+}
+
+// one kernel per feature map (see phi8)
+template <bool GATHER>
+cudaError_t launch_phi(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
+                       int block_tokens, int nblk, const int32_t* perm, const int32_t* bins, const int32_t* msort,
+                       int nbins, void* out, uint32_t* err, cudaStream_t st) {
+    switch (p.phi) {
+        case PHI_RELU1:
+            return launch_t<GATHER, PHI_RELU1>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort, nbins,
+                                               out, err, st);
+        case PHI_ELU1:
+            return launch_t<GATHER, PHI_ELU1>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort, nbins,
+                                              out, err, st);
+        default:
+            return launch_t<GATHER, PHI_IDENTITY>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort,
+                                                  nbins, out, err, st);
+    }
 }
 
 }  // namespace
 
 cudaError_t tc_chunked_t(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
                          int block_tokens, int nblk, const int32_t* perm, const int32_t* bins,
-                         const int32_t* mcl, int nbins, void* out, uint32_t* err, cudaStream_t st) {
+                         const int32_t* msort, int nbins, void* out, uint32_t* err, cudaStream_t st) {
     if (perm != nullptr)
-        return launch_t<true>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, mcl, nbins, out, err, st);
-    return launch_t<false>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, mcl, nbins, out, err, st);
+        return launch_phi<true>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort, nbins, out, err, st);
+    return launch_phi<false>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort, nbins, out, err, st);
 }
 
 }  // namespace la
