@@ -4,8 +4,9 @@ command to put under a profiler (ncu) when studying a single kernel.
     python -m kernelized_linear_attention_phi_b200.profile_case \\
         --op noncausal --B 1 --H 16 --N 16384 --d 64 --iters 3
 
-``--op`` is one of kv_summary, noncausal, causal, prefix, decode. Inputs come
-from the seeded generators in ``workloads``; nothing is checked or timed.
+``--op`` is one of kv_summary, noncausal, causal, prefix, decode,
+noncausal_bwd, causal_bwd. Inputs come from the seeded generators in
+``workloads``; nothing is checked or timed.
 """
 
 from __future__ import annotations
@@ -20,13 +21,14 @@ from . import workloads as W
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", required=True, choices=["kv_summary", "noncausal", "causal", "prefix", "decode"])
+    ap.add_argument("--op", required=True, choices=["kv_summary", "noncausal", "causal", "prefix", "decode",
+                                                      "noncausal_bwd", "causal_bwd"])
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--H", type=int, default=16)
     ap.add_argument("--N", type=int, default=16384)
     ap.add_argument("--d", type=int, default=64)
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f32"])
-    ap.add_argument("--phi", default="relu1", choices=["relu1", "identity"])
+    ap.add_argument("--phi", default="relu1", choices=["relu1", "identity", "elu1"])
     ap.add_argument("--unnormalized", action="store_true")
     ap.add_argument("--chunk", type=int, default=64)
     ap.add_argument("--iters", type=int, default=3)
@@ -34,7 +36,7 @@ def main():
     from . import build
     build.build()
     dev = torch.device("cuda", 0)
-    sigma = 1.0 if a.phi == "relu1" else a.d ** -0.5
+    sigma = a.d ** -0.5 if a.phi == "identity" else 1.0
     norm = not a.unnormalized
     q, k, v = W.qkv(a.B, a.H, a.N, a.d, sigma, 1, a.dtype, dev)
     desc = la._desc_of(q, a.phi, norm)
@@ -44,6 +46,12 @@ def main():
         q1, k1, v1 = (t[0].contiguous() for t in W.decode_tokens(1, a.B, a.H, a.d, sigma, 1, a.dtype, dev))
         out = torch.empty_like(q1)
         fn = lambda: la.la_decode_step(q1, k1, v1, S, z, out, a.phi, norm)
+    elif a.op.endswith("_bwd"):
+        ws = la.workspace(desc, a.op, a.chunk, dev)
+        dout = W.upstream_grad(a.B, a.H, a.N, a.d, 1, a.dtype, dev)
+        grads = [torch.empty_like(q) for _ in range(3)]
+        bwd = la.la_noncausal_backward if a.op == "noncausal_bwd" else la.la_causal_backward
+        fn = lambda: bwd(q, k, v, dout, *grads, phi=a.phi, normalize=norm, ws=ws)
     else:
         ws = la.workspace(desc, a.op, a.chunk, dev)
         out = torch.empty_like(q)
