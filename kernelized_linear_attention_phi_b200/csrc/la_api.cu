@@ -349,6 +349,9 @@ la_status backward_impl(const la_desc* desc, bool causal, const void* q, const v
     float* G = at<float>(ws, L.gtot);
     float* h = G + (size_t)p.bh() * p.d * p.d;
     LA_TRY(kv_summary_impl(p, k, v, S, z, ws, st));
+    if (tc_supported(p))  // tensor cores: the KV summary's record slots take the (G, h) records
+        return cuda_status(tc_noncausal_backward(p, q, k, v, dout, S, z, at<float>(ws, L.part), G, h, dq, dk, dv,
+                                                 at<uint32_t>(ws, 0), st));
     LA_TRY(cuda_status(bwd_q(p, false, q, k, v, dout, S, z, (long long)p.d * p.d, p.d, bp.block_tokens,
                              bp.nblk, dq, gn, gden, grec, st)));
     LA_TRY(cuda_status(state_reduce(p, grec, bp.nblk, G, h, st)));

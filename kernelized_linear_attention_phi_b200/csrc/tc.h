@@ -28,6 +28,9 @@ KvBalanced kv_balanced_plan(const Problem& p);
 // d*d + d floats), then a fixed-order reduction into S [bh][d*d], z [bh][d].
 cudaError_t tc_kv_summary(const Problem& p, const void* k, const void* v, float* part, float* S,
                           float* z, uint32_t* err, cudaStream_t st);
+// Sums balanced-split records (slot cta * K + j, d*d + d floats each) per
+// head in CTA order into S [bh][d*d] and z [bh][d].
+cudaError_t tc_reduce_records(const Problem& p, const float* part, float* S, float* z, cudaStream_t st);
 // KV summary per block: CTA (block, head) writes record (head*nblk + block)
 // over tokens [block*block_tokens, ...); block_tokens must be a multiple of 128.
 cudaError_t tc_kv_blocks(const Problem& p, const void* k, const void* v, int block_tokens, int nblk,
@@ -50,6 +53,13 @@ cudaError_t tc_chunked(const Problem& p, int chunk, const void* q, const void* k
 cudaError_t tc_chunked_t(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
                          int block_tokens, int nblk, const int32_t* perm, const int32_t* bins,
                          const int32_t* msort, int nbins, void* out, uint32_t* err, cudaStream_t st);
+
+// Gradients of the non-causal form (tc_bwd.cu): S, z are the KV summary of
+// the forward; `part` holds kv_balanced_plan(p) record slots, (G, h)
+// [bh][d*d], [bh][d] receive the reduced records. Writes dq, dk, dv.
+cudaError_t tc_noncausal_backward(const Problem& p, const void* q, const void* k, const void* v, const void* dout,
+                                  const float* S, const float* z, float* part, float* G, float* h, void* dq,
+                                  void* dk, void* dv, uint32_t* err, cudaStream_t st);
 
 // [BH, N, d] bf16 viewed as 3-D for TMA: 64-column x `rows` boxes, 128-byte
 // swizzle, zero fill outside the tensor.

@@ -656,6 +656,13 @@ cudaError_t tc_kv_summary(const Problem& p, const void* k, const void* v, float*
                       part, w.b, p.d, S, z);
 }
 
+cudaError_t tc_reduce_records(const Problem& p, const float* part, float* S, float* z, cudaStream_t st) {
+    const KvBalanced w = kv_balanced_plan(p);
+    const int rec4 = (p.d * p.d + p.d) / 4;
+    return launch_pdl(kv_reduce_balanced_kernel, dim3((rec4 + 127) / 128, (unsigned)p.bh()), dim3(128), 0, st, part,
+                      w, p.d, S, z);
+}
+
 cudaError_t tc_kv_blocks(const Problem& p, const void* k, const void* v, int block_tokens, int nblk, float* part,
                          uint32_t* err, cudaStream_t st) {
     if (block_tokens % kTile != 0) return cudaErrorInvalidValue;
