@@ -21,6 +21,8 @@
 // (all ones above the diagonal for the non-causal form, where the chunk
 // terms are folded into the totals instead and not formed).
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 #include "launch_util.h"
@@ -343,10 +345,10 @@ bwd_q_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restri
 // state of the blocks after blk (index bh * nblk + blk); non-causal, the
 // totals of the head (index bh). Causal chunks are swept last to first,
 // each adding its own queries to (G, h) after its keys are done.
-template <typename T, int D, bool CAUSAL>
+template <typename T, int D, bool CAUSAL, typename TG = float>
 __global__ void __launch_bounds__(kThreads)
 bwd_kv_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V,
-              const float* __restrict__ gn_in, const float* __restrict__ gden_in,
+              const TG* __restrict__ gn_in, const float* __restrict__ gden_in,
               const float* __restrict__ Gb, const float* __restrict__ hb, long long g_stride,
               long long h_stride, int N, int block_tokens, int nblk, int phi, T* __restrict__ dK,
               T* __restrict__ dV) {
@@ -382,7 +384,7 @@ bwd_kv_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restr
         tile_to_smem<T, D, LD>(sV, V + hoff + (long long)t0 * D, C, valid, false, phi);
         if (CAUSAL) {
             tile_to_smem<T, D, LD>(sA, Q + hoff + (long long)t0 * D, C, valid, true, phi);
-            tile_to_smem<float, D, LD>(sN, gn_in + hoff + (long long)t0 * D, C, valid, false, phi);
+            tile_to_smem<TG, D, LD>(sN, gn_in + hoff + (long long)t0 * D, C, valid, false, phi);
             if (threadIdx.x < C)
                 sGd[threadIdx.x] = threadIdx.x < valid ? gden_in[bh * (long long)N + t0 + threadIdx.x] : 0.f;
         }
@@ -512,7 +514,7 @@ cudaError_t launch_bwd(const Problem& p, bool causal, const void* q, const void*
                        const void* dout, const float* S, const float* z, long long s_stride, long long z_stride,
                        const float* G, const float* h, long long g_stride, long long h_stride, int block_tokens,
                        int nblk, void* dq, void* dk, void* dv, float* gn, float* gden, float* grec, bool q_pass,
-                       cudaStream_t st) {
+                       bool gn16, cudaStream_t st) {
     using CF = BwCfg<D>;
     if (block_tokens % CF::C != 0) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)nblk, (unsigned)p.bh());
@@ -528,6 +530,19 @@ cudaError_t launch_bwd(const Problem& p, bool causal, const void* q, const void*
                           s_stride, z_stride, p.N, block_tokens, nblk, p.phi, p.normalize, static_cast<T*>(dq), gn,
                           gden, grec);
     }
+    if (gn16) {
+        // gn in bf16 (from the tensor-core first sweep: causal, bf16, d = 64)
+        if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 64) {
+            if (!causal) return cudaErrorInvalidValue;
+            cudaError_t e = ensure_smem<bwd_kv_kernel<T, D, true, __nv_bfloat16>>(CF::SMEM);
+            if (e != cudaSuccess) return e;
+            return launch_pdl(bwd_kv_kernel<T, D, true, __nv_bfloat16>, grid, dim3(kThreads), CF::SMEM, st, Q, K, V,
+                              reinterpret_cast<const __nv_bfloat16*>(gn), static_cast<const float*>(gden), G, h,
+                              g_stride, h_stride, p.N, block_tokens, nblk, p.phi, static_cast<T*>(dk),
+                              static_cast<T*>(dv));
+        }
+        return cudaErrorInvalidValue;
+    }
     auto kern = causal ? bwd_kv_kernel<T, D, true> : bwd_kv_kernel<T, D, false>;
     cudaError_t e = causal ? ensure_smem<bwd_kv_kernel<T, D, true>>(CF::SMEM)
                            : ensure_smem<bwd_kv_kernel<T, D, false>>(CF::SMEM);
@@ -542,10 +557,10 @@ cudaError_t bwd_dispatch(const Problem& p, bool causal, const void* q, const voi
                          const void* dout, const float* S, const float* z, long long s_stride, long long z_stride,
                          const float* G, const float* h, long long g_stride, long long h_stride, int block_tokens,
                          int nblk, void* dq, void* dk, void* dv, float* gn, float* gden, float* grec, bool q_pass,
-                         cudaStream_t st) {
+                         bool gn16, cudaStream_t st) {
 #define LA_BW(D_)                                                                                             \
     return launch_bwd<T, D_>(p, causal, q, k, v, dout, S, z, s_stride, z_stride, G, h, g_stride, h_stride, \
-                             block_tokens, nblk, dq, dk, dv, gn, gden, grec, q_pass, st)
+                             block_tokens, nblk, dq, dk, dv, gn, gden, grec, q_pass, gn16, st)
     switch (p.d) {
         case 16: LA_BW(16);
         case 32: LA_BW(32);
@@ -565,15 +580,16 @@ cudaError_t bwd_q(const Problem& p, bool causal, const void* q, const void* k, c
                   int nblk, void* dq, float* gn, float* gden, float* grec, cudaStream_t st) {
     auto f = p.dtype == DT_F32 ? bwd_dispatch<float> : bwd_dispatch<__nv_bfloat16>;
     return f(p, causal, q, k, v, dout, S, z, s_stride, z_stride, nullptr, nullptr, 0, 0, block_tokens, nblk, dq,
-             nullptr, nullptr, gn, gden, grec, true, st);
+             nullptr, nullptr, gn, gden, grec, true, false, st);
 }
 
-cudaError_t bwd_kv(const Problem& p, bool causal, const void* q, const void* k, const void* v, const float* gn,
+cudaError_t bwd_kv(const Problem& p, bool causal, const void* q, const void* k, const void* v, const void* gn,
                    const float* gden, const float* G, const float* h, long long g_stride, long long h_stride,
-                   int block_tokens, int nblk, void* dk, void* dv, cudaStream_t st) {
+                   int block_tokens, int nblk, void* dk, void* dv, cudaStream_t st, bool gn_bf16) {
     auto f = p.dtype == DT_F32 ? bwd_dispatch<float> : bwd_dispatch<__nv_bfloat16>;
     return f(p, causal, q, k, v, nullptr, nullptr, nullptr, 0, 0, G, h, g_stride, h_stride, block_tokens, nblk,
-             nullptr, dk, dv, const_cast<float*>(gn), const_cast<float*>(gden), nullptr, false, st);
+             nullptr, dk, dv, static_cast<float*>(const_cast<void*>(gn)), const_cast<float*>(gden), nullptr, false,
+             gn_bf16, st);
 }
 
 }  // namespace la

@@ -75,10 +75,11 @@ cudaError_t bwd_q(const Problem& p, bool causal, const void* q, const void* k, c
                   int nblk, void* dq, float* gn, float* gden, float* grec, cudaStream_t st);
 // Reverse sweep: per block, from (G, h) of all later queries (causal: suffix
 // state at index bh*nblk + blk; non-causal: totals at index bh), writes dk
-// and dv.
-cudaError_t bwd_kv(const Problem& p, bool causal, const void* q, const void* k, const void* v, const float* gn,
+// and dv. gn is fp32, or bf16 with gn_bf16 (causal bf16 d = 64 only: the
+// tensor-core first sweep's output).
+cudaError_t bwd_kv(const Problem& p, bool causal, const void* q, const void* k, const void* v, const void* gn,
                    const float* gden, const float* G, const float* h, long long g_stride, long long h_stride,
-                   int block_tokens, int nblk, void* dk, void* dv, cudaStream_t st);
+                   int block_tokens, int nblk, void* dk, void* dv, cudaStream_t st, bool gn_bf16 = false);
 
 // ---- decode (decode.cu) -------------------------------------------------------
 cudaError_t decode_step(const Problem& p, const void* q, const void* k, const void* v, float* S,

@@ -338,11 +338,17 @@ la_status backward_impl(const la_desc* desc, bool causal, const void* q, const v
             LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
         }
         LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
-        LA_TRY(cuda_status(bwd_q(p, true, q, k, v, dout, part, part + (size_t)p.d * p.d, rec, rec,
-                                 bp.block_tokens, bp.nblk, dq, gn, gden, grec, st)));
+        const bool tcq = tc_causal_backward_supported(p, bp.block_tokens);
+        if (tcq) {  // tensor cores; gn in bf16
+            LA_TRY(cuda_status(tc_causal_backward_q(p, q, k, v, dout, part, bp.block_tokens, bp.nblk, dq, gn, gden,
+                                                    grec, flags, st)));
+        } else {
+            LA_TRY(cuda_status(bwd_q(p, true, q, k, v, dout, part, part + (size_t)p.d * p.d, rec, rec,
+                                     bp.block_tokens, bp.nblk, dq, gn, gden, grec, st)));
+        }
         LA_TRY(cuda_status(state_exclusive_scan(p, grec, bp.nblk, nullptr, nullptr, st, true)));
         return cuda_status(bwd_kv(p, true, q, k, v, gn, gden, grec, grec + (size_t)p.d * p.d, rec, rec,
-                                  bp.block_tokens, bp.nblk, dk, dv, st));
+                                  bp.block_tokens, bp.nblk, dk, dv, st, tcq));
     }
     float* S = at<float>(ws, L.sz);
     float* z = S + (size_t)p.bh() * p.d * p.d;

@@ -61,6 +61,15 @@ cudaError_t tc_noncausal_backward(const Problem& p, const void* q, const void* k
                                   const float* S, const float* z, float* part, float* G, float* h, void* dq,
                                   void* dk, void* dv, uint32_t* err, cudaStream_t st);
 
+// First sweep of the causal gradients on tensor cores (tc_bwd_causal.cu;
+// bf16, d = 64, block_tokens a multiple of 64): from the forward's exclusive
+// block prefixes, writes dq, gn (bf16 [bh][N][d]), gden (fp32 [bh][N]) and
+// the blocks' own (G, h) records grec[bh*nblk + blk], as bwd_q does.
+bool tc_causal_backward_supported(const Problem& p, int block_tokens);
+cudaError_t tc_causal_backward_q(const Problem& p, const void* q, const void* k, const void* v, const void* dout,
+                                 const float* prefix, int block_tokens, int nblk, void* dq, void* gn, float* gden,
+                                 float* grec, uint32_t* err, cudaStream_t st);
+
 // [BH, N, d] bf16 viewed as 3-D for TMA: 64-column x `rows` boxes, 128-byte
 // swizzle, zero fill outside the tensor.
 cudaError_t make_map(CUtensorMap* map, const void* base, int d, int N, long long bh, int rows);

@@ -47,35 +47,6 @@ __host__ __device__ __forceinline__ long long range_lo(long long total, int G, l
     return c * total / G;
 }
 
-// Bit e of the result is set when element e of eight packed bf16 values is
-// greater than zero (sign clear and not +0).
-__device__ __forceinline__ uint32_t positive_bits(const uint4& w) {
-    const uint32_t v[4] = {w.x, w.y, w.z, w.w};
-    uint32_t m = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = v[i] & 0xFFFFu, hi = v[i] >> 16;
-        m |= (((lo & 0x8000u) == 0 && lo != 0) ? 1u : 0u) << (2 * i);
-        m |= (((hi & 0x8000u) == 0 && hi != 0) ? 1u : 0u) << (2 * i + 1);
-    }
-    return m;
-}
-
-// f *= phi'(x) on eight values of one row: relu+1 from the sign bits,
-// elu+1 from phi(x) itself (packed bf16 in w), the identity leaves f alone.
-template <int PHI>
-__device__ __forceinline__ void times_phi_grad(float* f, uint32_t bits, const uint4& w) {
-    if constexpr (PHI == PHI_RELU1) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = ((bits >> e) & 1u) ? f[e] : 0.f;
-    } else if constexpr (PHI == PHI_ELU1) {
-        float p[8];
-        unpack8(w, p);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] *= fminf(p[e], 1.f);
-    }
-}
-
 // phi in place on one stage tile of 128 rows x D columns (16-byte chunks
 // et, et + 128, ...), recording relu+1's sign bits per row and logical
 // column group: sgn[row * D / 8 + group].

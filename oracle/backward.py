@@ -32,7 +32,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .linear_attention import (FORM_NONCAUSAL, PHI_ELU1, PHI_IDENTITY, PHI_RELU1, phi,
+from .linear_attention import (FORM_CAUSAL, FORM_NONCAUSAL, PHI_ELU1, PHI_IDENTITY, PHI_RELU1, phi,
                                visible)
 
 
@@ -51,10 +51,19 @@ def phi_grad(x, kind=PHI_RELU1):
 def backward_dense(Q, K, V, dO, form=FORM_NONCAUSAL, m=None, phi_kind=PHI_RELU1,
                    normalize=True, scales=False):
     """(dQ, dK, dV) of one head by the definition above. With scales=True
-    also (tq, tk, tv): per row, the sum of the norms of the terms that make up
-    that row of dQ (phi' times sum_j dnum_i.v_j b_j and times dden_i sum_j
-    b_j), of dK (the same two with the roles of queries and keys swapped) and
-    of dV (sum_i |w_ij| ||dnum_i||), the size of what rounding acts on."""
+    also (tq, tk, tv), per row the size of what rounding acts on. The rows
+    are products with the states a query or key sees,
+        dq_i = phi'(q_i) (S_i dnum_i + dden_i z_i),   S_i = sum_{j vis i} b_j v_j^T,
+        dk_j = phi'(k_j) (G_j v_j + h_j),   dv_j = G_j^T b_j,
+                                   G_j = sum_{i sees j} a_i dnum_i^T,
+    and the scale of each is the same product with every factor replaced by
+    its absolute value, the states summed exactly first (|S_i| |dnum_i| +
+    |dden_i| z_i, and so on): a product of rounded operands errs by at most
+    the unit roundoff times the product of the absolute values, and the
+    states are what a chunked computation rounds, not their single terms.
+    The norms of the exact terms are not such a scale (an inner product of
+    them can cancel while their rounding does not); a sum of absolute values
+    over keys would be one, but loose by a factor that grows with N."""
     Q, K, V, dO = (np.asarray(t, dtype=np.float64) for t in (Q, K, V, dO))
     n = Q.shape[0]
     A, Bk = phi(Q, phi_kind), phi(K, phi_kind)
@@ -75,13 +84,28 @@ def backward_dense(Q, K, V, dO, form=FORM_NONCAUSAL, m=None, phi_kind=PHI_RELU1,
     grads = (phi_grad(Q, phi_kind) * dA, phi_grad(K, phi_kind) * dB, dV)
     if not scales:
         return grads
-    vis = visible(n, form, m)
-    dnv = np.where(vis, dnum @ V.T, 0.0)   # dnum_i . v_j on visible entries
-    dd = np.where(vis, dden[:, None], 0.0)
-    pq, pk = phi_grad(Q, phi_kind), phi_grad(K, phi_kind)
-    tq = np.linalg.norm(pq * (dnv @ Bk), axis=1) + np.linalg.norm(pq * (dd @ Bk), axis=1)
-    tk = np.linalg.norm(pk * (dnv.T @ A), axis=1) + np.linalg.norm(pk * (dd.T @ A), axis=1)
-    tv = np.abs(W).T @ np.linalg.norm(dnum, axis=1)
+    vis = visible(n, form, m).astype(np.float64)
+    # per-row states: S_i, z_i over the keys query i sees; G_j, h_j over the
+    # queries that see key j
+    Sx = Bk[:, :, None] * V[:, None, :]      # b_j v_j^T
+    Gx = A[:, :, None] * dnum[:, None, :]    # a_i dnum_i^T
+    if form == FORM_NONCAUSAL:
+        S = np.broadcast_to(Sx.sum(0), Sx.shape)
+        z = np.broadcast_to(Bk.sum(0), Bk.shape)
+        G = np.broadcast_to(Gx.sum(0), Gx.shape)
+        h = np.broadcast_to((A * dden[:, None]).sum(0), A.shape)
+    elif form == FORM_CAUSAL:
+        S, z = np.cumsum(Sx, 0), np.cumsum(Bk, 0)
+        G = np.cumsum(Gx[::-1], 0)[::-1]
+        h = np.cumsum((A * dden[:, None])[::-1], 0)[::-1]
+    else:
+        S, z = np.einsum("ij,jkv->ikv", vis, Sx), vis @ Bk
+        G, h = np.einsum("ij,ikv->jkv", vis, Gx), vis.T @ (A * dden[:, None])
+    pq, pk = np.abs(phi_grad(Q, phi_kind)), np.abs(phi_grad(K, phi_kind))
+    tq = np.linalg.norm(pq * (np.einsum("ikv,iv->ik", np.abs(S), np.abs(dnum)) + np.abs(dden)[:, None] * np.abs(z)),
+                        axis=1)
+    tk = np.linalg.norm(pk * (np.einsum("jkv,jv->jk", np.abs(G), np.abs(V)) + np.abs(h)), axis=1)
+    tv = np.linalg.norm(np.einsum("jkv,jk->jv", np.abs(G), np.abs(Bk)), axis=1)
     return grads + (tq, tk, tv)
 
 

@@ -11,17 +11,19 @@ Gradients need a different floor: some of their entries are differences
 of terms of ordinary size that cancel exactly or nearly (a query that sees a
 single key: its normalized output does not depend on it, so d out / d q = 0
 while each of the two terms the kernels add is of order one). A result
-computed in fp32 returns rounding noise of the order of the terms there, which
-no relative error against the (zero) oracle row can accept. A gradient row
-is a sum of terms, so ``max_row_grad_err`` measures its error relative to the
-larger of its own norm and t_i, the sum of the norms of the terms that are
-added (from ``backward.backward_dense(..., scales=True)``):
+computed in finite precision returns rounding noise there, which no relative
+error against the (zero) oracle row can accept. ``max_row_grad_err``
+measures a row's error relative to the larger of its own norm and t_i, the
+rounding scale of the row (from ``backward.backward_dense(..., scales=True)``:
+the row's product with the states it sees, computed with every factor
+replaced by its absolute value, which bounds what rounding the operands can
+do to it):
 
     err = max_i ||g_i - r_i||_2 / max(||r_i||_2, t_i)
 
-Where the terms do not cancel, t_i is close to ||r_i|| and this is the plain
-relative row error; a wrong or missing term, or a small relative error in one
-of them (the state S, say), still shows up at its own size relative to t_i.
+A wrong or missing term still shows up at its own size relative to t_i, which
+for inputs with mixed signs is a sizeable fraction of t_i (a planted dropped
+term is pinned to fail by a wide margin).
 """
 
 import numpy as np

@@ -118,3 +118,30 @@ def test_gradient_metric_and_scales():
     assert np.all(tq >= np.linalg.norm(dq, axis=1) - 1e-12)
     assert np.all(tk >= np.linalg.norm(dk, axis=1) - 1e-12)
     assert np.all(tv >= np.linalg.norm(dv, axis=1) - 1e-12)
+
+
+@pytest.mark.parametrize("form", [la.FORM_NONCAUSAL, la.FORM_CAUSAL])
+def test_gradient_scale_bounds_terms_and_keeps_power(form):
+    """The rounding scale of a gradient row (its product with the states it
+    sees, in absolute values) dominates the norm of each exact term of the
+    row, and a row with a term dropped (planted here, in the oracle's own
+    arithmetic) still fails the metric by far more than the bf16 tolerance."""
+    from oracle.metrics import max_row_grad_err
+    rng = np.random.default_rng(21)
+    n, d = 300, 16
+    Q, K, V, G = (rng.standard_normal((n, d)) for _ in range(4))
+    dq, dk, dv, tq, tk, tv = bw.backward_dense(Q, K, V, G, form, scales=True)
+    A, B = la.phi(Q), la.phi(K)
+    vis = la.visible(n, form, None)
+    W = np.where(vis, A @ B.T, 0.0)
+    den = W.sum(axis=1)
+    out = (W @ V) / den[:, None]
+    gn, gden = G / den[:, None], -(G * out).sum(axis=1) / den
+    pq = bw.phi_grad(Q)
+    t1 = pq * (np.where(vis, gn @ V.T, 0.0) @ B)          # the gn . v term of dq
+    t2 = pq * (np.where(vis, gden[:, None], 0.0) @ B)     # the gden term of dq
+    assert np.allclose(t1 + t2, dq, atol=1e-10)
+    assert np.all(tq >= np.linalg.norm(t1, axis=1) - 1e-12)
+    assert np.all(tq >= np.linalg.norm(t2, axis=1) - 1e-12)
+    assert max_row_grad_err(t1, dq, tq) > 0.2             # gden term dropped
+    assert max_row_grad_err(t2, dq, tq) > 0.2             # gn . v term dropped
