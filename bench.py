@@ -58,7 +58,7 @@ CALL_KERNELS = {
     "noncausal_bwd": ["tc_kv_kernel", "kv_reduce_balanced_kernel", "tc_bwd_q_kernel", "kv_reduce_balanced_kernel",
                       "tc_bwd_kv_kernel"],
     "causal_bwd": ["tc_kv_kernel", "state_scan_kernel", "tc_bwd_causal_q_kernel", "state_scan_kernel",
-                   "bwd_kv_kernel"],
+                   "tc_bwd_causal_kv_kernel"],
 }
 # The same on the fp32 (CUDA-core) path.
 CALL_KERNELS_F32 = {
@@ -77,7 +77,7 @@ KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balan
                "state_scan_kernel": "scan", "tc_sweep": "sweep", "chunked_kernel": "sweep",
                "bin_kernel": "bin", "decode_kernel": "decode", "bwd_q_kernel": "bwd_q",
                "bwd_kv_kernel": "bwd_kv", "tc_bwd_q_kernel": "bwd_q", "tc_bwd_kv_kernel": "bwd_kv",
-               "tc_bwd_causal_q_kernel": "bwd_q"}
+               "tc_bwd_causal_q_kernel": "bwd_q", "tc_bwd_causal_kv_kernel": "bwd_kv"}
 
 
 def parse():

@@ -347,8 +347,11 @@ la_status backward_impl(const la_desc* desc, bool causal, const void* q, const v
                                      bp.block_tokens, bp.nblk, dq, gn, gden, grec, st)));
         }
         LA_TRY(cuda_status(state_exclusive_scan(p, grec, bp.nblk, nullptr, nullptr, st, true)));
+        if (tcq)
+            return cuda_status(tc_causal_backward_kv(p, q, k, v, gn, gden, grec, bp.block_tokens, bp.nblk, dk, dv,
+                                                     flags, st));
         return cuda_status(bwd_kv(p, true, q, k, v, gn, gden, grec, grec + (size_t)p.d * p.d, rec, rec,
-                                  bp.block_tokens, bp.nblk, dk, dv, st, tcq));
+                                  bp.block_tokens, bp.nblk, dk, dv, st));
     }
     float* S = at<float>(ws, L.sz);
     float* z = S + (size_t)p.bh() * p.d * p.d;

@@ -69,6 +69,11 @@ bool tc_causal_backward_supported(const Problem& p, int block_tokens);
 cudaError_t tc_causal_backward_q(const Problem& p, const void* q, const void* k, const void* v, const void* dout,
                                  const float* prefix, int block_tokens, int nblk, void* dq, void* gn, float* gden,
                                  float* grec, uint32_t* err, cudaStream_t st);
+// Second sweep (same support): from the blocks' suffix states (G, h)
+// (grec after the reverse exclusive scan), gn and gden, writes dk and dv.
+cudaError_t tc_causal_backward_kv(const Problem& p, const void* q, const void* k, const void* v, const void* gn,
+                                  const float* gden, const float* suffix, int block_tokens, int nblk, void* dk,
+                                  void* dv, uint32_t* err, cudaStream_t st);
 
 // [BH, N, d] bf16 viewed as 3-D for TMA: 64-column x `rows` boxes, 128-byte
 // swizzle, zero fill outside the tensor.
