@@ -12,8 +12,11 @@ pytestmark = pytest.mark.gpu
 
 # kernels per call on the bf16 tensor-core path (KV summary: partial records +
 # reduction; non-causal: those + readout; causal: block states, scan, sweep;
-# prefix mask: binning + the causal three; decode: one)
-TC_LAUNCHES = {"kv_summary": 2, "noncausal": 3, "causal": 3, "prefix": 4, "decode": 1}
+# prefix mask: binning + the causal three; decode: one; gradients: the
+# forward states, their reduction or scan, the dq sweep, the (G, h)
+# reduction or reverse scan, the dk/dv sweep)
+TC_LAUNCHES = {"kv_summary": 2, "noncausal": 3, "causal": 3, "prefix": 4, "decode": 1, "noncausal_bwd": 5,
+               "causal_bwd": 5}
 
 
 @pytest.fixture
@@ -33,13 +36,17 @@ def _calls(dev):
     q1, k1, v1 = (t[:, :, :1].contiguous() for t in (q, k, v))
     out1 = torch.empty_like(q1)
     desc = la._desc_of(q, "relu1", True)
-    ws = {op: la.workspace(desc, op, 64, dev) for op in ("kv_summary", "noncausal", "causal", "prefix")}
+    ws = {op: la.workspace(desc, op, 64, dev)
+          for op in ("kv_summary", "noncausal", "causal", "prefix", "noncausal_bwd", "causal_bwd")}
+    dout = torch.randn_like(q)
     return {
         "kv_summary": lambda: la.la_kv_summary(k, v, S, z, ws=ws["kv_summary"]),
         "noncausal": lambda: la.la_noncausal(q, k, v, out, ws=ws["noncausal"]),
         "causal": lambda: la.la_causal_chunked(q, k, v, out, 64, ws=ws["causal"]),
         "prefix": lambda: la.la_prefix_mask(q, k, v, m, out, 64, ws=ws["prefix"]),
         "decode": lambda: la.la_decode_step(q1, k1, v1, S, z, out1),
+        "noncausal_bwd": lambda: la.la_noncausal_backward(q, k, v, dout, ws=ws["noncausal_bwd"]),
+        "causal_bwd": lambda: la.la_causal_backward(q, k, v, dout, ws=ws["causal_bwd"]),
     }
 
 
