@@ -70,14 +70,28 @@ CALL_KERNELS_F32 = {
                       "bwd_kv_kernel"],
     "causal_bwd": ["kv_partial_kernel", "state_scan_kernel", "bwd_q_kernel", "state_scan_kernel", "bwd_kv_kernel"],
 }
-LAUNCHES = {k: len(v) for k, v in CALL_KERNELS.items()}
+
+
+def call_kernels(wl, dtype):
+    """The kernels of each call for this workload: the tables above, with the
+    non-causal form as one thread-block-cluster kernel where la_noncausal
+    takes that path (bf16, d = 64, B*H * 8 <= 288, N <= 8192)."""
+    if dtype != "bf16":
+        return CALL_KERNELS_F32
+    out = dict(CALL_KERNELS)
+    if wl.d == 64 and wl.B * wl.H * 8 <= 288 and wl.N <= 8192:
+        out["noncausal"] = ["tc_noncausal_cluster_kernel"]
+    return out
+
+
 # What each kernel does, for its algorithmic bytes (Step.kernel_bytes).
 KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balanced_kernel": "reduce",
                "state_reduce_kernel": "reduce", "tc_readout_kernel": "readout", "readout_kernel": "readout",
                "state_scan_kernel": "scan", "tc_sweep": "sweep", "chunked_kernel": "sweep",
                "bin_kernel": "bin", "decode_kernel": "decode", "bwd_q_kernel": "bwd_q",
                "bwd_kv_kernel": "bwd_kv", "tc_bwd_q_kernel": "bwd_q", "tc_bwd_kv_kernel": "bwd_kv",
-               "tc_bwd_causal_q_kernel": "bwd_q", "tc_bwd_causal_kv_kernel": "bwd_kv"}
+               "tc_bwd_causal_q_kernel": "bwd_q", "tc_bwd_causal_kv_kernel": "bwd_kv",
+               "tc_noncausal_cluster_kernel": "fused"}
 
 
 def parse():
@@ -242,7 +256,7 @@ class Step:
             causal = call == "causal_bwd"
             return {"kv": 2 * t, "bwd_q": (5 if causal else 3) * t,
                     "bwd_kv": (5 if causal else 4) * t}.get(role, 0)
-        return {"kv": 2 * t, "reduce": st, "readout": 2 * t + st, "scan": 0, "sweep": 4 * t,
+        return {"kv": 2 * t, "reduce": st, "readout": 2 * t + st, "scan": 0, "sweep": 4 * t, "fused": 4 * t,
                 "bin": self.B * self.N * 4, "decode": 2 * st + 4 * one}.get(role, 0)
 
     def host_io(self):
@@ -413,7 +427,7 @@ def run_ours(args, rank, world, local_rank):
 
     peaks = load_peaks()
     peak = peaks.get("hbm_gbs", 6650.0)
-    names = CALL_KERNELS if dtype == "bf16" else CALL_KERNELS_F32
+    names = call_kernels(wl, dtype)
     per_kernel = {}
     for name in per_call:
         s_call = per_call[name] / 1e3 / K
@@ -462,7 +476,7 @@ def run_ours(args, rank, world, local_rank):
                    "tokens_per_step_per_gpu": step.tokens},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": sum(LAUNCHES[n] for n, _ in calls) * K,
+        "gpu_launches": sum(len(names[n]) for n, _ in calls) * K,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": recorded_traffic(wl.name, dtype, f"{dom}/{di}"),
@@ -639,7 +653,8 @@ def record_traffic(csv_path, workload, dtype):
             rec["bytes"] += float(r[iv].replace(",", "")) * scale.get(r[iu], 1)
     seq = [launches[i] for i in sorted(launches)]
     forms = Step.ALL_FORMS if workload == "multi_head" else W.WORKLOADS[workload].forms
-    want = [(f, k) for f in forms for k in CALL_KERNELS[f]]
+    names = call_kernels(W.WORKLOADS[workload], dtype)
+    want = [(f, k) for f in forms for k in names[f]]
     for start in range(len(seq) - len(want), -1, -1):
         if all(k in seq[start + n]["name"] for n, (_, k) in enumerate(want)):
             break

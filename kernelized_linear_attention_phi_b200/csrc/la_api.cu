@@ -258,6 +258,9 @@ la_status la_noncausal(const la_desc* desc, const void* q, const void* k, const 
     LA_TRY(check_device());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     timing_begin(st);
+    // small problems: one kernel, a thread-block cluster per head
+    if (tc_noncausal_fused_supported(p))
+        return cuda_status(tc_noncausal_fused(p, q, k, v, out, S_out, z_out, at<uint32_t>(ws, 0), st));
     float* S = S_out;
     float* z = z_out;
     if (S == nullptr) {

@@ -28,6 +28,13 @@ KvBalanced kv_balanced_plan(const Problem& p);
 // d*d + d floats), then a fixed-order reduction into S [bh][d*d], z [bh][d].
 cudaError_t tc_kv_summary(const Problem& p, const void* k, const void* v, float* part, float* S,
                           float* z, uint32_t* err, cudaStream_t st);
+// Non-causal attention in one kernel for small problems (tc_fused.cu): bf16,
+// d = 64, B*H * 8 <= 288 (one wave of 8-CTA clusters, one per head),
+// N <= 8192. Writes
+// out and, when S / z are non-null, the KV summary [bh][d*d], [bh][d].
+bool tc_noncausal_fused_supported(const Problem& p);
+cudaError_t tc_noncausal_fused(const Problem& p, const void* q, const void* k, const void* v, void* out, float* S,
+                               float* z, uint32_t* err, cudaStream_t st);
 // Sums balanced-split records (slot cta * K + j, d*d + d floats each) per
 // head in CTA order into S [bh][d*d] and z [bh][d].
 cudaError_t tc_reduce_records(const Problem& p, const float* part, float* S, float* z, cudaStream_t st);

@@ -263,25 +263,38 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
                 fence_async_smem();
                 mbar_arrive(tdone + s);
             }
-            // column sums: the 16 threads of a column group add up their parts
+            // column sums: the 16 threads of a column group add up their parts;
+            // in a warp, lanes l, l^9, l^18, l^27 hold the same group
 #pragma unroll
             for (int b = 0; b < C::NB; ++b)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    red[(et * 2 + 0) * C::NB * 8 + b * 8 + e] = zk[b][e];
-                    red[(et * 2 + 1) * C::NB * 8 + b * 8 + e] = cv[b][e];
+                    zk[b][e] += __shfl_xor_sync(0xffffffffu, zk[b][e], 9);
+                    zk[b][e] += __shfl_xor_sync(0xffffffffu, zk[b][e], 18);
+                    cv[b][e] += __shfl_xor_sync(0xffffffffu, cv[b][e], 9);
+                    cv[b][e] += __shfl_xor_sync(0xffffffffu, cv[b][e], 18);
                 }
+            const int wq = et >> 5;  // warp of the group (0..3)
+            if (lane < 8) {
+                const int g = lane ^ ((4 * wq) & 7);  // group of lanes 0..7 in this warp
+#pragma unroll
+                for (int b = 0; b < C::NB; ++b)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        red[((wq * C::NB + b) * 8 + g) * 16 + e] = zk[b][e];
+                        red[((wq * C::NB + b) * 8 + g) * 16 + 8 + e] = cv[b][e];
+                    }
+            }
             named_bar(1, 128);
             float* rec = part + (size_t)sg.slot * REC;
             if (et < D) {
                 const int b = et / 64, g = (et % 64) / 8, e = et % 8;
                 float zs = relu ? (float)(sg.t1 - sg.t0) : 0.f;
                 float cs = 0.f;
-                for (int t = 0; t < 128; ++t) {
-                    if ((((t & 7) ^ ((t >> 3) & 7))) == g) {
-                        zs += red[(t * 2 + 0) * C::NB * 8 + b * 8 + e];
-                        cs += red[(t * 2 + 1) * C::NB * 8 + b * 8 + e];
-                    }
+#pragma unroll
+                for (int w4 = 0; w4 < 4; ++w4) {  // fixed order
+                    zs += red[((w4 * C::NB + b) * 8 + g) * 16 + e];
+                    cs += red[((w4 * C::NB + b) * 8 + g) * 16 + 8 + e];
                 }
                 rec[(size_t)D * D + et] = zs;
                 csum[et] = relu ? cs : 0.f;
