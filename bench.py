@@ -75,13 +75,29 @@ CALL_KERNELS_F32 = {
 def call_kernels(wl, dtype):
     """The kernels of each call for this workload: the tables above, with the
     non-causal form as one thread-block-cluster kernel where la_noncausal
-    takes that path (bf16, d = 64, B*H * 8 <= 288, N <= 8192)."""
+    takes that path (bf16, d = 64, B*H * 8 <= 288, N <= 8192), and without
+    the block-state scan kernel where the KV pass scans in its clusters."""
     if dtype != "bf16":
         return CALL_KERNELS_F32
     out = dict(CALL_KERNELS)
     if wl.d == 64 and wl.B * wl.H * 8 <= 288 and wl.N <= 8192:
         out["noncausal"] = ["tc_noncausal_cluster_kernel"]
+    if wl.d == 64 and block_count(wl) <= 16 and block_count(wl) * wl.B * wl.H <= 296:
+        # the KV pass scans the block states inside its clusters (prefix mask,
+        # causal gradients): no scan kernel
+        out["prefix"] = [k for k in out["prefix"] if k != "state_scan_kernel"]
+        out["causal_bwd"] = [k for i, k in enumerate(out["causal_bwd"]) if not (i == 1 and k == "state_scan_kernel")]
     return out
+
+
+def block_count(wl):
+    """Blocks per head of the chunked forms, as la_api.cu's block plan picks
+    them (one wave of 148 SMs x 2 CTAs, blocks of at least 256 tokens, a
+    multiple of 128)."""
+    per_sm = 1 if wl.d == 128 else 2
+    target = max(1, per_sm * 148 // (wl.B * wl.H))
+    bt = max(256, -(-(-(-wl.N // target)) // 128) * 128)
+    return -(-wl.N // bt)
 
 
 # What each kernel does, for its algorithmic bytes (Step.kernel_bytes).

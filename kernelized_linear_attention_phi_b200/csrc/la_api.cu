@@ -297,6 +297,8 @@ la_status causal_impl(const la_desc* desc, int32_t chunk, const void* q, const v
     // phase 1: per-block states; phase 2: exclusive prefix over blocks (and
     // the total); phase 3: each block's outputs from its prefix state.
     uint32_t* flags = at<uint32_t>(ws, 0);
+    // (the in-cluster scan of tc_kv_blocks_scan measured no faster here: the
+    // separate scan overlaps the sweep's prologue)
     if (tc_supported(p)) {
         LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
     } else {
@@ -335,12 +337,16 @@ la_status backward_impl(const la_desc* desc, bool causal, const void* q, const v
     if (causal) {
         float* part = at<float>(ws, L.part);
         uint32_t* flags = at<uint32_t>(ws, 0);
-        if (tc_supported(p)) {
-            LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
+        if (tc_kv_scan_supported(p, bp.block_tokens, bp.nblk)) {
+            LA_TRY(cuda_status(tc_kv_blocks_scan(p, k, v, bp.block_tokens, bp.nblk, part, nullptr, nullptr, flags, st)));
         } else {
-            LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
+            if (tc_supported(p)) {
+                LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
+            } else {
+                LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
+            }
+            LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
         }
-        LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
         const bool tcq = tc_causal_backward_supported(p, bp.block_tokens);
         if (tcq) {  // tensor cores; gn in bf16
             LA_TRY(cuda_status(tc_causal_backward_q(p, q, k, v, dout, part, bp.block_tokens, bp.nblk, dq, gn, gden,
@@ -427,15 +433,19 @@ la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, cons
     int32_t* bins = at<int32_t>(ws, L.bins);
     float* part = at<float>(ws, L.part);
     // the binning reads only m: launched after the KV pass it runs beside it
-    // (bin_kernel waits for its predecessor only at its end); the scan waits
-    // for both
-    if (tc) {
+    // (bin_kernel waits for its predecessor only at its end); the next
+    // kernel (the scan, or the sweep when the KV pass scans in-cluster)
+    // waits for both
+    const bool cscan = tc_kv_scan_supported(p, bp.block_tokens, bp.nblk);
+    if (cscan) {
+        LA_TRY(cuda_status(tc_kv_blocks_scan(p, k, v, bp.block_tokens, bp.nblk, part, nullptr, nullptr, flags, st)));
+    } else if (tc) {
         LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
     } else {
         LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
     }
     LA_TRY(cuda_status(bin_queries(p, m, kchunk, nbins, perm, bins, msort, flags, st)));
-    LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
+    if (!cscan) LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, nullptr, nullptr, st)));
     if (tc)
         return cuda_status(tc_chunked(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, perm, bins,
                                       msort, nbins, out, flags, st));

@@ -42,6 +42,13 @@ cudaError_t tc_reduce_records(const Problem& p, const float* part, float* S, flo
 // over tokens [block*block_tokens, ...); block_tokens must be a multiple of 128.
 cudaError_t tc_kv_blocks(const Problem& p, const void* k, const void* v, int block_tokens, int nblk,
                          float* part, uint32_t* err, cudaStream_t st);
+// tc_kv_blocks followed by the exclusive block-state scan, in one kernel with
+// a thread-block cluster per head (bf16, d = 64, nblk <= 16, nblk * B*H <=
+// 296): part[bh*nblk + blk] receives the prefix of the blocks before blk
+// (what state_exclusive_scan leaves), S_total / z_total (nullable) the total.
+bool tc_kv_scan_supported(const Problem& p, int block_tokens, int nblk);
+cudaError_t tc_kv_blocks_scan(const Problem& p, const void* k, const void* v, int block_tokens, int nblk, float* part,
+                              float* S_total, float* z_total, uint32_t* err, cudaStream_t st);
 // Same contract as simt_readout.
 cudaError_t tc_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,
                        uint32_t* err, cudaStream_t st);

@@ -106,23 +106,52 @@ __device__ __forceinline__ Seg kv_seg(const KvWork& w, int N, int j) {
 // ---------------------------------------------------------------------------
 // KV summary
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool SCAN = false>
 struct KvCfg {
     static constexpr int NB = D / 64;                 // 64-column boxes per tile
     static constexpr int TILE = kTile * D * 2;        // bytes of a K or V tile
-    static constexpr int STAGES = D == 64 ? 4 : 3;
+    // with the in-cluster scan (short blocks, several CTAs per SM) two stages
+    static constexpr int STAGES = SCAN ? 3 : (D == 64 ? 4 : 3);
     static constexpr int RED = 128 * 2 * NB * 8 * 4 + D * 4;  // per-thread column sums, colsum(V)
     static constexpr uint32_t TMEM_COLS = D <= 64 ? 64u : 128u;
     static constexpr int BARS = 3 * STAGES + 1;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * 2 * TILE + RED + 8 * BARS + 16;
     static_assert(SMEM <= 227 * 1024, "shared memory");
+    // the block's record is kept in the stage buffers once its MMAs are done
+    static_assert(!SCAN || (size_t)STAGES * 2 * TILE >= (size_t)(D * D + D) * 4, "record fits the stages");
+    // two resident CTAs per SM with the in-cluster scan: 228 KiB per SM, 1 KiB reserved per CTA
+    static_assert(!SCAN || 2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
-template <int D, int PHI>
-__global__ void __launch_bounds__(kThreads, 1)
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+// Cluster-wide barrier: arrive (release) then wait (acquire), every thread.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive;" ::: "memory");
+    asm volatile("barrier.cluster.wait;" ::: "memory");
+}
+
+// SCAN (blocks mode, one cluster of nblk CTAs per head): instead of its own
+// record each CTA writes the exclusive prefix of the records of its head,
+// computed across the cluster (see the end of the kernel); S_total, z_total
+// (nullable) receive the head's total.
+template <int D, int PHI, bool SCAN = false>
+__global__ void __launch_bounds__(kThreads, SCAN ? 2 : 1)
 tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV, int N,
-             KvWork w, float* __restrict__ part, uint32_t* __restrict__ err) {
-    using C = KvCfg<D>;
+             KvWork w, float* __restrict__ part, uint32_t* __restrict__ err, float* __restrict__ S_total,
+             float* __restrict__ z_total) {
+    using C = KvCfg<D, SCAN>;
     constexpr size_t REC = (size_t)D * D + D;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles = align1024(smem_raw);
@@ -286,7 +315,9 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
                     }
             }
             named_bar(1, 128);
-            float* rec = part + (size_t)sg.slot * REC;
+            // SCAN: the record goes to the stage buffers, after the MMAs are done
+            float* rec = SCAN ? reinterpret_cast<float*>(tiles) : part + (size_t)sg.slot * REC;
+            float zrow = 0.f;
             if (et < D) {
                 const int b = et / 64, g = (et % 64) / 8, e = et % 8;
                 float zs = relu ? (float)(sg.t1 - sg.t0) : 0.f;
@@ -296,7 +327,8 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
                     zs += red[((w4 * C::NB + b) * 8 + g) * 16 + e];
                     cs += red[((w4 * C::NB + b) * 8 + g) * 16 + 8 + e];
                 }
-                rec[(size_t)D * D + et] = zs;
+                if (!SCAN) rec[(size_t)D * D + et] = zs;
+                zrow = zs;
                 csum[et] = relu ? cs : 0.f;
             }
             named_bar(1, 128);
@@ -334,9 +366,52 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
                                         __uint_as_float(r[4 * q4 + 2]) + csum[c0 + 4 * q4 + 2],
                                         __uint_as_float(r[4 * q4 + 3]) + csum[c0 + 4 * q4 + 3]);
             }
+            if (SCAN && et < D) rec[(size_t)D * D + et] = zrow;
             tc_fence_before();
             named_bar(1, 128);  // `red` is reused by the next segment
         }
+    }
+    if constexpr (SCAN) {
+        // Exclusive prefix of the head's block records across the cluster
+        // (rank = block): CTA r takes float4s [r*chunk, (r+1)*chunk) of the
+        // record, reads them from every rank in order and writes rank r''s
+        // prefix (the sum over ranks before it) to its record slot, then the
+        // total. Every thread of every CTA reaches both cluster barriers.
+        cluster_sync();
+        if (warp >= 2) {
+            const int et = threadIdx.x - 64;
+            const int nblk = w.nblk, bh = blockIdx.y, r = blockIdx.x;
+            constexpr int E4 = (D * D + D) / 4;
+            const int chunk = (E4 + nblk - 1) / nblk;
+            const float* recs = reinterpret_cast<const float*>(tiles);
+            for (int f = r * chunk + et; f < min(E4, (r + 1) * chunk); f += 128) {
+                float4 x[16];
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr)
+                    if (rr < nblk) x[rr] = ld_cluster_f4(cluster_addr(recs + 4 * f, rr));
+                float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    if (rr < nblk) {
+                        reinterpret_cast<float4*>(part + ((size_t)bh * nblk + rr) * REC)[f] = run;
+                        run.x += x[rr].x;
+                        run.y += x[rr].y;
+                        run.z += x[rr].z;
+                        run.w += x[rr].w;
+                    }
+                }
+                if (S_total != nullptr) {
+                    const float t[4] = {run.x, run.y, run.z, run.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int idx = 4 * f + q;
+                        if (idx < D * D) S_total[(size_t)bh * D * D + idx] = t[q];
+                        else z_total[(size_t)bh * D + (idx - D * D)] = t[q];
+                    }
+                }
+            }
+        }
+        cluster_sync();  // no CTA leaves while another reads its record
     }
     tc_fence_before();
     __syncthreads();
@@ -608,7 +683,38 @@ cudaError_t launch_kv_phi(const Problem& p, const CUtensorMap& mk, const CUtenso
     constexpr size_t smem = KvCfg<D>::SMEM;
     cudaError_t e = ensure_smem<tc_kv_kernel<D, PHI>>(smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(tc_kv_kernel<D, PHI>, grid, dim3(kThreads), smem, st, mk, mv, p.N, w, part, err);
+    return launch_pdl(tc_kv_kernel<D, PHI>, grid, dim3(kThreads), smem, st, mk, mv, p.N, w, part, err,
+                      static_cast<float*>(nullptr), static_cast<float*>(nullptr));
+}
+
+// Blocks mode with the block-state scan inside: one cluster of nblk CTAs per head.
+template <int D, int PHI>
+cudaError_t launch_kv_scan(const Problem& p, const CUtensorMap& mk, const CUtensorMap& mv, const KvWork& w,
+                           float* part, float* S_total, float* z_total, uint32_t* err, cudaStream_t st) {
+    constexpr size_t smem = KvCfg<D, true>::SMEM;
+    cudaError_t e = ensure_smem<tc_kv_kernel<D, PHI, true>>(smem);
+    if (e != cudaSuccess) return e;
+    if (w.nblk > 8) {
+        e = cudaFuncSetAttribute(tc_kv_kernel<D, PHI, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)w.nblk, (unsigned)p.bh());
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)w.nblk;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, tc_kv_kernel<D, PHI, true>, mk, mv, p.N, w, part, err, S_total, z_total);
+    if (e == cudaSuccess) timing_mark(st);
+    return e;
 }
 
 // one kernel per feature map (see phi8)
@@ -674,6 +780,30 @@ cudaError_t tc_reduce_records(const Problem& p, const float* part, float* S, flo
     const int rec4 = (p.d * p.d + p.d) / 4;
     return launch_pdl(kv_reduce_balanced_kernel, dim3((rec4 + 127) / 128, (unsigned)p.bh()), dim3(128), 0, st, part,
                       w, p.d, S, z);
+}
+
+bool tc_kv_scan_supported(const Problem& p, int block_tokens, int nblk) {
+    // one cluster per head (at most 16 CTAs), one wave at two CTAs per SM
+    return tc_supported(p) && p.d == 64 && block_tokens % kTile == 0 && nblk >= 1 && nblk <= 16 &&
+           (long long)nblk * p.bh() <= 2 * 148;
+}
+
+cudaError_t tc_kv_blocks_scan(const Problem& p, const void* k, const void* v, int block_tokens, int nblk, float* part,
+                              float* S_total, float* z_total, uint32_t* err, cudaStream_t st) {
+    if (!tc_kv_scan_supported(p, block_tokens, nblk)) return cudaErrorInvalidValue;
+    KvWork w{};
+    w.balanced = 0;
+    w.block_tokens = block_tokens;
+    w.nblk = nblk;
+    CUtensorMap mk, mv;
+    cudaError_t e = make_map(&mk, k, 64, p.N, p.bh(), kTile);
+    if (e == cudaSuccess) e = make_map(&mv, v, 64, p.N, p.bh(), kTile);
+    if (e != cudaSuccess) return e;
+    switch (p.phi) {  // one kernel per feature map (see phi8)
+        case PHI_RELU1: return launch_kv_scan<64, PHI_RELU1>(p, mk, mv, w, part, S_total, z_total, err, st);
+        case PHI_ELU1: return launch_kv_scan<64, PHI_ELU1>(p, mk, mv, w, part, S_total, z_total, err, st);
+        default: return launch_kv_scan<64, PHI_IDENTITY>(p, mk, mv, w, part, S_total, z_total, err, st);
+    }
 }
 
 cudaError_t tc_kv_blocks(const Problem& p, const void* k, const void* v, int block_tokens, int nblk, float* part,

@@ -10,14 +10,14 @@ from tests.gpu_util import qkv
 
 pytestmark = pytest.mark.gpu
 
-# kernels per call on the bf16 tensor-core path at this size (KV summary:
-# partial records + reduction; non-causal: one thread-block-cluster kernel
-# (8 heads, d = 64); causal: block states, scan, sweep;
-# prefix mask: binning + the causal three; decode: one; gradients: the
-# forward states, their reduction or scan, the dq sweep, the (G, h)
-# reduction or reverse scan, the dk/dv sweep)
-TC_LAUNCHES = {"kv_summary": 2, "noncausal": 1, "causal": 3, "prefix": 4, "decode": 1, "noncausal_bwd": 5,
-               "causal_bwd": 5}
+# kernels per call on the bf16 tensor-core path at this size (8 heads of
+# 1024 tokens, d = 64): KV summary: partial records + reduction; non-causal:
+# one thread-block-cluster kernel; causal: block states, scan, sweep; prefix
+# mask: block states scanned inside a cluster per head, binning, sweep;
+# decode: one; gradients: forward states (non-causal: + reduction; causal:
+# scanned in-cluster), dq sweep, (G, h) reduction or reverse scan, dk/dv sweep
+TC_LAUNCHES = {"kv_summary": 2, "noncausal": 1, "causal": 3, "prefix": 3, "decode": 1, "noncausal_bwd": 5,
+               "causal_bwd": 4}
 
 
 @pytest.fixture
