@@ -140,13 +140,20 @@ WsLayout ws_layout(const Problem& p, int op) {
         const BlockPlan bp = block_plan(p);
         L.part = off;
         if (op == LA_OP_NONCAUSAL_BWD) {
-            // the KV summary's own scratch where kv_summary_impl expects it,
-            // then the totals (S, z) and (G, h)
+            // the KV summary's own scratch where kv_summary_impl expects it
+            // (on the tensor cores it then takes the gradient kernels' (G, h)
+            // records, whose split may have more slots), then the totals
+            // (S, z) and (G, h)
             off = ws_layout(p, LA_OP_KV_SUMMARY).total;
+            if (tc_supported(p)) off = std::max(off, round_up(L.part + tc_backward_record_slots(p) * rec, kAlign));
             L.sz = off;
             off = round_up(off + (size_t)p.bh() * rec, kAlign);
             L.gtot = off;
             off = round_up(off + (size_t)p.bh() * rec, kAlign);
+            if (tc_supported(p)) {  // the CUDA-core path's block states and gn, gden are not used
+                L.total = off;
+                return L;
+            }
         } else {
             off = round_up(off + (size_t)p.bh() * bp.nblk * rec, kAlign);  // block states (S, z)
         }

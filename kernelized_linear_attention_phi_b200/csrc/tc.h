@@ -22,7 +22,9 @@ struct KvBalanced {
     int G, K, tph;     // CTAs, record slots per CTA, tiles per head
     long long total;   // bh * tph
 };
-KvBalanced kv_balanced_plan(const Problem& p);
+// Balanced split of the bh * tph (head, 128-token tile) pairs over
+// min(total, 148 * per_sm) CTAs in contiguous ranges.
+KvBalanced kv_balanced_plan(const Problem& p, int per_sm = 1);
 
 // KV summary in balanced mode: partial records into `part` (G*K slots of
 // d*d + d floats), then a fixed-order reduction into S [bh][d*d], z [bh][d].
@@ -35,9 +37,10 @@ cudaError_t tc_kv_summary(const Problem& p, const void* k, const void* v, float*
 bool tc_noncausal_fused_supported(const Problem& p);
 cudaError_t tc_noncausal_fused(const Problem& p, const void* q, const void* k, const void* v, void* out, float* S,
                                float* z, uint32_t* err, cudaStream_t st);
-// Sums balanced-split records (slot cta * K + j, d*d + d floats each) per
-// head in CTA order into S [bh][d*d] and z [bh][d].
-cudaError_t tc_reduce_records(const Problem& p, const float* part, float* S, float* z, cudaStream_t st);
+// Sums balanced-split records of plan w (slot cta * K + j, d*d + d floats
+// each) per head in CTA order into S [bh][d*d] and z [bh][d].
+cudaError_t tc_reduce_records(const Problem& p, const KvBalanced& w, const float* part, float* S, float* z,
+                              cudaStream_t st);
 // KV summary per block: CTA (block, head) writes record (head*nblk + block)
 // over tokens [block*block_tokens, ...); block_tokens must be a multiple of 128.
 cudaError_t tc_kv_blocks(const Problem& p, const void* k, const void* v, int block_tokens, int nblk,
@@ -69,8 +72,9 @@ cudaError_t tc_chunked_t(const Problem& p, const void* q, const void* k, const v
                          const int32_t* msort, int nbins, void* out, uint32_t* err, cudaStream_t st);
 
 // Gradients of the non-causal form (tc_bwd.cu): S, z are the KV summary of
-// the forward; `part` holds kv_balanced_plan(p) record slots, (G, h)
+// the forward; `part` holds tc_backward_record_slots(p) records, (G, h)
 // [bh][d*d], [bh][d] receive the reduced records. Writes dq, dk, dv.
+size_t tc_backward_record_slots(const Problem& p);
 cudaError_t tc_noncausal_backward(const Problem& p, const void* q, const void* k, const void* v, const void* dout,
                                   const float* S, const float* z, float* part, float* G, float* h, void* dq,
                                   void* dk, void* dv, uint32_t* err, cudaStream_t st);

@@ -93,12 +93,17 @@ struct BqCfg {
     static constexpr int BARS = 3 * STAGES + 4 * 2 + 2;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 2 * BS + 2 * BZ + 2 * BG + STAGES * SGN + ZF +
                                    8 * BARS + 16;
+    // CTAs an SM holds (TMEM, shared memory and, through the launch bounds,
+    // registers): at d = 64 a second CTA hides the load of a stage behind
+    // the other CTA's epilogues
+    static constexpr int PER_SM = D == 64 ? 2 : 1;
     static_assert(COL_H + 16 <= (int)TMEM_COLS, "TMEM");
-    static_assert(SMEM <= 227 * 1024, "shared memory");
+    static_assert(PER_SM * TMEM_COLS <= 512, "TMEM per SM");
+    static_assert(PER_SM * (SMEM + 1024) <= 228 * 1024, "shared memory");
 };
 
 template <int D, int PHI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, BqCfg<D>::PER_SM)
 tc_bwd_q_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mGo,
                 const __grid_constant__ CUtensorMap mDq, const float* __restrict__ S, const float* __restrict__ z,
                 KvBalanced w, int normalize, float* __restrict__ part, uint32_t* __restrict__ err) {
@@ -413,11 +418,14 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             tc_fence_before();
             mbar_arrive(g_free);
         };
+        // gn of tile it before phi of tile it + 1: the load of it + 1 (issued
+        // once tile it - 1 was stored) lands meanwhile, and the dA MMA of
+        // tile it runs under the transform
         int seg = 0;
         if (ntile > 0) transform(0);
         for (int it = 0; it < ntile; ++it) {
-            if (it + 1 < ntile) transform(it + 1);
             const float gden = epi_gn(it);
+            if (it + 1 < ntile) transform(it + 1);
             epi_dq(it, gden);
             const long long g = lo + it;
             if (it + 1 == ntile || (g + 1) % w.tph == 0) epi_g(seg++);
@@ -629,10 +637,12 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
                 mbar_arrive(empty + s);
             }
         };
+        // the epilogue of tile it before phi of tile it + 1, whose load
+        // (issued once tile it - 1 was stored) lands meanwhile
         if (ntile > 0) transform(0);
         for (int it = 0; it < ntile; ++it) {
-            if (it + 1 < ntile) transform(it + 1);
             epilogue(it);
+            if (it + 1 < ntile) transform(it + 1);
         }
         if (et == 0) bulk_wait0();
     }
@@ -657,12 +667,12 @@ cudaError_t launch_bwd(const Problem& p, const void* q, const void* k, const voi
     if (e == cudaSuccess) e = make_map(&mdk, dk, D, p.N, p.bh(), kTile);
     if (e == cudaSuccess) e = make_map(&mdv, dv, D, p.N, p.bh(), kTile);
     if (e != cudaSuccess) return e;
-    const KvBalanced w = kv_balanced_plan(p);
+    const KvBalanced w = kv_balanced_plan(p, BqCfg<D>::PER_SM);
     e = ensure_smem<tc_bwd_q_kernel<D, PHI>>(BqCfg<D>::SMEM);
     if (e == cudaSuccess)
         e = launch_pdl(tc_bwd_q_kernel<D, PHI>, dim3(w.G), dim3(kThreads), BqCfg<D>::SMEM, st, mq, mg, mdq, S, z, w,
                        p.normalize, part, err);
-    if (e == cudaSuccess) e = tc_reduce_records(p, part, G, h, st);
+    if (e == cudaSuccess) e = tc_reduce_records(p, w, part, G, h, st);
     if (e != cudaSuccess) return e;
     e = ensure_smem<tc_bwd_kv_kernel<D, PHI>>(BkCfg<D>::SMEM);
     if (e != cudaSuccess) return e;
@@ -683,6 +693,11 @@ cudaError_t bwd_phi(const Problem& p, const void* q, const void* k, const void* 
 }
 
 }  // namespace
+
+size_t tc_backward_record_slots(const Problem& p) {
+    const KvBalanced w = kv_balanced_plan(p, p.d == 64 ? BqCfg<64>::PER_SM : BqCfg<128>::PER_SM);
+    return (size_t)w.G * w.K;
+}
 
 cudaError_t tc_noncausal_backward(const Problem& p, const void* q, const void* k, const void* v, const void* dout,
                                   const float* S, const float* z, float* part, float* G, float* h, void* dq,

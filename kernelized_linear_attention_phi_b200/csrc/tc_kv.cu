@@ -34,11 +34,11 @@
 
 namespace la {
 
-KvBalanced kv_balanced_plan(const Problem& p) {
+KvBalanced kv_balanced_plan(const Problem& p, int per_sm) {
     KvBalanced w;
     w.tph = (p.N + tc::kTile - 1) / tc::kTile;
     w.total = p.bh() * w.tph;
-    w.G = (int)std::min<long long>(w.total, 148);
+    w.G = (int)std::min<long long>(w.total, 148LL * per_sm);
     const long long per = (w.total + w.G - 1) / w.G;  // most tiles a CTA gets
     w.K = (int)std::min<long long>(p.bh(), (per + w.tph - 1) / w.tph + 1);
     return w;
@@ -775,8 +775,8 @@ cudaError_t tc_kv_summary(const Problem& p, const void* k, const void* v, float*
                       part, w.b, p.d, S, z);
 }
 
-cudaError_t tc_reduce_records(const Problem& p, const float* part, float* S, float* z, cudaStream_t st) {
-    const KvBalanced w = kv_balanced_plan(p);
+cudaError_t tc_reduce_records(const Problem& p, const KvBalanced& w, const float* part, float* S, float* z,
+                              cudaStream_t st) {
     const int rec4 = (p.d * p.d + p.d) / 4;
     return launch_pdl(kv_reduce_balanced_kernel, dim3((rec4 + 127) / 128, (unsigned)p.bh()), dim3(128), 0, st, part,
                       w, p.d, S, z);
