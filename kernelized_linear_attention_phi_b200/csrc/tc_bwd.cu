@@ -91,8 +91,15 @@ struct BqCfg {
     static constexpr int COL_G = 2 * ACC, COL_H = COL_G + D;
     static constexpr uint32_t TMEM_COLS = D == 64 ? 256u : 512u;
     static constexpr int BARS = 3 * STAGES + 4 * 2 + 2;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 2 * BS + 2 * BZ + 2 * BG + STAGES * SGN + ZF +
-                                   8 * BARS + 16;
+    // d = 64: dq is staged in a tile of its own, so a stage is free for the
+    // next load as soon as the MMAs have read it (for relu+1 and identity,
+    // whose derivative comes from the sign bits; elu+1's reads phi(Q) back,
+    // so there the stage also waits for the dq epilogue). At d = 128 there is
+    // no room for it and dq is written over the dO tile.
+    static constexpr bool STG_DQ = D == 64;
+    static constexpr int STG = STG_DQ ? TILE : 0;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + STG + 2 * BS + 2 * BZ + 2 * BG + STAGES * SGN +
+                                   ZF + 8 * BARS + 16;
     // CTAs an SM holds (TMEM, shared memory and, through the launch bounds,
     // registers): at d = 64 a second CTA hides the load of a stage behind
     // the other CTA's epilogues
@@ -100,6 +107,7 @@ struct BqCfg {
     static_assert(COL_H + 16 <= (int)TMEM_COLS, "TMEM");
     static_assert(PER_SM * TMEM_COLS <= 512, "TMEM per SM");
     static_assert(PER_SM * (SMEM + 1024) <= 228 * 1024, "shared memory");
+    static_assert(STAGE % 1024 == 0 && STG % 1024 == 0 && BS % 1024 == 0, "1024-byte aligned swizzled tiles");
 };
 
 template <int D, int PHI>
@@ -110,14 +118,16 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     using C = BqCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* stages = align1024(smem_raw);
-    uint8_t* bS = stages + C::STAGES * C::STAGE;
+    uint8_t* stg = stages + C::STAGES * C::STAGE;  // dq staging (STG_DQ)
+    uint8_t* bS = stg + C::STG;
     uint8_t* bZ = bS + 2 * C::BS;
     uint8_t* bG = bZ + 2 * C::BZ;
     uint8_t* sgn = bG + 2 * C::BG;
     float* zf = reinterpret_cast<float*>(sgn + C::STAGES * C::SGN);
     uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(zf) + C::ZF);
     uint64_t* tdone = full + C::STAGES;    // phi(Q) and the head's S, z operands ready
-    uint64_t* empty = tdone + C::STAGES;   // MMA done with the stage and dq stored from it
+    uint64_t* empty = tdone + C::STAGES;   // MMA done with the stage (and, see STG_DQ, dq done with it)
+    constexpr uint32_t kEmptyArrivals = (C::STG_DQ && PHI != PHI_ELU1) ? 1u : 2u;
     uint64_t* acc_full = empty + C::STAGES;  // [2] O, den
     uint64_t* gn_ready = acc_full + 2;       // [2] GN and gden operands written (O read)
     uint64_t* da_full = gn_ready + 2;        // [2] dA (and the tile's G, h terms) done
@@ -137,7 +147,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(full + s, 1);
             mbar_init(tdone + s, 128);
-            mbar_init(empty + s, 2);
+            mbar_init(empty + s, kEmptyArrivals);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(acc_full + a, 1);
@@ -335,16 +345,21 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             mbar_arrive(gn_ready + ab);
             return gden;
         };
-        // dq of row r over the dO tile, then the tile's TMA store
+        // dq of row r into the staging tile (STG_DQ) or over the dO tile,
+        // then the tile's TMA store
         auto epi_dq = [&](int it, float gden) {
             const int ab = it & 1, s = it % C::STAGES;
             const long long g = lo + it;
             const int buf = (int)((g / w.tph - h0) & 1);
+            if (C::STG_DQ) {  // the previous tile's store has read the staging tile
+                if (et == 0) bulk_wait_read0();
+                named_bar(2, 128);
+            }
             ok = ok && mbar_wait(da_full + ab, (it >> 1) & 1, err);
             tc_fence_after();
             const uint32_t acc = tmem + ab * C::ACC + lane_base;
             uint8_t* qt = stages + s * C::STAGE;
-            uint8_t* gt = qt + C::TILE;
+            uint8_t* gt = C::STG_DQ ? stg : qt + C::TILE;
             const uint8_t* sg = sgn + s * C::SGN + r * (D / 8);
             const float* zb = zf + buf * D;
 #pragma unroll
@@ -367,16 +382,16 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             tc_fence_before();
             mbar_arrive(acc_empty + ab);
             fence_async_smem();
-            named_bar(2, 128);  // the dq tile is complete and nothing else reads the stage
+            named_bar(2, 128);  // the dq tile is complete and no thread reads the stage any more
             if (et == 0) {
                 if (ok) {
 #pragma unroll
                     for (int b = 0; b < C::NB; ++b)
                         tma_store_3d(&mDq, gt + b * kTile * 128, b * 64, (int)(g % w.tph) * kTile, (int)(g / w.tph));
                     bulk_commit();
-                    bulk_wait_read0();
+                    if (!C::STG_DQ) bulk_wait_read0();  // the store reads the stage
                 }
-                mbar_arrive(empty + s);
+                if (kEmptyArrivals == 2) mbar_arrive(empty + s);
             }
         };
         // the segment's (G, h) from TMEM into its record (S, z layout: G[d_k][d_v], h[d_k])
