@@ -34,38 +34,6 @@ using namespace tc;
 constexpr int kThreads = 192;
 constexpr int kCluster = 8;
 
-__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
-}
-__device__ __forceinline__ float ld_cluster_f(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_cluster_u4(uint32_t addr, const uint4& v) {
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
-                 "r"(v.w)
-                 : "memory");
-}
-__device__ __forceinline__ void st_cluster_u16(uint32_t addr, uint16_t v) {
-    asm volatile("st.shared::cluster.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
-}
-// Cluster-wide barrier: arrive (release) then wait (acquire), every thread.
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive;" ::: "memory");
-    asm volatile("barrier.cluster.wait;" ::: "memory");
-}
-
 struct FnCfg {
     static constexpr int D = 64;
     static constexpr int TILE = kTile * D * 2;   // one [128 x 64] bf16 tile
@@ -434,23 +402,8 @@ cudaError_t launch_fused(const Problem& p, const CUtensorMap& mk, const CUtensor
                          const CUtensorMap& mo, int tpc, float* S, float* z, uint32_t* err, cudaStream_t st) {
     cudaError_t e = ensure_smem<tc_noncausal_cluster_kernel<PHI>>(FnCfg::SMEM);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kCluster, (unsigned)p.bh());
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = FnCfg::SMEM;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = kCluster;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, tc_noncausal_cluster_kernel<PHI>, mk, mv, mq, mo, p.N, tpc, p.normalize, S, z, err);
-    if (e == cudaSuccess) timing_mark(st);
-    return e;
+    return launch_cluster_pdl(tc_noncausal_cluster_kernel<PHI>, dim3(kCluster, (unsigned)p.bh()), dim3(kThreads),
+                              FnCfg::SMEM, st, (unsigned)kCluster, mk, mv, mq, mo, p.N, tpc, p.normalize, S, z, err);
 }
 
 }  // namespace

@@ -123,25 +123,6 @@ struct KvCfg {
     static_assert(!SCAN || 2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
-__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
-}
-// Cluster-wide barrier: arrive (release) then wait (acquire), every thread.
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive;" ::: "memory");
-    asm volatile("barrier.cluster.wait;" ::: "memory");
-}
-
 // SCAN (blocks mode, one cluster of nblk CTAs per head): instead of its own
 // record each CTA writes the exclusive prefix of the records of its head,
 // computed across the cluster (see the end of the kernel); S_total, z_total
@@ -692,29 +673,10 @@ template <int D, int PHI>
 cudaError_t launch_kv_scan(const Problem& p, const CUtensorMap& mk, const CUtensorMap& mv, const KvWork& w,
                            float* part, float* S_total, float* z_total, uint32_t* err, cudaStream_t st) {
     constexpr size_t smem = KvCfg<D, true>::SMEM;
-    cudaError_t e = ensure_smem<tc_kv_kernel<D, PHI, true>>(smem);
+    const cudaError_t e = ensure_smem<tc_kv_kernel<D, PHI, true>>(smem);
     if (e != cudaSuccess) return e;
-    if (w.nblk > 8) {
-        e = cudaFuncSetAttribute(tc_kv_kernel<D, PHI, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)w.nblk, (unsigned)p.bh());
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = (unsigned)w.nblk;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, tc_kv_kernel<D, PHI, true>, mk, mv, p.N, w, part, err, S_total, z_total);
-    if (e == cudaSuccess) timing_mark(st);
-    return e;
+    return launch_cluster_pdl(tc_kv_kernel<D, PHI, true>, dim3((unsigned)w.nblk, (unsigned)p.bh()), dim3(kThreads),
+                              smem, st, (unsigned)w.nblk, mk, mv, p.N, w, part, err, S_total, z_total);
 }
 
 // one kernel per feature map (see phi8)

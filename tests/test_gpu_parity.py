@@ -271,3 +271,29 @@ def test_causal_prefill_then_decode(dt, d, phi):
     assert oracle.max_row_rel_err(f64(got), ref) < TOL[DT[dt]]
     ref_pre = oracle.batched(oracle.causal, Q[:, :, :N0], K[:, :, :N0], V[:, :, :N0], phi_kind=phi)
     assert oracle.max_row_rel_err(f64(out), ref_pre) < TOL[DT[dt]]
+
+
+@pytest.mark.parametrize("B,H,N", [(1, 16, 4096), (1, 2, 2300), (4, 37, 512), (1, 1, 64)])
+def test_causal_and_prefix_block_counts(B, H, N):
+    """bf16, d = 64 with 16, 9, 2 and 1 blocks per head (148 heads of 2
+    blocks fill the wave; the prefix mask scans the block states inside a
+    cluster per head, up to the non-portable size 16): 64- and 128-token
+    chunks agree with each other and with the oracle, the prefill's outputs
+    are those of the causal call and its state is the KV summary."""
+    d = 64
+    q, k, v = qkv(B, H, N, d, "bf16", seed=B + H + N)
+    ref = oracle.batched(oracle.causal, f64(q), f64(k), f64(v))
+    out = la.la_causal_chunked(q, k, v, chunk=64)
+    assert oracle.max_row_rel_err(f64(out), ref) < 2e-2
+    assert oracle.max_row_rel_err(f64(out), f64(la.la_causal_chunked(q, k, v, chunk=128))) < 2e-2
+    out_p, S, z = la.la_causal_prefill(q, k, v, chunk=64)
+    assert torch.equal(out_p, out)
+    S_ref, z_ref = oracle.kv_summary_batched(f64(k), f64(v))
+    assert oracle.max_row_rel_err(f64(S), S_ref) < 1e-4
+    np.testing.assert_allclose(f64(z), z_ref, rtol=1e-4)
+    m = workloads.prefix_mask_uniform(B, N, seed=N, device="cuda")
+    ws = la.workspace(la._desc_of(q, "relu1", True), "prefix", 64)
+    out_m = la.la_prefix_mask(q, k, v, m, chunk=64, ws=ws)
+    assert la.la_last_error(ws) == (0, 0)
+    ref_m = oracle.batched(oracle.prefix_mask, f64(q), f64(k), f64(v), m=m.cpu().numpy())
+    assert oracle.max_row_rel_err(f64(out_m), ref_m) < 2e-2
