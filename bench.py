@@ -75,12 +75,12 @@ CALL_KERNELS_F32 = {
 def call_kernels(wl, dtype):
     """The kernels of each call for this workload: the tables above, with the
     non-causal form as one thread-block-cluster kernel where la_noncausal
-    takes that path (bf16, d = 64, B*H * 8 <= 288, N <= 8192), and without
+    takes that path (bf16, d = 64, B*H <= 33, N <= 8192), and without
     the block-state scan kernel where the KV pass scans in its clusters."""
     if dtype != "bf16":
         return CALL_KERNELS_F32
     out = dict(CALL_KERNELS)
-    if wl.d == 64 and wl.B * wl.H * 8 <= 288 and wl.N <= 8192:
+    if wl.d == 64 and wl.B * wl.H <= 33 and wl.N <= 8192:
         out["noncausal"] = ["tc_noncausal_cluster_kernel"]
     if wl.d == 64 and block_count(wl) <= 16 and block_count(wl) * wl.B * wl.H <= 296:
         # the KV pass scans the block states inside its clusters (prefix mask,

@@ -31,7 +31,7 @@ KvBalanced kv_balanced_plan(const Problem& p, int per_sm = 1);
 cudaError_t tc_kv_summary(const Problem& p, const void* k, const void* v, float* part, float* S,
                           float* z, uint32_t* err, cudaStream_t st);
 // Non-causal attention in one kernel for small problems (tc_fused.cu): bf16,
-// d = 64, B*H * 8 <= 288 (one wave of 8-CTA clusters, one per head),
+// d = 64, B*H <= 33 (one wave of 8-CTA clusters, one per head),
 // N <= 8192. Writes
 // out and, when S / z are non-null, the KV summary [bh][d*d], [bh][d].
 bool tc_noncausal_fused_supported(const Problem& p);
