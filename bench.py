@@ -76,18 +76,32 @@ def call_kernels(wl, dtype):
     """The kernels of each call for this workload: the tables above, with the
     non-causal form as one thread-block-cluster kernel where la_noncausal
     takes that path (bf16, d = 64, B*H <= 33, N <= 8192), and without
-    the block-state scan kernel where the KV pass scans in its clusters."""
+    the block-state scan kernel where the KV pass scans in its clusters
+    (scan_in_cluster)."""
     if dtype != "bf16":
         return CALL_KERNELS_F32
     out = dict(CALL_KERNELS)
     if wl.d == 64 and wl.B * wl.H <= 33 and wl.N <= 8192:
         out["noncausal"] = ["tc_noncausal_cluster_kernel"]
-    if wl.d == 64 and block_count(wl) <= 16 and block_count(wl) * wl.B * wl.H <= 296:
-        # the KV pass scans the block states inside its clusters (prefix mask,
-        # causal gradients): no scan kernel
+    if wl.d == 64 and scan_in_cluster(wl):
+        # the KV pass scans the block states inside its clusters (causal,
+        # prefix mask, causal gradients): no forward scan kernel
+        out["causal"] = [k for k in out["causal"] if k != "state_scan_kernel"]
         out["prefix"] = [k for k in out["prefix"] if k != "state_scan_kernel"]
         out["causal_bwd"] = [k for i, k in enumerate(out["causal_bwd"]) if not (i == 1 and k == "state_scan_kernel")]
     return out
+
+
+def scan_in_cluster(wl):
+    """Whether the KV pass scans the block states in a cluster per head, as
+    tc_kv.cu decides it: at most 16 blocks, and every head's cluster (one or
+    two blocks per CTA) resident at once; a B200 holds 71 clusters of 4, 33
+    of 8 and 14 of 16 at two CTAs per SM."""
+    nblk, bh = block_count(wl), wl.B * wl.H
+
+    def capacity(cs):
+        return 296 if cs <= 1 else 148 if cs <= 2 else 71 if cs <= 4 else 33 if cs <= 8 else 14
+    return nblk <= 16 and any(bh <= capacity(-(-nblk // bpc)) for bpc in (1, 2))
 
 
 def block_count(wl):

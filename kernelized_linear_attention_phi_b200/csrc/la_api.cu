@@ -304,14 +304,16 @@ la_status causal_impl(const la_desc* desc, int32_t chunk, const void* q, const v
     // phase 1: per-block states; phase 2: exclusive prefix over blocks (and
     // the total); phase 3: each block's outputs from its prefix state.
     uint32_t* flags = at<uint32_t>(ws, 0);
-    // (the in-cluster scan of tc_kv_blocks_scan measured no faster here: the
-    // separate scan overlaps the sweep's prologue)
-    if (tc_supported(p)) {
-        LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
+    if (tc_kv_scan_supported(p, bp.block_tokens, bp.nblk)) {  // phases 1 and 2 in one kernel
+        LA_TRY(cuda_status(tc_kv_blocks_scan(p, k, v, bp.block_tokens, bp.nblk, part, S_total, z_total, flags, st)));
     } else {
-        LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
+        if (tc_supported(p)) {
+            LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
+        } else {
+            LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
+        }
+        LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, S_total, z_total, st)));
     }
-    LA_TRY(cuda_status(state_exclusive_scan(p, part, bp.nblk, S_total, z_total, st)));
     if (tc_supported(p))
         return cuda_status(tc_chunked(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, nullptr,
                                       nullptr, nullptr, 0, out, flags, st));

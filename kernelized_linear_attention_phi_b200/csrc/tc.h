@@ -46,9 +46,10 @@ cudaError_t tc_reduce_records(const Problem& p, const KvBalanced& w, const float
 cudaError_t tc_kv_blocks(const Problem& p, const void* k, const void* v, int block_tokens, int nblk,
                          float* part, uint32_t* err, cudaStream_t st);
 // tc_kv_blocks followed by the exclusive block-state scan, in one kernel with
-// a thread-block cluster per head (bf16, d = 64, nblk <= 16, nblk * B*H <=
-// 296): part[bh*nblk + blk] receives the prefix of the blocks before blk
-// (what state_exclusive_scan leaves), S_total / z_total (nullable) the total.
+// a thread-block cluster per head (bf16, d = 64, nblk <= 16, every head's
+// cluster resident at once, with one or two blocks per CTA): part[bh*nblk +
+// blk] receives the prefix of the blocks before blk (what
+// state_exclusive_scan leaves), S_total / z_total (nullable) the total.
 bool tc_kv_scan_supported(const Problem& p, int block_tokens, int nblk);
 cudaError_t tc_kv_blocks_scan(const Problem& p, const void* k, const void* v, int block_tokens, int nblk, float* part,
                               float* S_total, float* z_total, uint32_t* err, cudaStream_t st);

@@ -67,6 +67,7 @@ __device__ __forceinline__ int cta_of(const KvBalanced& w, long long t) {
 struct KvWork {
     int balanced;
     int block_tokens, nblk;  // blocks mode
+    int bpc;                 // blocks mode: consecutive blocks per CTA (1 or 2)
     KvBalanced b;            // balanced mode
 };
 
@@ -76,7 +77,7 @@ struct Seg {
 };
 
 __device__ __forceinline__ int kv_nseg(const KvWork& w) {
-    if (!w.balanced) return 1;
+    if (!w.balanced) return max(0, min(w.bpc, w.nblk - (int)blockIdx.x * w.bpc));
     const long long lo = range_lo(w.b.total, w.b.G, blockIdx.x);
     const long long hi = range_lo(w.b.total, w.b.G, blockIdx.x + 1);
     return hi > lo ? (int)((hi - 1) / w.b.tph - lo / w.b.tph + 1) : 0;
@@ -85,10 +86,11 @@ __device__ __forceinline__ int kv_nseg(const KvWork& w) {
 __device__ __forceinline__ Seg kv_seg(const KvWork& w, int N, int j) {
     Seg s;
     if (!w.balanced) {
+        const int blk = blockIdx.x * w.bpc + j;
         s.bh = blockIdx.y;
-        s.t0 = blockIdx.x * w.block_tokens;
+        s.t0 = blk * w.block_tokens;
         s.t1 = min(N, s.t0 + w.block_tokens);
-        s.slot = blockIdx.y * w.nblk + blockIdx.x;
+        s.slot = blockIdx.y * w.nblk + blk;
     } else {
         const long long lo = range_lo(w.b.total, w.b.G, blockIdx.x);
         const long long hi = range_lo(w.b.total, w.b.G, blockIdx.x + 1);
@@ -117,16 +119,15 @@ struct KvCfg {
     static constexpr int BARS = 3 * STAGES + 1;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * 2 * TILE + RED + 8 * BARS + 16;
     static_assert(SMEM <= 227 * 1024, "shared memory");
-    // the block's record is kept in the stage buffers once its MMAs are done
-    static_assert(!SCAN || (size_t)STAGES * 2 * TILE >= (size_t)(D * D + D) * 4, "record fits the stages");
     // two resident CTAs per SM with the in-cluster scan: 228 KiB per SM, 1 KiB reserved per CTA
     static_assert(!SCAN || 2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
-// SCAN (blocks mode, one cluster of nblk CTAs per head): instead of its own
-// record each CTA writes the exclusive prefix of the records of its head,
-// computed across the cluster (see the end of the kernel); S_total, z_total
-// (nullable) receive the head's total.
+// SCAN (blocks mode, one cluster of the CTAs of a head, each taking bpc
+// consecutive blocks): the block records are replaced by their exclusive
+// prefix over the head's blocks, computed across the cluster after its
+// barrier (see the end of the kernel); S_total, z_total (nullable) receive
+// the head's total.
 template <int D, int PHI, bool SCAN = false>
 __global__ void __launch_bounds__(kThreads, SCAN ? 2 : 1)
 tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV, int N,
@@ -296,9 +297,7 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
                     }
             }
             named_bar(1, 128);
-            // SCAN: the record goes to the stage buffers, after the MMAs are done
-            float* rec = SCAN ? reinterpret_cast<float*>(tiles) : part + (size_t)sg.slot * REC;
-            float zrow = 0.f;
+            float* rec = part + (size_t)sg.slot * REC;
             if (et < D) {
                 const int b = et / 64, g = (et % 64) / 8, e = et % 8;
                 float zs = relu ? (float)(sg.t1 - sg.t0) : 0.f;
@@ -308,8 +307,7 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
                     zs += red[((w4 * C::NB + b) * 8 + g) * 16 + e];
                     cs += red[((w4 * C::NB + b) * 8 + g) * 16 + 8 + e];
                 }
-                if (!SCAN) rec[(size_t)D * D + et] = zs;
-                zrow = zs;
+                rec[(size_t)D * D + et] = zs;
                 csum[et] = relu ? cs : 0.f;
             }
             named_bar(1, 128);
@@ -347,34 +345,36 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
                                         __uint_as_float(r[4 * q4 + 2]) + csum[c0 + 4 * q4 + 2],
                                         __uint_as_float(r[4 * q4 + 3]) + csum[c0 + 4 * q4 + 3]);
             }
-            if (SCAN && et < D) rec[(size_t)D * D + et] = zrow;
             tc_fence_before();
             named_bar(1, 128);  // `red` is reused by the next segment
         }
     }
     if constexpr (SCAN) {
-        // Exclusive prefix of the head's block records across the cluster
-        // (rank = block): CTA r takes float4s [r*chunk, (r+1)*chunk) of the
-        // record, reads them from every rank in order and writes rank r''s
-        // prefix (the sum over ranks before it) to its record slot, then the
-        // total. Every thread of every CTA reaches both cluster barriers.
+        // Exclusive prefix of the head's block records across the cluster:
+        // after the barrier (release / acquire at cluster scope, so every
+        // record written above is visible) CTA r of the nc in the cluster
+        // takes float4s [r*chunk, (r+1)*chunk) of the records, reads them
+        // for every block in order (L2) and overwrites each with the sum over
+        // the blocks before it, then writes the total. Each element has one
+        // owner, so the in-place update needs no second barrier. Every thread
+        // of every CTA reaches the barrier.
         cluster_sync();
         if (warp >= 2) {
             const int et = threadIdx.x - 64;
-            const int nblk = w.nblk, bh = blockIdx.y, r = blockIdx.x;
+            const int nblk = w.nblk, bh = blockIdx.y, r = blockIdx.x, nc = gridDim.x;
             constexpr int E4 = (D * D + D) / 4;
-            const int chunk = (E4 + nblk - 1) / nblk;
-            const float* recs = reinterpret_cast<const float*>(tiles);
+            const int chunk = (E4 + nc - 1) / nc;
+            float4* recs = reinterpret_cast<float4*>(part + (size_t)bh * nblk * REC);
             for (int f = r * chunk + et; f < min(E4, (r + 1) * chunk); f += 128) {
                 float4 x[16];
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr)
-                    if (rr < nblk) x[rr] = ld_cluster_f4(cluster_addr(recs + 4 * f, rr));
+                    if (rr < nblk) x[rr] = recs[(size_t)rr * (REC / 4) + f];
                 float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) {
                     if (rr < nblk) {
-                        reinterpret_cast<float4*>(part + ((size_t)bh * nblk + rr) * REC)[f] = run;
+                        recs[(size_t)rr * (REC / 4) + f] = run;
                         run.x += x[rr].x;
                         run.y += x[rr].y;
                         run.z += x[rr].z;
@@ -392,7 +392,6 @@ tc_kv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUt
                 }
             }
         }
-        cluster_sync();  // no CTA leaves while another reads its record
     }
     tc_fence_before();
     __syncthreads();
@@ -675,8 +674,9 @@ cudaError_t launch_kv_scan(const Problem& p, const CUtensorMap& mk, const CUtens
     constexpr size_t smem = KvCfg<D, true>::SMEM;
     const cudaError_t e = ensure_smem<tc_kv_kernel<D, PHI, true>>(smem);
     if (e != cudaSuccess) return e;
-    return launch_cluster_pdl(tc_kv_kernel<D, PHI, true>, dim3((unsigned)w.nblk, (unsigned)p.bh()), dim3(kThreads),
-                              smem, st, (unsigned)w.nblk, mk, mv, p.N, w, part, err, S_total, z_total);
+    const unsigned nc = (unsigned)((w.nblk + w.bpc - 1) / w.bpc);  // CTAs of a head's cluster
+    return launch_cluster_pdl(tc_kv_kernel<D, PHI, true>, dim3(nc, (unsigned)p.bh()), dim3(kThreads), smem, st, nc,
+                              mk, mv, p.N, w, part, err, S_total, z_total);
 }
 
 // one kernel per feature map (see phi8)
@@ -744,10 +744,28 @@ cudaError_t tc_reduce_records(const Problem& p, const KvBalanced& w, const float
                       w, p.d, S, z);
 }
 
+namespace {
+// Clusters of cs CTAs (two per SM, the scanning KV pass's threads and shared
+// memory) that a B200 holds at once, from the occupancy of a plain kernel of
+// the same shape: 71 of 4, 33 of 8, 14 of 16. A cluster of up to 2^k CTAs
+// fits wherever one of 2^k does, so other sizes take the next power of two.
+int cluster_capacity(int cs) {
+    return cs <= 1 ? 296 : cs <= 2 ? 148 : cs <= 4 ? 71 : cs <= 8 ? 33 : 14;
+}
+// Blocks per CTA of the scanning KV pass: one while every head's cluster
+// fits one wave, else two (half the CTAs, twice the tiles each); 0 when
+// neither fits (the separate scan kernel is used then).
+int kv_scan_bpc(const Problem& p, int nblk) {
+    for (int bpc = 1; bpc <= 2; ++bpc)
+        if (p.bh() <= cluster_capacity((nblk + bpc - 1) / bpc)) return bpc;
+    return 0;
+}
+}  // namespace
+
 bool tc_kv_scan_supported(const Problem& p, int block_tokens, int nblk) {
-    // one cluster per head (at most 16 CTAs), one wave at two CTAs per SM
+    // one cluster per head (at most 16 blocks), all clusters in one wave
     return tc_supported(p) && p.d == 64 && block_tokens % kTile == 0 && nblk >= 1 && nblk <= 16 &&
-           (long long)nblk * p.bh() <= 2 * 148;
+           kv_scan_bpc(p, nblk) > 0;
 }
 
 cudaError_t tc_kv_blocks_scan(const Problem& p, const void* k, const void* v, int block_tokens, int nblk, float* part,
@@ -757,6 +775,7 @@ cudaError_t tc_kv_blocks_scan(const Problem& p, const void* k, const void* v, in
     w.balanced = 0;
     w.block_tokens = block_tokens;
     w.nblk = nblk;
+    w.bpc = kv_scan_bpc(p, nblk);
     CUtensorMap mk, mv;
     cudaError_t e = make_map(&mk, k, 64, p.N, p.bh(), kTile);
     if (e == cudaSuccess) e = make_map(&mv, v, 64, p.N, p.bh(), kTile);
@@ -775,6 +794,7 @@ cudaError_t tc_kv_blocks(const Problem& p, const void* k, const void* v, int blo
     w.balanced = 0;
     w.block_tokens = block_tokens;
     w.nblk = nblk;
+    w.bpc = 1;
     const dim3 grid(nblk, (unsigned)p.bh());
     return p.d == 64 ? launch_kv<64>(p, k, v, w, grid, part, err, st)
                      : launch_kv<128>(p, k, v, w, grid, part, err, st);

@@ -12,11 +12,11 @@ pytestmark = pytest.mark.gpu
 
 # kernels per call on the bf16 tensor-core path at this size (8 heads of
 # 1024 tokens, d = 64): KV summary: partial records + reduction; non-causal:
-# one thread-block-cluster kernel; causal: block states, scan, sweep; prefix
-# mask: block states scanned inside a cluster per head, binning, sweep;
+# one thread-block-cluster kernel; causal: block states scanned inside a
+# cluster per head, sweep; prefix mask: the same plus the binning;
 # decode: one; gradients: forward states (non-causal: + reduction; causal:
 # scanned in-cluster), dq sweep, (G, h) reduction or reverse scan, dk/dv sweep
-TC_LAUNCHES = {"kv_summary": 2, "noncausal": 1, "causal": 3, "prefix": 3, "decode": 1, "noncausal_bwd": 5,
+TC_LAUNCHES = {"kv_summary": 2, "noncausal": 1, "causal": 2, "prefix": 3, "decode": 1, "noncausal_bwd": 5,
                "causal_bwd": 4}
 
 
