@@ -105,3 +105,14 @@ def test_noncausal_gradients_split_across_heads(d, phi, normalize):
     for name, gt, rf, sc in zip(("dq", "dk", "dv"), got, ref[:3], ref[3:]):
         err = oracle.max_row_grad_err(f64(gt), rf, sc)
         assert err < TOL[torch.bfloat16], (name, err)
+
+
+def test_causal_gradients_with_two_blocks_per_cta():
+    """15 heads of 2500 tokens (10 blocks each): 15 clusters of 10 CTAs would
+    not all be resident, so the forward block states are formed and scanned
+    with two blocks per CTA (clusters of 5)."""
+    got, ref = _case("causal", "bf16", 64, 2500, "relu1", True, B=1, H=15, seed=12)
+    for name, gt, rf, sc in zip(("dq", "dk", "dv"), got, ref[:3], ref[3:]):
+        err = oracle.max_row_grad_err(f64(gt), rf, sc)
+        assert err < TOL[torch.bfloat16], (name, err)
+

@@ -273,13 +273,15 @@ def test_causal_prefill_then_decode(dt, d, phi):
     assert oracle.max_row_rel_err(f64(out), ref_pre) < TOL[DT[dt]]
 
 
-@pytest.mark.parametrize("B,H,N", [(1, 16, 4096), (1, 2, 2300), (4, 37, 512), (1, 1, 64)])
+@pytest.mark.parametrize("B,H,N", [(1, 16, 4096), (1, 16, 3800), (1, 2, 2300), (4, 37, 512), (1, 1, 64)])
 def test_causal_and_prefix_block_counts(B, H, N):
-    """bf16, d = 64 with 16, 9, 2 and 1 blocks per head (148 heads of 2
-    blocks fill the wave; the prefix mask scans the block states inside a
-    cluster per head, up to the non-portable size 16): 64- and 128-token
-    chunks agree with each other and with the oracle, the prefill's outputs
-    are those of the causal call and its state is the KV summary."""
+    """bf16, d = 64 with 16, 15, 9, 2 and 1 blocks per head (148 heads of 2
+    blocks fill the wave). The KV pass scans the block states inside a
+    cluster per head: one block per CTA up to the non-portable cluster size 9
+    here, two blocks per CTA for 16 heads of 16 or 15 blocks (the last CTA
+    then takes one, partial block). 64- and 128-token chunks agree with each
+    other and with the oracle, the prefill's outputs are those of the causal
+    call and its state is the KV summary."""
     d = 64
     q, k, v = qkv(B, H, N, d, "bf16", seed=B + H + N)
     ref = oracle.batched(oracle.causal, f64(q), f64(k), f64(v))
