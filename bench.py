@@ -75,7 +75,8 @@ CALL_KERNELS_F32 = {
 def call_kernels(wl, dtype):
     """The kernels of each call for this workload: the tables above, with the
     non-causal form as one thread-block-cluster kernel where la_noncausal
-    takes that path (bf16, d = 64, B*H <= 33, N <= 8192), and without
+    takes that path (bf16, d = 64, B*H <= 33, N <= 8192; the non-causal
+    gradient then forms its KV summary with it too), and without
     the block-state scan kernel where the KV pass scans in its clusters
     (scan_in_cluster)."""
     if dtype != "bf16":
@@ -83,6 +84,8 @@ def call_kernels(wl, dtype):
     out = dict(CALL_KERNELS)
     if wl.d == 64 and wl.B * wl.H <= 33 and wl.N <= 8192:
         out["noncausal"] = ["tc_noncausal_cluster_kernel"]
+        # the gradient's KV summary: the same kernel without its readout
+        out["noncausal_bwd"] = ["tc_noncausal_cluster_kernel"] + out["noncausal_bwd"][2:]
     if wl.d == 64 and scan_in_cluster(wl):
         # the KV pass scans the block states inside its clusters (causal,
         # prefix mask, causal gradients): no forward scan kernel
@@ -284,7 +287,7 @@ class Step:
             # q, k, v, dout -> dq; q, k, v -> dk, dv); the reductions of
             # (G, h) move scratch only
             causal = call == "causal_bwd"
-            return {"kv": 2 * t, "bwd_q": (5 if causal else 3) * t,
+            return {"kv": 2 * t, "fused": 2 * t, "bwd_q": (5 if causal else 3) * t,
                     "bwd_kv": (5 if causal else 4) * t}.get(role, 0)
         return {"kv": 2 * t, "reduce": st, "readout": 2 * t + st, "scan": 0, "sweep": 4 * t, "fused": 4 * t,
                 "bin": self.B * self.N * 4, "decode": 2 * st + 4 * one}.get(role, 0)

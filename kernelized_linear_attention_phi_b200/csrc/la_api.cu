@@ -196,6 +196,8 @@ la_status check_ws(const WsLayout& L, void* ws, size_t ws_bytes) {
 la_status kv_summary_impl(const Problem& p, const void* k, const void* v, float* S, float* z,
                           void* ws, cudaStream_t st) {
     float* part = at<float>(ws, ws_layout(p, LA_OP_KV_SUMMARY).part);
+    if (tc_noncausal_fused_supported(p))  // small problems: one launch, reduced in a cluster per head
+        return cuda_status(tc_noncausal_fused(p, nullptr, k, v, nullptr, S, z, at<uint32_t>(ws, 0), st));
     if (tc_supported(p)) return cuda_status(tc_kv_summary(p, k, v, part, S, z, at<uint32_t>(ws, 0), st));
     const SplitPlan sp = kv_plan(p);
     LA_TRY(cuda_status(simt_kv_partial(p, k, v, sp.tps, sp.nsplit, part, st)));

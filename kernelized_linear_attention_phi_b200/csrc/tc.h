@@ -33,7 +33,8 @@ cudaError_t tc_kv_summary(const Problem& p, const void* k, const void* v, float*
 // Non-causal attention in one kernel for small problems (tc_fused.cu): bf16,
 // d = 64, B*H <= 33 (one wave of 8-CTA clusters, one per head),
 // N <= 8192. Writes
-// out and, when S / z are non-null, the KV summary [bh][d*d], [bh][d].
+// out and, when S / z are non-null, the KV summary [bh][d*d], [bh][d]; with
+// out null (q then unused) only the KV summary, into S and z (both needed).
 bool tc_noncausal_fused_supported(const Problem& p);
 cudaError_t tc_noncausal_fused(const Problem& p, const void* q, const void* k, const void* v, void* out, float* S,
                                float* z, uint32_t* err, cudaStream_t st);

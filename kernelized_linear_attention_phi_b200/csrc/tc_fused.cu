@@ -15,7 +15,8 @@
 //      after (hardware barriers: every thread of every CTA reaches both on
 //      every path);
 //   3. readout of the CTA's tokens against the full S, z (the readout
-//      pipeline), output tiles stored by TMA.
+//      pipeline), output tiles stored by TMA; skipped when only the KV
+//      summary is asked for (readout = 0: S, z written, Q never loaded).
 // The Q tiles of phase 3 are loaded while phases 1 and 2 finish (the stages
 // are shared, and the first ones free up as the phase-1 MMAs complete).
 //
@@ -64,8 +65,8 @@ template <int PHI>
 __global__ void __launch_bounds__(kThreads, 2)
 tc_noncausal_cluster_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
                             const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mOut, int N,
-                            int tpc, int normalize, float* __restrict__ S_out, float* __restrict__ z_out,
-                            uint32_t* __restrict__ err) {
+                            int tpc, int normalize, int readout, float* __restrict__ S_out,
+                            float* __restrict__ z_out, uint32_t* __restrict__ err) {
     using C = FnCfg;
     constexpr int D = C::D;
     constexpr bool relu = PHI == PHI_RELU1;
@@ -90,7 +91,8 @@ tc_noncausal_cluster_kernel(const __grid_constant__ CUtensorMap mK, const __grid
     const int bh = blockIdx.y;
     const int t0 = rank * tpc;
     const int t1 = min(N, t0 + tpc);
-    const int nt = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;  // tiles in each phase
+    const int nt = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;  // tiles of phase 1
+    const int nq = readout ? nt : 0;                              // tiles of phase 3
 
     if (threadIdx.x == 0) {
         cta_abort_reset();
@@ -145,12 +147,12 @@ tc_noncausal_cluster_kernel(const __grid_constant__ CUtensorMap mK, const __grid
         if (lane == 0) {
             for (int i = 0; i < nt && ok; ++i) load(i, i, false);
             // the first Q tiles wait only for phase-1 MMAs to free their stages
-            for (int i = 0; i < min(nt, C::STAGES) && ok; ++i) load(nt + i, i, true);
+            for (int i = 0; i < min(nq, C::STAGES) && ok; ++i) load(nt + i, i, true);
         }
         cluster_sync();
         cluster_sync();
         if (lane == 0) {
-            for (int i = C::STAGES; i < nt && ok; ++i) load(nt + i, i, true);
+            for (int i = C::STAGES; i < nq && ok; ++i) load(nt + i, i, true);
             for (int s = 0; s < C::STAGES; ++s)
                 if (issued[s] > 0) mbar_wait(full + s, (issued[s] - 1) & 1, err, false);
         }
@@ -182,7 +184,7 @@ tc_noncausal_cluster_kernel(const __grid_constant__ CUtensorMap mK, const __grid
             constexpr uint32_t id_o = idesc_bf16(128, D, false, true);    // O = phi(Q) S
             constexpr uint32_t id_z = idesc_bf16(128, 16, false, false);  // den = phi(Q) [z]
             const uint32_t sb = smem_u32(bS), zb = smem_u32(bZ);
-            for (int i = 0; i < nt && ok; ++i) {
+            for (int i = 0; i < nq && ok; ++i) {
                 const int ring = nt + i, s = ring % C::STAGES, u = ring / C::STAGES;
                 const int ab = i & 1, ua = i >> 1;
                 if (!(ok = mbar_wait(tdone + s, u & 1, err))) break;
@@ -382,9 +384,9 @@ tc_noncausal_cluster_kernel(const __grid_constant__ CUtensorMap mK, const __grid
                 bulk_commit();
             }
         };
-        if (nt > 0) transform(0);
-        for (int i = 0; i < nt; ++i) {
-            if (i + 1 < nt) transform(i + 1);
+        if (nq > 0) transform(0);
+        for (int i = 0; i < nq; ++i) {
+            if (i + 1 < nq) transform(i + 1);
             epilogue(i);
         }
         if (et == 0) bulk_wait0();
@@ -399,11 +401,13 @@ tc_noncausal_cluster_kernel(const __grid_constant__ CUtensorMap mK, const __grid
 
 template <int PHI>
 cudaError_t launch_fused(const Problem& p, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mq,
-                         const CUtensorMap& mo, int tpc, float* S, float* z, uint32_t* err, cudaStream_t st) {
+                         const CUtensorMap& mo, int tpc, int readout, float* S, float* z, uint32_t* err,
+                         cudaStream_t st) {
     cudaError_t e = ensure_smem<tc_noncausal_cluster_kernel<PHI>>(FnCfg::SMEM);
     if (e != cudaSuccess) return e;
     return launch_cluster_pdl(tc_noncausal_cluster_kernel<PHI>, dim3(kCluster, (unsigned)p.bh()), dim3(kThreads),
-                              FnCfg::SMEM, st, (unsigned)kCluster, mk, mv, mq, mo, p.N, tpc, p.normalize, S, z, err);
+                              FnCfg::SMEM, st, (unsigned)kCluster, mk, mv, mq, mo, p.N, tpc, p.normalize, readout, S,
+                              z, err);
 }
 
 }  // namespace
@@ -420,17 +424,21 @@ cudaError_t tc_noncausal_fused(const Problem& p, const void* q, const void* k, c
                                float* z, uint32_t* err, cudaStream_t st) {
     if (!tc_noncausal_fused_supported(p)) return cudaErrorInvalidValue;
     constexpr int D = FnCfg::D;
+    // KV summary only (no out): the Q and output maps are never used and
+    // are encoded over K
+    const int readout = out != nullptr ? 1 : 0;
+    if (!readout && (S == nullptr || z == nullptr)) return cudaErrorInvalidValue;
     CUtensorMap mk, mv, mq, mo;
     cudaError_t e = make_map(&mk, k, D, p.N, p.bh(), kTile);
     if (e == cudaSuccess) e = make_map(&mv, v, D, p.N, p.bh(), kTile);
-    if (e == cudaSuccess) e = make_map(&mq, q, D, p.N, p.bh(), kTile);
-    if (e == cudaSuccess) e = make_map(&mo, out, D, p.N, p.bh(), kTile);
+    if (e == cudaSuccess) e = make_map(&mq, readout ? q : k, D, p.N, p.bh(), kTile);
+    if (e == cudaSuccess) e = make_map(&mo, readout ? out : k, D, p.N, p.bh(), kTile);
     if (e != cudaSuccess) return e;
     const int tpc = ((p.N + kCluster - 1) / kCluster + kTile - 1) / kTile * kTile;  // tokens per CTA
     switch (p.phi) {  // one kernel per feature map (see phi8)
-        case PHI_RELU1: return launch_fused<PHI_RELU1>(p, mk, mv, mq, mo, tpc, S, z, err, st);
-        case PHI_ELU1: return launch_fused<PHI_ELU1>(p, mk, mv, mq, mo, tpc, S, z, err, st);
-        default: return launch_fused<PHI_IDENTITY>(p, mk, mv, mq, mo, tpc, S, z, err, st);
+        case PHI_RELU1: return launch_fused<PHI_RELU1>(p, mk, mv, mq, mo, tpc, readout, S, z, err, st);
+        case PHI_ELU1: return launch_fused<PHI_ELU1>(p, mk, mv, mq, mo, tpc, readout, S, z, err, st);
+        default: return launch_fused<PHI_IDENTITY>(p, mk, mv, mq, mo, tpc, readout, S, z, err, st);
     }
 }
 

@@ -26,6 +26,8 @@ def test_in_cluster_scan_takes_two_blocks_per_cta_when_one_would_not_fit():
     assert k["causal_bwd"] == ["tc_kv_kernel", "tc_bwd_causal_q_kernel", "state_scan_kernel",
                                "tc_bwd_causal_kv_kernel"]
     assert k["noncausal"] == ["tc_noncausal_cluster_kernel"]
+    assert k["noncausal_bwd"] == ["tc_noncausal_cluster_kernel", "tc_bwd_q_kernel", "kv_reduce_balanced_kernel",
+                                  "tc_bwd_kv_kernel"]
 
 
 def test_long_and_fp32_workloads_keep_the_separate_kernels():
