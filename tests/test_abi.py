@@ -154,3 +154,22 @@ def test_backward_validation(lib):
     assert B.la_workspace_size(dsc, "noncausal_bwd") > 0
     assert B.la_workspace_size(dsc, "causal_bwd") > 0
     assert lib.la_workspace_size(ctypes.byref(dsc), 7, 64) == 0
+
+
+def test_gradient_workspace_sizes(lib):
+    """The tensor-core non-causal gradient (bf16, d = 64 / 128) keeps the
+    record slots of its balanced splits and the totals (S, z), (G, h), but
+    not the CUDA-core path's per-token scaled gradient (fp32 [B,H,N,d]) and
+    block states: at a long sequence it needs less than the fp32 request of
+    the same shape, whose per-token buffer alone exceeds it."""
+    B_, H, N = 1, 2, 65536
+    per_token = B_ * H * N * 64 * 4  # fp32 gn of the CUDA-core path
+    tc = B.la_workspace_size(B.la_desc(B_, H, N, 64, 1, 0, 1), "noncausal_bwd")
+    simt = B.la_workspace_size(B.la_desc(B_, H, N, 64, 0, 0, 1), "noncausal_bwd")
+    assert 0 < tc < per_token <= simt
+    B_, H, N = 2, 3, 4096
+    # both gradients hold at least the totals of both states
+    for dt in (0, 1):
+        for op in ("noncausal_bwd", "causal_bwd"):
+            n = B.la_workspace_size(B.la_desc(B_, H, N, 64, dt, 0, 1), op)
+            assert n % 256 == 0 and n >= 2 * B_ * H * (64 * 64 + 64) * 4

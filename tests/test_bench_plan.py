@@ -43,3 +43,25 @@ def test_kernel_roles_cover_every_listed_kernel():
         for names in table.values():
             for n in names:
                 assert any(n.startswith(r) for r in bench.KERNEL_ROLE), n
+
+
+def test_kernel_bytes_of_the_gradient_calls():
+    """Algorithmic bytes per kernel of the gradient calls: the KV summary
+    reads K and V (whether the balanced KV pass or the cluster kernel without
+    its readout forms it), the query side Q, dO and dq (causal: also K, V),
+    the key side K, V, dk, dv (causal: also Q); reductions move scratch only."""
+    wl = W.WORKLOADS["multi_head_bwd"]
+    t = wl.B * wl.H * wl.N * wl.d * 2
+
+    class S:  # the fields kernel_bytes reads
+        B, H, N, d, elem = wl.B, wl.H, wl.N, wl.d, 2
+    kb = lambda call, k: bench.Step.kernel_bytes(S, call, k)
+    assert kb("noncausal_bwd", "tc_noncausal_cluster_kernel") == 2 * t
+    assert kb("noncausal_bwd", "tc_kv_kernel") == 2 * t
+    assert kb("noncausal_bwd", "tc_bwd_q_kernel") == 3 * t
+    assert kb("noncausal_bwd", "tc_bwd_kv_kernel") == 4 * t
+    assert kb("noncausal_bwd", "kv_reduce_balanced_kernel") == 0
+    assert kb("causal_bwd", "tc_bwd_causal_q_kernel") == 5 * t
+    assert kb("causal_bwd", "tc_bwd_causal_kv_kernel") == 5 * t
+    assert kb("noncausal", "tc_noncausal_cluster_kernel") == 4 * t
+
