@@ -1,29 +1,40 @@
 """Throughput of the kernelized linear attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload multi_head] [--dtype bf16]
+                    [--case NAME] [--no-configs] [--no-cpu-baseline]
 
-One step is one pass of every form of the path over one batch of the
-workload: non-causal (KV summary + readout), causal (chunked), prefix mask
-(queries binned by m_i) and one decode step on the state the non-causal pass
-produced. The default workload is multi-head attention with B=2, H=8,
-N=4096, d=64 (the lineartile quick-start shape), phi = relu+1, normalized,
-bf16, chunk 64, m_i uniform in [0, N-1]. Other workloads (--workload) run
-only the forms they are defined for.
+One run measures every workload of the pages (kernelized_linear_attention_phi_b200/
+workloads.py) and prints ONE JSON line. Its headline (``value``, ``e2e``,
+``roofline``, ``cpu_baseline``) is the largest workload that one GPU holds,
+the long-context case: a step is one non-causal call on B=4, H=16, N=16384
+(128x128 latent tokens), d=64 plus one causal call on B=1, H=16, N=131072,
+d=128, both bf16, phi = relu+1, normalized. ``per_config`` holds the same
+fields for every other workload:
 
-Tokens counted per step: B*N for each full-sequence form plus B for a decode
-step. ``value`` is tokens/s over all ranks (weak scaling: each rank runs its
-own batch; the path has no exchange step, so there is no data-path
-collective). Each library call is captured once into a CUDA graph and the
-graphs are replayed. Timing: CUDA events between the calls of every step on
-the launching stream, L2 flushed (a 256 MiB write) between steps outside the
-events, W untimed warm-up steps, max over ranks. ``e2e`` repeats the step
-through the plain API calls with pinned host inputs copied in and the
-outputs copied back inside the timed region. ``roofline`` is the dominant
-kernel's: after the timed steps every call is replayed again from a graph
-captured with the library's per-kernel timing events (la_timing_enable), L2
-flushed before each replay, and the kernel with the largest mean time has its
-algorithmic bytes divided by that time.
+* ``single_head``: 1x1x256x16 fp32, non-causal;
+* ``multi_head_bf16`` / ``multi_head_f32``: 2x8x4096x64, non-causal + causal
+  (chunk 64);
+* ``prefix_mask``: 8x8x2048x64 bf16, identity map, unnormalized, m_i uniform
+  in [0, N-1]; ``prefix_mask_arange``: the same with m = arange(N);
+* ``decode``: 64 sequences x 32 heads, d=128, fp32 state prefilled from 2048
+  bf16 tokens; a step is 1024 one-token decode steps;
+* ``multi_head_bwd_bf16``: the gradients (dq, dk, dv) of both 2x8x4096x64
+  forms.
+
+Tokens per step: B*N per full-sequence call, sequences x steps for decode.
+``value`` is tokens/s over all ranks (weak scaling: each rank runs its own
+batch; the path has no exchange step, so there is no data-path collective).
+Each library call is captured once into a CUDA graph (decode: the 1024
+steps in one graph) and the graphs are replayed. Timing: CUDA events around
+every call on the launching stream, L2 flushed (a 256 MiB write) before
+every call outside the events, W untimed warm-up steps, max over ranks.
+``e2e`` repeats the step through the plain API calls with pinned host inputs
+copied in and the outputs copied back inside the timed region.
+``roofline`` is the dominant kernel's: after the timed steps every call is
+replayed from a graph captured with the library's per-kernel timing events
+(la_timing_enable), L2 flushed before each replay, and the kernel with the
+largest mean time has its algorithmic bytes divided by that time (decode:
+the 1024-step call time over 1024).
 """
 
 from __future__ import annotations
@@ -46,78 +57,64 @@ import torch  # noqa: E402
 from kernelized_linear_attention_phi_b200 import workloads as W  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20
+METRIC = "tokens/sec (fwd, 1xB200) and % of HBM / bf16 tensor-core roofline per kernel"
 
-# Kernels each library call launches on the bf16 tensor-core path, in launch
-# order; kept in step with la_api.cu's dispatch and checked against the ncu
-# launch list (--record-traffic matches them there).
-CALL_KERNELS = {
-    "noncausal": ["tc_kv_kernel", "kv_reduce_balanced_kernel", "tc_readout_kernel"],
-    "causal": ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"],
-    "prefix": ["tc_kv_kernel", "bin_kernel", "state_scan_kernel", "tc_sweep"],
-    "decode": ["decode_kernel"],
-    "noncausal_bwd": ["tc_kv_kernel", "kv_reduce_balanced_kernel", "tc_bwd_q_kernel", "kv_reduce_balanced_kernel",
-                      "tc_bwd_kv_kernel"],
-    "causal_bwd": ["tc_kv_kernel", "state_scan_kernel", "tc_bwd_causal_q_kernel", "state_scan_kernel",
-                   "tc_bwd_causal_kv_kernel"],
+# The calls of each case: (workload, dtype, form, mask kind).
+CASES = {
+    "long": [("long_noncausal", "bf16", "noncausal", None), ("long_causal", "bf16", "causal", None)],
+    "single_head": [("single_head", "f32", "noncausal", None)],
+    "multi_head_bf16": [("multi_head", "bf16", "noncausal", None), ("multi_head", "bf16", "causal", None)],
+    "multi_head_f32": [("multi_head", "f32", "noncausal", None), ("multi_head", "f32", "causal", None)],
+    "prefix_mask": [("prefix_mask", "bf16", "prefix", "uniform")],
+    "prefix_mask_arange": [("prefix_mask", "bf16", "prefix", "arange")],
+    "decode": [("decode", "bf16", "decode", None)],
+    "multi_head_bwd_bf16": [("multi_head_bwd", "bf16", "noncausal_bwd", None),
+                            ("multi_head_bwd", "bf16", "causal_bwd", None)],
 }
-# The same on the fp32 (CUDA-core) path.
-CALL_KERNELS_F32 = {
-    "noncausal": ["kv_partial_kernel", "state_reduce_kernel", "readout_kernel"],
-    "causal": ["kv_partial_kernel", "state_scan_kernel", "chunked_kernel"],
-    "prefix": ["kv_partial_kernel", "bin_kernel", "state_scan_kernel", "chunked_kernel"],
-    "decode": ["decode_kernel"],
-    "noncausal_bwd": ["kv_partial_kernel", "state_reduce_kernel", "bwd_q_kernel", "state_reduce_kernel",
-                      "bwd_kv_kernel"],
-    "causal_bwd": ["kv_partial_kernel", "state_scan_kernel", "bwd_q_kernel", "state_scan_kernel", "bwd_kv_kernel"],
+HEADLINE = "long"
+CASE_TEXT = {
+    "long": "long-context: non-causal 4x16x16384x64 (128x128 latent tokens) + causal 1x16x131072x128, bf16, "
+            "phi=relu1, normalized",
+    "single_head": "single head: non-causal 1x1x256x16 fp32, phi=relu1, normalized",
+    "multi_head_bf16": "multi-head: non-causal + causal (chunk 64) 2x8x4096x64 bf16, phi=relu1, normalized",
+    "multi_head_f32": "multi-head: non-causal + causal (chunk 64) 2x8x4096x64 fp32, phi=relu1, normalized",
+    "prefix_mask": "prefix mask: 8x8x2048x64 bf16, identity map, unnormalized, m_i uniform in [0, N-1]",
+    "prefix_mask_arange": "prefix mask: 8x8x2048x64 bf16, identity map, unnormalized, m = arange(N)",
+    "decode": "decode: 64 sequences x 32 heads, d=128, fp32 state prefilled from 2048 bf16 tokens, "
+              "1024 one-token steps per step",
+    "multi_head_bwd_bf16": "gradients: dq, dk, dv of non-causal + causal 2x8x4096x64 bf16, upstream N(0,1)",
 }
 
+# Kernels each call launches, in launch order, by the number the library's
+# timing events report (the dispatch in la_api.cu takes one-launch or
+# in-cluster-scan paths where the problem allows; the count tells which).
+TC_KERNELS = {
+    "noncausal": {1: ["tc_noncausal_cluster_kernel"],
+                  3: ["tc_kv_kernel", "kv_reduce_balanced_kernel", "tc_readout_kernel"]},
+    "causal": {2: ["tc_kv_kernel", "tc_sweep"], 3: ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"]},
+    "prefix": {3: ["tc_kv_kernel", "bin_kernel", "tc_sweep"],
+               4: ["tc_kv_kernel", "bin_kernel", "state_scan_kernel", "tc_sweep"]},
+    "decode": {1: ["decode_kernel"]},
+    "noncausal_bwd": {4: ["tc_noncausal_cluster_kernel", "tc_bwd_q_kernel", "kv_reduce_balanced_kernel",
+                          "tc_bwd_kv_kernel"],
+                      5: ["tc_kv_kernel", "kv_reduce_balanced_kernel", "tc_bwd_q_kernel",
+                          "kv_reduce_balanced_kernel", "tc_bwd_kv_kernel"]},
+    "causal_bwd": {4: ["tc_kv_kernel", "tc_bwd_causal_q_kernel", "state_scan_kernel", "tc_bwd_causal_kv_kernel"],
+                   5: ["tc_kv_kernel", "state_scan_kernel", "tc_bwd_causal_q_kernel", "state_scan_kernel",
+                       "tc_bwd_causal_kv_kernel"]},
+}
+SIMT_KERNELS = {
+    "noncausal": {3: ["kv_partial_kernel", "state_reduce_kernel", "readout_kernel"]},
+    "causal": {3: ["kv_partial_kernel", "state_scan_kernel", "chunked_kernel"]},
+    "prefix": {4: ["kv_partial_kernel", "bin_kernel", "state_scan_kernel", "chunked_kernel"]},
+    "decode": {1: ["decode_kernel"]},
+    "noncausal_bwd": {5: ["kv_partial_kernel", "state_reduce_kernel", "bwd_q_kernel", "state_reduce_kernel",
+                          "bwd_kv_kernel"]},
+    "causal_bwd": {5: ["kv_partial_kernel", "state_scan_kernel", "bwd_q_kernel", "state_scan_kernel",
+                       "bwd_kv_kernel"]},
+}
 
-def call_kernels(wl, dtype):
-    """The kernels of each call for this workload: the tables above, with the
-    non-causal form as one thread-block-cluster kernel where la_noncausal
-    takes that path (bf16, d = 64, B*H <= 33, N <= 8192; the non-causal
-    gradient then forms its KV summary with it too), and without
-    the block-state scan kernel where the KV pass scans in its clusters
-    (scan_in_cluster)."""
-    if dtype != "bf16":
-        return CALL_KERNELS_F32
-    out = dict(CALL_KERNELS)
-    if wl.d == 64 and wl.B * wl.H <= 33 and wl.N <= 8192:
-        out["noncausal"] = ["tc_noncausal_cluster_kernel"]
-        # the gradient's KV summary: the same kernel without its readout
-        out["noncausal_bwd"] = ["tc_noncausal_cluster_kernel"] + out["noncausal_bwd"][2:]
-    if wl.d == 64 and scan_in_cluster(wl):
-        # the KV pass scans the block states inside its clusters (causal,
-        # prefix mask, causal gradients): no forward scan kernel
-        out["causal"] = [k for k in out["causal"] if k != "state_scan_kernel"]
-        out["prefix"] = [k for k in out["prefix"] if k != "state_scan_kernel"]
-        out["causal_bwd"] = [k for i, k in enumerate(out["causal_bwd"]) if not (i == 1 and k == "state_scan_kernel")]
-    return out
-
-
-def scan_in_cluster(wl):
-    """Whether the KV pass scans the block states in a cluster per head, as
-    tc_kv.cu decides it: at most 16 blocks, and every head's cluster (one or
-    two blocks per CTA) resident at once; a B200 holds 71 clusters of 4, 33
-    of 8 and 14 of 16 at two CTAs per SM."""
-    nblk, bh = block_count(wl), wl.B * wl.H
-
-    def capacity(cs):
-        return 296 if cs <= 1 else 148 if cs <= 2 else 71 if cs <= 4 else 33 if cs <= 8 else 14
-    return nblk <= 16 and any(bh <= capacity(-(-nblk // bpc)) for bpc in (1, 2))
-
-
-def block_count(wl):
-    """Blocks per head of the chunked forms, as la_api.cu's block plan picks
-    them (one wave of 148 SMs x 2 CTAs, blocks of at least 256 tokens, a
-    multiple of 128)."""
-    per_sm = 1 if wl.d == 128 else 2
-    target = max(1, per_sm * 148 // (wl.B * wl.H))
-    bt = max(256, -(-(-(-wl.N // target)) // 128) * 128)
-    return -(-wl.N // bt)
-
-
-# What each kernel does, for its algorithmic bytes (Step.kernel_bytes).
+# What each kernel does, for its algorithmic bytes (Call.kernel_bytes).
 KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balanced_kernel": "reduce",
                "state_reduce_kernel": "reduce", "tc_readout_kernel": "readout", "readout_kernel": "readout",
                "state_scan_kernel": "scan", "tc_sweep": "sweep", "chunked_kernel": "sweep",
@@ -127,20 +124,34 @@ KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balan
                "tc_noncausal_cluster_kernel": "fused"}
 
 
-def parse():
+def kernel_names(form, dtype, d, count):
+    """Names of the `count` kernels a call of `form` launched (tensor cores:
+    bf16 with d = 64 or 128; CUDA cores otherwise)."""
+    table = TC_KERNELS if dtype == "bf16" and d in (64, 128) else SIMT_KERNELS
+    names = table.get(form, {}).get(count)
+    return names if names else [f"kernel{i}" for i in range(count)]
+
+
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="multi_head")
-    ap.add_argument("--dtype", default="bf16", choices=["bf16", "f32"])
+    ap.add_argument("--case", default=HEADLINE, choices=sorted(CASES),
+                    help="the case the headline fields measure (default: the long-context step)")
+    ap.add_argument("--no-configs", action="store_true", help="measure the headline case only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--record-traffic", metavar="NCU_CSV",
-                    help="read an ncu launch list with dram__bytes_read.sum and "
-                         "dram__bytes_write.sum of this workload's bench run and store "
-                         "each call's DRAM bytes in profiles/traffic.json")
-    return ap.parse_args()
+                    help="read an ncu launch list with dram__bytes_read.sum and dram__bytes_write.sum "
+                         "of a --case run (--no-configs) and store its calls' DRAM bytes in "
+                         "profiles/traffic.json; --traffic-scale multiplies them (a capture of a "
+                         "smaller problem scaled to the case's size)")
+    ap.add_argument("--traffic-scale", type=float, default=1.0)
+    ap.add_argument("--scale-heads", type=int, default=0,
+                    help="run the case with this many heads instead of the workload's (for a "
+                         "reduced-size ncu capture; never a bench number)")
+    return ap.parse_args(argv)
 
 
 def dist_env():
@@ -161,6 +172,7 @@ class ClockSampler:
     def __init__(self, device):
         self.samples, self.reasons, self.max_mhz = [], 0, None
         self._stop = threading.Event()
+        self._active = threading.Event()
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -182,20 +194,33 @@ class ClockSampler:
 
     def _run(self):
         while not self._stop.is_set():
-            self._sample()
+            if self._active.is_set():
+                self._sample()
             time.sleep(0.01)
 
-    def __enter__(self):
+    def start(self):
         if self.nv:
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
-        return self
 
-    def __exit__(self, *a):
+    def timed(self):
+        """Context manager: sample while a timed region runs."""
+        sampler = self
+
+        class _Region:
+            def __enter__(self):
+                sampler._active.set()
+
+            def __exit__(self, *a):
+                if sampler.nv:
+                    sampler._sample()
+                sampler._active.clear()
+        return _Region()
+
+    def stop(self):
         if self.nv:
             self._stop.set()
             self._t.join()
-            self._sample()
 
     def summary(self):
         if not self.nv or not self.samples:
@@ -206,132 +231,130 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-# The step
+# One library call on its own seeded inputs
 # ---------------------------------------------------------------------------
 
-class Step:
-    """Device buffers and the four library calls of one step."""
+class Call:
+    """Device buffers and the library call of one (workload, dtype, form)."""
 
-    ALL_FORMS = ("noncausal", "causal", "prefix", "decode")
-
-    def __init__(self, wl, dtype, seed, device, forms):
+    def __init__(self, wl, dtype, form, mask, seed, device, heads=0):
         from kernelized_linear_attention_phi_b200 import binding as la
-        self.la = la
-        self.forms = forms
-        B, H, N, d = wl.B, wl.H, wl.N, wl.d
-        self.wl, self.B, self.H, self.N, self.d = wl, B, H, N, d
+        self.la, self.wl, self.dtype, self.form, self.mask = la, wl, dtype, form, mask
+        B, H, N, d = wl.B, (heads or wl.H), wl.N, wl.d
+        self.B, self.H, self.N, self.d = B, H, N, d
+        self.name = wl.name if form != "prefix" or mask == "uniform" else f"{wl.name}_{mask}"
         self.phi, self.normalize, self.chunk = wl.phi, wl.normalize, wl.chunk
-        self.q, self.k, self.v = W.qkv(B, H, N, d, wl.sigma, seed, dtype, device)
-        self.m = W.prefix_mask_uniform(B, N, seed, device)
-        q1, k1, v1 = W.decode_tokens(1, B, H, d, wl.sigma, seed, dtype, device)
-        self.q1, self.k1, self.v1 = q1[0].contiguous(), k1[0].contiguous(), v1[0].contiguous()
-        self.out_nc = torch.empty_like(self.q)
-        self.out_c = torch.empty_like(self.q)
-        self.out_m = torch.empty_like(self.q)
-        self.out_d = torch.empty_like(self.q1)
-        if any(f.endswith("_bwd") for f in forms):
-            self.dout = W.upstream_grad(B, H, N, d, seed, dtype, device)
-            self.grads = {f: tuple(torch.empty_like(self.q) for _ in range(3)) for f in forms}
-        self.S = torch.empty(B, H, d, d, dtype=torch.float32, device=device)
-        self.z = torch.empty(B, H, d, dtype=torch.float32, device=device)
-        desc = la._desc_of(self.q, self.phi, self.normalize)
-        self.ws = {op: la.workspace(desc, op, self.chunk, device)
-                   for op in ("noncausal", "causal", "prefix") + tuple(f for f in forms if f.endswith("_bwd"))}
-        self.tokens = sum(B if f == "decode" else B * N for f in forms)
-        self.elem = self.q.element_size()
-        if "decode" in forms and "noncausal" not in forms:
-            # the cached state the decode steps continue from: a prefill of N tokens
-            la.la_kv_summary(self.k, self.v, self.S, self.z, self.phi)
+        self.seed = seed
+        self.ws = None
+        self.elem = 2 if dtype == "bf16" else 4
+        desc = la.make_desc(B, H, N, d, W.TORCH_DTYPES[dtype], self.phi, self.normalize)
+        if form == "decode":
+            T = wl.decode_steps
+            self.steps = T
+            _, k0, v0 = W.qkv(B, H, N, d, wl.sigma, seed, dtype, device)
+            self.S = torch.empty(B, H, d, d, dtype=torch.float32, device=device)
+            self.z = torch.empty(B, H, d, dtype=torch.float32, device=device)
+            la.la_kv_summary(k0, v0, self.S, self.z, self.phi)  # the cached state: a prefill of N tokens
+            del k0, v0
+            self.qs, self.ks, self.vs = W.decode_tokens(T, B, H, d, wl.sigma, seed + 1, dtype, device)
+            self.outs = torch.empty_like(self.qs)
+            self.tokens = B * T
+        else:
+            self.steps = 1
+            self.q, self.k, self.v = W.qkv(B, H, N, d, wl.sigma, seed, dtype, device)
+            if form == "prefix":
+                self.m = (W.prefix_mask_uniform(B, N, seed, device) if mask == "uniform"
+                          else W.prefix_mask_arange(B, N, device))
+            if form.endswith("_bwd"):
+                self.dout = W.upstream_grad(B, H, N, d, seed, dtype, device)
+                self.grads = tuple(torch.empty_like(self.q) for _ in range(3))
+            else:
+                self.out = torch.empty_like(self.q)
+            op = {"prefix": "prefix", "causal": "causal"}.get(form, form)
+            self.ws = la.workspace(desc, op, self.chunk, device)
+            self.tokens = B * N
 
-    def calls(self):
+    def run(self):
         la = self.la
-        table = {
-            "noncausal": lambda: la.la_noncausal(self.q, self.k, self.v, self.out_nc, self.S, self.z,
-                                                 self.phi, self.normalize, self.ws["noncausal"]),
-            "causal": lambda: la.la_causal_chunked(self.q, self.k, self.v, self.out_c, self.chunk,
-                                                   self.phi, self.normalize, self.ws["causal"]),
-            "prefix": lambda: la.la_prefix_mask(self.q, self.k, self.v, self.m, self.out_m, self.chunk,
-                                                self.phi, self.normalize, self.ws["prefix"]),
-            "decode": lambda: la.la_decode_step(self.q1, self.k1, self.v1, self.S, self.z, self.out_d,
-                                                self.phi, self.normalize),
-            "noncausal_bwd": lambda: la.la_noncausal_backward(self.q, self.k, self.v, self.dout,
-                                                              *self.grads["noncausal_bwd"], self.phi,
-                                                              self.normalize, self.ws["noncausal_bwd"]),
-            "causal_bwd": lambda: la.la_causal_backward(self.q, self.k, self.v, self.dout,
-                                                        *self.grads["causal_bwd"], self.phi, self.normalize,
-                                                        self.ws["causal_bwd"]),
-        }
-        return [(f, table[f]) for f in self.forms]
+        f = self.form
+        if f == "noncausal":
+            la.la_noncausal(self.q, self.k, self.v, self.out, None, None, self.phi, self.normalize, self.ws)
+        elif f == "causal":
+            la.la_causal_chunked(self.q, self.k, self.v, self.out, self.chunk, self.phi, self.normalize, self.ws)
+        elif f == "prefix":
+            la.la_prefix_mask(self.q, self.k, self.v, self.m, self.out, self.chunk, self.phi, self.normalize,
+                              self.ws)
+        elif f == "decode":
+            for t in range(self.steps):
+                la.la_decode_step(self.qs[t], self.ks[t], self.vs[t], self.S, self.z, self.outs[t], self.phi,
+                                  self.normalize)
+        elif f == "noncausal_bwd":
+            la.la_noncausal_backward(self.q, self.k, self.v, self.dout, *self.grads, self.phi, self.normalize,
+                                     self.ws)
+        elif f == "causal_bwd":
+            la.la_causal_backward(self.q, self.k, self.v, self.dout, *self.grads, self.phi, self.normalize, self.ws)
+
+    def run_from_host(self, h_ins, h_outs):
+        """The call through the public API with its inputs copied in from
+        pinned host memory and its outputs copied back (decode: per step)."""
+        if self.form == "decode":
+            hq, hk, hv = h_ins
+            (ho,) = h_outs
+            for t in range(self.steps):
+                self.qs[t].copy_(hq[t], non_blocking=True)
+                self.ks[t].copy_(hk[t], non_blocking=True)
+                self.vs[t].copy_(hv[t], non_blocking=True)
+                self.la.la_decode_step(self.qs[t], self.ks[t], self.vs[t], self.S, self.z, self.outs[t], self.phi,
+                                       self.normalize)
+                ho[t].copy_(self.outs[t], non_blocking=True)
+            return
+        ins, outs = self.device_io()
+        for d_t, h_t in zip(ins, h_ins):
+            d_t.copy_(h_t, non_blocking=True)
+        self.run()
+        for h_t, d_t in zip(h_outs, outs):
+            h_t.copy_(d_t, non_blocking=True)
+
+    def device_io(self):
+        if self.form == "decode":
+            return [self.qs, self.ks, self.vs], [self.outs]
+        ins = [self.q, self.k, self.v] + ([self.m] if self.form == "prefix" else []) \
+            + ([self.dout] if self.form.endswith("_bwd") else [])
+        outs = list(self.grads) if self.form.endswith("_bwd") else [self.out]
+        return ins, outs
 
     def algorithmic_bytes(self):
-        """Bytes each call must move at least: its inputs once and outputs once."""
+        """Bytes the call must move at least: its inputs once and outputs once."""
         t = self.B * self.H * self.N * self.d * self.elem     # one [B,H,N,d] tensor
         st = self.B * self.H * (self.d * self.d + self.d) * 4  # fp32 (S, z)
         one = self.B * self.H * self.d * self.elem
-        return {"noncausal": 4 * t + st, "causal": 4 * t, "prefix": 4 * t + self.B * self.N * 4,
-                "decode": 2 * st + 4 * one, "noncausal_bwd": 7 * t, "causal_bwd": 7 * t}
+        return {"noncausal": 4 * t, "causal": 4 * t, "prefix": 4 * t + self.B * self.N * 4,
+                "decode": self.steps * (2 * st + 4 * one), "noncausal_bwd": 7 * t, "causal_bwd": 7 * t}[self.form]
 
-    def kernel_bytes(self, call, kernel):
-        """Algorithmic bytes of one kernel of a call: the method's tensors it
-        must read or write once (Q, K, V, out, S, z, m). Scratch the library
-        keeps between its kernels (partial and block-state records, the
-        binning tables) is not counted, so a kernel that only moves scratch
-        (the prefix scan over block states) has none."""
-        t = self.B * self.H * self.N * self.d * self.elem
-        st = self.B * self.H * (self.d * self.d + self.d) * 4
-        one = self.B * self.H * self.d * self.elem
-        role = KERNEL_ROLE.get(kernel)
-        if call.endswith("_bwd"):
-            # gradients: q, k, v, dout read and dq, dk, dv written once over
-            # the sweeps (non-causal: q, dout -> dq; k, v -> dk, dv; causal:
-            # q, k, v, dout -> dq; q, k, v -> dk, dv); the reductions of
-            # (G, h) move scratch only
-            causal = call == "causal_bwd"
-            return {"kv": 2 * t, "fused": 2 * t, "bwd_q": (5 if causal else 3) * t,
-                    "bwd_kv": (5 if causal else 4) * t}.get(role, 0)
-        return {"kv": 2 * t, "reduce": st, "readout": 2 * t + st, "scan": 0, "sweep": 4 * t, "fused": 4 * t,
-                "bin": self.B * self.N * 4, "decode": 2 * st + 4 * one}.get(role, 0)
-
-    def host_io(self):
-        full = [f for f in self.forms if f != "decode"]
-        bwd = [f for f in self.forms if f.endswith("_bwd")]
-        ins = ([self.q, self.k, self.v] if full else []) + ([self.m] if "prefix" in self.forms else []) \
-            + ([self.q1, self.k1, self.v1] if "decode" in self.forms else []) + ([self.dout] if bwd else [])
-        outs = []
-        for f in self.forms:
-            if f.endswith("_bwd"):
-                outs += list(self.grads[f])
-            else:
-                outs.append({"noncausal": self.out_nc, "causal": self.out_c, "prefix": self.out_m,
-                             "decode": self.out_d}[f])
-        return ins, outs
+    def kernel_bytes(self, kernel):
+        """Algorithmic bytes of one kernel launch of the call: the method's
+        tensors it must read or write once (Q, K, V, out, S, z, m). Scratch
+        the library keeps between its kernels (partial and block-state
+        records, the binning tables) is not counted, so a kernel that only
+        moves scratch (the prefix scan over block states) has none."""
+        return kernel_bytes(self.form, kernel, self.B, self.H, self.N, self.d, self.elem)
 
 
-def kernel_times(step, calls, flush, reps):
-    """Per call: the mean duration (ms) of each kernel it launches, from the
-    library's timing events over `reps` replays of a graph of the call."""
-    la = step.la
-    la.la_timing_enable(True)
-    out = {}
-    try:
-        for name, fn in calls:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                fn()
-            for _ in range(3):
-                g.replay()
-            torch.cuda.synchronize()
-            acc = None
-            for _ in range(reps):
-                flush_l2(flush)
-                g.replay()
-                ms = la.la_timing_read()
-                acc = ms if acc is None else [a + b for a, b in zip(acc, ms)]
-            out[name] = [a / reps for a in acc]
-            del g
-    finally:
-        la.la_timing_enable(False)
-    return out
+def kernel_bytes(form, kernel, B, H, N, d, elem):
+    t = B * H * N * d * elem
+    st = B * H * (d * d + d) * 4
+    one = B * H * d * elem
+    role = KERNEL_ROLE.get(kernel)
+    if form.endswith("_bwd"):
+        # gradients: q, k, v, dout read and dq, dk, dv written once over
+        # the sweeps (non-causal: q, dout -> dq; k, v -> dk, dv; causal:
+        # q, k, v, dout -> dq; q, k, v -> dk, dv); the reductions of
+        # (G, h) move scratch only
+        causal = form == "causal_bwd"
+        return {"kv": 2 * t, "fused": 2 * t, "bwd_q": (5 if causal else 3) * t,
+                "bwd_kv": (5 if causal else 4) * t}.get(role, 0)
+    return {"kv": 2 * t, "reduce": st, "readout": 2 * t + st, "scan": 0, "sweep": 4 * t, "fused": 4 * t,
+            "bin": B * N * 4, "decode": 2 * st + 4 * one}.get(role, 0)
 
 
 def flush_l2(buf):
@@ -359,6 +382,179 @@ def aggregate_tokens_per_s(tokens_per_step, steps, world, seconds):
     return tokens_per_step * steps * world / seconds
 
 
+def kernel_times(call, flush, reps):
+    """Mean duration (ms) of each kernel the call launches, from the
+    library's timing events over `reps` replays of a graph of the call, L2
+    flushed before each. Decode: the 1024-step call's time over 1024 (one
+    kernel, back to back)."""
+    la = call.la
+    g = torch.cuda.CUDAGraph()
+    if call.form == "decode":
+        with torch.cuda.graph(g):
+            call.run()
+        g.replay()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            flush_l2(flush)
+            a.record()
+            g.replay()
+            b.record()
+        torch.cuda.synchronize()
+        return [sum(a.elapsed_time(b) for a, b in ev) / reps / call.steps]
+    la.la_timing_enable(True)
+    try:
+        with torch.cuda.graph(g):
+            call.run()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        acc = None
+        for _ in range(reps):
+            flush_l2(flush)
+            g.replay()
+            ms = la.la_timing_read()
+            acc = ms if acc is None else [a + b for a, b in zip(acc, ms)]
+    finally:
+        la.la_timing_enable(False)
+    del g
+    return [a / reps for a in acc]
+
+
+def measure_case(case, args, rank, world, device, flush, sampler, peak, heads=0):
+    """Times one case; returns its JSON fields (value, roofline, e2e, ...)."""
+    calls = [Call(W.WORKLOADS[w], dt, form, mask, rank_seed(W.WORKLOADS[w], rank), device, heads)
+             for w, dt, form, mask in CASES[case]]
+    warm = max(args.warmup, 3)
+    for _ in range(warm):
+        for c in calls:
+            c.run()
+    torch.cuda.synchronize()
+    graphs = []
+    for c in calls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            c.run()
+        graphs.append(g)
+    for _ in range(warm):
+        for g in graphs:
+            g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(device)
+
+    K = args.steps
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    # Every call starts with a cold L2 (a 256 MiB write before each call,
+    # outside the events), so each reads its inputs from HBM; a step's time
+    # is the sum of its calls' times.
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+          for _ in range(K)]
+    with sampler.timed():
+        for i in range(K):
+            for j, g in enumerate(graphs):
+                flush_l2(flush)
+                ev[i][j][0].record(stream)
+                g.replay()
+                ev[i][j][1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    per_call_ms = [sum(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(K)) / K for j in range(len(calls))]
+    del graphs
+
+    # end to end through the public API: pinned host inputs in, outputs back
+    h_io = []
+    h2d = d2h = 0
+    for c in calls:
+        ins, outs = c.device_io()
+        h_ins = [t.cpu().pin_memory() for t in ins]
+        h_outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        h2d += sum(t.numel() * t.element_size() for t in h_ins)
+        d2h += sum(t.numel() * t.element_size() for t in h_outs)
+        h_io.append((h_ins, h_outs))
+    Ke = max(1, min(K, 20))
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+    torch.cuda.synchronize()
+    for i in range(Ke):
+        flush_l2(flush)
+        e_ev[i][0].record(stream)
+        for c, (h_ins, h_outs) in zip(calls, h_io):
+            c.run_from_host(h_ins, h_outs)
+        e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_s = sum(a.elapsed_time(b) for a, b in e_ev) / 1e3
+    del h_io
+
+    # each kernel's own duration (per-kernel timing events)
+    kt = [kernel_times(c, flush, max(3, min(K, 20))) for c in calls]
+
+    # every call reports expired bounded waits in its workspace error word
+    bad_flags = {}
+    for c in calls:
+        if c.ws is not None:
+            f = c.la.la_last_error(c.ws)[1]
+            if f:
+                bad_flags[f"{c.name}/{c.form}"] = f
+
+    step_ms = sum(per_call_ms)
+    t_s, e2e_s = max_over_ranks([step_ms / 1e3 * K, e2e_s], device)
+    tokens = sum(c.tokens for c in calls)
+    value = aggregate_tokens_per_s(tokens, K, world, t_s)
+    e2e_value = aggregate_tokens_per_s(tokens, Ke, world, e2e_s)
+
+    per_call, cands, launches = {}, [], 0
+    for c, ms, ktimes in zip(calls, per_call_ms, kt):
+        names = ["decode_kernel"] if c.form == "decode" else kernel_names(c.form, c.dtype, c.d, len(ktimes))
+        launches += len(names) * c.steps
+        s_call = ms / 1e3
+        a = c.algorithmic_bytes()
+        entry = {"us": round(ms * 1e3, 2), "GB_s": round(a / s_call / 1e9, 1),
+                 "frac_hbm": round(a / s_call / 1e9 / peak, 4), "share": round(ms / step_ms, 3), "kernels": []}
+        for i, (kn, kms) in enumerate(zip(names, ktimes)):
+            kb = c.kernel_bytes(kn)
+            entry["kernels"].append({"kernel": kn, "us": round(kms * 1e3, 2),
+                                     "GB_s": round(kb / (kms / 1e3) / 1e9, 1) if kb else None,
+                                     "frac_hbm": round(kb / (kms / 1e3) / 1e9 / peak, 4) if kb else None})
+            if kb:
+                cands.append((kms * c.steps, kms, c, kn, i, kb))
+        per_call[f"{c.name}/{c.form}"] = entry
+
+    # roofline of the dominant kernel: the one with the largest time in the
+    # step, its algorithmic bytes over its own timed duration
+    _, dom_ms, dom_call, dom_kernel, di, dom_bytes = max(cands, key=lambda x: x[0])
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+    dtypes = sorted({c.dtype for c in calls})
+    out = {
+        "value": value,
+        "unit": "tokens/s",
+        "ms_per_step": step_ms,
+        "dtype": dtypes[0] if len(dtypes) == 1 else "+".join(dtypes),
+        "config": {"workload": CASE_TEXT[case] + (f" (scaled to {heads} heads)" if heads else ""),
+                   "calls": [f"{c.name}: B={c.B} H={c.H} N={c.N} d={c.d} {c.dtype} {c.form}" for c in calls],
+                   "global_batch": sum(c.B for c in calls) * world,
+                   "seq_len": max(c.N for c in calls), "parallelism": f"dp{world}",
+                   "l2": "flushed before every call (256 MiB write)",
+                   "launch": "one CUDA graph per call" + (" (decode: 1024 steps in one graph)"
+                                                          if any(c.form == "decode" for c in calls) else ""),
+                   "tokens_per_step_per_gpu": tokens},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches * K,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "traffic": recorded_traffic(dom_call.name, dom_call.dtype, f"{dom_call.form}/{di}"),
+                     "kernel": f"{dom_kernel} (kernel {di} of {dom_call.name}/{dom_call.form})",
+                     "kernel_us": round(dom_ms * 1e3, 2), "algorithmic_bytes": dom_bytes},
+        "per_call": per_call,
+    }
+    if bad_flags:
+        out["error_flags"] = bad_flags
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(calls, min_seconds=10.0 if case == HEADLINE else 3.0)
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
@@ -370,165 +566,40 @@ def run_ours(args, rank, world, local_rank):
         build_mod.build()
     if world > 1:
         torch.distributed.barrier()
-    wl = W.WORKLOADS[args.workload]
-    dtype = args.dtype if args.dtype in wl.dtypes else wl.dtypes[0]
-    forms = Step.ALL_FORMS if args.workload == "multi_head" else wl.forms
-    step = Step(wl, dtype, rank_seed(wl, rank), device, forms)
-    calls = step.calls()
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
-
-    for _ in range(max(args.warmup, 3)):
-        for _, fn in calls:
-            fn()
-    torch.cuda.synchronize()
-    graphs = []
-    for _, fn in calls:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        graphs.append(g)
-    for _ in range(max(args.warmup, 3)):
-        for g in graphs:
-            g.replay()
-    torch.cuda.synchronize()
-    stream = torch.cuda.current_stream(device)
-
-    K = args.steps
-    sampler = ClockSampler(device)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    # Every call starts with a cold L2 (a 256 MiB write between calls, outside
-    # the events), so each call reads its inputs from HBM; a step's time is
-    # the sum of its calls' times.
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(len(calls))] for _ in range(K)]
-    with sampler:
-        for i in range(K):
-            for j, g in enumerate(graphs):
-                flush_l2(flush)
-                ev[i][j][0].record(stream)
-                g.replay()
-                ev[i][j][1].record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    per_call = {name: 0.0 for name, _ in calls}
-    total_ms = 0.0
-    for i in range(K):
-        for j, (name, _) in enumerate(calls):
-            ms = ev[i][j][0].elapsed_time(ev[i][j][1])
-            per_call[name] += ms
-            total_ms += ms
-    t_s = total_ms / 1e3
-
-    # end to end through the public API: pinned host inputs in, outputs back
-    ins, outs = step.host_io()
-    h_ins = [t.cpu().pin_memory() for t in ins]
-    h_outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
-    h2d = sum(t.numel() * t.element_size() for t in h_ins)
-    d2h = sum(t.numel() * t.element_size() for t in h_outs)
-    Ke = max(1, min(K, 50))
-    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
-    torch.cuda.synchronize()
-    for i in range(Ke):
-        flush_l2(flush)
-        e_ev[i][0].record(stream)
-        for d_t, h_t in zip(ins, h_ins):
-            d_t.copy_(h_t, non_blocking=True)
-        for _, fn in calls:
-            fn()
-        for h_t, d_t in zip(h_outs, outs):
-            h_t.copy_(d_t, non_blocking=True)
-        e_ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_s = sum(a.elapsed_time(b) for a, b in e_ev) / 1e3
-
-    # each kernel's own duration: the calls replayed again from graphs
-    # captured with the library's per-kernel timing events (an event node
-    # between two kernels; the call-level numbers above come from graphs
-    # without them), L2 flushed before every replay, averaged over the replays
-    kt = kernel_times(step, calls, flush, max(3, min(K, 20)))
-
-    # every call reports expired bounded waits in its workspace error word
-    flags = {op: step.la.la_last_error(ws)[1] for op, ws in step.ws.items()}
-    bad_flags = {op: f for op, f in flags.items() if f}
-
-    t_s, e2e_s = max_over_ranks([t_s, e2e_s], device)
-    value = aggregate_tokens_per_s(step.tokens, K, world, t_s)
-    e2e_value = aggregate_tokens_per_s(step.tokens, Ke, world, e2e_s)
-
     peaks = load_peaks()
     peak = peaks.get("hbm_gbs", 6650.0)
-    names = call_kernels(wl, dtype)
-    per_kernel = {}
-    for name in per_call:
-        s_call = per_call[name] / 1e3 / K
-        a = step.algorithmic_bytes()[name]
-        entry = {"us": round(s_call * 1e6, 2), "GB_s": round(a / s_call / 1e9, 1),
-                 "frac_hbm": round(a / s_call / 1e9 / peak, 3),
-                 "share": round(per_call[name] / sum(per_call.values()), 3), "kernels": []}
-        for i, ms in enumerate(kt.get(name, [])):
-            kn = names[name][i] if i < len(names[name]) else f"kernel{i}"
-            kb = step.kernel_bytes(name, kn)
-            entry["kernels"].append({"kernel": kn, "us": round(ms * 1e3, 2),
-                                     "GB_s": round(kb / (ms / 1e3) / 1e9, 1) if kb else None,
-                                     "frac_hbm": round(kb / (ms / 1e3) / 1e9 / peak, 3) if kb else None})
-        per_kernel[name] = entry
-
-    # roofline of the dominant kernel: the (call, kernel) with the largest
-    # time in the step, its algorithmic bytes over its own timed duration
-    cands = [(ms, name, i) for name, lst in kt.items() for i, ms in enumerate(lst)
-             if step.kernel_bytes(name, names[name][i] if i < len(names[name]) else "") > 0]
-    dom_ms, dom, di = max(cands)
-    dom_kernel = names[dom][di]
-    dom_bytes = step.kernel_bytes(dom, dom_kernel)
-    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-    result = {
-        "metric": "tokens/sec (fwd, 1xB200) and % of HBM / bf16 tensor-core roofline per kernel",
-        "value": value,
-        "unit": "tokens/s",
-        "n_gpus": world,
-        "steps": K,
-        "warmup": max(args.warmup, 3),
-        "ms_per_step": total_ms / K,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": dtype,
-        "data": "synthetic",
-        "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} N={wl.N} d={wl.d} {dtype} phi={wl.phi} "
-                               f"normalize={int(wl.normalize)} chunk={wl.chunk}; step = "
-                               + " + ".join({"noncausal": "noncausal", "causal": "causal",
-                                             "prefix": "prefix mask (m uniform)",
-                                             "decode": "1 decode step",
-                                             "noncausal_bwd": "noncausal gradients",
-                                             "causal_bwd": "causal gradients"}[f] for f in forms),
-                   "global_batch": wl.B * world, "seq_len": wl.N, "parallelism": f"dp{world}",
-                   "l2": "flushed between steps (256 MiB write)", "launch": "one CUDA graph per call",
-                   "tokens_per_step_per_gpu": step.tokens},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": sum(len(names[n]) for n, _ in calls) * K,
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": recorded_traffic(wl.name, dtype, f"{dom}/{di}"),
-                     "kernel": f"{dom_kernel} (kernel {di} of la_{dom})",
-                     "kernel_us": round(dom_ms * 1e3, 2), "peak_source": peaks.get("_src"),
-                     "algorithmic_bytes": dom_bytes},
-        "per_call": per_kernel,
-        "clocks": sampler.summary(),
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(step, heads=2)
-    if bad_flags:
-        result["error_flags"] = bad_flags
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    sampler = ClockSampler(device)
+    sampler.start()
+    try:
+        head = measure_case(args.case, args, rank, world, device, flush, sampler, peak, args.scale_heads)
+        torch.cuda.empty_cache()  # the case's buffers are released once it returns
+        others = {}
+        if not args.no_configs:
+            for case in CASES:
+                if case != args.case:
+                    others[case] = measure_case(case, args, rank, world, device, flush, sampler, peak)
+                    torch.cuda.empty_cache()
+    finally:
+        sampler.stop()
+    result = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+              "warmup": max(args.warmup, 3), "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+              "scaling": "weak", "vs_baseline": None, "dtype": head["dtype"], "data": "synthetic"}
+    for key in ("config", "e2e", "gpu_launches", "roofline", "per_call", "cpu_baseline", "error_flags"):
+        if key in head:
+            result[key] = head[key]
+    result["roofline"]["peak_source"] = peaks.get("_src")
+    result["clocks"] = sampler.summary()
+    if others:
+        result["per_config"] = others
+    bad = {k: v for k, v in [(args.case, head.get("error_flags"))] + [(c, o.get("error_flags"))
+                                                                        for c, o in others.items()] if v}
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
-    if bad_flags:
-        raise SystemExit(f"library error flags set during the run: {bad_flags}")
+    if bad:
+        raise SystemExit(f"library error flags set during the run: {bad}")
 
 
 def library_source_hash():
@@ -544,8 +615,8 @@ def library_source_hash():
 
 
 def recorded_traffic(workload, dtype, key):
-    """DRAM bytes (read + write) of one call ("causal") or one of its kernels
-    ("causal/2", by launch index) from the ncu capture in
+    """DRAM bytes (read + written) of one launch of a call's kernel
+    ("causal/2": kernel 2 of the causal call) from the ncu launch list in
     profiles/traffic.json; None when none was taken for this workload and
     key, or the kernels changed since."""
     try:
@@ -582,122 +653,192 @@ def _blas_threads():
         return 1
 
 
-def oracle_sample(q, k, v, m, q1, k1, v1, phi, normalize, heads, forms, dout=None):
-    """Runs the oracle's forms on the first `heads` heads of sequence 0.
-    Returns (seconds, tokens processed), tokens counted like the GPU step
-    (B*N per full-sequence form, B per decode step) scaled by heads/H."""
+# Tokens of one head the oracle's sample takes per call: all of them where
+# the oracle's form is a few matrix products, a prefix of the sequence where
+# it is a per-token loop (causal, prefix mask), the first steps of decode.
+SAMPLE_TOKENS = {"noncausal": None, "causal": 4096, "prefix": 2048, "decode": 256,
+                 "noncausal_bwd": 1024, "causal_bwd": 1024}
+
+
+def oracle_sample(call_specs):
+    """Runs the oracle, as it stands, on one head of each call (sequence 0,
+    head 0; a prefix of the tokens where SAMPLE_TOKENS says so). Returns
+    (seconds, tokens), tokens counted like the GPU step (B*N per
+    full-sequence call, sequences x steps for decode) in the proportion of
+    the work sampled: one head of H, n of N tokens, t of T steps."""
     import oracle
+    total_t, tokens = 0.0, 0.0
+    for spec in call_specs:
+        form, phi, normalize, H = spec["form"], spec["phi"], spec["normalize"], spec["H"]
+        Q, K, V = spec["Q"], spec["K"], spec["V"]
+        n = Q.shape[0]
+        t0 = time.perf_counter()
+        if form == "noncausal":
+            oracle.noncausal(Q, K, V, phi, normalize)
+        elif form == "causal":
+            oracle.causal(Q, K, V, phi, normalize)
+        elif form == "prefix":
+            oracle.prefix_mask(Q, K, V, spec["m"], phi, normalize)
+        elif form == "decode":
+            S, z = spec["S"], spec["z"]
+            for t in range(n):
+                _, S, z = oracle.decode_step(S, z, Q[t], K[t], V[t], phi, normalize)
+        else:
+            oracle.backward_dense(Q, K, V, spec["G"], form[:-4], None, phi, normalize)
+        total_t += time.perf_counter() - t0
+        if form == "decode":
+            tokens += spec["B"] * n / H
+        else:
+            tokens += spec["B"] * spec["N"] * (n / spec["N"]) / H
+    return total_t, tokens
+
+
+def sample_specs(calls_or_cases):
+    """The oracle's inputs for each call: head 0 of sequence 0, exact fp64
+    copies of the GPU inputs (or, for the reference arm, of the same seeded
+    inputs drawn on the host)."""
+    specs = []
     f = lambda t: t.detach().to(torch.float64).cpu().numpy()
-    H = q.shape[1]
-    Q, K, V = f(q[0, :heads]), f(k[0, :heads]), f(v[0, :heads])
-    M = m[0].cpu().numpy()
-    q1_, k1_, v1_ = f(q1[0, :heads, 0]), f(k1[0, :heads, 0]), f(v1[0, :heads, 0])
-    G = f(dout[0, :heads]) if dout is not None else None
-    N = Q.shape[1]
-    t0 = time.perf_counter()
-    for h in range(heads):
-        S = z = None
-        if "noncausal" in forms:
-            _, S, z = oracle.noncausal(Q[h], K[h], V[h], phi, normalize)
-        if "causal" in forms:
-            oracle.causal(Q[h], K[h], V[h], phi, normalize)
-        if "prefix" in forms:
-            oracle.prefix_mask(Q[h], K[h], V[h], M, phi, normalize)
-        if "decode" in forms:
-            if S is None:
-                S, z = oracle.kv_summary(K[h], V[h], phi)
-            oracle.decode_step(S, z, q1_[h], k1_[h], v1_[h], phi, normalize)
-        for fm in ("noncausal_bwd", "causal_bwd"):
-            if fm in forms:
-                oracle.backward_dense(Q[h], K[h], V[h], G[h], fm[:-4], None, phi, normalize)
-    dt = time.perf_counter() - t0
-    per_seq = sum(1 if fm == "decode" else N for fm in forms)
-    return dt, per_seq * heads / H
+    for c in calls_or_cases:
+        n = SAMPLE_TOKENS[c.form] or c.N
+        spec = {"form": c.form, "phi": c.phi, "normalize": c.normalize, "H": c.H, "B": c.B, "N": c.N}
+        if c.form == "decode":
+            n = min(n, c.steps)
+            spec.update(Q=f(c.qs[:n, 0, 0, 0]), K=f(c.ks[:n, 0, 0, 0]), V=f(c.vs[:n, 0, 0, 0]),
+                        S=f(c.S[0, 0]), z=f(c.z[0, 0]))
+            spec["N"] = c.steps
+        else:
+            n = min(n, c.N)
+            spec.update(Q=f(c.q[0, 0, :n]), K=f(c.k[0, 0, :n]), V=f(c.v[0, 0, :n]))
+            if c.form == "prefix":
+                spec["m"] = np.minimum(c.m[0, :n].cpu().numpy(), n - 1) if n < c.N else c.m[0].cpu().numpy()
+            if c.form.endswith("_bwd"):
+                spec["G"] = f(c.dout[0, 0, :n])
+        specs.append(spec)
+    return specs
 
 
-def cpu_baseline(step, heads=2, min_seconds=10.0):
+def cpu_baseline(calls, min_seconds=10.0):
     """The oracle, as it is, on the host cores: repeated passes over a
-    sample of heads until about `min_seconds` of CPU work."""
+    sample of the case until about `min_seconds` of CPU work."""
+    specs = sample_specs(calls)
     total_t, total_tok, passes = 0.0, 0.0, 0
     while total_t < min_seconds:
-        dt, tok = oracle_sample(step.q, step.k, step.v, step.m, step.q1, step.k1, step.v1,
-                                step.phi, step.normalize, heads, step.forms, getattr(step, "dout", None))
+        dt, tok = oracle_sample(specs)
         total_t += dt
         total_tok += tok
         passes += 1
+    what = ", ".join(f"{c.name}/{c.form}: head 0 of {c.H}, "
+                     + (f"{min(SAMPLE_TOKENS[c.form], c.steps)} of {c.steps} steps" if c.form == "decode"
+                        else f"{min(SAMPLE_TOKENS[c.form] or c.N, c.N)} of {c.N} tokens")
+                     for c in calls)
     return {"value": total_tok / total_t, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"oracle (numpy fp64) on {heads} of {step.H} heads of sequence 0, forms "
-                      f"{'+'.join(step.forms)}, N={step.N}, {passes} passes, {total_t:.1f} s; tokens "
-                      f"scaled by heads/H; Python loops single-threaded, BLAS calls may use the cores"}
+            "sample": f"oracle (numpy fp64) on {what}; {passes} passes, {total_t:.1f} s; tokens scaled by the "
+                      f"share of the work sampled; Python loops single-threaded, BLAS calls may use the cores"}
+
+
+class _HostCall:
+    """The inputs of one call of a case drawn on the host (reference arm):
+    one head of the workload from the same seeded generators, drawn by the
+    host's generator (the same distributions and shapes; the values differ
+    from the device's draw), only what the oracle's sample reads."""
+
+    def __init__(self, wl, dtype, form, mask):
+        self.wl, self.form, self.name = wl, form, wl.name
+        self.B, self.H, self.N, self.d = wl.B, wl.H, wl.N, wl.d
+        self.phi, self.normalize, self.dtype = wl.phi, wl.normalize, dtype
+        n = SAMPLE_TOKENS[form] or wl.N
+        if form == "decode":
+            self.steps = wl.decode_steps
+            n = min(n, self.steps)
+            qs, ks, vs = W.decode_tokens(n, 1, 1, wl.d, wl.sigma, wl.seed + 1, dtype, "cpu")
+            self.qs, self.ks, self.vs = qs, ks, vs
+            _, k0, v0 = W.qkv(1, 1, wl.N, wl.d, wl.sigma, wl.seed, dtype, "cpu")
+            import oracle
+            S, z = oracle.kv_summary(k0[0, 0].double().numpy(), v0[0, 0].double().numpy(), wl.phi)
+            self.S, self.z = torch.from_numpy(S)[None, None], torch.from_numpy(z)[None, None]
+        else:
+            q, k, v = W.qkv(1, 1, wl.N, wl.d, wl.sigma, wl.seed, dtype, "cpu")
+            self.q, self.k, self.v = q, k, v
+            if form == "prefix":
+                self.m = (W.prefix_mask_uniform(wl.B, wl.N, wl.seed, "cpu") if mask == "uniform"
+                          else W.prefix_mask_arange(wl.B, wl.N, "cpu"))
+            if form.endswith("_bwd"):
+                self.dout = W.upstream_grad(1, 1, wl.N, wl.d, wl.seed, dtype, "cpu")
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    wl = W.WORKLOADS[args.workload]
-    dtype = args.dtype if args.dtype in wl.dtypes else wl.dtypes[0]
-    forms = Step.ALL_FORMS if args.workload == "multi_head" else wl.forms
-    q, k, v = W.qkv(1, wl.H, wl.N, wl.d, wl.sigma, wl.seed, dtype, "cpu")
-    m = W.prefix_mask_uniform(1, wl.N, wl.seed, "cpu")
-    q1, k1, v1 = (t[0] for t in W.decode_tokens(1, 1, wl.H, wl.d, wl.sigma, wl.seed, dtype, "cpu"))
-    dout = W.upstream_grad(1, wl.H, wl.N, wl.d, wl.seed, dtype, "cpu")
-    heads = 1
+    calls = [_HostCall(W.WORKLOADS[w], dt, form, mask) for w, dt, form, mask in CASES[args.case]]
+    specs = sample_specs(calls)
     for _ in range(args.warmup):
-        oracle_sample(q, k, v, m, q1, k1, v1, wl.phi, wl.normalize, heads, forms, dout)
+        oracle_sample(specs)
     total, tokens = 0.0, 0.0
     for _ in range(args.steps):
-        dt, tok = oracle_sample(q, k, v, m, q1, k1, v1, wl.phi, wl.normalize, heads, forms, dout)
+        dt, tok = oracle_sample(specs)
         total += dt
         tokens += tok
     value = tokens / total
     cores = _blas_threads()
-    sample = (f"oracle (numpy fp64) on {heads} of {wl.H} heads of one sequence per step, forms "
-              f"{'+'.join(forms)}, N={wl.N}; tokens scaled by heads/H")
+    what = ", ".join(f"{c.name}/{c.form}: head 0 of {c.H}, "
+                     + (f"{min(SAMPLE_TOKENS[c.form], c.steps)} of {c.steps} steps" if c.form == "decode"
+                        else f"{min(SAMPLE_TOKENS[c.form] or c.N, c.N)} of {c.N} tokens") for c in calls)
+    sample = (f"oracle (numpy fp64) per step on {what}; tokens scaled by the share of the work sampled")
     print(json.dumps({
-        "impl": "reference",
-        "metric": "tokens/sec (fwd, 1xB200) and % of HBM / bf16 tensor-core roofline per kernel",
+        "impl": "reference", "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} N={wl.N} d={wl.d} {dtype} inputs",
-                   "global_batch": wl.B, "seq_len": wl.N, "parallelism": "host cores"},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+        "config": {"workload": CASE_TEXT[args.case] + " (inputs; the oracle computes in fp64)",
+                   "global_batch": sum(c.B for c in calls), "seq_len": max(c.N for c in calls),
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
 
-def record_traffic(csv_path, workload, dtype):
-    """Per call of the last complete step in an ncu launch list: the sum of
-    dram__bytes_read.sum + dram__bytes_write.sum over the call's kernels."""
+def record_traffic(csv_path, case, scale):
+    """Per kernel launch of the last complete step of `case` in an ncu launch
+    list: dram__bytes_read.sum + dram__bytes_write.sum, times `scale` (a
+    capture of a smaller problem scaled to the case's size by the units each
+    kernel processes), stored per workload/dtype/call/kernel index."""
     import csv
     with open(csv_path) as f:
         rows = [r for r in csv.reader(f)]
     head = next(i for i, r in enumerate(rows) if r and r[0] == "ID")
     h = rows[head]
     ik, im, iv, iu = (h.index(c) for c in ("Kernel Name", "Metric Name", "Metric Value", "Metric Unit"))
-    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    units = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
     launches = {}
     for r in rows[head + 1:]:
         if len(r) <= iv or "la::" not in r[ik]:
             continue
         rec = launches.setdefault(int(r[0]), {"name": r[ik], "bytes": 0.0})
         if r[im] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
-            rec["bytes"] += float(r[iv].replace(",", "")) * scale.get(r[iu], 1)
+            rec["bytes"] += float(r[iv].replace(",", "")) * units.get(r[iu], 1)
     seq = [launches[i] for i in sorted(launches)]
-    forms = Step.ALL_FORMS if workload == "multi_head" else W.WORKLOADS[workload].forms
-    names = call_kernels(W.WORKLOADS[workload], dtype)
-    want = [(f, k) for f in forms for k in names[f]]
-    for start in range(len(seq) - len(want), -1, -1):
-        if all(k in seq[start + n]["name"] for n, (_, k) in enumerate(want)):
-            break
-    else:
-        raise SystemExit("the launch list holds no complete step of this workload")
-    per_call, per_kernel = {}, {}
-    for n, (f, _) in enumerate(want):
-        per_call[f] = per_call.get(f, 0.0) + seq[start + n]["bytes"]
-        i = sum(1 for g, _ in want[:n] if g == f)  # the kernel's index within its call
-        per_kernel[f"{f}/{i}"] = seq[start + n]["bytes"]
+    out_bytes = {}
+    for w, dt, form, mask in CASES[case]:
+        # the last complete launch of this call in the list (the bench's
+        # per-kernel timing replays each call in turn after the timed steps)
+        wl = W.WORKLOADS[w]
+        name = wl.name if form != "prefix" or mask == "uniform" else f"{wl.name}_{mask}"
+        table = (TC_KERNELS if dt == "bf16" and wl.d in (64, 128) else SIMT_KERNELS)[form]
+        found = None
+        for start in range(len(seq) - 1, -1, -1):
+            for count in sorted(table, reverse=True):
+                names = kernel_names(form, dt, wl.d, count)
+                if start + len(names) <= len(seq) and all(k in seq[start + n]["name"] for n, k in enumerate(names)):
+                    found = (start, names)
+                    break
+            if found:
+                break
+        if not found:
+            raise SystemExit(f"the launch list holds no complete {name}/{form} call")
+        start, names = found
+        for n in range(len(names)):
+            out_bytes[f"{name}/{dt}/{form}/{n}"] = int(seq[start + n]["bytes"] * scale)
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -706,23 +847,19 @@ def record_traffic(csv_path, workload, dtype):
         out = {}
     if out.get("source_hash") != library_source_hash():
         out = {"source_hash": library_source_hash(), "bytes": {}}
-    out["note"] = ("DRAM bytes read + written per library call (workload/dtype/call, summed over "
-                   "the call's kernels) and per kernel (workload/dtype/call/index in launch order), "
-                   "from an ncu launch list (cold cache per kernel); valid for the CUDA sources "
-                   "with this hash")
-    for f, b in per_call.items():
-        out["bytes"][f"{workload}/{dtype}/{f}"] = int(b)
-    for key, b in per_kernel.items():
-        out["bytes"][f"{workload}/{dtype}/{key}"] = int(b)
+    out["note"] = ("DRAM bytes read + written per kernel launch (workload/dtype/call/index in launch order) "
+                   "from an ncu launch list (cold cache per kernel); valid for the CUDA sources with this "
+                   "hash; launches of a reduced-size capture are scaled to the workload's size")
+    out["bytes"].update(out_bytes)
     with open(path, "w") as f:
         json.dump(out, f, indent=1, sort_keys=True)
-    print(json.dumps(per_call))
+    print(json.dumps(out_bytes))
 
 
 def main():
     args = parse()
     if args.record_traffic:
-        record_traffic(args.record_traffic, args.workload, args.dtype)
+        record_traffic(args.record_traffic, args.case, args.traffic_scale)
         return
     rank, world, local_rank = dist_env()
     if args.impl == "reference":

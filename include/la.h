@@ -99,9 +99,14 @@ typedef struct {
 } la_desc;
 
 /* Bytes of workspace `op` needs for `desc` (chunk is used by LA_OP_CAUSAL and
- * LA_OP_PREFIX only; it must be 64 or 128 for those and is ignored otherwise). Returns 0 when the request is invalid or unsupported,
- * and for ops that need none (LA_OP_DECODE). A valid request that needs a
- * workspace always gets a non-zero size. Pure host function. */
+ * LA_OP_PREFIX only; it must be 64 or 128 for those and is ignored
+ * otherwise). Returns 0 when the request is invalid or unsupported, and for
+ * ops that need none (LA_OP_DECODE). A valid request that needs a workspace
+ * always gets a non-zero size. Host function; launches nothing. The work is
+ * split to fill the SMs of the current device, so the size is for that
+ * device (with no CUDA device, for a 148-SM B200): a workspace sized on one
+ * device can be too small for another, which the call then rejects with
+ * LA_ERR_WORKSPACE. */
 LA_API size_t la_workspace_size(const la_desc* desc, int32_t op, int32_t chunk);
 
 /* KV summary of every head (nx source, KV-summary loop):
@@ -200,21 +205,24 @@ LA_API la_status la_decode_step(const la_desc* desc, const void* q, const void* 
  * its tensors). The pages describe no such variant; it exists for these
  * callers only.
  *
- * Same inputs, outputs and result as la_kv_summary. The scratch the KV
- * summary needs lives in a device array of 32 MiB inside the library, which
- * every GPU that loads the library holds until the process exits; a problem
- * whose la_workspace_size(desc, LA_OP_KV_SUMMARY, 0) exceeds 32 MiB is
- * rejected with LA_ERR_WORKSPACE before anything is launched. The call
- * allocates nothing: it issues a 4-byte cudaMemsetAsync (clearing the
- * array's error word) and the kernels.
- * - The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, once per device, with that device current); make
- *   that first call before any stream capture.
+ * Same inputs, outputs, result and argument checks as la_kv_summary. The
+ * scratch the KV summary needs lives in a device array of 32 MiB inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits; a problem whose la_workspace_size(desc, LA_OP_KV_SUMMARY, 0)
+ * exceeds 32 MiB is rejected with LA_ERR_WORKSPACE before anything is
+ * launched. The call allocates nothing: it issues a 4-byte cudaMemsetAsync
+ * (clearing the array's error word), the KV-summary kernels and one small
+ * kernel that checks the error word.
+ * - The first call in each CUDA context looks up the array's device address
+ *   (cudaGetSymbolAddress, with that context current) and keeps it for that
+ *   context; make that first call before any stream capture. A device reset
+ *   creates a new context, whose first call looks the address up again.
  * - All calls share the one array, which keeps the last call's contents:
  *   calls that may overlap on the GPU (different streams, or different host
  *   threads) race and give undefined results; serialize them.
- * - An expired bounded wait leaves S_out and z_out undefined and is recorded
- *   only in the array's error word, which no entry point reads. */
+ * - An expired bounded wait (an internal error; see LA_ERR_TIMEOUT) fills
+ *   S_out and z_out with NaN: this call has no workspace that la_last_error
+ *   could read. */
 LA_API la_status la_kv_summary_static(const la_desc* desc, const void* k, const void* v,
                                       float* S_out, float* z_out, void* stream);
 

@@ -129,6 +129,26 @@ def _same(ref, *ts):
             raise ValueError("q, k, v and out must share shape, dtype and device")
 
 
+def _state(S, z, ref):
+    """S [B,H,d,d] and z [B,H,d]: contiguous float32 on ref's device (the
+    library writes or reads exactly that many floats)."""
+    B, H, _, d = ref.shape
+    if S.dtype != torch.float32 or tuple(S.shape) != (B, H, d, d) or S.device != ref.device:
+        raise ValueError(f"S must be float32 [{B}, {H}, {d}, {d}] on {ref.device}")
+    if z.dtype != torch.float32 or tuple(z.shape) != (B, H, d) or z.device != ref.device:
+        raise ValueError(f"z must be float32 [{B}, {H}, {d}] on {ref.device}")
+    if not S.is_contiguous() or not z.is_contiguous():
+        raise ValueError("S and z must be contiguous")
+
+
+def _ws(ws, ref):
+    """A workspace: a contiguous uint8 buffer on ref's device (the library
+    checks its size)."""
+    if ws.dtype != torch.uint8 or ws.device != ref.device or not ws.is_contiguous():
+        raise ValueError(f"the workspace must be a contiguous uint8 tensor on {ref.device}")
+    return ws
+
+
 def la_version() -> int:
     return int(lib().la_version())
 
@@ -158,8 +178,8 @@ def la_kv_summary(k, v, S_out=None, z_out=None, phi="relu1", ws=None, stream=Non
         S_out = torch.empty(B, H, d, d, dtype=torch.float32, device=k.device)
     if z_out is None:
         z_out = torch.empty(B, H, d, dtype=torch.float32, device=k.device)
-    if ws is None:
-        ws = workspace(desc, "kv_summary", device=k.device)
+    _state(S_out, z_out, k)
+    ws = workspace(desc, "kv_summary", device=k.device) if ws is None else _ws(ws, k)
     _check("la_kv_summary", lib().la_kv_summary(
         ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(S_out), _ptr(z_out), _ptr(ws), ws.numel(),
         _stream(k, stream)))
@@ -172,6 +192,7 @@ def la_kv_summary_static(k, v, S_out, z_out, phi="relu1", stream=None):
     nothing; S_out [B,H,d,d] and z_out [B,H,d] float32 are the caller's.
     Calls that overlap on the GPU race (they share the scratch)."""
     _same(k, v)
+    _state(S_out, z_out, k)
     desc = _desc_of(k, phi, True)
     _check("la_kv_summary_static", lib().la_kv_summary_static(
         ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(S_out), _ptr(z_out), _stream(k, stream)))
@@ -184,9 +205,12 @@ def la_noncausal(q, k, v, out=None, S_out=None, z_out=None, phi="relu1", normali
     if out is None:
         out = torch.empty_like(q)
     _same(q, k, v, out)
+    if (S_out is None) != (z_out is None):
+        raise ValueError("give both S_out and z_out, or neither")
+    if S_out is not None:
+        _state(S_out, z_out, q)
     desc = _desc_of(q, phi, normalize)
-    if ws is None:
-        ws = workspace(desc, "noncausal", device=q.device)
+    ws = workspace(desc, "noncausal", device=q.device) if ws is None else _ws(ws, q)
     _check("la_noncausal", lib().la_noncausal(
         ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(S_out), _ptr(z_out),
         _ptr(ws), ws.numel(), _stream(q, stream)))
@@ -200,8 +224,7 @@ def la_causal_chunked(q, k, v, out=None, chunk=64, phi="relu1", normalize=True, 
         out = torch.empty_like(q)
     _same(q, k, v, out)
     desc = _desc_of(q, phi, normalize)
-    if ws is None:
-        ws = workspace(desc, "causal", chunk, device=q.device)
+    ws = workspace(desc, "causal", chunk, device=q.device) if ws is None else _ws(ws, q)
     _check("la_causal_chunked", lib().la_causal_chunked(
         ctypes.byref(desc), int(chunk), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(ws),
         ws.numel(), _stream(q, stream)))
@@ -220,13 +243,9 @@ def la_causal_prefill(q, k, v, out=None, S_out=None, z_out=None, chunk=64, phi="
         S_out = torch.empty(B, H, d, d, dtype=torch.float32, device=q.device)
     if z_out is None:
         z_out = torch.empty(B, H, d, dtype=torch.float32, device=q.device)
-    if S_out.dtype != torch.float32 or tuple(S_out.shape) != (B, H, d, d) or not S_out.is_contiguous():
-        raise ValueError("S_out must be contiguous float32 [B, H, d, d]")
-    if z_out.dtype != torch.float32 or tuple(z_out.shape) != (B, H, d) or not z_out.is_contiguous():
-        raise ValueError("z_out must be contiguous float32 [B, H, d]")
+    _state(S_out, z_out, q)
     desc = _desc_of(q, phi, normalize)
-    if ws is None:
-        ws = workspace(desc, "causal", chunk, device=q.device)
+    ws = workspace(desc, "causal", chunk, device=q.device) if ws is None else _ws(ws, q)
     _check("la_causal_prefill", lib().la_causal_prefill(
         ctypes.byref(desc), int(chunk), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(S_out), _ptr(z_out),
         _ptr(ws), ws.numel(), _stream(q, stream)))
@@ -242,9 +261,10 @@ def la_prefix_mask(q, k, v, m, out=None, chunk=64, phi="relu1", normalize=True, 
     B, _, N, _ = q.shape
     if m.dtype != torch.int32 or tuple(m.shape) != (B, N) or m.device != q.device:
         raise ValueError("m must be an int32 [B, N] tensor on the same device")
+    if not m.is_contiguous():
+        raise ValueError("m must be contiguous")
     desc = _desc_of(q, phi, normalize)
-    if ws is None:
-        ws = workspace(desc, "prefix", chunk, device=q.device)
+    ws = workspace(desc, "prefix", chunk, device=q.device) if ws is None else _ws(ws, q)
     _check("la_prefix_mask", lib().la_prefix_mask(
         ctypes.byref(desc), int(chunk), _ptr(q), _ptr(k), _ptr(v), _ptr(m), _ptr(out), _ptr(ws),
         ws.numel(), _stream(q, stream)))
@@ -256,11 +276,7 @@ def la_decode_step(q, k, v, S, z, out=None, phi="relu1", normalize=True, stream=
     if out is None:
         out = torch.empty_like(q)
     _same(q, k, v, out)
-    B, H, _, d = q.shape
-    if S.dtype != torch.float32 or tuple(S.shape) != (B, H, d, d):
-        raise ValueError("S must be float32 [B, H, d, d]")
-    if z.dtype != torch.float32 or tuple(z.shape) != (B, H, d):
-        raise ValueError("z must be float32 [B, H, d]")
+    _state(S, z, q)
     desc = _desc_of(q, phi, normalize)
     _check("la_decode_step", lib().la_decode_step(
         ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(S), _ptr(z), _ptr(out),
@@ -297,8 +313,7 @@ def _backward(name, op, q, k, v, dout, dq, dk, dv, phi, normalize, ws, stream):
     dv = torch.empty_like(v) if dv is None else dv
     _same(q, k, v, dout, dq, dk, dv)
     desc = _desc_of(q, phi, normalize)
-    if ws is None:
-        ws = workspace(desc, op, 64, device=q.device)
+    ws = workspace(desc, op, 64, device=q.device) if ws is None else _ws(ws, q)
     _check(name, getattr(lib(), name)(
         ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
         ws.numel(), _stream(q, stream)))

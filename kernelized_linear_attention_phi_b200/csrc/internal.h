@@ -8,8 +8,11 @@
 
 namespace la {
 
-// la_kv_summary after its argument checks: validation, then the KV summary
-// with `ws` as workspace (la_api.cu).
+// la_kv_summary's checks of the descriptor and the four pointers (no CUDA
+// call); LA_OK or the status la_kv_summary returns for them (la_api.cu).
+la_status kv_summary_args(const la_desc* desc, const void* k, const void* v, const float* S_out,
+                          const float* z_out);
+// la_kv_summary: validation, then the KV summary with `ws` as workspace.
 la_status kv_summary_checked(const la_desc* desc, const void* k, const void* v, float* S_out,
                              float* z_out, void* ws, size_t ws_bytes, cudaStream_t st);
 

@@ -10,8 +10,10 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "device.h"
 #include "internal.h"
 #include "launch_util.h"
+#include "plan.h"
 #include "tc.h"
 #include "tc_common.cuh"
 
@@ -19,7 +21,6 @@ namespace la {
 namespace {
 
 constexpr int kSimtChunk = 64;     // chunk length the SIMT chunked kernel runs at
-constexpr int kNumSMs = 148;       // B200
 constexpr size_t kAlign = 256;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -72,31 +73,12 @@ Problem to_problem(const la_desc* d) {
 
 // ---- work plans (pure functions of the problem, shared by sizing and launch) ----
 
-struct SplitPlan {
-    int nsplit, tps;  // splits per head, tokens per split
-};
-SplitPlan kv_plan(const Problem& p) {
-    const long long target = std::max(1LL, cdiv(2 * kNumSMs, p.bh()));
-    const long long max_splits = std::max(1LL, cdiv(p.N, 256));
-    long long ns = std::min(target, max_splits);
-    const long long tps = (long long)round_up((size_t)cdiv(p.N, ns), 128);
-    ns = cdiv(p.N, tps);
-    return SplitPlan{(int)ns, (int)tps};
-}
-
-struct BlockPlan {
-    int block_tokens, nblk;
-};
-// Blocks of the chunked forms: every (block, head) is one CTA of the chunk
-// sweep, so the block count per head is chosen to fill one wave (CTAs that
-// fit on an SM at once x 148 SMs) without spilling into a second.
-BlockPlan block_plan(const Problem& p) {
-    const int per_sm = (p.dtype == LA_BF16 && p.d == 128) ? 1 : 2;
-    const long long target = std::max(1LL, (long long)(per_sm * kNumSMs) / p.bh());
-    long long bt = (long long)round_up((size_t)cdiv(p.N, target), 128);
-    bt = std::max(bt, 256LL);
-    return BlockPlan{(int)bt, (int)cdiv(p.N, bt)};
-}
+// Plans for the current device's SM count (plan.h): a workspace sized on a
+// device fits every launch on that device.
+plan::SplitPlan kv_plan(const Problem& p) { return plan::kv_plan(p, device_sms()); }
+plan::BlockPlan block_plan(const Problem& p) { return plan::block_plan(p, device_sms()); }
+using plan::BlockPlan;
+using plan::SplitPlan;
 
 int prefix_nbins(const Problem& p, int kchunk) { return p.N / kchunk + 1; }
 
@@ -206,12 +188,17 @@ la_status kv_summary_impl(const Problem& p, const void* k, const void* v, float*
 
 }  // namespace
 
-la_status kv_summary_checked(const la_desc* desc, const void* k, const void* v, float* S_out,
-                             float* z_out, void* ws, size_t ws_bytes, cudaStream_t st) {
+la_status kv_summary_args(const la_desc* desc, const void* k, const void* v, const float* S_out,
+                          const float* z_out) {
     LA_TRY(check_desc(desc));
     if (!k || !v || !S_out || !z_out) return LA_ERR_INVALID_ARG;
-    if (!aligned16(k) || !aligned16(v) || !aligned16(S_out) || !aligned16(z_out))
-        return LA_ERR_MISALIGNED;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(S_out) || !aligned16(z_out)) return LA_ERR_MISALIGNED;
+    return LA_OK;
+}
+
+la_status kv_summary_checked(const la_desc* desc, const void* k, const void* v, float* S_out,
+                             float* z_out, void* ws, size_t ws_bytes, cudaStream_t st) {
+    LA_TRY(kv_summary_args(desc, k, v, S_out, z_out));
     const Problem p = to_problem(desc);
     LA_TRY(check_ws(ws_layout(p, LA_OP_KV_SUMMARY), ws, ws_bytes));
     LA_TRY(check_device());

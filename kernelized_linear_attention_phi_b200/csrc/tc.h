@@ -4,6 +4,7 @@
 #include <cuda.h>
 
 #include "internal.h"
+#include "plan.h"
 
 namespace la {
 
@@ -13,17 +14,13 @@ bool tc_supported(const Problem& p);
 // Every kernel below bounds its waits; an expired wait sets
 // tc::FLAG_TIMEOUT in *err (the workspace error word) and the kernel returns.
 
-// Balanced split of the KV summary: a 1-D grid of G CTAs (one per SM) cuts
-// the flattened sequence of (head, 128-token tile) pairs into G contiguous
-// ranges of equal length. A range that touches several heads writes one
-// partial record per head; slot (cta * K + j) holds the record of the
-// j-th head the CTA touches.
-struct KvBalanced {
-    int G, K, tph;     // CTAs, record slots per CTA, tiles per head
-    long long total;   // bh * tph
-};
-// Balanced split of the bh * tph (head, 128-token tile) pairs over
-// min(total, 148 * per_sm) CTAs in contiguous ranges.
+// Balanced split of the KV summary (plan::KvBalanced): a 1-D grid of G CTAs
+// cuts the flattened sequence of (head, 128-token tile) pairs into G
+// contiguous ranges of equal length; a range that touches several heads
+// writes one partial record per head, slot (cta * K + j) holding the record
+// of the j-th head the CTA touches. Planned for the current device's SMs,
+// per_sm ranges per SM.
+using KvBalanced = plan::KvBalanced;
 KvBalanced kv_balanced_plan(const Problem& p, int per_sm = 1);
 
 // KV summary in balanced mode: partial records into `part` (G*K slots of
@@ -31,8 +28,8 @@ KvBalanced kv_balanced_plan(const Problem& p, int per_sm = 1);
 cudaError_t tc_kv_summary(const Problem& p, const void* k, const void* v, float* part, float* S,
                           float* z, uint32_t* err, cudaStream_t st);
 // Non-causal attention in one kernel for small problems (tc_fused.cu): bf16,
-// d = 64, B*H <= 33 (one wave of 8-CTA clusters, one per head),
-// N <= 8192. Writes
+// d = 64, N <= 8192, and one 8-CTA cluster per head all resident at once
+// (B*H <= 33 on a B200). Writes
 // out and, when S / z are non-null, the KV summary [bh][d*d], [bh][d]; with
 // out null (q then unused) only the KV summary, into S and z (both needed).
 bool tc_noncausal_fused_supported(const Problem& p);

@@ -32,6 +32,7 @@
 
 #include <algorithm>
 
+#include "device.h"
 #include "launch_util.h"
 #include "tc.h"
 #include "tc_common.cuh"
@@ -691,7 +692,7 @@ cudaError_t launch_bwd(const Problem& p, const void* q, const void* k, const voi
     if (e != cudaSuccess) return e;
     e = ensure_smem<tc_bwd_kv_kernel<D, PHI>>(BkCfg<D>::SMEM);
     if (e != cudaSuccess) return e;
-    const int Gk = (int)std::min<long long>(w.total, 148LL * BkCfg<D>::PER_SM);
+    const int Gk = plan::balanced_ctas(w.total, device_sms(), BkCfg<D>::PER_SM);
     return launch_pdl(tc_bwd_kv_kernel<D, PHI>, dim3(Gk), dim3(kThreads), BkCfg<D>::SMEM, st, mk, mv, mdk, mdv, G, h,
                       w.total, w.tph, err);
 }

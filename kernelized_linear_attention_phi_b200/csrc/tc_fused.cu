@@ -23,6 +23,7 @@
 // Warp roles (192 threads): warp 0 TMA, warp 1 TMEM owner and MMA issuer,
 // warps 2-5 transforms, column sums, the reduction and epilogues.
 
+#include "device.h"
 #include "launch_util.h"
 #include "tc.h"
 #include "tc_common.cuh"
@@ -413,11 +414,12 @@ cudaError_t launch_fused(const Problem& p, const CUtensorMap& mk, const CUtensor
 }  // namespace
 
 bool tc_noncausal_fused_supported(const Problem& p) {
-    // one wave of 8-CTA clusters at two CTAs per SM (B200 holds 33 such
-    // clusters at once: measured 36 heads at 36.9 us here against 35.8 us on
-    // the three-kernel path), at most 1024 tokens per CTA (beyond that the
-    // balanced three-kernel path spreads better)
-    return p.dtype == DT_BF16 && p.d == FnCfg::D && p.bh() <= 33 && p.N <= 8 * 1024;
+    // one wave of 8-CTA clusters, one per head (a B200 holds 33 at two CTAs
+    // per SM; measured 36 heads, two waves, at 36.9 us here against 35.8 us
+    // on the three-kernel path), at most 1024 tokens per CTA (beyond that
+    // the balanced three-kernel path spreads better)
+    return p.dtype == DT_BF16 && p.d == FnCfg::D && p.N <= 8 * 1024 &&
+           p.bh() <= max_active_clusters(kCluster, kThreads, FnCfg::SMEM);
 }
 
 cudaError_t tc_noncausal_fused(const Problem& p, const void* q, const void* k, const void* v, void* out, float* S,

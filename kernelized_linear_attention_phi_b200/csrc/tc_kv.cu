@@ -28,21 +28,17 @@
 
 #include <algorithm>
 
+#include "device.h"
 #include "launch_util.h"
+#include "plan.h"
 #include "tc.h"
 #include "tc_common.cuh"
 
 namespace la {
 
-KvBalanced kv_balanced_plan(const Problem& p, int per_sm) {
-    KvBalanced w;
-    w.tph = (p.N + tc::kTile - 1) / tc::kTile;
-    w.total = p.bh() * w.tph;
-    w.G = (int)std::min<long long>(w.total, 148LL * per_sm);
-    const long long per = (w.total + w.G - 1) / w.G;  // most tiles a CTA gets
-    w.K = (int)std::min<long long>(p.bh(), (per + w.tph - 1) / w.tph + 1);
-    return w;
-}
+static_assert(plan::kTileTokens == tc::kTile, "the plans and the kernels tile tokens alike");
+
+KvBalanced kv_balanced_plan(const Problem& p, int per_sm) { return plan::kv_balanced_plan(p, device_sms(), per_sm); }
 
 namespace {
 
@@ -702,7 +698,7 @@ cudaError_t launch_readout_phi(const Problem& p, const CUtensorMap& mq, const CU
     if (e != cudaSuccess) return e;
     const int tph = (p.N + kTile - 1) / kTile;
     const long long total = p.bh() * tph;
-    const int G = (int)std::min<long long>(total, 148LL * RoCfg<D>::PER_SM);
+    const int G = plan::balanced_ctas(total, device_sms(), RoCfg<D>::PER_SM);
     return launch_pdl(tc_readout_kernel<D, PHI>, dim3(G), dim3(kThreads), smem, st, mq, mo, S, z, p.N, total, tph,
                       p.normalize, err);
 }
@@ -745,13 +741,10 @@ cudaError_t tc_reduce_records(const Problem& p, const KvBalanced& w, const float
 }
 
 namespace {
-// Clusters of cs CTAs (two per SM, the scanning KV pass's threads and shared
-// memory) that a B200 holds at once, from the occupancy of a plain kernel of
-// the same shape: 71 of 4, 33 of 8, 14 of 16. A cluster of up to 2^k CTAs
-// fits wherever one of 2^k does, so other sizes take the next power of two.
-int cluster_capacity(int cs) {
-    return cs <= 1 ? 296 : cs <= 2 ? 148 : cs <= 4 ? 71 : cs <= 8 ? 33 : 14;
-}
+// Clusters of cs CTAs with the scanning KV pass's threads and shared memory
+// that the device holds at once (on a B200 at two CTAs per SM: 71 of 4, 33
+// of 8, 14 of 16).
+int cluster_capacity(int cs) { return max_active_clusters(cs, kThreads, KvCfg<64, true>::SMEM); }
 // Blocks per CTA of the scanning KV pass: one while every head's cluster
 // fits one wave, else two (half the CTAs, twice the tiles each); 0 when
 // neither fits (the separate scan kernel is used then).

@@ -247,6 +247,29 @@ def prefix_mask(Q, K, V, m, phi_kind=PHI_RELU1, normalize=True):
     return out
 
 
+def causal_rows(Q, K, V, rows, phi_kind=PHI_RELU1, normalize=True):
+    """Selected rows of causal attention by the nx recurrence, for long
+    sequences: keys are added to (S, z) in order, the keys between two
+    requested rows as one KV summary of that stretch (the same sum over j,
+    grouped), and each requested row i reads out once (S, z) holds keys
+    0..i. O(N d^2) for any number of rows, against O(i d) per row for
+    ``attention_rows``."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    rows = np.asarray(rows, dtype=np.int64)
+    S = np.zeros((K.shape[1], V.shape[1]))
+    z = np.zeros(K.shape[1])
+    out = np.empty((len(rows), V.shape[1]))
+    added = 0  # keys 0..added-1 are in (S, z)
+    for r in np.argsort(rows, kind="stable"):
+        i = int(rows[r])
+        if i + 1 > added:
+            dS, dz = kv_summary(K[added:i + 1], V[added:i + 1], phi_kind)
+            S, z = S + dS, z + dz
+            added = i + 1
+        out[r] = readout(Q[i], S, z, phi_kind, normalize)
+    return out
+
+
 # ---------------------------------------------------------------------------
 # Batched helpers over [B, H, N, d]
 # ---------------------------------------------------------------------------

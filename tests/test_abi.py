@@ -173,3 +173,44 @@ def test_gradient_workspace_sizes(lib):
         for op in ("noncausal_bwd", "causal_bwd"):
             n = B.la_workspace_size(B.la_desc(B_, H, N, 64, dt, 0, 1), op)
             assert n % 256 == 0 and n >= 2 * B_ * H * (64 * 64 + 64) * 4
+
+
+def test_static_kv_summary_validates_before_any_cuda_call(lib):
+    """la_kv_summary_static checks the descriptor and the pointers first, with
+    the statuses la_kv_summary gives, before it looks up its scratch array or
+    enqueues anything; a valid request then fails cleanly without a GPU."""
+    dsc = desc()
+    f = lib.la_kv_summary_static
+    assert f(None, P16, P16, P16, P16, NULL) == 1
+    assert f(ctypes.byref(desc(d=48)), P16, P16, P16, P16, NULL) == 2
+    assert f(ctypes.byref(dsc), P16, P16, NULL, P16, NULL) == 1
+    assert f(ctypes.byref(dsc), P16, NULL, P16, P16, NULL) == 1
+    assert f(ctypes.byref(dsc), P16, P16, P_MIS, P16, NULL) == 3
+    assert f(ctypes.byref(dsc), P16, P16, P16, P_MIS, NULL) == 3
+    for bad in (dict(d=48), dict(N=0)):
+        d_ = desc(**bad)
+        assert f(ctypes.byref(d_), P16, P16, NULL, P16, NULL) == \
+            lib.la_kv_summary(ctypes.byref(d_), P16, P16, NULL, P16, P16, 1 << 30, NULL)
+    if not torch.cuda.is_available():
+        assert f(ctypes.byref(dsc), P16, P16, P16, P16, NULL) == 5
+
+
+def test_binding_rejects_wrong_state_tensors(lib):
+    """The binding refuses S / z buffers of the wrong dtype, shape or
+    device before calling the library (which would write B*H*(d*d + d)
+    floats through them)."""
+    k = torch.zeros(2, 3, 256, 64, dtype=torch.bfloat16)
+    ok_S = torch.zeros(2, 3, 64, 64)
+    ok_z = torch.zeros(2, 3, 64)
+    for S, z in ((ok_S.bfloat16(), ok_z), (ok_S[:, :2], ok_z), (ok_S, ok_z[..., :32]),
+                 (ok_S.double(), ok_z)):
+        with pytest.raises(ValueError):
+            B.la_kv_summary_static(k, k, S, z)
+        with pytest.raises(ValueError):
+            B.la_kv_summary(k, k, S, z)
+        with pytest.raises(ValueError):
+            B.la_noncausal(k, k, k, torch.empty_like(k), S, z)
+    with pytest.raises(ValueError):
+        B.la_noncausal(k, k, k, torch.empty_like(k), ok_S, None)
+    with pytest.raises(ValueError):  # a workspace must be uint8 bytes
+        B.la_causal_chunked(k, k, k, torch.empty_like(k), ws=torch.zeros(16, dtype=torch.float32))

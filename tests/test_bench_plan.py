@@ -1,67 +1,82 @@
-"""Host logic of bench.py that mirrors the library's dispatch: the kernels
-each call of a workload launches (the labels of the per-kernel roofline),
-the block count of the chunked forms and when the KV pass scans the block
-states inside its clusters. Checked on CPU against the figures the dispatch
-is written from."""
+"""Host logic of bench.py: the cases one run measures (every workload of the
+pages, the long-context step as the headline), the names it gives the
+kernels of each call from the count the library's timing events report, and
+the algorithmic bytes of each kernel. Checked on CPU."""
+
+import json
+import subprocess
+import sys
 
 import bench
 from kernelized_linear_attention_phi_b200 import workloads as W
 
 
-def test_block_count_follows_the_block_plan():
-    # one wave of 2 x 148 CTAs, blocks of at least 256 tokens in multiples of 128
-    assert bench.block_count(W.WORKLOADS["multi_head"]) == 16      # 16 heads x 4096: 256-token blocks
-    assert bench.block_count(W.WORKLOADS["prefix_mask"]) == 4      # 64 heads x 2048: 512-token blocks
-    assert bench.block_count(W.WORKLOADS["long_causal"]) == 9      # d = 128, one CTA per SM
+def test_one_run_covers_every_workload_with_the_long_step_as_headline():
+    assert bench.HEADLINE == "long"
+    assert bench.CASES["long"] == [("long_noncausal", "bf16", "noncausal", None),
+                                   ("long_causal", "bf16", "causal", None)]
+    covered = {w for calls in bench.CASES.values() for w, *_ in calls}
+    assert {"single_head", "multi_head", "prefix_mask", "long_noncausal", "long_causal", "decode"} <= covered
+    assert ("multi_head", "f32", "causal", None) in bench.CASES["multi_head_f32"]
+    assert [c[3] for c in bench.CASES["prefix_mask"] + bench.CASES["prefix_mask_arange"]] == ["uniform", "arange"]
+    assert set(bench.CASE_TEXT) == set(bench.CASES)
+    assert W.WORKLOADS["decode"].decode_steps == 1024
 
 
-def test_in_cluster_scan_takes_two_blocks_per_cta_when_one_would_not_fit():
-    wl = W.WORKLOADS["multi_head"]
-    # 16 heads x 16 blocks: 16 clusters of 16 exceed the 14 a B200 holds, 16
-    # clusters of 8 (two blocks per CTA) fit the 33
-    assert bench.scan_in_cluster(wl)
-    k = bench.call_kernels(wl, "bf16")
-    assert k["causal"] == ["tc_kv_kernel", "tc_sweep"]
-    assert k["prefix"] == ["tc_kv_kernel", "bin_kernel", "tc_sweep"]
-    assert k["causal_bwd"] == ["tc_kv_kernel", "tc_bwd_causal_q_kernel", "state_scan_kernel",
-                               "tc_bwd_causal_kv_kernel"]
-    assert k["noncausal"] == ["tc_noncausal_cluster_kernel"]
-    assert k["noncausal_bwd"] == ["tc_noncausal_cluster_kernel", "tc_bwd_q_kernel", "kv_reduce_balanced_kernel",
-                                  "tc_bwd_kv_kernel"]
-
-
-def test_long_and_fp32_workloads_keep_the_separate_kernels():
-    k = bench.call_kernels(W.WORKLOADS["long_causal"], "bf16")  # d = 128: no in-cluster scan
-    assert k["causal"] == ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"]
-    k = bench.call_kernels(W.WORKLOADS["long_noncausal"], "bf16")  # 64 heads: the balanced split
-    assert k["noncausal"] == ["tc_kv_kernel", "kv_reduce_balanced_kernel", "tc_readout_kernel"]
-    assert bench.call_kernels(W.WORKLOADS["multi_head"], "f32") == bench.CALL_KERNELS_F32
+def test_kernel_names_follow_the_count_of_launches():
+    kn = bench.kernel_names
+    assert kn("noncausal", "bf16", 64, 1) == ["tc_noncausal_cluster_kernel"]
+    assert kn("noncausal", "bf16", 64, 3) == ["tc_kv_kernel", "kv_reduce_balanced_kernel", "tc_readout_kernel"]
+    assert kn("causal", "bf16", 128, 3) == ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"]
+    assert kn("causal", "bf16", 64, 2) == ["tc_kv_kernel", "tc_sweep"]
+    assert kn("prefix", "bf16", 64, 3)[-1] == "tc_sweep"
+    # fp32 and small d run on the CUDA cores
+    assert kn("causal", "f32", 64, 3) == ["kv_partial_kernel", "state_scan_kernel", "chunked_kernel"]
+    assert kn("noncausal", "bf16", 16, 3)[0] == "kv_partial_kernel"
+    # a count the table does not know keeps neutral labels
+    assert kn("causal", "bf16", 64, 7) == [f"kernel{i}" for i in range(7)]
 
 
 def test_kernel_roles_cover_every_listed_kernel():
-    for table in (bench.CALL_KERNELS, bench.CALL_KERNELS_F32):
-        for names in table.values():
-            for n in names:
-                assert any(n.startswith(r) for r in bench.KERNEL_ROLE), n
+    for table in (bench.TC_KERNELS, bench.SIMT_KERNELS):
+        for by_count in table.values():
+            for names in by_count.values():
+                for n in names:
+                    assert n in bench.KERNEL_ROLE, n
 
 
-def test_kernel_bytes_of_the_gradient_calls():
-    """Algorithmic bytes per kernel of the gradient calls: the KV summary
-    reads K and V (whether the balanced KV pass or the cluster kernel without
-    its readout forms it), the query side Q, dO and dq (causal: also K, V),
-    the key side K, V, dk, dv (causal: also Q); reductions move scratch only."""
-    wl = W.WORKLOADS["multi_head_bwd"]
-    t = wl.B * wl.H * wl.N * wl.d * 2
-
-    class S:  # the fields kernel_bytes reads
-        B, H, N, d, elem = wl.B, wl.H, wl.N, wl.d, 2
-    kb = lambda call, k: bench.Step.kernel_bytes(S, call, k)
+def test_kernel_bytes():
+    """Algorithmic bytes per kernel: the KV pass reads K and V, a sweep reads
+    Q, K, V and writes out, the readout reads Q and S, z and writes out, the
+    gradient sweeps move their tensors once; scratch-only kernels have none."""
+    B, H, N, d, e = 2, 8, 4096, 64, 2
+    t = B * H * N * d * e
+    st = B * H * (d * d + d) * 4
+    kb = lambda form, k: bench.kernel_bytes(form, k, B, H, N, d, e)
+    assert kb("causal", "tc_kv_kernel") == 2 * t
+    assert kb("causal", "tc_sweep") == 4 * t
+    assert kb("causal", "state_scan_kernel") == 0
+    assert kb("noncausal", "tc_readout_kernel") == 2 * t + st
+    assert kb("noncausal", "tc_noncausal_cluster_kernel") == 4 * t
+    assert kb("prefix", "bin_kernel") == B * N * 4
+    assert kb("decode", "decode_kernel") == 2 * st + 4 * B * H * d * e
     assert kb("noncausal_bwd", "tc_noncausal_cluster_kernel") == 2 * t
-    assert kb("noncausal_bwd", "tc_kv_kernel") == 2 * t
     assert kb("noncausal_bwd", "tc_bwd_q_kernel") == 3 * t
     assert kb("noncausal_bwd", "tc_bwd_kv_kernel") == 4 * t
     assert kb("noncausal_bwd", "kv_reduce_balanced_kernel") == 0
     assert kb("causal_bwd", "tc_bwd_causal_q_kernel") == 5 * t
     assert kb("causal_bwd", "tc_bwd_causal_kv_kernel") == 5 * t
-    assert kb("noncausal", "tc_noncausal_cluster_kernel") == 4 * t
 
+
+def test_reference_arm_runs_on_the_host_and_prints_one_line():
+    """--impl reference times the oracle on a sample of the headline case,
+    on the host alone, and prints the contract's JSON line."""
+    r = subprocess.run([sys.executable, bench.__file__, "--impl", "reference", "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["value"] > 0 and rec["unit"] == "tokens/s"
+    assert rec["metric"] == bench.METRIC and rec["e2e"]["h2d_bytes_per_step"] == 0
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] >= 1

@@ -1,8 +1,8 @@
 """The five workloads at full size, in the launch configuration bench.py uses
 (the library's work plans depend only on the problem shape), against the
 fp64 oracle: every row where the oracle's O(N d^2) form is quick, sampled rows
-(by the O(i d) definition) for the long causal sequence, sampled heads over
-all 1024 steps for the decode workload."""
+(block edges, whole chunks, random rows; by the recurrence) for the long
+causal sequence, 64 heads over all 1024 steps for the decode workload."""
 
 import numpy as np
 import pytest
@@ -74,17 +74,37 @@ def test_long_noncausal():
     assert max(errs) < 2e-2
 
 
+def _block_starts(wl, sms):
+    """Token starts of the blocks the library's block plan cuts a head into
+    on a device with `sms` SMs (one wave of CTAs; d = 128 bf16 sweeps one
+    CTA per SM; blocks of at least 256 tokens in multiples of 128)."""
+    per_sm = 1 if wl.d == 128 else 2
+    target = max(1, per_sm * sms // (wl.B * wl.H))
+    bt = max(256, -(-(-(-wl.N // target)) // 128) * 128)
+    return list(range(0, wl.N, bt))
+
+
 def test_long_causal_sampled_rows():
+    """Every head: the first and last token of every block and every token
+    of one 64-token chunk per block (with the tokens on either side of it),
+    the first 130 and last 2 tokens of the head, and random rows, against the
+    oracle's recurrence."""
     wl = W.WORKLOADS["long_causal"]
     q, k, v = _inputs(wl, "bf16")
     out = la.la_causal_chunked(q, k, v, chunk=wl.chunk)
+    starts = _block_starts(wl, torch.cuda.get_device_properties(0).multi_processor_count)
+    ends = starts[1:] + [wl.N]
     rng = np.random.default_rng(0)
     errs = []
     for h in range(wl.H):
-        rows = sorted(set([0, 1, 127, 128, 129, wl.N - 1] +
-                          rng.integers(0, wl.N, size=10).tolist()))
-        ref = oracle.attention_rows(f64(q[0, h]), f64(k[0, h]), f64(v[0, h]), rows,
-                                    form=oracle.FORM_CAUSAL)
+        rows = set(range(130)) | {wl.N - 2, wl.N - 1}
+        for s0, s1 in zip(starts, ends):
+            rows |= {s0, s1 - 1}
+            c0 = s0 + 64 * int(rng.integers(0, (s1 - s0) // 64))  # one chunk of the block
+            rows |= set(range(max(0, c0 - 1), min(wl.N, c0 + 65)))
+        rows |= set(rng.integers(0, wl.N, size=16).tolist())
+        rows = sorted(rows)
+        ref = oracle.causal_rows(f64(q[0, h]), f64(k[0, h]), f64(v[0, h]), rows)
         errs.append(oracle.max_row_rel_err(f64(out[0, h, rows]), ref))
     assert max(errs) < 2e-2
 
@@ -95,7 +115,8 @@ def test_decode_workload():
     _, k0, v0 = W.qkv(B, H, N0, d, wl.sigma, wl.seed, "bf16", "cuda")
     S, z = la.la_kv_summary(k0, v0)
     S0_sample = {}
-    heads = [(0, 0), (17, 5), (40, 31), (63, 30)]
+    # 64 heads: every sequence, its head spread over H
+    heads = [(b, (7 * b + 3) % H) for b in range(B)]
     for b, h in heads:
         S0_sample[(b, h)] = (f64(S[b, h]), f64(z[b, h]))
     qs, ks, vs = W.decode_tokens(T, B, H, d, wl.sigma, wl.seed + 1, "bf16", "cuda")

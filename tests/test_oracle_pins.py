@@ -416,3 +416,18 @@ def test_planted_mistakes_fail_the_worked_example(golden_dir, monkeypatch):
         S, z = la.kv_summary(K, V)
         return la.readout(Q, S, S.sum(axis=1))
     assert not _gate2_ok(golden_dir, wrong_den)
+
+
+@pytest.mark.parametrize("phi_kind,normalize", [("relu1", True), ("identity", False), ("elu1", True)])
+def test_causal_rows_match_definition(phi_kind, normalize):
+    """causal_rows (segment sums of the KV summary between requested rows)
+    gives the definition's rows, in any order and with repeats."""
+    rng = np.random.default_rng(21)
+    n, d = 300, 8
+    Q, K, V = (rng.standard_normal((n, d)) for _ in range(3))
+    rows = [299, 0, 5, 5, 64, 63, 127, 128, 1, 250]
+    got = la.causal_rows(Q, K, V, rows, phi_kind, normalize)
+    ref = la.attention_rows(Q, K, V, rows, la.FORM_CAUSAL, phi_kind=phi_kind, normalize=normalize)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+    dense = la.attention_dense(Q, K, V, la.FORM_CAUSAL, phi_kind=phi_kind, normalize=normalize)
+    np.testing.assert_allclose(got, dense[rows], rtol=1e-12, atol=1e-12)

@@ -1,8 +1,9 @@
 """la_kv_summary_static, the KV summary for callers that cannot allocate
 device memory (its scratch is a fixed device array inside the library), must
-give what la_kv_summary gives. Collected last, so that a run that stops at the
-first failure has run every other test; it must also pass on its own in a
-fresh process (the first call sets up the array's device address)."""
+give what la_kv_summary gives, and what the oracle gives. Collected last, so
+that a run that stops at the first failure has run every other test; it must
+also pass on its own in a fresh process (the first call in a context looks up
+the array's device address)."""
 
 import ctypes
 
@@ -25,19 +26,32 @@ def _built():
     la.lib()
 
 
+# S and z are fp32 sums; bf16 elu+1 rounds phi(K) before the products, the
+# other maps are exact to fp32 accumulation (the library's KV-summary tolerance)
+TOL = 1e-5
+
+
 @pytest.mark.parametrize("dtype,d", [("bf16", 64), ("bf16", 128), ("f32", 64)])
-def test_static_scratch_matches_workspace_entry_point(dtype, d):
-    """Two calls in a row on different inputs, each against la_kv_summary."""
+def test_static_scratch_matches_workspace_entry_point_and_oracle(dtype, d):
+    """Two calls in a row on different inputs, each against la_kv_summary
+    and against the oracle's KV summary; the calls allocate nothing through
+    torch's allocator."""
     B, H, N = 2, 4, 3000
     for seed in (1, 2):
         _, k, v = W.qkv(B, H, N, d, 1.0, seed, dtype, "cuda")
         S_ref, z_ref = la.la_kv_summary(k, v)
         S = torch.full((B, H, d, d), float("nan"), device="cuda")
         z = torch.full((B, H, d), float("nan"), device="cuda")
+        torch.cuda.synchronize()
+        before = torch.cuda.memory_allocated()
         la.la_kv_summary_static(k, v, S, z)
         torch.cuda.synchronize()
-        assert oracle.max_row_rel_err(f64(S), f64(S_ref)) < 1e-5
-        assert oracle.max_row_rel_err(f64(z)[..., None, :], f64(z_ref)[..., None, :]) < 1e-5
+        assert torch.cuda.memory_allocated() == before
+        assert oracle.max_row_rel_err(f64(S), f64(S_ref)) < TOL
+        assert oracle.max_row_rel_err(f64(z)[..., None, :], f64(z_ref)[..., None, :]) < TOL
+        S_o, z_o = oracle.kv_summary_batched(f64(k), f64(v))
+        assert oracle.max_row_rel_err(f64(S), S_o) < TOL
+        assert oracle.max_row_rel_err(f64(z)[..., None, :], z_o[..., None, :]) < TOL
 
 
 def test_static_scratch_rejects_problems_beyond_its_size():
