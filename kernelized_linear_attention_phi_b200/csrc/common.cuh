@@ -92,6 +92,11 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // start by then, so an early dependent never takes an SM from this grid;
 // one that is resident on an SM where this grid still holds TMEM waits in its
 // allocation until that CTA releases it.)
+// A kernel may read memory before its pdl_wait() only when no earlier kernel
+// still running can write it: a later kernel of a call may prefetch the
+// caller's inputs (no kernel of the call writes them), but the first kernel of
+// a call may not, because the kernel before it on the stream can be the last
+// kernel of an earlier call whose outputs are this call's inputs.
 __device__ __forceinline__ void pdl_wait() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

@@ -421,6 +421,13 @@ la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, cons
     LA_TRY(check_device());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     timing_begin(st);
+    {
+        // sequences of at most 4096 tokens at d = 64: binning, block states,
+        // their prefix and the sweep in one kernel (a cluster per head)
+        int fbt = 0, fnc = 0;
+        if (tc_prefix_fused_plan(p, &fbt, &fnc))
+            return cuda_status(tc_prefix_fused(p, q, k, v, m, out, at<uint32_t>(ws, 0), st));
+    }
     const BlockPlan bp = block_plan(p);
     const bool tc = tc_supported(p);
     const int kchunk = tc ? tc_chunk(p, chunk) : kSimtChunk;  // chunk length of the kernel used

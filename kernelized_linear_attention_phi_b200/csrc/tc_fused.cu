@@ -120,9 +120,11 @@ tc_noncausal_cluster_kernel(const __grid_constant__ CUtensorMap mK, const __grid
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // The TMA producer loads only the caller's inputs; every other warp waits
-    // for the previous kernel on the stream first (the epilogue writes out).
-    if (warp != 0) pdl_wait();
+    // This kernel is the first of its call: the kernel before it on the stream
+    // may be the last kernel of an earlier call whose outputs are this call's
+    // inputs (and that kernel lets its dependents launch early). So every warp,
+    // the TMA producer included, waits for it before reading anything.
+    pdl_wait();
 
     // Ring of stages shared by both phases: phase-1 tile i is ring index i,
     // phase-3 tile i is ring index nt + i (stage ring % STAGES, use ring / STAGES).
