@@ -91,8 +91,9 @@ CASE_TEXT = {
 TC_KERNELS = {
     "noncausal": {1: ["tc_noncausal_cluster_kernel"],
                   3: ["tc_kv_kernel", "kv_reduce_balanced_kernel", "tc_readout_kernel"]},
-    "causal": {2: ["tc_kv_kernel", "tc_sweep"], 3: ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"]},
-    "prefix": {3: ["tc_kv_kernel", "bin_kernel", "tc_sweep"],
+    "causal": {1: ["tc_prefix_fused_kernel"], 2: ["tc_kv_kernel", "tc_sweep"],
+               3: ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"]},
+    "prefix": {1: ["tc_prefix_fused_kernel"], 3: ["tc_kv_kernel", "bin_kernel", "tc_sweep"],
                4: ["tc_kv_kernel", "bin_kernel", "state_scan_kernel", "tc_sweep"]},
     "decode": {1: ["decode_kernel"]},
     "noncausal_bwd": {4: ["tc_noncausal_cluster_kernel", "tc_bwd_q_kernel", "kv_reduce_balanced_kernel",
@@ -121,7 +122,17 @@ KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balan
                "bin_kernel": "bin", "decode_kernel": "decode", "bwd_q_kernel": "bwd_q",
                "bwd_kv_kernel": "bwd_kv", "tc_bwd_q_kernel": "bwd_q", "tc_bwd_kv_kernel": "bwd_kv",
                "tc_bwd_causal_q_kernel": "bwd_q", "tc_bwd_causal_kv_kernel": "bwd_kv",
-               "tc_noncausal_cluster_kernel": "fused"}
+               "tc_noncausal_cluster_kernel": "fused", "tc_prefix_fused_kernel": "prefix_fused"}
+
+
+def block_plan(B, H, N, d, dtype, sms):
+    """(block_tokens, nblk) of the chunked forms, as the library plans them
+    (csrc/plan.h block_plan): one wave of CTAs (one per SM for bf16 d = 128,
+    else two), blocks of at least 256 tokens in multiples of 128."""
+    per_sm = 1 if dtype == "bf16" and d == 128 else 2
+    target = max(1, per_sm * sms // (B * H))
+    bt = max(256, -(-(-(-N // target)) // 128) * 128)
+    return bt, -(-N // bt)
 
 
 def kernel_names(form, dtype, d, count):
@@ -245,6 +256,7 @@ class Call:
         self.name = wl.name if form != "prefix" or mask == "uniform" else f"{wl.name}_{mask}"
         self.phi, self.normalize, self.chunk = wl.phi, wl.normalize, wl.chunk
         self.seed = seed
+        self.sms = torch.cuda.get_device_properties(device).multi_processor_count
         self.ws = None
         self.elem = 2 if dtype == "bf16" else 4
         desc = la.make_desc(B, H, N, d, W.TORCH_DTYPES[dtype], self.phi, self.normalize)
@@ -337,7 +349,14 @@ class Call:
         the library keeps between its kernels (partial and block-state
         records, the binning tables) is not counted, so a kernel that only
         moves scratch (the prefix scan over block states) has none."""
-        return kernel_bytes(self.form, kernel, self.B, self.H, self.N, self.d, self.elem)
+        kb = kernel_bytes(self.form, kernel, self.B, self.H, self.N, self.d, self.elem)
+        if self.form == "causal" and self.dtype == "bf16" and self.d == 128 and KERNEL_ROLE.get(kernel) == "kv":
+            # the d = 128 causal call forms the states of every block but the
+            # last (no prefix holds it): the KV pass reads those keys only
+            bt, nblk = block_plan(self.B, self.H, self.N, self.d, self.dtype, self.sms)
+            if nblk >= 2:
+                kb = kb * min(self.N, (nblk - 1) * bt) // self.N
+        return kb
 
 
 def kernel_bytes(form, kernel, B, H, N, d, elem):
@@ -354,7 +373,8 @@ def kernel_bytes(form, kernel, B, H, N, d, elem):
         return {"kv": 2 * t, "fused": 2 * t, "bwd_q": (5 if causal else 3) * t,
                 "bwd_kv": (5 if causal else 4) * t}.get(role, 0)
     return {"kv": 2 * t, "reduce": st, "readout": 2 * t + st, "scan": 0, "sweep": 4 * t, "fused": 4 * t,
-            "bin": B * N * 4, "decode": 2 * st + 4 * one}.get(role, 0)
+            "prefix_fused": 4 * t + (B * N * 4 if form == "prefix" else 0), "bin": B * N * 4,
+            "decode": 2 * st + 4 * one}.get(role, 0)
 
 
 def flush_l2(buf):
@@ -523,6 +543,8 @@ def measure_case(case, args, rank, world, device, flush, sampler, peak, heads=0)
 
     # roofline of the dominant kernel: the one with the largest time in the
     # step, its algorithmic bytes over its own timed duration
+    if not cands:
+        raise SystemExit(f"no kernel of case {case} has algorithmic bytes: unknown kernel labels {per_call}")
     _, dom_ms, dom_call, dom_kernel, di, dom_bytes = max(cands, key=lambda x: x[0])
     achieved = dom_bytes / (dom_ms / 1e3) / 1e9
     dtypes = sorted({c.dtype for c in calls})

@@ -293,6 +293,17 @@ la_status causal_impl(const la_desc* desc, int32_t chunk, const void* q, const v
     // phase 1: per-block states; phase 2: exclusive prefix over blocks (and
     // the total); phase 3: each block's outputs from its prefix state.
     uint32_t* flags = at<uint32_t>(ws, 0);
+    int fbt = 0, fnc = 0;
+    if (tc_prefix_fused_plan(p, &fbt, &fnc))  // short sequences at d = 64: one kernel
+        return cuda_status(tc_causal_fused(p, q, k, v, out, S_total, z_total, flags, st));
+    if (tc_supported(p) && p.d == 128 && S_total == nullptr && bp.nblk >= 2) {
+        // the states of every block but the last (no block's prefix holds
+        // it), then the sweep, whose CTAs each sum the states before their
+        // block: no scan kernel in between
+        LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st, bp.nblk - 1)));
+        return cuda_status(tc_chunked_t(p, q, k, v, part, bp.block_tokens, bp.nblk, nullptr, nullptr, nullptr, 0,
+                                        out, flags, st, true));
+    }
     if (tc_kv_scan_supported(p, bp.block_tokens, bp.nblk)) {  // phases 1 and 2 in one kernel
         LA_TRY(cuda_status(tc_kv_blocks_scan(p, k, v, bp.block_tokens, bp.nblk, part, S_total, z_total, flags, st)));
     } else {

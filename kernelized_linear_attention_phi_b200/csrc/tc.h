@@ -41,8 +41,9 @@ cudaError_t tc_reduce_records(const Problem& p, const KvBalanced& w, const float
                               cudaStream_t st);
 // KV summary per block: CTA (block, head) writes record (head*nblk + block)
 // over tokens [block*block_tokens, ...); block_tokens must be a multiple of 128.
+// Only blocks 0..nform-1 are formed (nform <= nblk; -1: all).
 cudaError_t tc_kv_blocks(const Problem& p, const void* k, const void* v, int block_tokens, int nblk,
-                         float* part, uint32_t* err, cudaStream_t st);
+                         float* part, uint32_t* err, cudaStream_t st, int nform = -1);
 // tc_kv_blocks followed by the exclusive block-state scan, in one kernel with
 // a thread-block cluster per head (bf16, d = 64, nblk <= 16, every head's
 // cluster resident at once, with one or two blocks per CTA): part[bh*nblk +
@@ -74,11 +75,20 @@ cudaError_t tc_chunked(const Problem& p, int chunk, const void* q, const void* k
 bool tc_prefix_fused_plan(const Problem& p, int* block_tokens, int* nc);
 cudaError_t tc_prefix_fused(const Problem& p, const void* q, const void* k, const void* v, const int32_t* m, void* out,
                             uint32_t* err, cudaStream_t st);
+// The causal form through the same kernel (m_i = i, no binning), under the
+// same plan; S_total / z_total (both or neither) receive the state after the
+// last token.
+cudaError_t tc_causal_fused(const Problem& p, const void* q, const void* k, const void* v, void* out, float* S_total,
+                            float* z_total, uint32_t* err, cudaStream_t st);
 
 // The d = 128 kernel behind tc_chunked (64-token chunks, state kept as S^T).
+// With raw_prefix, `prefix` holds each block's own state (as tc_kv_blocks
+// writes it; the last block's record is not read) and every CTA sums the
+// records of the blocks before it, so no scan runs in between.
 cudaError_t tc_chunked_t(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
                          int block_tokens, int nblk, const int32_t* perm, const int32_t* bins,
-                         const int32_t* msort, int nbins, void* out, uint32_t* err, cudaStream_t st);
+                         const int32_t* msort, int nbins, void* out, uint32_t* err, cudaStream_t st,
+                         bool raw_prefix = false);
 
 // Gradients of the non-causal form (tc_bwd.cu): S, z are the KV summary of
 // the forward; `part` holds tc_backward_record_slots(p) records, (G, h)

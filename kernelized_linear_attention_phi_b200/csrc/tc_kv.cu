@@ -781,14 +781,17 @@ cudaError_t tc_kv_blocks_scan(const Problem& p, const void* k, const void* v, in
 }
 
 cudaError_t tc_kv_blocks(const Problem& p, const void* k, const void* v, int block_tokens, int nblk, float* part,
-                         uint32_t* err, cudaStream_t st) {
+                         uint32_t* err, cudaStream_t st, int nform) {
     if (block_tokens % kTile != 0) return cudaErrorInvalidValue;
+    if (nform < 0) nform = nblk;
+    if (nform > nblk) return cudaErrorInvalidValue;
+    if (nform == 0) return cudaSuccess;
     KvWork w{};
     w.balanced = 0;
     w.block_tokens = block_tokens;
     w.nblk = nblk;
     w.bpc = 1;
-    const dim3 grid(nblk, (unsigned)p.bh());
+    const dim3 grid(nform, (unsigned)p.bh());  // records keep the stride of nblk blocks per head
     return p.d == 64 ? launch_kv<64>(p, k, v, w, grid, part, err, st)
                      : launch_kv<128>(p, k, v, w, grid, part, err, st);
 }

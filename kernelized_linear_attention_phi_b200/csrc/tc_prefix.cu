@@ -10,7 +10,10 @@
 // answers every query whose key limit m_i lies in its block [r*BT, r*BT+BT):
 //
 //   phase A  the block's state T_r = phi(K_r)^T V_r, z_r = phi(K_r)^T 1
-//            (tensor cores, over the block's 128-key sub-blocks); meanwhile
+//            (tensor cores, over the block's 128-key sub-blocks; for relu+1
+//            as relu(K)^T V + 1 (x) colsum(V) and colsum(relu K) + count,
+//            relu(K) being exact in bf16, so the state carries no rounding of
+//            phi(K)); meanwhile
 //            the mask warps bin the sequence's queries: those with m_i in
 //            the block, stably sorted by the sub-block holding m_i;
 //   phase B  the block prefix S_bp = sum_{r' < r} T_r' (and z) over
@@ -103,12 +106,15 @@ __device__ __forceinline__ int op_sub(int op) { return (op >> 8) & 0xFF; }
 __device__ __forceinline__ bool op_opens(int op) { return op & 1; }
 __device__ __forceinline__ bool op_closes(int op) { return op & 2; }
 
-template <int PHI>
+// CAUSAL: the causal form (m_i = i) without a mask: the queries of the block
+// are its own tokens, so no binning; tile t is sub-block t (loaded as a TMA
+// tile, not gathered) and has exactly one op.
+template <int PHI, bool CAUSAL>
 __global__ void __launch_bounds__(PfCfg::THREADS, 1)
-tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_constant__ CUtensorMap mK,
+tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                        const __grid_constant__ CUtensorMap mV, const int32_t* __restrict__ m, int H, int N,
-                       int block_tokens, int normalize, __nv_bfloat16* __restrict__ out,
-                       uint32_t* __restrict__ err) {
+                       int block_tokens, int normalize, __nv_bfloat16* __restrict__ out, float* __restrict__ S_total,
+                       float* __restrict__ z_total, uint32_t* __restrict__ err) {
     using CF = PfCfg;
     constexpr int D = CF::D, KC = CF::KC;
     extern __shared__ uint8_t smem_raw[];
@@ -173,7 +179,7 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
             mbar_init(qempty + j, 1);
         }
         fence_mbar_init();
-        tma_prefetch_map(&mQrow);
+        tma_prefetch_map(&mQ);
         tma_prefetch_map(&mK);
         tma_prefetch_map(&mV);
     }
@@ -222,15 +228,23 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
                 const int t = op_tile(op), qb = t % CF::QB, u = t / CF::QB;
                 if (t >= CF::QB) ok = ok && __all_sync(0xffffffffu, mbar_wait(qempty + qb, (u - 1) & 1, err));
                 if (!ok) break;
-                int tok[4];
+                if (CAUSAL) {
+                    // the block's own tokens (rows past N arrive as zeros)
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(qfull + qb, CF::TILE);
+                        tma_load_3d(qbuf + qb * CF::TILE, &mQ, qfull + qb, 0, k0 + t * KC, bh);
+                    }
+                } else {
+                    int tok[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int pos = t * KC + 4 * lane + e;
-                    tok[e] = pos < nq ? (tab[pos] >> CF::LIM_BITS) : -1;
+                    for (int e = 0; e < 4; ++e) {
+                        const int pos = t * KC + 4 * lane + e;
+                        tok[e] = pos < nq ? (tab[pos] >> CF::LIM_BITS) : -1;
+                    }
+                    if (lane == 0) mbar_arrive_expect_tx(qfull + qb, CF::TILE);
+                    __syncwarp();
+                    gather_tile<KC, 1>(qbuf + qb * CF::TILE, &mQ, qfull + qb, bh * N, tok, lane);
                 }
-                if (lane == 0) mbar_arrive_expect_tx(qfull + qb, CF::TILE);
-                __syncwarp();
-                gather_tile<KC, 1>(qbuf + qb * CF::TILE, &mQrow, qfull + qb, bh * N, tok, lane);
                 tq = t + 1;
             }
         }
@@ -251,20 +265,27 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
             constexpr uint32_t id_p = idesc_bf16(KC, KC, false, false);  // P = Q K^T
             constexpr uint32_t id_o = idesc_bf16(KC, D, false, true);    // O = Q S_k, O += P~ V
             constexpr uint32_t id_oz = idesc_bf16(KC, 16, false, false); // Oz = Q [z]
+            constexpr uint32_t id_cs = idesc_bf16(D, D, false, true);    // 1 (x) colsum(V)
             const uint32_t onesa = smem_u32(ones), pta = smem_u32(pt), qa0 = smem_u32(qbuf);
             bool ok = true;
-            // state MMAs over the sub-block in load `ld` (accumulating unless `first`)
-            auto state_update = [&](int ld, bool first) {
+            // state MMAs over the sub-block in load `ld` (accumulating unless
+            // `first`); with `colsum`, also colsum(V) into every row of the P
+            // columns (an all-ones A operand; phase A of relu+1)
+            auto state_update = [&](int ld, bool first, bool with_z, bool colsum) {
                 const int s = ld % CF::STAGES;
                 const uint32_t kt = smem_u32(ring + s * CF::STAGE), vt = kt + CF::TILE;
 #pragma unroll
                 for (int kk = 0; kk < KC / 16; ++kk) {
                     const uint64_t a = sdesc(kt + kk * 2048, KC * 128, 1024);
-                    mma_bf16(tmem + CF::COL_S, a, sdesc(vt + kk * 2048, KC * 128, 1024), id_su,
-                             (first && kk == 0) ? 0u : 1u);
-                    if (normalize)
+                    const uint64_t bv = sdesc(vt + kk * 2048, KC * 128, 1024);
+                    const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+                    mma_bf16(tmem + CF::COL_S, a, bv, id_su, acc);
+                    if (with_z)
                         mma_bf16(tmem + CF::COL_Z, a, sdesc(onesa + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024), id_zu,
-                                 (first && kk == 0) ? 0u : 1u);
+                                 acc);
+                    if (colsum)
+                        mma_bf16(tmem + CF::COL_P, sdesc(pta + (kk / 4) * (D * 128) + (kk % 4) * 32, 16, 1024), bv,
+                                 id_cs, acc);
                 }
             };
             // phase A: the block's own state
@@ -273,7 +294,7 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
                 ok = mbar_wait(kready + s, (ld / CF::STAGES) & 1, err);
                 if (!ok) break;
                 tc_fence_after();
-                state_update(ld, ld == 0);
+                state_update(ld, ld == 0, true, PHI == PHI_RELU1);
                 mma_commit(empty + s);
             }
             mma_commit(bsdone);
@@ -313,7 +334,7 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
                 ok = mbar_wait(bprep, k & 1, err) && mbar_wait(kready + s, (ld / CF::STAGES) & 1, err);
                 if (!ok) break;
                 tc_fence_after();
-                state_update(ld, false);
+                state_update(ld, false, normalize != 0, false);
                 mma_commit(bsdone);
                 const uint32_t kt = smem_u32(ring + s * CF::STAGE);
                 const uint32_t b3a = smem_u32(b3 + (k & 1) * CF::B3), bza = smem_u32(bz + (k & 1) * CF::BZ);
@@ -359,8 +380,11 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
         const uint4 one8 = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
         for (int c = et; c < CF::ONES / 16; c += 128) reinterpret_cast<uint4*>(ones)[c] = one8;
         for (int c = et; c < 2 * CF::BZ / 16; c += 128) reinterpret_cast<uint4*>(bz)[c] = make_uint4(0, 0, 0, 0);
+        if (PHI == PHI_RELU1)  // phase A: an all-ones [64 x 128] A operand in the (idle) P~ buffers
+            for (int c = et; c < 2 * D * 128 / 16; c += 128) reinterpret_cast<uint4*>(pt)[c] = one8;
         fence_async_smem();
-        // phi on the K tile of load ld, rows past the sequence zeroed
+        // phi on the K tile of load ld (phase A of relu+1: relu alone), rows
+        // past the sequence zeroed
         auto transform_k = [&](int ld) {
             const int s = ld % CF::STAGES;
             mbar_wait(full + s, (ld / CF::STAGES) & 1, err);
@@ -368,13 +392,14 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
             if (mapped || kvalid < KC) {
                 uint4* kt = reinterpret_cast<uint4*>(ring + s * CF::STAGE);
                 constexpr int NL = CF::TILE / 16 / 128;
+                const bool split = PHI == PHI_RELU1 && ld < nsub;
                 uint4 w[NL];
 #pragma unroll
                 for (int j = 0; j < NL; ++j) w[j] = kt[et + 128 * j];
 #pragma unroll
                 for (int j = 0; j < NL; ++j) {
                     const int r = (et + 128 * j) >> 3;
-                    kt[et + 128 * j] = r < kvalid ? phi8<PHI>(w[j]) : make_uint4(0, 0, 0, 0);
+                    kt[et + 128 * j] = r >= kvalid ? make_uint4(0, 0, 0, 0) : split ? relu_x8(w[j]) : phi8<PHI>(w[j]);
                 }
                 fence_async_smem();
             }
@@ -417,6 +442,17 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
         {
             float f[32], zv;
             read_state(f, zv);
+            if (PHI == PHI_RELU1) {
+                // + 1 (x) colsum(V) (every row of the P columns holds it) and
+                // z = colsum(relu K) + the block's key count
+                uint32_t r[32];
+                tmem_ld16x2<32>(tmem + CF::COL_P + lane_base, *reinterpret_cast<uint32_t(*)[16]>(r));
+                tmem_ld16x2<32>(tmem + CF::COL_P + lane_base + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) f[e] += __uint_as_float(r[e]);
+                zv += (float)nkeys;
+            }
 #pragma unroll
             for (int g = 0; g < 8; ++g)
                 *reinterpret_cast<float4*>(xch + a * D + cb + 4 * g) = make_float4(f[4 * g], f[4 * g + 1], f[4 * g + 2],
@@ -438,6 +474,15 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
                 acc.w += x.w;
             }
             reinterpret_cast<float4*>(sbp)[e4] = acc;
+            if (S_total != nullptr && rank == (int)gridDim.x - 1) {
+                // the head's total (the state a decode continues from)
+                const float4 own = reinterpret_cast<const float4*>(xch)[e4];
+                const float4 tot = make_float4(acc.x + own.x, acc.y + own.y, acc.z + own.z, acc.w + own.w);
+                if (4 * e4 < D * D)
+                    reinterpret_cast<float4*>(S_total + (size_t)bh * D * D)[e4] = tot;
+                else
+                    reinterpret_cast<float4*>(z_total + (size_t)bh * D)[e4 - D * D / 4] = tot;
+            }
         }
         named_bar(1, 128);
         {
@@ -498,6 +543,20 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
         const int mw = mt >> 5;            // mask warp 0..3
         // binning: the queries with m_i in [k0, k0 + nkeys), stably sorted by
         // the sub-block of m_i (each mask warp takes a quarter of the sequence)
+        if (CAUSAL) {
+            // queries = the block's tokens; tile t = sub-block t, one op each
+            if (mt == 0) {
+                for (int k = 0; k < nsub; ++k) {
+                    step_begin[k] = k;
+                    ops[k] = op_pack(k, k, true, true);
+                }
+                step_begin[nsub] = nsub;
+                misc[0] = nkeys;
+                misc[1] = nsub;
+                misc[2] = nsub;
+                mbar_arrive(binned);
+            }
+        } else {
         const int32_t* mb = m + (size_t)b * N;
         for (int c = mt; c < 4 * CF::MAX_SUB; c += 128) hist[c] = 0;
         named_bar(2, 128);
@@ -568,6 +627,7 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
             misc[2] = nops;
             mbar_arrive(binned);
         }
+        }  // !CAUSAL
         asm volatile("barrier.cluster.arrive;" ::: "memory");
         mbar_wait(binned, 0, err);
         const int nops = misc[2];
@@ -577,10 +637,12 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
         const int i = sp * 32 + lane;  // row of the M = 128 accumulators this thread reads
         float rs[2] = {0.f, 0.f};      // denominator row sums per O slot
         bool ok = true;
+        const int nq = misc[0];
         for (int n = 0; n < nops; ++n) {
             const int op = ops[n], t = op_tile(op), k = op_sub(op), j = n & 1, os = t & 1;
             const int pos = t * KC + i;
-            const int lim = pos < nq ? (tab[pos] & ((1 << CF::LIM_BITS) - 1)) - k * KC : -1;  // keys 0..lim visible
+            // keys 0..lim of sub-block k visible (causal: the diagonal and before)
+            const int lim = pos >= nq ? -1 : (CAUSAL ? pos : (tab[pos] & ((1 << CF::LIM_BITS) - 1))) - k * KC;
             ok = mbar_wait(pfull + j, (n >> 1) & 1, err) && ok;
             tc_fence_after();
             uint8_t* ptj = pt + j * CF::PT;
@@ -624,7 +686,7 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
                 const float inv = normalize ? __frcp_rn(den) : 1.0f;
                 rs[os] = 0.f;
                 if (ok && pos < nq) {
-                    const int tok = tab[pos] >> CF::LIM_BITS;
+                    const int tok = CAUSAL ? k0 + pos : tab[pos] >> CF::LIM_BITS;
                     uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)bh * N + tok) * D);
 #pragma unroll
                     for (int g = 0; g < D / 8; ++g) {
@@ -648,15 +710,33 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQrow, const __grid_c
     }
 }
 
-template <int PHI>
+template <int PHI, bool CAUSAL>
 cudaError_t launch_prefix_fused(const Problem& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                                const int32_t* m, int block_tokens, int nc, void* out, uint32_t* err,
-                                cudaStream_t st) {
-    cudaError_t e = ensure_smem<tc_prefix_fused_kernel<PHI>>(PfCfg::SMEM);
+                                const int32_t* m, int block_tokens, int nc, void* out, float* S_total, float* z_total,
+                                uint32_t* err, cudaStream_t st) {
+    cudaError_t e = ensure_smem<tc_prefix_fused_kernel<PHI, CAUSAL>>(PfCfg::SMEM);
     if (e != cudaSuccess) return e;
-    return launch_cluster_pdl(tc_prefix_fused_kernel<PHI>, dim3(nc, (unsigned)p.bh()), dim3(PfCfg::THREADS),
+    return launch_cluster_pdl(tc_prefix_fused_kernel<PHI, CAUSAL>, dim3(nc, (unsigned)p.bh()), dim3(PfCfg::THREADS),
                               PfCfg::SMEM, st, (unsigned)nc, mq, mk, mv, m, p.H, p.N, block_tokens, p.normalize,
-                              static_cast<__nv_bfloat16*>(out), err);
+                              static_cast<__nv_bfloat16*>(out), S_total, z_total, err);
+}
+
+template <bool CAUSAL>
+cudaError_t fused_phi(const Problem& p, const void* q, const void* k, const void* v, const int32_t* m, void* out,
+                      float* S_total, float* z_total, uint32_t* err, cudaStream_t st) {
+    int bt = 0, nc = 0;
+    if (!tc_prefix_fused_plan(p, &bt, &nc)) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv;
+    // causal: Q tiles of the block's own tokens; prefix mask: a 2-D row map for tile::gather4
+    cudaError_t e = CAUSAL ? make_map(&mq, q, PfCfg::D, p.N, p.bh(), PfCfg::KC) : make_row_map(&mq, q, PfCfg::D, p.bh() * p.N);
+    if (e == cudaSuccess) e = make_map(&mk, k, PfCfg::D, p.N, p.bh(), PfCfg::KC);
+    if (e == cudaSuccess) e = make_map(&mv, v, PfCfg::D, p.N, p.bh(), PfCfg::KC);
+    if (e != cudaSuccess) return e;
+    switch (p.phi) {  // one kernel per feature map (see phi8)
+        case PHI_RELU1: return launch_prefix_fused<PHI_RELU1, CAUSAL>(p, mq, mk, mv, m, bt, nc, out, S_total, z_total, err, st);
+        case PHI_ELU1: return launch_prefix_fused<PHI_ELU1, CAUSAL>(p, mq, mk, mv, m, bt, nc, out, S_total, z_total, err, st);
+        default: return launch_prefix_fused<PHI_IDENTITY, CAUSAL>(p, mq, mk, mv, m, bt, nc, out, S_total, z_total, err, st);
+    }
 }
 
 }  // namespace
@@ -677,18 +757,12 @@ bool tc_prefix_fused_plan(const Problem& p, int* block_tokens, int* nc) {
 
 cudaError_t tc_prefix_fused(const Problem& p, const void* q, const void* k, const void* v, const int32_t* m, void* out,
                             uint32_t* err, cudaStream_t st) {
-    int bt = 0, nc = 0;
-    if (!tc_prefix_fused_plan(p, &bt, &nc)) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mv;
-    cudaError_t e = make_row_map(&mq, q, PfCfg::D, p.bh() * p.N);
-    if (e == cudaSuccess) e = make_map(&mk, k, PfCfg::D, p.N, p.bh(), PfCfg::KC);
-    if (e == cudaSuccess) e = make_map(&mv, v, PfCfg::D, p.N, p.bh(), PfCfg::KC);
-    if (e != cudaSuccess) return e;
-    switch (p.phi) {  // one kernel per feature map (see phi8)
-        case PHI_RELU1: return launch_prefix_fused<PHI_RELU1>(p, mq, mk, mv, m, bt, nc, out, err, st);
-        case PHI_ELU1: return launch_prefix_fused<PHI_ELU1>(p, mq, mk, mv, m, bt, nc, out, err, st);
-        default: return launch_prefix_fused<PHI_IDENTITY>(p, mq, mk, mv, m, bt, nc, out, err, st);
-    }
+    return fused_phi<false>(p, q, k, v, m, out, nullptr, nullptr, err, st);
+}
+
+cudaError_t tc_causal_fused(const Problem& p, const void* q, const void* k, const void* v, void* out, float* S_total,
+                            float* z_total, uint32_t* err, cudaStream_t st) {
+    return fused_phi<true>(p, q, k, v, nullptr, out, S_total, z_total, err, st);
 }
 
 }  // namespace la

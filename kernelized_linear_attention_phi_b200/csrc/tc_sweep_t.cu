@@ -73,7 +73,7 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                   const float* __restrict__ prefix, int H, int N,
                   int block_tokens, int nblk, const int32_t* __restrict__ perm,
                   const int32_t* __restrict__ bin_start, const int32_t* __restrict__ msort, int nbins,
-                  int normalize, __nv_bfloat16* __restrict__ out, uint32_t* __restrict__ err) {
+                  int normalize, int raw_prefix, __nv_bfloat16* __restrict__ out, uint32_t* __restrict__ err) {
     using CF = StCfg<GATHER>;
     constexpr int D = CF::D, C = CF::C;
     extern __shared__ uint8_t smem_raw[];
@@ -297,7 +297,12 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
         const int sp = warp & 3;
         const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
         const int a = sp * 32 + lane;  // the S^T row (d_v index) this thread owns in TMEM
-        const float* pre = prefix + ((size_t)bh * nblk + blk) * (size_t)(D * D + D);
+        // the block's prefix: its record of the exclusive block scan, or with
+        // raw_prefix the records of the blocks before it (their own states),
+        // summed here in block order (the order the scan adds them in)
+        constexpr size_t kRec = (size_t)D * D + D;
+        const float* pre = prefix + ((size_t)bh * nblk + (raw_prefix ? 0 : blk)) * kRec;
+        const int npre = raw_prefix ? blk : 1;
         // rows 66..79 of every extended K box stay zero (TMA writes rows 0..63)
         for (int x = et; x < CF::STAGES * CF::NB * 14 * 8; x += 128) {
             const int s = x / (CF::NB * 112), bx = (x / 112) % CF::NB, r = 66 + (x % 112) / 8, q16 = x % 8;
@@ -307,14 +312,23 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
         // seed S^T with the block's prefix record (S stored [d_k][d_v])
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
+            float f[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) f[e] = 0.f;
+            for (int rb = 0; rb < npre; ++rb) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) f[e] += pre[rb * kRec + (size_t)(c0 + e) * D + a];
+            }
             uint32_t r[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(pre[(size_t)(c0 + e) * D + a]);
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(f[e]);
             tmem_st16(tmem + CF::COL_S + lane_base + c0, *reinterpret_cast<uint32_t(*)[16]>(r));
             tmem_st16(tmem + CF::COL_S + lane_base + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
         }
         tmem_st_wait();
-        float zp = normalize ? pre[(size_t)D * D + et] : 0.f;  // z_prev[d_k = et]
+        float zp = 0.f;  // z_prev[d_k = et]
+        if (normalize)
+            for (int rb = 0; rb < npre; ++rb) zp += pre[rb * kRec + (size_t)D * D + et];
         // column group (of 8) of the K chunks this thread transforms: the
         // 128-byte swizzle maps 16-byte chunk (lane & 7) of its rows (all with
         // the same row & 7) to logical columns 8 * g .. 8 * g + 7
@@ -542,7 +556,7 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
 template <bool GATHER, int PHI>
 cudaError_t launch_t(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
                      int block_tokens, int nblk, const int32_t* perm, const int32_t* bins, const int32_t* msort,
-                     int nbins, void* out, uint32_t* err, cudaStream_t st) {
+                     int nbins, int raw_prefix, void* out, uint32_t* err, cudaStream_t st) {
     using CF = StCfg<GATHER>;
     if (p.d != CF::D || block_tokens % CF::C != 0) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv, mo;
@@ -556,7 +570,7 @@ cudaError_t launch_t(const Problem& p, const void* q, const void* k, const void*
     if (e != cudaSuccess) return e;
     dim3 grid(nblk, (unsigned)p.bh());
     return launch_pdl(tc_sweep_t_kernel<GATHER, PHI>, grid, dim3(CF::THREADS), CF::SMEM, st, mq, mk, mv, mo,
-                      prefix, p.H, p.N, block_tokens, nblk, perm, bins, msort, nbins, p.normalize,
+                      prefix, p.H, p.N, block_tokens, nblk, perm, bins, msort, nbins, p.normalize, raw_prefix,
                       static_cast<__nv_bfloat16*>(out), err);
 }
 
@@ -564,17 +578,17 @@ cudaError_t launch_t(const Problem& p, const void* q, const void* k, const void*
 template <bool GATHER>
 cudaError_t launch_phi(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
                        int block_tokens, int nblk, const int32_t* perm, const int32_t* bins, const int32_t* msort,
-                       int nbins, void* out, uint32_t* err, cudaStream_t st) {
+                       int nbins, int raw_prefix, void* out, uint32_t* err, cudaStream_t st) {
     switch (p.phi) {
         case PHI_RELU1:
             return launch_t<GATHER, PHI_RELU1>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort, nbins,
-                                               out, err, st);
+                                               raw_prefix, out, err, st);
         case PHI_ELU1:
             return launch_t<GATHER, PHI_ELU1>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort, nbins,
-                                              out, err, st);
+                                              raw_prefix, out, err, st);
         default:
             return launch_t<GATHER, PHI_IDENTITY>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort,
-                                                  nbins, out, err, st);
+                                                  nbins, raw_prefix, out, err, st);
     }
 }
 
@@ -582,10 +596,13 @@ cudaError_t launch_phi(const Problem& p, const void* q, const void* k, const voi
 
 cudaError_t tc_chunked_t(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
                          int block_tokens, int nblk, const int32_t* perm, const int32_t* bins,
-                         const int32_t* msort, int nbins, void* out, uint32_t* err, cudaStream_t st) {
+                         const int32_t* msort, int nbins, void* out, uint32_t* err, cudaStream_t st,
+                         bool raw_prefix) {
     if (perm != nullptr)
-        return launch_phi<true>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort, nbins, out, err, st);
-    return launch_phi<false>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort, nbins, out, err, st);
+        return launch_phi<true>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort, nbins, raw_prefix ? 1 : 0,
+                                out, err, st);
+    return launch_phi<false>(p, q, k, v, prefix, block_tokens, nblk, perm, bins, msort, nbins, raw_prefix ? 1 : 0, out,
+                             err, st);
 }
 
 }  // namespace la

@@ -7,6 +7,8 @@
 // call: plan.h is plain host code).
 
 #include <cstdio>
+#include <cstdlib>
+#include <string>
 #include <vector>
 
 #include "plan.h"
@@ -68,7 +70,17 @@ static void check_balanced(const Problem& p, int sms, int per_sm) {
     EXPECT(plan::balanced_ctas(w.total, sms, per_sm) == w.G, "balanced_ctas");
 }
 
-int main() {
+// "plan B H N d dtype sms" on the command line: print that block plan as
+// "block_tokens nblk" (for the Python mirror in bench.py) and exit.
+static int print_block_plan(char** argv) {
+    const Problem p{atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]), atoi(argv[6]), 0, 1};
+    const plan::BlockPlan b = plan::block_plan(p, atoi(argv[7]));
+    std::printf("%d %d\n", b.block_tokens, b.nblk);
+    return 0;
+}
+
+int main(int argc, char** argv) {
+    if (argc == 8 && std::string(argv[1]) == "plan") return print_block_plan(argv);
     const std::vector<int> sms_list = {1, 2, 7, 16, 20, 66, 78, 114, 132, 148, 160, 264};
     const std::vector<int> Ns = {1, 2, 127, 128, 129, 255, 256, 257, 1000, 2048, 3000, 4096, 16384, 65537, 131072};
     const std::vector<std::pair<int, int>> BHs = {{1, 1}, {1, 3}, {2, 8}, {4, 16}, {8, 8}, {1, 16}, {64, 32}, {3, 37}};

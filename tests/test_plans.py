@@ -30,3 +30,18 @@ def test_plans_cover_every_token_for_any_sm_count(plan_check):
     r = subprocess.run([plan_check], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout[-4000:]
     assert r.stdout.strip().splitlines()[-1].startswith("checked ")
+
+
+def test_bench_mirror_of_the_block_plan(plan_check):
+    """bench.py counts the bytes of a KV pass that skips the last block from
+    its own copy of the block plan: it must agree with the library's."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    for B, H, N, d, dt in [(1, 16, 131072, 128, 1), (2, 8, 4096, 64, 1), (8, 8, 2048, 64, 1), (1, 3, 1000, 128, 1),
+                           (64, 32, 2048, 128, 1), (1, 1, 300, 64, 0), (4, 16, 16384, 64, 1)]:
+        for sms in (148, 132, 100, 16, 1):
+            out = subprocess.run([plan_check, "plan", str(B), str(H), str(N), str(d), str(dt), str(sms)],
+                                 capture_output=True, text=True, check=True).stdout.split()
+            want = (int(out[0]), int(out[1]))
+            assert bench.block_plan(B, H, N, d, "bf16" if dt == 1 else "f32", sms) == want, (B, H, N, d, dt, sms)
