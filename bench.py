@@ -127,9 +127,9 @@ KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balan
 
 def block_plan(B, H, N, d, dtype, sms):
     """(block_tokens, nblk) of the chunked forms, as the library plans them
-    (csrc/plan.h block_plan): one wave of CTAs (one per SM for bf16 d = 128,
-    else two), blocks of at least 256 tokens in multiples of 128."""
-    per_sm = 1 if dtype == "bf16" and d == 128 else 2
+    (csrc/plan.h block_plan): one wave of CTAs (one per SM for d = 128, else
+    two), blocks of at least 256 tokens in multiples of 128."""
+    per_sm = 1 if d == 128 else 2
     target = max(1, per_sm * sms // (B * H))
     bt = max(256, -(-(-(-N // target)) // 128) * 128)
     return bt, -(-N // bt)

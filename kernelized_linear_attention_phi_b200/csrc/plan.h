@@ -41,7 +41,9 @@ inline SplitPlan kv_plan(const Problem& p, int sms) {
 struct BlockPlan {
     int block_tokens, nblk;
 };
-inline int sweep_ctas_per_sm(const Problem& p) { return (p.dtype == LA_BF16 && p.d == 128) ? 1 : 2; }
+// The d = 128 sweeps (tensor-core and CUDA-core alike) hold one CTA per SM
+// (shared memory and TMEM); the others two.
+inline int sweep_ctas_per_sm(const Problem& p) { return p.d == 128 ? 1 : 2; }
 inline BlockPlan block_plan(const Problem& p, int sms) {
     const long long target = std::max(1LL, (long long)sweep_ctas_per_sm(p) * sms / p.bh());
     long long bt = round_up(cdiv(p.N, target), 128);

@@ -20,7 +20,6 @@ namespace la {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kTT = 32;  // tokens per shared-memory tile in kv_partial
 constexpr int kC = 64;   // chunk length of the SIMT chunked kernel
 
 template <int R>
@@ -48,8 +47,12 @@ __global__ void __launch_bounds__(kThreads)
 kv_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int N, int tps, int nsplit,
                   int phi, float* __restrict__ part) {
     constexpr int R = D / 16;
-    __shared__ __align__(16) float sK[kTT * D];
-    __shared__ __align__(16) float sV[kTT * D];
+    constexpr int kTT = D == 128 ? 16 : 32;              // tokens per tile (static shared memory <= 32 KB)
+    constexpr int EPV = Vec16<T>::N, VPR = D / EPV;
+    constexpr int NV = kTT * VPR;                        // 16-byte vectors per tile and tensor
+    constexpr int PER = (NV + kThreads - 1) / kThreads;  // of them per thread
+    __shared__ __align__(16) float sK[2][kTT * D];
+    __shared__ __align__(16) float sV[2][kTT * D];
     const int s = blockIdx.x;
     const long long bh = blockIdx.y;
     const int t0 = s * tps;
@@ -59,6 +62,40 @@ kv_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int N, int t
     const T* Vh = V + bh * (long long)N * D;
     const int ta = threadIdx.x / 16, tb = threadIdx.x % 16;
 
+    // this thread's vectors of the tile at `base`, held in registers so that
+    // the next tile's loads are in flight while the current one is summed
+    uint4 rk[PER], rv[PER];
+    auto fetch = [&](int base) {
+        const int valid = min(kTT, t1 - base);
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int t = threadIdx.x + j * kThreads;
+            const int r = t / VPR, col = (t % VPR) * EPV;
+            const bool in = t < NV && r < valid;
+            rk[j] = in ? ldg_stream(Kh + (size_t)(base + r) * D + col) : make_uint4(0, 0, 0, 0);
+            rv[j] = in ? ldg_stream(Vh + (size_t)(base + r) * D + col) : make_uint4(0, 0, 0, 0);
+        }
+        return valid;
+    };
+    auto stage = [&](int buf, int valid) {
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int t = threadIdx.x + j * kThreads;
+            if (t >= NV) continue;
+            const int r = t / VPR, col = (t % VPR) * EPV;
+            float fk[EPV], fv[EPV];
+            Vec16<T>::unpack(rk[j], fk);
+            Vec16<T>::unpack(rv[j], fv);
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) fk[e] = r < valid ? phi_apply(fk[e], phi) : 0.f;
+#pragma unroll
+            for (int e = 0; e < EPV; e += 4) {
+                *reinterpret_cast<float4*>(&sK[buf][r * D + col + e]) = make_float4(fk[e], fk[e + 1], fk[e + 2], fk[e + 3]);
+                *reinterpret_cast<float4*>(&sV[buf][r * D + col + e]) = make_float4(fv[e], fv[e + 1], fv[e + 2], fv[e + 3]);
+            }
+        }
+    };
+
     float acc[R][R];
     float zacc[R];
 #pragma unroll
@@ -67,24 +104,27 @@ kv_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int N, int t
 #pragma unroll
         for (int c = 0; c < R; ++c) acc[r][c] = 0.f;
     }
+    int buf = 0;
+    if (t0 < t1) stage(0, fetch(t0));
+    __syncthreads();
     for (int base = t0; base < t1; base += kTT) {
-        const int valid = min(kTT, t1 - base);
-        tile_to_smem<T, D, D>(sK, Kh + (long long)base * D, kTT, valid, true, phi);
-        tile_to_smem<T, D, D>(sV, Vh + (long long)base * D, kTT, valid, false, phi);
-        __syncthreads();
+        const bool more = base + kTT < t1;
+        const int nvalid = more ? fetch(base + kTT) : 0;
 #pragma unroll 4
         for (int t = 0; t < kTT; ++t) {
-            float a[R], b[R];
-            lds<R>(sK + t * D + ta * R, a);
-            lds<R>(sV + t * D + tb * R, b);
+            float a[R], bb[R];
+            lds<R>(&sK[buf][t * D + ta * R], a);
+            lds<R>(&sV[buf][t * D + tb * R], bb);
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 zacc[r] += a[r];
 #pragma unroll
-                for (int c = 0; c < R; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+                for (int c = 0; c < R; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
             }
         }
+        if (more) stage(buf ^ 1, nvalid);
         __syncthreads();
+        buf ^= 1;
     }
     float* o = part + ((size_t)bh * nsplit + s) * (size_t)(D * D + D);
 #pragma unroll
@@ -159,71 +199,160 @@ __global__ void state_scan_kernel(float* __restrict__ part, int nblk, int D,
 // ---------------------------------------------------------------------------
 template <int D>
 constexpr size_t readout_smem() {
-    return sizeof(float) * ((size_t)D * D + D + 64 * (D + 4) + 64);
+    return sizeof(float) * ((size_t)D * (D + 4) + D + (size_t)D * (64 + 4) + 64);
 }
 
+// 64 queries per CTA: phi(Q)^T staged k-major, then O = phi(Q) S as 4 x D/16
+// register blocks (one 16-byte load of each operand per step over d_k), the
+// denominator phi(q).z summed in d_k order.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 readout_kernel(const T* __restrict__ Q, const float* __restrict__ S, const float* __restrict__ z,
                T* __restrict__ out, int N, int phi, int normalize) {
-    constexpr int TQ = 64, LDQ = D + 4, RC = D / 16, RT = TQ / 16;
+    constexpr int TQ = 64, LC = TQ + 4, LDD = D + 4, RC = D / 16;
     extern __shared__ __align__(16) float sm[];
     float* sS = sm;
-    float* sz = sS + D * D;
-    float* sQ = sz + D;
-    float* sDen = sQ + TQ * LDQ;
+    float* sz = sS + D * LDD;
+    float* sQT = sz + D;
+    float* sDen = sQT + D * LC;
     const int tile = blockIdx.x;
     const long long bh = blockIdx.y;
     pdl_wait();
-    const float4* S4 = reinterpret_cast<const float4*>(S + (size_t)bh * D * D);
-    for (int e = threadIdx.x; e < D * D / 4; e += kThreads) reinterpret_cast<float4*>(sS)[e] = S4[e];
+    const float* Sh = S + (size_t)bh * D * D;
+    for (int e = threadIdx.x; e < D * D / 4; e += kThreads) {
+        const int a = (4 * e) / D, bcol = (4 * e) % D;
+        *reinterpret_cast<float4*>(sS + a * LDD + bcol) = reinterpret_cast<const float4*>(Sh)[e];
+    }
     for (int e = threadIdx.x; e < D; e += kThreads) sz[e] = z[(size_t)bh * D + e];
     const int row0 = tile * TQ;
-    const T* Qh = Q + bh * (long long)N * D;
-    tile_to_smem<T, D, LDQ>(sQ, Qh + (long long)row0 * D, TQ, min(TQ, N - row0), true, phi);
+    const int nq = min(TQ, N - row0);
+    const T* Qh = Q + bh * (long long)N * D + (long long)row0 * D;
+    {
+        constexpr int EPV = Vec16<T>::N, VPR = D / EPV;
+        for (int t = threadIdx.x; t < TQ * VPR; t += kThreads) {
+            const int r = t / VPR, col = (t % VPR) * EPV;
+            float f[EPV];
+            if (r < nq) {
+                Vec16<T>::unpack(ldg_stream(Qh + (size_t)r * D + col), f);
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) f[e] = phi_apply(f[e], phi);
+            } else {
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) f[e] = 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) sQT[(col + e) * LC + r] = f[e];
+        }
+    }
     __syncthreads();
     if (normalize && threadIdx.x < TQ) {
         float den = 0.f;
-        for (int a = 0; a < D; ++a) den = fmaf(sQ[threadIdx.x * LDQ + a], sz[a], den);
+        for (int a = 0; a < D; ++a) den = fmaf(sQT[a * LC + threadIdx.x], sz[a], den);
         sDen[threadIdx.x] = den;
     }
-    const int tc = threadIdx.x % 16, tt = threadIdx.x / 16;
-    float acc[RT][RC];
-#pragma unroll
-    for (int i = 0; i < RT; ++i)
-#pragma unroll
-        for (int c = 0; c < RC; ++c) acc[i][c] = 0.f;
+    const int ti = threadIdx.x % 16, tj = threadIdx.x / 16;
+    float acc[4][RC] = {};
 #pragma unroll 4
     for (int a = 0; a < D; ++a) {
-        float sv[RC];
-        lds<RC>(sS + a * D + tc * RC, sv);
+        float qa[4], sv[RC];
+        lds<4>(sQT + a * LC + 4 * ti, qa);
+        lds<RC>(sS + a * LDD + RC * tj, sv);
 #pragma unroll
-        for (int i = 0; i < RT; ++i) {
-            const float qa = sQ[(tt * RT + i) * LDQ + a];
+        for (int r = 0; r < 4; ++r)
 #pragma unroll
-            for (int c = 0; c < RC; ++c) acc[i][c] = fmaf(qa, sv[c], acc[i][c]);
-        }
+            for (int c = 0; c < RC; ++c) acc[r][c] = fmaf(qa[r], sv[c], acc[r][c]);
     }
     __syncthreads();
     T* Oh = out + bh * (long long)N * D;
 #pragma unroll
-    for (int i = 0; i < RT; ++i) {
-        const int row = row0 + tt * RT + i;
-        if (row >= N) continue;
-        const float den = normalize ? sDen[tt * RT + i] : 1.f;
+    for (int r = 0; r < 4; ++r) {
+        const int i = 4 * ti + r;
+        if (i >= nq) continue;
+        const float inv = normalize ? 1.f / sDen[i] : 1.f;
 #pragma unroll
-        for (int c = 0; c < RC; ++c)
-            Oh[(long long)row * D + tc * RC + c] = from_f32<T>(normalize ? acc[i][c] / den : acc[i][c]);
+        for (int c = 0; c < RC; ++c) Oh[(long long)(row0 + i) * D + RC * tj + c] = from_f32<T>(acc[r][c] * inv);
     }
 }
 
 // ---------------------------------------------------------------------------
 // Chunked causal / prefix-mask outputs.
+//
+// Every product is a small matrix product over shared-memory tiles stored
+// with the output's row index contiguous along the contraction ("k-major"),
+// so that a thread reads four consecutive rows (or columns) with one 16-byte
+// load per contraction step and accumulates a 4 x RC block in registers:
+//   P^T  = (phi(Q)^T)^T (phi(K)^T)      queries x keys, masked, stored [key][query]
+//   O    = phi(Q) S + P V               queries x d_v
+//   S   += phi(K)^T V,  z += phi(K)^T 1
 // ---------------------------------------------------------------------------
 template <int D>
+struct ChCfg {
+    static constexpr int C = kC;
+    static constexpr int LC = C + 4;        // row length of the [D][C] and [C][C] tiles
+    static constexpr int LDD = D + 4;       // row length of the [C][D] and [D][D] tiles
+    static constexpr int RC = D / 16;       // output columns per thread (O, S)
+    static constexpr int OFF_S = 0, OFF_Z = OFF_S + D * LDD, OFF_QT = OFF_Z + D, OFF_KT = OFF_QT + D * LC,
+                         OFF_KN = OFF_KT + D * LC, OFF_VN = OFF_KN + C * LDD, OFF_PT = OFF_VN + C * LDD,
+                         OFF_DEN = OFF_PT + C * LC, FLOATS = OFF_DEN + C;
+    static constexpr size_t SMEM = sizeof(float) * (size_t)FLOATS + 2 * sizeof(int) * C;
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+template <int D>
 constexpr size_t chunked_smem() {
-    return sizeof(float) * ((size_t)D * D + D + 3 * kC * (D + 4) + kC * (kC + 4) + kC) +
-           2 * sizeof(int) * kC;
+    return ChCfg<D>::SMEM;
+}
+
+// acc[r][c] += sum_k A[k][i0 + r] * B[k][j0 + c], r < RI, c < RJ; A and B
+// k-major with row lengths lda, ldb (multiples of 4 floats).
+template <int RI, int RJ>
+__device__ __forceinline__ void kmajor_acc(float (&acc)[RI][RJ], const float* A, int lda, int i0, const float* B,
+                                           int ldb, int j0, int K) {
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+        float a[RI], b[RJ];
+        lds<RI>(A + k * lda + i0, a);
+        lds<RJ>(B + k * ldb + j0, b);
+#pragma unroll
+        for (int r = 0; r < RI; ++r)
+#pragma unroll
+            for (int c = 0; c < RJ; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+    }
+}
+
+// Rows of a [C x D] input tile into shared memory, phi applied when asked:
+// transposed (dstT[col][row], row length LC) and/or natural (dstN[row][col],
+// row length LDD). Row r of the tile is src row `rowidx(r)`; a negative
+// index, or r >= valid, gives a zero row.
+template <typename T, int D, typename RowIdx>
+__device__ __forceinline__ void load_rows(const T* src, int valid, RowIdx rowidx, bool apply_phi, int phi,
+                                          float* dstT, float* dstN) {
+    using CF = ChCfg<D>;
+    constexpr int EPV = Vec16<T>::N, VPR = D / EPV;
+    for (int t = threadIdx.x; t < CF::C * VPR; t += kThreads) {
+        const int r = t / VPR, col = (t % VPR) * EPV;
+        const int row = r < valid ? rowidx(r) : -1;
+        float f[EPV];
+        if (row >= 0) {
+            Vec16<T>::unpack(ldg_stream(src + (size_t)row * D + col), f);
+            if (apply_phi) {
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) f[e] = phi_apply(f[e], phi);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) f[e] = 0.f;
+        }
+        if (dstT) {
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) dstT[(col + e) * CF::LC + r] = f[e];
+        }
+        if (dstN) {
+#pragma unroll
+            for (int e = 0; e < EPV; e += 4)
+                *reinterpret_cast<float4*>(dstN + r * CF::LDD + col + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+        }
+    }
 }
 
 template <typename T, int D, bool GATHER>
@@ -233,19 +362,19 @@ chunked_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __rest
                const int32_t* __restrict__ perm, const int32_t* __restrict__ bin_start,
                const int32_t* __restrict__ msort, int nbins, int phi, int normalize,
                T* __restrict__ out) {
-    constexpr int LD = D + 4, LDP = kC + 4;
-    constexpr int R = D / 16;               // state-update block per thread (R x R)
-    constexpr int RT = kC / 16, RC = D / 16;  // output block per thread (RT rows x RC cols)
+    using CF = ChCfg<D>;
+    constexpr int C = CF::C, LC = CF::LC, LDD = CF::LDD, RC = CF::RC;
     extern __shared__ __align__(16) float sm[];
-    float* sS = sm;
-    float* sz = sS + D * D;
-    float* sQ = sz + D;
-    float* sK = sQ + kC * LD;
-    float* sV = sK + kC * LD;
-    float* sP = sV + kC * LD;
-    float* sDen = sP + kC * LDP;
-    int* sRow = reinterpret_cast<int*>(sDen + kC);
-    int* sLim = sRow + kC;
+    float* sS = sm + CF::OFF_S;
+    float* sz = sm + CF::OFF_Z;
+    float* sQT = sm + CF::OFF_QT;
+    float* sKT = sm + CF::OFF_KT;
+    float* sKn = sm + CF::OFF_KN;
+    float* sVn = sm + CF::OFF_VN;
+    float* sPT = sm + CF::OFF_PT;
+    float* sDen = sm + CF::OFF_DEN;
+    int* sRow = reinterpret_cast<int*>(sm + CF::FLOATS);
+    int* sLim = sRow + C;
 
     const int blk = blockIdx.x;
     const long long bh = blockIdx.y;
@@ -258,27 +387,22 @@ chunked_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __rest
 
     pdl_wait();
     const float* pre = prefix + ((size_t)bh * nblk + blk) * (size_t)(D * D + D);
-    for (int e = threadIdx.x; e < D * D + D; e += kThreads) {
-        if (e < D * D) sS[e] = pre[e];
-        else sz[e - D * D] = pre[e];
-    }
-    const int nchunks = (N + kC - 1) / kC;
-    const int c_begin = blk * (block_tokens / kC);
-    int c_end = min(nchunks, c_begin + block_tokens / kC);
+    for (int e = threadIdx.x; e < D * D; e += kThreads) sS[(e / D) * LDD + e % D] = pre[e];
+    for (int e = threadIdx.x; e < D; e += kThreads) sz[e] = pre[D * D + e];
+    const int nchunks = (N + C - 1) / C;
+    const int c_begin = blk * (block_tokens / C);
+    int c_end = min(nchunks, c_begin + block_tokens / C);
     if (GATHER && blk == nblk - 1) c_end = nbins;  // the last block also answers the all-keys bin
 
-    const int ta = threadIdx.x / 16, tb = threadIdx.x % 16;
-    const int tc = threadIdx.x % 16, tt = threadIdx.x / 16;
+    // output blocks: rows 4*ti .. 4*ti + 3 (queries), columns RC*tb .. (of d_v)
+    // P blocks: rows 4*ti, keys 4*tj .. 4*tj + 3; state blocks: rows RC*ti (d_k)
+    const int ti = threadIdx.x % 16, tj = threadIdx.x / 16;
 
     for (int c = c_begin; c < c_end; ++c) {
-        const int kvalid = c < nchunks ? min(kC, N - c * kC) : 0;
-        __syncthreads();
-        if (kvalid > 0) {
-            tile_to_smem<T, D, LD>(sK, Kh + (long long)c * kC * D, kC, kvalid, true, phi);
-            tile_to_smem<T, D, LD>(sV, Vh + (long long)c * kC * D, kC, kvalid, false, phi);
-        } else {
-            for (int e = threadIdx.x; e < kC * LD; e += kThreads) { sK[e] = 0.f; sV[e] = 0.f; }
-        }
+        const int kvalid = c < nchunks ? min(C, N - c * C) : 0;
+        __syncthreads();  // the previous chunk's tiles are no longer read
+        load_rows<T, D>(Kh + (long long)c * C * D, kvalid, [](int r) { return r; }, true, phi, sKT, sKn);
+        load_rows<T, D>(Vh + (long long)c * C * D, kvalid, [](int r) { return r; }, false, phi, nullptr, sVn);
         int qbeg, qend;
         if (GATHER) {
             qbeg = bin_start[(size_t)b * (nbins + 1) + c];
@@ -287,134 +411,80 @@ chunked_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __rest
             qbeg = 0;
             qend = kvalid;
         }
-        for (int qt = qbeg; qt < qend; qt += kC) {
-            const int nq = min(kC, qend - qt);
-            __syncthreads();
-            if (threadIdx.x < kC) {
+        for (int qt = qbeg; qt < qend; qt += C) {
+            const int nq = min(C, qend - qt);
+            __syncthreads();  // the previous tile's queries, P and row table are no longer read
+            if (threadIdx.x < C) {
                 const int r = threadIdx.x;
                 if (r < nq) {
-                    if (GATHER) {
-                        sRow[r] = perm[(size_t)b * N + qt + r];
-                        sLim[r] = msort[(size_t)b * N + qt + r] - c * kC;  // in [-1, kvalid-1]
-                    } else {
-                        sRow[r] = c * kC + r;
-                        sLim[r] = r;
-                    }
+                    sRow[r] = GATHER ? perm[(size_t)b * N + qt + r] : c * C + r;
+                    sLim[r] = GATHER ? msort[(size_t)b * N + qt + r] - c * C : r;  // keys 0..lim visible
                 } else {
                     sRow[r] = -1;
                     sLim[r] = -1;
                 }
             }
             __syncthreads();
-            // phi(Q) rows of this tile
+            load_rows<T, D>(Qh, nq, [&](int r) { return sRow[r]; }, true, phi, sQT, nullptr);
+            __syncthreads();
+            // P^T: queries x keys, masked
             {
-                constexpr int EPV = Vec16<T>::N, VPR = D / EPV;
-                for (int t = threadIdx.x; t < kC * VPR; t += kThreads) {
-                    const int r = t / VPR, col = (t % VPR) * EPV;
-                    float f[EPV];
-                    const int i = sRow[r];
-                    if (i >= 0) {
-                        Vec16<T>::unpack(ldg_stream(Qh + (long long)i * D + col), f);
+                float p[4][4] = {};
+                kmajor_acc<4, 4>(p, sQT, LC, 4 * ti, sKT, LC, 4 * tj, D);
+                int lim[4];
 #pragma unroll
-                        for (int e = 0; e < EPV; ++e) f[e] = phi_apply(f[e], phi);
-                    } else {
+                for (int r = 0; r < 4; ++r) lim[r] = sLim[4 * ti + r];
 #pragma unroll
-                        for (int e = 0; e < EPV; ++e) f[e] = 0.f;
-                    }
-                    float4* o = reinterpret_cast<float4*>(sQ + r * LD + col);
-#pragma unroll
-                    for (int e = 0; e < EPV; e += 4) o[e / 4] = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int j = 4 * tj + cc;
+                    *reinterpret_cast<float4*>(sPT + j * LC + 4 * ti) =
+                        make_float4(j <= lim[0] ? p[0][cc] : 0.f, j <= lim[1] ? p[1][cc] : 0.f,
+                                    j <= lim[2] ? p[2][cc] : 0.f, j <= lim[3] ? p[3][cc] : 0.f);
                 }
             }
             __syncthreads();
-            // P[i][j] = phi(q_i).phi(k_j) for visible j, else 0
-            for (int idx = threadIdx.x; idx < kC * kC; idx += kThreads) {
-                const int i = idx / kC, j = idx % kC;
-                float p = 0.f;
-                if (j <= sLim[i]) {
-                    const float* qi = sQ + i * LD;
-                    const float* kj = sK + j * LD;
-#pragma unroll 8
-                    for (int a = 0; a < D; ++a) p = fmaf(qi[a], kj[a], p);
-                }
-                sP[i * LDP + j] = p;
-            }
-            __syncthreads();
-            if (normalize && threadIdx.x < kC) {
+            // denominators: the row sums of P~ in key order, then phi(q).z
+            if (normalize && threadIdx.x < C) {
                 const int i = threadIdx.x;
                 float den = 0.f;
-                for (int j = 0; j < kC; ++j) den += sP[i * LDP + j];
+                for (int j = 0; j < C; ++j) den += sPT[j * LC + i];
                 float dz = 0.f;
-                for (int a = 0; a < D; ++a) dz = fmaf(sQ[i * LD + a], sz[a], dz);
+                for (int a = 0; a < D; ++a) dz = fmaf(sQT[a * LC + i], sz[a], dz);
                 sDen[i] = den + dz;
             }
-            float acc[RT][RC];
+            // O = phi(Q) S + P V
+            float o[4][RC] = {};
+            kmajor_acc<4, RC>(o, sQT, LC, 4 * ti, sS, LDD, RC * tj, D);
+            kmajor_acc<4, RC>(o, sPT, LC, 4 * ti, sVn, LDD, RC * tj, C);
+            __syncthreads();  // sDen
 #pragma unroll
-            for (int i = 0; i < RT; ++i)
-#pragma unroll
-                for (int cc = 0; cc < RC; ++cc) acc[i][cc] = 0.f;
-            for (int j = 0; j < kC; ++j) {
-                float vv[RC];
-                lds<RC>(sV + j * LD + tc * RC, vv);
-#pragma unroll
-                for (int i = 0; i < RT; ++i) {
-                    const float pij = sP[(tt * RT + i) * LDP + j];
-#pragma unroll
-                    for (int cc = 0; cc < RC; ++cc) acc[i][cc] = fmaf(pij, vv[cc], acc[i][cc]);
-                }
-            }
-#pragma unroll 4
-            for (int a = 0; a < D; ++a) {
-                float sv[RC];
-                lds<RC>(sS + a * D + tc * RC, sv);
-#pragma unroll
-                for (int i = 0; i < RT; ++i) {
-                    const float qa = sQ[(tt * RT + i) * LD + a];
-#pragma unroll
-                    for (int cc = 0; cc < RC; ++cc) acc[i][cc] = fmaf(qa, sv[cc], acc[i][cc]);
-                }
-            }
-            __syncthreads();
-#pragma unroll
-            for (int i = 0; i < RT; ++i) {
-                const int r = tt * RT + i;
-                const int row = sRow[r];
+            for (int r = 0; r < 4; ++r) {
+                const int i = 4 * ti + r;
+                const int row = sRow[i];
                 if (row < 0) continue;
-                const float den = normalize ? sDen[r] : 1.f;
+                const float inv = normalize ? 1.f / sDen[i] : 1.f;
+                float f[RC];
 #pragma unroll
-                for (int cc = 0; cc < RC; ++cc)
-                    Oh[(long long)row * D + tc * RC + cc] =
-                        from_f32<T>(normalize ? acc[i][cc] / den : acc[i][cc]);
+                for (int cc = 0; cc < RC; ++cc) f[cc] = o[r][cc] * inv;
+                T* dst = Oh + (long long)row * D + RC * tj;
+#pragma unroll
+                for (int cc = 0; cc < RC; ++cc) dst[cc] = from_f32<T>(f[cc]);
             }
         }
         // fold this chunk's keys into the running state
         if (kvalid > 0) {
             __syncthreads();
-            float up[R][R];
-            float zu[R];
+            float up[RC][RC] = {};
+            kmajor_acc<RC, RC>(up, sKn, LDD, RC * ti, sVn, LDD, RC * tj, C);
+            float zu = 0.f;
+            if (threadIdx.x < D)
+                for (int j = 0; j < C; ++j) zu += sKn[j * LDD + threadIdx.x];
+            __syncthreads();  // every read of the old state is done
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                zu[r] = 0.f;
+            for (int r = 0; r < RC; ++r)
 #pragma unroll
-                for (int cc = 0; cc < R; ++cc) up[r][cc] = 0.f;
-            }
-            for (int j = 0; j < kC; ++j) {
-                float a[R], bb[R];
-                lds<R>(sK + j * LD + ta * R, a);
-                lds<R>(sV + j * LD + tb * R, bb);
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    zu[r] += a[r];
-#pragma unroll
-                    for (int cc = 0; cc < R; ++cc) up[r][cc] = fmaf(a[r], bb[cc], up[r][cc]);
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-#pragma unroll
-                for (int cc = 0; cc < R; ++cc) sS[(ta * R + r) * D + tb * R + cc] += up[r][cc];
-                if (tb == 0) sz[ta * R + r] += zu[r];
-            }
+                for (int cc = 0; cc < RC; ++cc) sS[(RC * ti + r) * LDD + RC * tj + cc] += up[r][cc];
+            if (threadIdx.x < D) sz[threadIdx.x] += zu;
         }
     }
 }

@@ -87,7 +87,8 @@ struct PfCfg {
     static_assert(OFF_Q % 1024 == 0 && OFF_PT % 1024 == 0 && OFF_B3 % 1024 == 0 && OFF_BZ % 1024 == 0 &&
                       OFF_ONES % 1024 == 0,
                   "128-byte-swizzled tiles start on 1024-byte boundaries");
-    static_assert(XCH <= 2 * PT, "the block prefix is staged in the P~ buffers");
+    static_assert(XCH <= PT, "the block prefix is staged in the first P~ buffer");
+    static_assert(NMAX * 4 <= PT, "the mask row is staged in the second P~ buffer");
     static_assert(OFF_XCH % 16 == 0 && OFF_BAR % 8 == 0, "alignment");
     // TMEM columns: S (M = 64) and z, two P slots (M = 128, N = 128), two O
     // slots (O, then Oz)
@@ -465,13 +466,21 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         phase_b_waited = true;
         float* sbp = reinterpret_cast<float*>(pt);  // staged in the (idle) P~ buffers
         for (int e4 = et; e4 < (D * D + D) / 4; e4 += 128) {
+            // the lower ranks' pieces, eight loads in flight, summed in rank order
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int r = 0; r < rank; ++r) {
-                const float4 x = ld_cluster_f4(cluster_addr(xch + 4 * e4, r));
-                acc.x += x.x;
-                acc.y += x.y;
-                acc.z += x.z;
-                acc.w += x.w;
+            for (int r0 = 0; r0 < rank; r0 += 8) {
+                float4 x[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (r0 + q < rank) x[q] = ld_cluster_f4(cluster_addr(xch + 4 * e4, r0 + q));
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (r0 + q < rank) {
+                        acc.x += x[q].x;
+                        acc.y += x[q].y;
+                        acc.z += x[q].z;
+                        acc.w += x[q].w;
+                    }
             }
             reinterpret_cast<float4*>(sbp)[e4] = acc;
             if (S_total != nullptr && rank == (int)gridDim.x - 1) {
@@ -557,7 +566,21 @@ tc_prefix_fused_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
                 mbar_arrive(binned);
             }
         } else {
-        const int32_t* mb = m + (size_t)b * N;
+        // the sequence's m row into shared memory first (the second half of
+        // the P~ buffers, idle until phase D), every load in flight at once
+        int* mb = reinterpret_cast<int*>(pt + CF::PT);
+        {
+            // coalesced 4-byte loads (rows of m start anywhere), all issued
+            // before the first store
+            const int32_t* mg = m + (size_t)b * N;
+            constexpr int PER = CF::NMAX / 128;
+            int w[PER];
+#pragma unroll
+            for (int j = 0; j < PER; ++j) w[j] = mt + 128 * j < N ? mg[mt + 128 * j] : 0;
+#pragma unroll
+            for (int j = 0; j < PER; ++j)
+                if (mt + 128 * j < N) mb[mt + 128 * j] = w[j];
+        }
         for (int c = mt; c < 4 * CF::MAX_SUB; c += 128) hist[c] = 0;
         named_bar(2, 128);
         const int qlen = (N + 3) / 4, i0 = mw * qlen, i1 = min(N, i0 + qlen);
@@ -744,15 +767,19 @@ cudaError_t fused_phi(const Problem& p, const void* q, const void* k, const void
 bool tc_prefix_fused_plan(const Problem& p, int* block_tokens, int* nc) {
     if (p.dtype != DT_BF16 || p.d != PfCfg::D || p.N > PfCfg::NMAX) return false;
     // one CTA per SM: as many blocks per head as fill the SMs, at most 8 (a
-    // portable cluster)
-    const long long per_head = std::max(1LL, std::min(8LL, (long long)device_sms() / p.bh()));
-    const int bt = (int)(((p.N + per_head - 1) / per_head + PfCfg::KC - 1) / PfCfg::KC * PfCfg::KC);
-    const int n = (p.N + bt - 1) / bt;
-    // every head's cluster resident at once
-    if (p.bh() > max_active_clusters(n, PfCfg::THREADS, PfCfg::SMEM)) return false;
-    *block_tokens = bt;
-    *nc = n;
-    return true;
+    // portable cluster), fewer while the heads' clusters would not all be
+    // resident at once (a cluster lives inside one GPC)
+    for (long long per_head = std::max(1LL, std::min(8LL, (long long)device_sms() / p.bh())); per_head >= 1;
+         --per_head) {
+        const int bt = (int)(((p.N + per_head - 1) / per_head + PfCfg::KC - 1) / PfCfg::KC * PfCfg::KC);
+        const int n = (p.N + bt - 1) / bt;
+        if (p.bh() <= max_active_clusters(n, PfCfg::THREADS, PfCfg::SMEM)) {
+            *block_tokens = bt;
+            *nc = n;
+            return true;
+        }
+    }
+    return false;
 }
 
 cudaError_t tc_prefix_fused(const Problem& p, const void* q, const void* k, const void* v, const int32_t* m, void* out,

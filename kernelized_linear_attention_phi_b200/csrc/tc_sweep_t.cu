@@ -311,19 +311,17 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
         }
         // seed S^T with the block's prefix record (S stored [d_k][d_v])
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-            float f[32];
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            uint32_t r[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) f[e] = 0.f;
+            for (int e = 0; e < 16; ++e) r[e] = 0u;
+#pragma unroll 1
             for (int rb = 0; rb < npre; ++rb) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) f[e] += pre[rb * kRec + (size_t)(c0 + e) * D + a];
+                for (int e = 0; e < 16; ++e)
+                    r[e] = __float_as_uint(__uint_as_float(r[e]) + pre[rb * kRec + (size_t)(c0 + e) * D + a]);
             }
-            uint32_t r[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(f[e]);
-            tmem_st16(tmem + CF::COL_S + lane_base + c0, *reinterpret_cast<uint32_t(*)[16]>(r));
-            tmem_st16(tmem + CF::COL_S + lane_base + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+            tmem_st16(tmem + CF::COL_S + lane_base + c0, r);
         }
         tmem_st_wait();
         float zp = 0.f;  // z_prev[d_k = et]
@@ -351,6 +349,16 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
             float* rp = red + (ci & 1) * 4 * D;
 #pragma unroll
             for (int bx = 0; bx < CF::NB; ++bx) {
+                // the box's K chunks loaded before any is stored (then its Q
+                // chunks likewise): a load after a shared store could not be
+                // moved ahead of it, and with the tensor core reading operands
+                // each load is slow, so four are in flight at a time
+                uint4 kx[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int w = et + 128 * i;  // 16-byte chunk within the box
+                    kx[i] = *reinterpret_cast<const uint4*>(kt + bx * CF::KBOX + w * 16);
+                }
                 float cs[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) cs[e] = 0.f;
@@ -358,24 +366,27 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                 for (int i = 0; i < 4; ++i) {
                     const int w = et + 128 * i;  // 16-byte chunk within the box
                     const int r = w >> 3;
-                    uint4* kp = reinterpret_cast<uint4*>(kt + bx * CF::KBOX + w * 16);
-                    uint4 x = *kp;
+                    uint4 x = kx[i];
                     if (r < kvalid) {
                         if (mapped) x = phi8<PHI>(x);
                     } else {
                         x = make_uint4(0, 0, 0, 0);
                     }
-                    *kp = x;
+                    *reinterpret_cast<uint4*>(kt + bx * CF::KBOX + w * 16) = x;
                     if (normalize) {
                         float f[8];
                         unpack8(x, f);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) cs[e] += f[e];
                     }
-                    if (!GATHER && mapped) {
-                        uint4* qp = reinterpret_cast<uint4*>(st + bx * CF::BOX + w * 16);
-                        *qp = phi8<PHI>(*qp);
-                    }
+                }
+                if (!GATHER && mapped) {  // the Q chunks of the box, loads first as well
+                    uint4 qx[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) qx[i] = *reinterpret_cast<const uint4*>(st + bx * CF::BOX + (et + 128 * i) * 16);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        *reinterpret_cast<uint4*>(st + bx * CF::BOX + (et + 128 * i) * 16) = phi8<PHI>(qx[i]);
                 }
                 if (normalize) {
                     // lanes l, l^9, l^18, l^27 hold the same column group g
