@@ -91,9 +91,8 @@ CASE_TEXT = {
 TC_KERNELS = {
     "noncausal": {1: ["tc_noncausal_cluster_kernel"],
                   3: ["tc_kv_kernel", "kv_reduce_balanced_kernel", "tc_readout_kernel"]},
-    "causal": {1: ["tc_prefix_fused_kernel"], 2: ["tc_kv_kernel", "tc_sweep"],
-               3: ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"]},
-    "prefix": {1: ["tc_prefix_fused_kernel"], 3: ["tc_kv_kernel", "bin_kernel", "tc_sweep"],
+    "causal": {2: ["tc_kv_kernel", "tc_sweep"], 3: ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"]},
+    "prefix": {3: ["tc_kv_kernel", "bin_kernel", "tc_sweep"],
                4: ["tc_kv_kernel", "bin_kernel", "state_scan_kernel", "tc_sweep"]},
     "decode": {1: ["decode_kernel"]},
     "noncausal_bwd": {4: ["tc_noncausal_cluster_kernel", "tc_bwd_q_kernel", "kv_reduce_balanced_kernel",
@@ -122,7 +121,7 @@ KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balan
                "bin_kernel": "bin", "decode_kernel": "decode", "bwd_q_kernel": "bwd_q",
                "bwd_kv_kernel": "bwd_kv", "tc_bwd_q_kernel": "bwd_q", "tc_bwd_kv_kernel": "bwd_kv",
                "tc_bwd_causal_q_kernel": "bwd_q", "tc_bwd_causal_kv_kernel": "bwd_kv",
-               "tc_noncausal_cluster_kernel": "fused", "tc_prefix_fused_kernel": "prefix_fused"}
+               "tc_noncausal_cluster_kernel": "fused"}
 
 
 def block_plan(B, H, N, d, dtype, sms):
@@ -373,8 +372,7 @@ def kernel_bytes(form, kernel, B, H, N, d, elem):
         return {"kv": 2 * t, "fused": 2 * t, "bwd_q": (5 if causal else 3) * t,
                 "bwd_kv": (5 if causal else 4) * t}.get(role, 0)
     return {"kv": 2 * t, "reduce": st, "readout": 2 * t + st, "scan": 0, "sweep": 4 * t, "fused": 4 * t,
-            "prefix_fused": 4 * t + (B * N * 4 if form == "prefix" else 0), "bin": B * N * 4,
-            "decode": 2 * st + 4 * one}.get(role, 0)
+            "bin": B * N * 4, "decode": 2 * st + 4 * one}.get(role, 0)
 
 
 def flush_l2(buf):

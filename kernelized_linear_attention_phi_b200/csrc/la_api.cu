@@ -293,9 +293,6 @@ la_status causal_impl(const la_desc* desc, int32_t chunk, const void* q, const v
     // phase 1: per-block states; phase 2: exclusive prefix over blocks (and
     // the total); phase 3: each block's outputs from its prefix state.
     uint32_t* flags = at<uint32_t>(ws, 0);
-    int fbt = 0, fnc = 0;
-    if (tc_prefix_fused_plan(p, &fbt, &fnc))  // short sequences at d = 64: one kernel
-        return cuda_status(tc_causal_fused(p, q, k, v, out, S_total, z_total, flags, st));
     if (tc_supported(p) && p.d == 128 && S_total == nullptr && bp.nblk >= 2) {
         // the states of every block but the last (no block's prefix holds
         // it), then the sweep, whose CTAs each sum the states before their
@@ -432,13 +429,6 @@ la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, cons
     LA_TRY(check_device());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     timing_begin(st);
-    {
-        // sequences of at most 4096 tokens at d = 64: binning, block states,
-        // their prefix and the sweep in one kernel (a cluster per head)
-        int fbt = 0, fnc = 0;
-        if (tc_prefix_fused_plan(p, &fbt, &fnc))
-            return cuda_status(tc_prefix_fused(p, q, k, v, m, out, at<uint32_t>(ws, 0), st));
-    }
     const BlockPlan bp = block_plan(p);
     const bool tc = tc_supported(p);
     const int kchunk = tc ? tc_chunk(p, chunk) : kSimtChunk;  // chunk length of the kernel used

@@ -199,78 +199,61 @@ __global__ void state_scan_kernel(float* __restrict__ part, int nblk, int D,
 // ---------------------------------------------------------------------------
 template <int D>
 constexpr size_t readout_smem() {
-    return sizeof(float) * ((size_t)D * (D + 4) + D + (size_t)D * (64 + 4) + 64);
+    return sizeof(float) * ((size_t)D * D + D + 64 * (D + 4) + 64);
 }
 
-// 64 queries per CTA: phi(Q)^T staged k-major, then O = phi(Q) S as 4 x D/16
-// register blocks (one 16-byte load of each operand per step over d_k), the
-// denominator phi(q).z summed in d_k order.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 readout_kernel(const T* __restrict__ Q, const float* __restrict__ S, const float* __restrict__ z,
                T* __restrict__ out, int N, int phi, int normalize) {
-    constexpr int TQ = 64, LC = TQ + 4, LDD = D + 4, RC = D / 16;
+    constexpr int TQ = 64, LDQ = D + 4, RC = D / 16, RT = TQ / 16;
     extern __shared__ __align__(16) float sm[];
     float* sS = sm;
-    float* sz = sS + D * LDD;
-    float* sQT = sz + D;
-    float* sDen = sQT + D * LC;
+    float* sz = sS + D * D;
+    float* sQ = sz + D;
+    float* sDen = sQ + TQ * LDQ;
     const int tile = blockIdx.x;
     const long long bh = blockIdx.y;
     pdl_wait();
-    const float* Sh = S + (size_t)bh * D * D;
-    for (int e = threadIdx.x; e < D * D / 4; e += kThreads) {
-        const int a = (4 * e) / D, bcol = (4 * e) % D;
-        *reinterpret_cast<float4*>(sS + a * LDD + bcol) = reinterpret_cast<const float4*>(Sh)[e];
-    }
+    const float4* S4 = reinterpret_cast<const float4*>(S + (size_t)bh * D * D);
+    for (int e = threadIdx.x; e < D * D / 4; e += kThreads) reinterpret_cast<float4*>(sS)[e] = S4[e];
     for (int e = threadIdx.x; e < D; e += kThreads) sz[e] = z[(size_t)bh * D + e];
     const int row0 = tile * TQ;
-    const int nq = min(TQ, N - row0);
-    const T* Qh = Q + bh * (long long)N * D + (long long)row0 * D;
-    {
-        constexpr int EPV = Vec16<T>::N, VPR = D / EPV;
-        for (int t = threadIdx.x; t < TQ * VPR; t += kThreads) {
-            const int r = t / VPR, col = (t % VPR) * EPV;
-            float f[EPV];
-            if (r < nq) {
-                Vec16<T>::unpack(ldg_stream(Qh + (size_t)r * D + col), f);
-#pragma unroll
-                for (int e = 0; e < EPV; ++e) f[e] = phi_apply(f[e], phi);
-            } else {
-#pragma unroll
-                for (int e = 0; e < EPV; ++e) f[e] = 0.f;
-            }
-#pragma unroll
-            for (int e = 0; e < EPV; ++e) sQT[(col + e) * LC + r] = f[e];
-        }
-    }
+    const T* Qh = Q + bh * (long long)N * D;
+    tile_to_smem<T, D, LDQ>(sQ, Qh + (long long)row0 * D, TQ, min(TQ, N - row0), true, phi);
     __syncthreads();
     if (normalize && threadIdx.x < TQ) {
         float den = 0.f;
-        for (int a = 0; a < D; ++a) den = fmaf(sQT[a * LC + threadIdx.x], sz[a], den);
+        for (int a = 0; a < D; ++a) den = fmaf(sQ[threadIdx.x * LDQ + a], sz[a], den);
         sDen[threadIdx.x] = den;
     }
-    const int ti = threadIdx.x % 16, tj = threadIdx.x / 16;
-    float acc[4][RC] = {};
+    const int tc = threadIdx.x % 16, tt = threadIdx.x / 16;
+    float acc[RT][RC];
+#pragma unroll
+    for (int i = 0; i < RT; ++i)
+#pragma unroll
+        for (int c = 0; c < RC; ++c) acc[i][c] = 0.f;
 #pragma unroll 4
     for (int a = 0; a < D; ++a) {
-        float qa[4], sv[RC];
-        lds<4>(sQT + a * LC + 4 * ti, qa);
-        lds<RC>(sS + a * LDD + RC * tj, sv);
+        float sv[RC];
+        lds<RC>(sS + a * D + tc * RC, sv);
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int i = 0; i < RT; ++i) {
+            const float qa = sQ[(tt * RT + i) * LDQ + a];
 #pragma unroll
-            for (int c = 0; c < RC; ++c) acc[r][c] = fmaf(qa[r], sv[c], acc[r][c]);
+            for (int c = 0; c < RC; ++c) acc[i][c] = fmaf(qa, sv[c], acc[i][c]);
+        }
     }
     __syncthreads();
     T* Oh = out + bh * (long long)N * D;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int i = 4 * ti + r;
-        if (i >= nq) continue;
-        const float inv = normalize ? 1.f / sDen[i] : 1.f;
+    for (int i = 0; i < RT; ++i) {
+        const int row = row0 + tt * RT + i;
+        if (row >= N) continue;
+        const float den = normalize ? sDen[tt * RT + i] : 1.f;
 #pragma unroll
-        for (int c = 0; c < RC; ++c) Oh[(long long)(row0 + i) * D + RC * tj + c] = from_f32<T>(acc[r][c] * inv);
+        for (int c = 0; c < RC; ++c)
+            Oh[(long long)row * D + tc * RC + c] = from_f32<T>(normalize ? acc[i][c] / den : acc[i][c]);
     }
 }
 

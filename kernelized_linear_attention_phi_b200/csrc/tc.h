@@ -66,21 +66,6 @@ cudaError_t tc_chunked(const Problem& p, int chunk, const void* q, const void* k
                        const int32_t* bins, const int32_t* msort, int nbins, void* out, uint32_t* err,
                        cudaStream_t st);
 
-// Prefix-mask attention in one kernel (tc_prefix.cu): bf16, d = 64, N <= 4096,
-// a cluster of up to 8 CTAs per head (block_tokens keys each, nc blocks)
-// with every head's cluster resident at once. tc_prefix_fused_plan says
-// whether the kernel takes the problem and with which blocks; the kernel
-// needs no workspace beyond the error word *err (it sets FLAG_MASK_RANGE for
-// an m outside [0, N-1], which it clamps).
-bool tc_prefix_fused_plan(const Problem& p, int* block_tokens, int* nc);
-cudaError_t tc_prefix_fused(const Problem& p, const void* q, const void* k, const void* v, const int32_t* m, void* out,
-                            uint32_t* err, cudaStream_t st);
-// The causal form through the same kernel (m_i = i, no binning), under the
-// same plan; S_total / z_total (both or neither) receive the state after the
-// last token.
-cudaError_t tc_causal_fused(const Problem& p, const void* q, const void* k, const void* v, void* out, float* S_total,
-                            float* z_total, uint32_t* err, cudaStream_t st);
-
 // The d = 128 kernel behind tc_chunked (64-token chunks, state kept as S^T).
 // With raw_prefix, `prefix` holds each block's own state (as tc_kv_blocks
 // writes it; the last block's record is not read) and every CTA sums the

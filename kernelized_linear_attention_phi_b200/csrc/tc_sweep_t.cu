@@ -349,16 +349,6 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
             float* rp = red + (ci & 1) * 4 * D;
 #pragma unroll
             for (int bx = 0; bx < CF::NB; ++bx) {
-                // the box's K chunks loaded before any is stored (then its Q
-                // chunks likewise): a load after a shared store could not be
-                // moved ahead of it, and with the tensor core reading operands
-                // each load is slow, so four are in flight at a time
-                uint4 kx[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int w = et + 128 * i;  // 16-byte chunk within the box
-                    kx[i] = *reinterpret_cast<const uint4*>(kt + bx * CF::KBOX + w * 16);
-                }
                 float cs[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) cs[e] = 0.f;
@@ -366,27 +356,24 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                 for (int i = 0; i < 4; ++i) {
                     const int w = et + 128 * i;  // 16-byte chunk within the box
                     const int r = w >> 3;
-                    uint4 x = kx[i];
+                    uint4* kp = reinterpret_cast<uint4*>(kt + bx * CF::KBOX + w * 16);
+                    uint4 x = *kp;
                     if (r < kvalid) {
                         if (mapped) x = phi8<PHI>(x);
                     } else {
                         x = make_uint4(0, 0, 0, 0);
                     }
-                    *reinterpret_cast<uint4*>(kt + bx * CF::KBOX + w * 16) = x;
+                    *kp = x;
                     if (normalize) {
                         float f[8];
                         unpack8(x, f);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) cs[e] += f[e];
                     }
-                }
-                if (!GATHER && mapped) {  // the Q chunks of the box, loads first as well
-                    uint4 qx[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) qx[i] = *reinterpret_cast<const uint4*>(st + bx * CF::BOX + (et + 128 * i) * 16);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        *reinterpret_cast<uint4*>(st + bx * CF::BOX + (et + 128 * i) * 16) = phi8<PHI>(qx[i]);
+                    if (!GATHER && mapped) {
+                        uint4* qp = reinterpret_cast<uint4*>(st + bx * CF::BOX + w * 16);
+                        *qp = phi8<PHI>(*qp);
+                    }
                 }
                 if (normalize) {
                     // lanes l, l^9, l^18, l^27 hold the same column group g

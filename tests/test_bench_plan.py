@@ -30,7 +30,6 @@ def test_kernel_names_follow_the_count_of_launches():
     assert kn("causal", "bf16", 128, 3) == ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"]
     assert kn("causal", "bf16", 64, 2) == ["tc_kv_kernel", "tc_sweep"]
     assert kn("prefix", "bf16", 64, 3)[-1] == "tc_sweep"
-    assert kn("prefix", "bf16", 64, 1) == ["tc_prefix_fused_kernel"]
     # fp32 and small d run on the CUDA cores
     assert kn("causal", "f32", 64, 3) == ["kv_partial_kernel", "state_scan_kernel", "chunked_kernel"]
     assert kn("noncausal", "bf16", 16, 3)[0] == "kv_partial_kernel"
@@ -60,8 +59,6 @@ def test_kernel_bytes():
     assert kb("noncausal", "tc_readout_kernel") == 2 * t + st
     assert kb("noncausal", "tc_noncausal_cluster_kernel") == 4 * t
     assert kb("prefix", "bin_kernel") == B * N * 4
-    assert kb("prefix", "tc_prefix_fused_kernel") == 4 * t + B * N * 4
-    assert kb("causal", "tc_prefix_fused_kernel") == 4 * t
     assert kb("decode", "decode_kernel") == 2 * st + 4 * B * H * d * e
     assert kb("noncausal_bwd", "tc_noncausal_cluster_kernel") == 2 * t
     assert kb("noncausal_bwd", "tc_bwd_q_kernel") == 3 * t

@@ -12,12 +12,12 @@ pytestmark = pytest.mark.gpu
 
 # kernels per call on the bf16 tensor-core path at this size (8 heads of
 # 1024 tokens, d = 64): KV summary and non-causal: one thread-block-cluster
-# kernel (a cluster per head reduces the summary); causal and prefix mask: one
-# kernel (binning for the mask, block states, their prefix and the sweep, a
-# cluster per head); decode: one; gradients: forward states (non-causal: the
-# cluster kernel without its readout; causal: scanned in-cluster), dq sweep,
-# (G, h) reduction or reverse scan, dk/dv sweep
-TC_LAUNCHES = {"kv_summary": 1, "noncausal": 1, "causal": 1, "prefix": 1, "decode": 1, "noncausal_bwd": 4,
+# kernel (a cluster per head reduces the summary); causal: block states
+# scanned inside a cluster per head, sweep; prefix mask: the same plus the
+# binning; decode: one; gradients: forward states (non-causal: the cluster
+# kernel without its readout; causal: scanned in-cluster), dq sweep, (G, h)
+# reduction or reverse scan, dk/dv sweep
+TC_LAUNCHES = {"kv_summary": 1, "noncausal": 1, "causal": 2, "prefix": 3, "decode": 1, "noncausal_bwd": 4,
                "causal_bwd": 4}
 
 
