@@ -257,12 +257,6 @@ la_status la_noncausal(const la_desc* desc, const void* q, const void* k, const 
     // small problems: one kernel, a thread-block cluster per head
     if (tc_noncausal_fused_supported(p))
         return cuda_status(tc_noncausal_fused(p, q, k, v, out, S_out, z_out, at<uint32_t>(ws, 0), st));
-    if (tc_supported(p) && S_out == nullptr) {
-        // no state asked for: the readout sums the KV pass's records itself
-        float* part = at<float>(ws, L.part);
-        LA_TRY(cuda_status(tc_kv_partials(p, k, v, part, at<uint32_t>(ws, 0), st)));
-        return cuda_status(tc_readout_partials(p, q, part, out, at<uint32_t>(ws, 0), st));
-    }
     float* S = S_out;
     float* z = z_out;
     if (S == nullptr) {

@@ -21,7 +21,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kC = 64;   // chunk length of the SIMT chunked kernel
-constexpr int kReadoutTiles = 4;  // 64-query tiles per CTA of the readout
 
 template <int R>
 __device__ __forceinline__ void lds(const float* p, float* o) {
@@ -213,51 +212,48 @@ readout_kernel(const T* __restrict__ Q, const float* __restrict__ S, const float
     float* sz = sS + D * D;
     float* sQ = sz + D;
     float* sDen = sQ + TQ * LDQ;
+    const int tile = blockIdx.x;
     const long long bh = blockIdx.y;
     pdl_wait();
     const float4* S4 = reinterpret_cast<const float4*>(S + (size_t)bh * D * D);
     for (int e = threadIdx.x; e < D * D / 4; e += kThreads) reinterpret_cast<float4*>(sS)[e] = S4[e];
     for (int e = threadIdx.x; e < D; e += kThreads) sz[e] = z[(size_t)bh * D + e];
+    const int row0 = tile * TQ;
     const T* Qh = Q + bh * (long long)N * D;
-    // kReadoutTiles query tiles per CTA: the head's S is staged once for all of them
-    for (int tile = blockIdx.x * kReadoutTiles; tile < (blockIdx.x + 1) * kReadoutTiles && tile * TQ < N; ++tile) {
-        const int row0 = tile * TQ;
-        __syncthreads();  // the previous tile's queries and denominators are no longer read
-        tile_to_smem<T, D, LDQ>(sQ, Qh + (long long)row0 * D, TQ, min(TQ, N - row0), true, phi);
-        __syncthreads();
-        if (normalize && threadIdx.x < TQ) {
-            float den = 0.f;
-            for (int a = 0; a < D; ++a) den = fmaf(sQ[threadIdx.x * LDQ + a], sz[a], den);
-            sDen[threadIdx.x] = den;
-        }
-        const int tc = threadIdx.x % 16, tt = threadIdx.x / 16;
-        float acc[RT][RC];
+    tile_to_smem<T, D, LDQ>(sQ, Qh + (long long)row0 * D, TQ, min(TQ, N - row0), true, phi);
+    __syncthreads();
+    if (normalize && threadIdx.x < TQ) {
+        float den = 0.f;
+        for (int a = 0; a < D; ++a) den = fmaf(sQ[threadIdx.x * LDQ + a], sz[a], den);
+        sDen[threadIdx.x] = den;
+    }
+    const int tc = threadIdx.x % 16, tt = threadIdx.x / 16;
+    float acc[RT][RC];
 #pragma unroll
-        for (int i = 0; i < RT; ++i)
+    for (int i = 0; i < RT; ++i)
 #pragma unroll
-            for (int c = 0; c < RC; ++c) acc[i][c] = 0.f;
+        for (int c = 0; c < RC; ++c) acc[i][c] = 0.f;
 #pragma unroll 4
-        for (int a = 0; a < D; ++a) {
-            float sv[RC];
-            lds<RC>(sS + a * D + tc * RC, sv);
-#pragma unroll
-            for (int i = 0; i < RT; ++i) {
-                const float qa = sQ[(tt * RT + i) * LDQ + a];
-#pragma unroll
-                for (int c = 0; c < RC; ++c) acc[i][c] = fmaf(qa, sv[c], acc[i][c]);
-            }
-        }
-        __syncthreads();
-        T* Oh = out + bh * (long long)N * D;
+    for (int a = 0; a < D; ++a) {
+        float sv[RC];
+        lds<RC>(sS + a * D + tc * RC, sv);
 #pragma unroll
         for (int i = 0; i < RT; ++i) {
-            const int row = row0 + tt * RT + i;
-            if (row >= N) continue;
-            const float den = normalize ? sDen[tt * RT + i] : 1.f;
+            const float qa = sQ[(tt * RT + i) * LDQ + a];
 #pragma unroll
-            for (int c = 0; c < RC; ++c)
-                Oh[(long long)row * D + tc * RC + c] = from_f32<T>(normalize ? acc[i][c] / den : acc[i][c]);
+            for (int c = 0; c < RC; ++c) acc[i][c] = fmaf(qa, sv[c], acc[i][c]);
         }
+    }
+    __syncthreads();
+    T* Oh = out + bh * (long long)N * D;
+#pragma unroll
+    for (int i = 0; i < RT; ++i) {
+        const int row = row0 + tt * RT + i;
+        if (row >= N) continue;
+        const float den = normalize ? sDen[tt * RT + i] : 1.f;
+#pragma unroll
+        for (int c = 0; c < RC; ++c)
+            Oh[(long long)row * D + tc * RC + c] = from_f32<T>(normalize ? acc[i][c] / den : acc[i][c]);
     }
 }
 
@@ -307,13 +303,13 @@ __device__ __forceinline__ void kmajor_acc(float (&acc)[RI][RJ], const float* A,
     }
 }
 
-// Rows of a [C x D] input tile into shared memory, phi applied when asked,
-// in natural layout (dstN[row][col], row length LDD; consecutive threads take
-// consecutive 16-byte column groups of a row). Row r of the tile is src row
-// `rowidx(r)`; a negative index, or r >= valid, gives a zero row.
+// Rows of a [C x D] input tile into shared memory, phi applied when asked:
+// transposed (dstT[col][row], row length LC) and/or natural (dstN[row][col],
+// row length LDD). Row r of the tile is src row `rowidx(r)`; a negative
+// index, or r >= valid, gives a zero row.
 template <typename T, int D, typename RowIdx>
 __device__ __forceinline__ void load_rows(const T* src, int valid, RowIdx rowidx, bool apply_phi, int phi,
-                                          float* dstN) {
+                                          float* dstT, float* dstN) {
     using CF = ChCfg<D>;
     constexpr int EPV = Vec16<T>::N, VPR = D / EPV;
     for (int t = threadIdx.x; t < CF::C * VPR; t += kThreads) {
@@ -330,42 +326,15 @@ __device__ __forceinline__ void load_rows(const T* src, int valid, RowIdx rowidx
 #pragma unroll
             for (int e = 0; e < EPV; ++e) f[e] = 0.f;
         }
+        if (dstT) {
 #pragma unroll
-        for (int e = 0; e < EPV; e += 4)
-            *reinterpret_cast<float4*>(dstN + r * CF::LDD + col + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
-    }
-}
-
-// The same rows transposed (dstT[col][row], row length LC), built from
-// blocks of 4 rows x one 16-byte column group per thread: a warp's loads
-// cover whole 32-byte sectors and its stores of four consecutive rows per
-// column are conflict-free float4s.
-template <typename T, int D, typename RowIdx>
-__device__ __forceinline__ void load_rows_t(const T* src, int valid, RowIdx rowidx, bool apply_phi, int phi,
-                                            float* dstT) {
-    using CF = ChCfg<D>;
-    constexpr int EPV = Vec16<T>::N, VPR = D / EPV, RB = CF::C / 4;
-    for (int t = threadIdx.x; t < RB * VPR; t += kThreads) {
-        const int rb = t % RB, col = (t / RB) * EPV;
-        float f[4][EPV];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = 4 * rb + i;
-            const int row = r < valid ? rowidx(r) : -1;
-            if (row >= 0) {
-                Vec16<T>::unpack(ldg_stream(src + (size_t)row * D + col), f[i]);
-                if (apply_phi) {
-#pragma unroll
-                    for (int e = 0; e < EPV; ++e) f[i][e] = phi_apply(f[i][e], phi);
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < EPV; ++e) f[i][e] = 0.f;
-            }
+            for (int e = 0; e < EPV; ++e) dstT[(col + e) * CF::LC + r] = f[e];
         }
+        if (dstN) {
 #pragma unroll
-        for (int e = 0; e < EPV; ++e)
-            *reinterpret_cast<float4*>(dstT + (col + e) * CF::LC + 4 * rb) = make_float4(f[0][e], f[1][e], f[2][e], f[3][e]);
+            for (int e = 0; e < EPV; e += 4)
+                *reinterpret_cast<float4*>(dstN + r * CF::LDD + col + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+        }
     }
 }
 
@@ -415,9 +384,8 @@ chunked_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __rest
     for (int c = c_begin; c < c_end; ++c) {
         const int kvalid = c < nchunks ? min(C, N - c * C) : 0;
         __syncthreads();  // the previous chunk's tiles are no longer read
-        load_rows_t<T, D>(Kh + (long long)c * C * D, kvalid, [](int r) { return r; }, true, phi, sKT);
-        load_rows<T, D>(Kh + (long long)c * C * D, kvalid, [](int r) { return r; }, true, phi, sKn);
-        load_rows<T, D>(Vh + (long long)c * C * D, kvalid, [](int r) { return r; }, false, phi, sVn);
+        load_rows<T, D>(Kh + (long long)c * C * D, kvalid, [](int r) { return r; }, true, phi, sKT, sKn);
+        load_rows<T, D>(Vh + (long long)c * C * D, kvalid, [](int r) { return r; }, false, phi, nullptr, sVn);
         int qbeg, qend;
         if (GATHER) {
             qbeg = bin_start[(size_t)b * (nbins + 1) + c];
@@ -440,7 +408,7 @@ chunked_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __rest
                 }
             }
             __syncthreads();
-            load_rows_t<T, D>(Qh, nq, [&](int r) { return sRow[r]; }, true, phi, sQT);
+            load_rows<T, D>(Qh, nq, [&](int r) { return sRow[r]; }, true, phi, sQT, nullptr);
             __syncthreads();
             // P^T: queries x keys, masked
             {
@@ -518,7 +486,7 @@ cudaError_t launch_readout(const Problem& p, const void* q, const float* S, cons
     constexpr size_t smem = readout_smem<D>();
     cudaError_t e = ensure_smem<readout_kernel<T, D>>(smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((p.N + 64 * kReadoutTiles - 1) / (64 * kReadoutTiles), (unsigned)p.bh());
+    dim3 grid((p.N + 63) / 64, (unsigned)p.bh());
     return launch_pdl(readout_kernel<T, D>, grid, dim3(kThreads), smem, st, static_cast<const T*>(q), S, z,
                       static_cast<T*>(out), p.N, p.phi, p.normalize);
 }

@@ -55,14 +55,6 @@ cudaError_t tc_kv_blocks_scan(const Problem& p, const void* k, const void* v, in
 // Same contract as simt_readout.
 cudaError_t tc_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,
                        uint32_t* err, cudaStream_t st);
-// Non-causal attention without the reduction kernel in between: the KV
-// pass's partial records (balanced split, as tc_kv_summary writes them into
-// `part`), then the readout, whose CTAs sum the records of each head they
-// answer in CTA order (the order the reduction adds them in).
-cudaError_t tc_kv_partials(const Problem& p, const void* k, const void* v, float* part, uint32_t* err,
-                           cudaStream_t st);
-cudaError_t tc_readout_partials(const Problem& p, const void* q, const float* part, void* out, uint32_t* err,
-                                cudaStream_t st);
 
 // Chunk length the tensor-core chunked kernel runs at for a requested chunk
 // (d = 128 always runs 64-token chunks: the shared-memory budget).

@@ -463,8 +463,8 @@ struct RoCfg {
 template <int D, int PHI>
 __global__ void __launch_bounds__(kThreads, RoCfg<D>::PER_SM)
 tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mOut,
-                  const float* __restrict__ S, const float* __restrict__ z, const float* __restrict__ part,
-                  KvBalanced wkv, int N, long long total, int tph, int normalize, uint32_t* __restrict__ err) {
+                  const float* __restrict__ S, const float* __restrict__ z, int N, long long total,
+                  int tph, int normalize, uint32_t* __restrict__ err) {
     using C = RoCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles = align1024(smem_raw);
@@ -571,47 +571,20 @@ tc_readout_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                 // first tile of a head: its S and z into operand buffer (h - h0) & 1
                 uint8_t* sb = bS + ((h - h0) & 1) * C::BS;
                 uint8_t* zb = bZ + ((h - h0) & 1) * C::BZ;
-                // eight consecutive floats of the head's record (S then z):
-                // from S, z, or with `part` the KV pass's partial records of
-                // the head summed in CTA order (as kv_reduce_balanced_kernel
-                // sums them)
-                int c0 = 0, c1 = -1;
-                if (part != nullptr) {
-                    c0 = cta_of(wkv, h * wkv.tph);
-                    c1 = cta_of(wkv, (h + 1) * wkv.tph - 1);
-                }
-                auto state8 = [&](int idx, float (&f)[8]) {
-                    if (part == nullptr) {
-                        const float* src = idx < D * D ? S + (size_t)h * D * D + idx : z + (size_t)h * D + (idx - D * D);
-                        const float4 x0 = reinterpret_cast<const float4*>(src)[0];
-                        const float4 x1 = reinterpret_cast<const float4*>(src)[1];
-                        f[0] = x0.x, f[1] = x0.y, f[2] = x0.z, f[3] = x0.w, f[4] = x1.x, f[5] = x1.y, f[6] = x1.z, f[7] = x1.w;
-                        return;
-                    }
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = 0.f;
-                    for (int c = c0; c <= c1; ++c) {
-                        const long long j = h - range_lo(wkv.total, wkv.G, c) / wkv.tph;
-                        const float* rec = part + ((size_t)c * wkv.K + j) * (size_t)(D * D + D) + idx;
-                        const float4 x0 = reinterpret_cast<const float4*>(rec)[0];
-                        const float4 x1 = reinterpret_cast<const float4*>(rec)[1];
-                        f[0] += x0.x, f[1] += x0.y, f[2] += x0.z, f[3] += x0.w;
-                        f[4] += x1.x, f[5] += x1.y, f[6] += x1.z, f[7] += x1.w;
-                    }
-                };
+                const float* Sh = S + (size_t)h * D * D;
                 for (int c = et; c < D * D / 8; c += 128) {
                     const int a = c / (D / 8), col = (c % (D / 8)) * 8;
-                    float f[8];
-                    state8(a * D + col, f);
+                    const float4 x0 = reinterpret_cast<const float4*>(Sh + (size_t)a * D + col)[0];
+                    const float4 x1 = reinterpret_cast<const float4*>(Sh + (size_t)a * D + col)[1];
+                    const float f[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
                     *reinterpret_cast<uint4*>(sb + (col / 64) * (D * 128) + sw128_off(a, col % 64)) = pack8(f);
                 }
                 for (int c = et; c < D / 8; c += 128) {
                     const int col = c * 8;
-                    float fh[8], fl[8], zs[8];
-                    state8(D * D + col, zs);
+                    float fh[8], fl[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float zv = zs[e];
+                        const float zv = z[(size_t)h * D + col + e];
                         fh[e] = __bfloat162float(__float2bfloat16_rn(zv));
                         fl[e] = zv - fh[e];
                     }
@@ -719,29 +692,28 @@ cudaError_t launch_kv(const Problem& p, const void* k, const void* v, const KvWo
 
 template <int D, int PHI>
 cudaError_t launch_readout_phi(const Problem& p, const CUtensorMap& mq, const CUtensorMap& mo, const float* S,
-                               const float* z, const float* part, const KvBalanced& wkv, uint32_t* err,
-                               cudaStream_t st) {
+                               const float* z, uint32_t* err, cudaStream_t st) {
     constexpr size_t smem = RoCfg<D>::SMEM;
     cudaError_t e = ensure_smem<tc_readout_kernel<D, PHI>>(smem);
     if (e != cudaSuccess) return e;
     const int tph = (p.N + kTile - 1) / kTile;
     const long long total = p.bh() * tph;
     const int G = plan::balanced_ctas(total, device_sms(), RoCfg<D>::PER_SM);
-    return launch_pdl(tc_readout_kernel<D, PHI>, dim3(G), dim3(kThreads), smem, st, mq, mo, S, z, part, wkv, p.N,
-                      total, tph, p.normalize, err);
+    return launch_pdl(tc_readout_kernel<D, PHI>, dim3(G), dim3(kThreads), smem, st, mq, mo, S, z, p.N, total, tph,
+                      p.normalize, err);
 }
 
 template <int D>
-cudaError_t launch_readout(const Problem& p, const void* q, const float* S, const float* z, const float* part,
-                           const KvBalanced& wkv, void* out, uint32_t* err, cudaStream_t st) {
+cudaError_t launch_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,
+                           uint32_t* err, cudaStream_t st) {
     CUtensorMap mq, mo;
     cudaError_t e = make_map(&mq, q, D, p.N, p.bh(), kTile);
     if (e == cudaSuccess) e = make_map(&mo, out, D, p.N, p.bh(), kTile);
     if (e != cudaSuccess) return e;
     switch (p.phi) {  // one kernel per feature map (see phi8)
-        case PHI_RELU1: return launch_readout_phi<D, PHI_RELU1>(p, mq, mo, S, z, part, wkv, err, st);
-        case PHI_ELU1: return launch_readout_phi<D, PHI_ELU1>(p, mq, mo, S, z, part, wkv, err, st);
-        default: return launch_readout_phi<D, PHI_IDENTITY>(p, mq, mo, S, z, part, wkv, err, st);
+        case PHI_RELU1: return launch_readout_phi<D, PHI_RELU1>(p, mq, mo, S, z, err, st);
+        case PHI_ELU1: return launch_readout_phi<D, PHI_ELU1>(p, mq, mo, S, z, err, st);
+        default: return launch_readout_phi<D, PHI_IDENTITY>(p, mq, mo, S, z, err, st);
     }
 }
 
@@ -826,25 +798,8 @@ cudaError_t tc_kv_blocks(const Problem& p, const void* k, const void* v, int blo
 
 cudaError_t tc_readout(const Problem& p, const void* q, const float* S, const float* z, void* out, uint32_t* err,
                        cudaStream_t st) {
-    const KvBalanced none{};
-    return p.d == 64 ? launch_readout<64>(p, q, S, z, nullptr, none, out, err, st)
-                     : launch_readout<128>(p, q, S, z, nullptr, none, out, err, st);
-}
-
-cudaError_t tc_kv_partials(const Problem& p, const void* k, const void* v, float* part, uint32_t* err,
-                           cudaStream_t st) {
-    KvWork w{};
-    w.balanced = 1;
-    w.b = kv_balanced_plan(p);
-    const dim3 grid(w.b.G);
-    return p.d == 64 ? launch_kv<64>(p, k, v, w, grid, part, err, st) : launch_kv<128>(p, k, v, w, grid, part, err, st);
-}
-
-cudaError_t tc_readout_partials(const Problem& p, const void* q, const float* part, void* out, uint32_t* err,
-                                cudaStream_t st) {
-    const KvBalanced wkv = kv_balanced_plan(p);
-    return p.d == 64 ? launch_readout<64>(p, q, nullptr, nullptr, part, wkv, out, err, st)
-                     : launch_readout<128>(p, q, nullptr, nullptr, part, wkv, out, err, st);
+    return p.d == 64 ? launch_readout<64>(p, q, S, z, out, err, st)
+                     : launch_readout<128>(p, q, S, z, out, err, st);
 }
 
 }  // namespace la
