@@ -282,6 +282,21 @@ __device__ __forceinline__ void tmem_ld2(uint32_t taddr, uint32_t (&r)[2]) {
                  : "=r"(r[0]), "=r"(r[1])
                  : "r"(taddr));
 }
+// Warp-wide, 16 TMEM lanes, eight repetitions of 8 columns (the 16x256b
+// shape): for repetition k, lane i receives in r[4k], r[4k + 1] TMEM lane
+// (base + i / 4) at columns col + 8k + 2 (i % 4) + {0, 1}, and in r[4k + 2],
+// r[4k + 3] the same columns of TMEM lane (base + 8 + i / 4).
+__device__ __forceinline__ void tmem_ld16x256_x8(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+          "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -295,6 +310,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Warp-wide: four 8x8 16-bit matrices stored transposed. In register m,
+// lane i holds the packed pair (row i / 4, columns 2 (i % 4) and 2 (i % 4) + 1)
+// of matrix m; the pair lands in stored rows 2 (i % 4) and 2 (i % 4) + 1 at
+// column i / 4. Lanes 8m .. 8m + 7 give the shared addresses of stored rows
+// 0..7 of matrix m (16 bytes each, 16-byte aligned).
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t p0, uint32_t p1, uint32_t p2,
+                                                  uint32_t p3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(saddr), "r"(p0),
+                 "r"(p1), "r"(p2), "r"(p3)
+                 : "memory");
 }
 
 // Named barrier over `nthreads` threads (multiple of 32).

@@ -441,7 +441,6 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
         const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
         const int i = sp * 16 + (lane & 15);  // P row (query) of this thread: M = 64 layout
         const int half = lane >= 16 ? 1 : 0;  // the two warp halves take the two column halves
-        const int a = sp * 32 + lane;         // O^T row (d_v index) of this thread
         const int et2 = threadIdx.x - 192;
         // No early exit in this warpgroup (named barrier 3); a failed wait
         // only suppresses the output stores.
@@ -495,28 +494,39 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
                 if (GATHER && et2 < C) orows[slot * C + et2] = srow[et2];
                 if (!GATHER && et2 == 0) bulk_wait_read0();  // the previous tile's store has read stg
                 named_bar(3, 128);  // also: the previous copy-out is done, inv[] is written
-                uint8_t* sbx = stg + (a / 64) * CF::BOX;
-                const int col = a % 64;
+                // O^T rows (d_v) a0 .. a0 + 15 per lane half, 16 columns (queries)
+                // at a time: the 16x256b TMEM shape hands each lane two rows x two
+                // adjacent columns, which is the fragment stmatrix .trans stores as
+                // 8 x 8 blocks with the queries as rows (16 bytes of d_v each).
+                const int mi = lane >> 3, mj = lane & 7;  // the block, and its row, this lane addresses
+                const int q2 = 2 * (lane & 3);           // this lane's first column within 8
+                const uint32_t stg_u = smem_u32(stg);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int hl = 0; hl < 2; ++hl) {
+                    const int a0 = sp * 32 + 16 * hl;
                     uint32_t o[32];
-                    tmem_ld16(tmem + CF::COL_O + slot * C + lane_base + 32 * h, *reinterpret_cast<uint32_t(*)[16]>(o));
-                    tmem_ld16(tmem + CF::COL_O + slot * C + lane_base + 32 * h + 16,
-                              *reinterpret_cast<uint32_t(*)[16]>(o + 16));
+                    tmem_ld16x256_x8(tmem + CF::COL_O + slot * C + (static_cast<uint32_t>(a0) << 16), o);
                     tmem_ld_wait();
-                    if (h == 1) {
+                    if (hl == 1) {
                         tc_fence_before();
                         mbar_arrive(bofree + slot);  // O^T[slot] read (and, gathered, the row table)
                     }
+                    const uint32_t box = stg_u + (a0 / 64) * CF::BOX;
+                    const int ch = (a0 % 64) / 8 + (mi & 1);  // 16-byte column chunk of the addressed block
 #pragma unroll
-                    for (int q = 0; q < 32; q += 4) {
-                        const float4 iv = normalize ? *reinterpret_cast<const float4*>(inv + 32 * h + q)
-                                                    : make_float4(1.f, 1.f, 1.f, 1.f);
-                        const float sc[4] = {iv.x, iv.y, iv.z, iv.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            *reinterpret_cast<__nv_bfloat16*>(sbx + sw128_off(32 * h + q + e, col)) =
-                                __float2bfloat16_rn(__uint_as_float(o[q + e]) * sc[e]);
+                    for (int cb = 0; cb < C; cb += 16) {
+                        const float2 i0 = normalize ? *reinterpret_cast<const float2*>(inv + cb + q2)
+                                                    : make_float2(1.f, 1.f);
+                        const float2 i1 = normalize ? *reinterpret_cast<const float2*>(inv + cb + 8 + q2)
+                                                    : make_float2(1.f, 1.f);
+                        const uint32_t* r = o + (cb / 8) * 4;
+                        const uint32_t p0 = pack_bf16(__uint_as_float(r[0]) * i0.x, __uint_as_float(r[1]) * i0.y);
+                        const uint32_t p1 = pack_bf16(__uint_as_float(r[2]) * i0.x, __uint_as_float(r[3]) * i0.y);
+                        const uint32_t p2 = pack_bf16(__uint_as_float(r[4]) * i1.x, __uint_as_float(r[5]) * i1.y);
+                        const uint32_t p3 = pack_bf16(__uint_as_float(r[6]) * i1.x, __uint_as_float(r[7]) * i1.y);
+                        const uint32_t row = cb + 8 * (mi >> 1) + mj;
+                        stmatrix_x4_trans(box + row * 128u + ((static_cast<uint32_t>(ch) ^ (row & 7u)) << 4), p0, p1,
+                                          p2, p3);
                     }
                 }
                 fence_async_smem();
