@@ -113,6 +113,18 @@ SIMT_KERNELS = {
     "causal_bwd": {5: ["kv_partial_kernel", "state_scan_kernel", "bwd_q_kernel", "state_scan_kernel",
                        "bwd_kv_kernel"]},
 }
+# fp32 at d = 64: the split-precision tensor-core kernel in its three modes
+# (block / split states, causal sweep, readout); the prefix mask and decode
+# stay on the CUDA cores
+F32_TC_KERNELS = dict(SIMT_KERNELS)
+F32_TC_KERNELS.update({
+    "noncausal": {3: ["tc_f32_kernel<0", "state_reduce_kernel", "tc_f32_kernel<2"]},
+    "causal": {3: ["tc_f32_kernel<0", "state_scan_kernel", "tc_f32_kernel<1"]},
+    "noncausal_bwd": {5: ["tc_f32_kernel<0", "state_reduce_kernel", "bwd_q_kernel", "state_reduce_kernel",
+                          "bwd_kv_kernel"]},
+    "causal_bwd": {5: ["tc_f32_kernel<0", "state_scan_kernel", "bwd_q_kernel", "state_scan_kernel",
+                       "bwd_kv_kernel"]},
+})
 
 # What each kernel does, for its algorithmic bytes (Call.kernel_bytes).
 KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balanced_kernel": "reduce",
@@ -121,7 +133,8 @@ KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balan
                "bin_kernel": "bin", "decode_kernel": "decode", "bwd_q_kernel": "bwd_q",
                "bwd_kv_kernel": "bwd_kv", "tc_bwd_q_kernel": "bwd_q", "tc_bwd_kv_kernel": "bwd_kv",
                "tc_bwd_causal_q_kernel": "bwd_q", "tc_bwd_causal_kv_kernel": "bwd_kv",
-               "tc_noncausal_cluster_kernel": "fused"}
+               "tc_noncausal_cluster_kernel": "fused", "tc_f32_kernel<0": "kv", "tc_f32_kernel<1": "sweep",
+               "tc_f32_kernel<2": "readout"}
 
 
 def block_plan(B, H, N, d, dtype, sms):
@@ -134,11 +147,17 @@ def block_plan(B, H, N, d, dtype, sms):
     return bt, -(-N // bt)
 
 
+def kernel_table(dtype, d):
+    """The kernels the library runs a problem on: tensor cores for bf16 with
+    d = 64 or 128 and (split precision) fp32 with d = 64; CUDA cores otherwise."""
+    if dtype == "bf16" and d in (64, 128):
+        return TC_KERNELS
+    return F32_TC_KERNELS if dtype == "f32" and d == 64 else SIMT_KERNELS
+
+
 def kernel_names(form, dtype, d, count):
-    """Names of the `count` kernels a call of `form` launched (tensor cores:
-    bf16 with d = 64 or 128; CUDA cores otherwise)."""
-    table = TC_KERNELS if dtype == "bf16" and d in (64, 128) else SIMT_KERNELS
-    names = table.get(form, {}).get(count)
+    """Names of the `count` kernels a call of `form` launched."""
+    names = kernel_table(dtype, d).get(form, {}).get(count)
     return names if names else [f"kernel{i}" for i in range(count)]
 
 
@@ -844,7 +863,7 @@ def record_traffic(csv_path, case, scale):
         # per-kernel timing replays each call in turn after the timed steps)
         wl = W.WORKLOADS[w]
         name = wl.name if form != "prefix" or mask == "uniform" else f"{wl.name}_{mask}"
-        table = (TC_KERNELS if dt == "bf16" and wl.d in (64, 128) else SIMT_KERNELS)[form]
+        table = kernel_table(dt, wl.d)[form]
         found = None
         for start in range(len(seq) - 1, -1, -1):
             for count in sorted(table, reverse=True):

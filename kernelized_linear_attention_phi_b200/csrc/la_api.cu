@@ -182,7 +182,11 @@ la_status kv_summary_impl(const Problem& p, const void* k, const void* v, float*
         return cuda_status(tc_noncausal_fused(p, nullptr, k, v, nullptr, S, z, at<uint32_t>(ws, 0), st));
     if (tc_supported(p)) return cuda_status(tc_kv_summary(p, k, v, part, S, z, at<uint32_t>(ws, 0), st));
     const SplitPlan sp = kv_plan(p);
-    LA_TRY(cuda_status(simt_kv_partial(p, k, v, sp.tps, sp.nsplit, part, st)));
+    if (tc_f32_supported(p)) {
+        LA_TRY(cuda_status(tc_f32_states(p, k, v, sp.tps, sp.nsplit, part, at<uint32_t>(ws, 0), st)));
+    } else {
+        LA_TRY(cuda_status(simt_kv_partial(p, k, v, sp.tps, sp.nsplit, part, st)));
+    }
     return cuda_status(state_reduce(p, part, sp.nsplit, S, z, st));
 }
 
@@ -265,6 +269,10 @@ la_status la_noncausal(const la_desc* desc, const void* q, const void* k, const 
     }
     LA_TRY(kv_summary_impl(p, k, v, S, z, ws, st));
     if (tc_supported(p)) return cuda_status(tc_readout(p, q, S, z, out, at<uint32_t>(ws, 0), st));
+    if (tc_f32_supported(p)) {
+        const BlockPlan bp = block_plan(p);
+        return cuda_status(tc_f32_readout(p, q, S, z, bp.block_tokens, bp.nblk, out, at<uint32_t>(ws, 0), st));
+    }
     return cuda_status(simt_readout(p, q, S, z, out, st));
 }
 
@@ -306,6 +314,8 @@ la_status causal_impl(const la_desc* desc, int32_t chunk, const void* q, const v
     } else {
         if (tc_supported(p)) {
             LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
+        } else if (tc_f32_supported(p)) {
+            LA_TRY(cuda_status(tc_f32_states(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
         } else {
             LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
         }
@@ -314,6 +324,8 @@ la_status causal_impl(const la_desc* desc, int32_t chunk, const void* q, const v
     if (tc_supported(p))
         return cuda_status(tc_chunked(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, nullptr,
                                       nullptr, nullptr, 0, out, flags, st));
+    if (tc_f32_supported(p))
+        return cuda_status(tc_f32_chunked(p, q, k, v, part, bp.block_tokens, bp.nblk, out, flags, st));
     return cuda_status(simt_chunked(p, q, k, v, part, bp.block_tokens, bp.nblk, nullptr, nullptr,
                                     nullptr, 0, out, st));
 }
@@ -348,6 +360,8 @@ la_status backward_impl(const la_desc* desc, bool causal, const void* q, const v
         } else {
             if (tc_supported(p)) {
                 LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
+            } else if (tc_f32_supported(p)) {
+                LA_TRY(cuda_status(tc_f32_states(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
             } else {
                 LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
             }

@@ -100,6 +100,22 @@ cudaError_t tc_causal_backward_kv(const Problem& p, const void* q, const void* k
 // [BH, N, d] bf16 viewed as 3-D for TMA: 64-column x `rows` boxes, 128-byte
 // swizzle, zero fill outside the tensor.
 cudaError_t make_map(CUtensorMap* map, const void* base, int d, int N, long long bh, int rows);
+// Same, for any element type: boxes of box_cols x box_rows elements (box_cols
+// * elem_bytes = 128 for the 128-byte swizzle).
+cudaError_t make_map_box(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes, int d,
+                         int N, long long bh, int box_cols, int box_rows);
+
+// fp32 forms at d = 64 on the tensor cores with split bf16 operands (tc_f32.cu).
+bool tc_f32_supported(const Problem& p);
+// (S, z) of each block of block_tokens keys: record (bh * nblk + blk) of part.
+cudaError_t tc_f32_states(const Problem& p, const void* k, const void* v, int block_tokens, int nblk, float* part,
+                          uint32_t* err, cudaStream_t st);
+// Causal outputs of each block from its exclusive prefix record in `prefix`.
+cudaError_t tc_f32_chunked(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
+                           int block_tokens, int nblk, void* out, uint32_t* err, cudaStream_t st);
+// Non-causal outputs from each head's total S [bh][d][d] and z [bh][d].
+cudaError_t tc_f32_readout(const Problem& p, const void* q, const float* S, const float* z, int block_tokens,
+                           int nblk, void* out, uint32_t* err, cudaStream_t st);
 // The same tensor viewed as 2-D [rows = BH * N, d] for row gathers
 // (tile::gather4): 64-column x 1-row boxes, 128-byte swizzle.
 cudaError_t make_row_map(CUtensorMap* map, const void* base, int d, long long rows);

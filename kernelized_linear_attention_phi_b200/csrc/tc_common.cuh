@@ -297,6 +297,12 @@ __device__ __forceinline__ void tmem_ld16x256_x8(uint32_t taddr, uint32_t (&r)[3
           "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
+// Warp-wide: lane i receives TMEM lane (base + i), 4 columns.
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }

@@ -48,12 +48,16 @@ def test_noncausal(dt, d, N, phi, normalize):
 
 
 def _state_tol(dt, phi):
-    """Tolerance on a KV summary. relu+1 and the identity are exact in bf16
-    (relu(K) and K are bf16 values; the +1 is added exactly in fp32), so S
-    and z carry only fp32 accumulation error. elu+1 has no such split: the
-    bf16 path multiplies phi(K) rounded to bf16, and its state is held to the
-    bf16 tolerance of the outputs."""
-    return TOL[DT[dt]] if (phi == "elu1" and dt == "bf16") else 1e-5
+    """Tolerance on a KV summary. bf16 inputs: relu+1 and the identity are
+    exact in bf16 (relu(K) and K are bf16 values; the +1 is added exactly in
+    fp32), so S and z carry only fp32 accumulation error; elu+1 has no such
+    split (phi(K) is rounded to bf16) and is held to the bf16 output
+    tolerance. fp32 inputs: the fp32 bar on every result, 1e-4 (the tensor-core
+    path forms each product from two-part bf16 splits of its fp32 operands,
+    within about 3 * 2^-16 of exact, so S carries about 1e-5)."""
+    if dt == "f32":
+        return TOL[DT[dt]]
+    return TOL[DT[dt]] if phi == "elu1" else 1e-5
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
@@ -63,7 +67,7 @@ def test_kv_summary(dt, d, N):
     _, k, v = qkv(1, 2, N, d, dt, seed=7 * N + d)
     S, z = la.la_kv_summary(k, v)
     S_ref, z_ref = oracle.kv_summary_batched(f64(k), f64(v))
-    assert oracle.max_row_rel_err(f64(S), S_ref) < 1e-5
+    assert oracle.max_row_rel_err(f64(S), S_ref) < _state_tol(dt, "relu1")
     np.testing.assert_allclose(f64(z), z_ref, rtol=1e-5)
 
 
@@ -157,7 +161,7 @@ def test_decode_from_prefill(dt, d):
             ref[b, h] = oracle.causal(Q[b, h, N0:], K[b, h, N0:], V[b, h, N0:], S0=S0, z0=z0)[0]
     assert oracle.max_row_rel_err(f64(got), ref) < TOL[DT[dt]]
     S_ref, z_ref = oracle.kv_summary_batched(K, V)
-    assert oracle.max_row_rel_err(f64(S), S_ref) < 1e-5
+    assert oracle.max_row_rel_err(f64(S), S_ref) < _state_tol(dt, "relu1")
 
 
 def test_decode_from_empty_cache_equals_causal():

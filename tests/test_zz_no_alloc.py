@@ -26,9 +26,12 @@ def _built():
     la.lib()
 
 
-# S and z are fp32 sums; bf16 elu+1 rounds phi(K) before the products, the
-# other maps are exact to fp32 accumulation (the library's KV-summary tolerance)
+# S and z are fp32 sums. bf16 inputs with relu+1: exact features, so only
+# fp32 accumulation error. fp32 inputs: S is formed on the tensor cores from
+# two-part bf16 splits of the fp32 operands (about 1e-5) and is held to the
+# fp32 bar of 1e-4; z is summed in fp32 on the CUDA cores.
 TOL = 1e-5
+TOL_S = {"bf16": 1e-5, "f32": 1e-4}
 
 
 @pytest.mark.parametrize("dtype,d", [("bf16", 64), ("bf16", 128), ("f32", 64)])
@@ -50,7 +53,7 @@ def test_static_scratch_matches_workspace_entry_point_and_oracle(dtype, d):
         assert oracle.max_row_rel_err(f64(S), f64(S_ref)) < TOL
         assert oracle.max_row_rel_err(f64(z)[..., None, :], f64(z_ref)[..., None, :]) < TOL
         S_o, z_o = oracle.kv_summary_batched(f64(k), f64(v))
-        assert oracle.max_row_rel_err(f64(S), S_o) < TOL
+        assert oracle.max_row_rel_err(f64(S), S_o) < TOL_S[dtype]
         assert oracle.max_row_rel_err(f64(z)[..., None, :], z_o[..., None, :]) < TOL
 
 
