@@ -19,14 +19,15 @@ constexpr int kTileTokens = 128;
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 inline long long round_up(long long x, long long a) { return (x + a - 1) / a * a; }
 
-// Split of the CUDA-core KV summary: nsplit splits per head of tps tokens
-// each (a multiple of 128; the last split may be shorter), about two CTAs
-// per SM in all.
+// Split of the KV summary that is not balanced across heads (CUDA cores,
+// fp32 tensor cores): nsplit splits per head of tps tokens each (a multiple
+// of 128; the last split may be shorter), at most two CTAs per SM in all
+// (one wave of two-per-SM kernels) unless the heads alone are more.
 struct SplitPlan {
     int nsplit, tps;
 };
 inline SplitPlan kv_plan(const Problem& p, int sms) {
-    const long long target = std::max(1LL, cdiv(2LL * sms, p.bh()));
+    const long long target = std::max(1LL, 2LL * sms / p.bh());
     const long long max_splits = std::max(1LL, cdiv(p.N, 256));
     long long ns = std::min(target, max_splits);
     const long long tps = round_up(cdiv(p.N, ns), 128);

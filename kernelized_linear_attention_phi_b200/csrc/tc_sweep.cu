@@ -14,16 +14,18 @@ using namespace tc;
 // Chunked causal / prefix-mask outputs of one block
 // ---------------------------------------------------------------------------
 // The block's chunks are swept in order with the running state of all
-// earlier keys kept in TMEM: S (fp32, M = d_k rows) and z (fp32, every column
-// of a 16-column block equal to z), both seeded from the block's prefix
-// record. For chunk c (C keys) and each tile of up to C queries answered
-// there:
-//   S_prev, z_prev -> bf16 operands (z as hi + lo rows)      [prep warps]
-//   S += phi(K_c)^T V_c ;  z += phi(K_c)^T 1                   [MMA]
+// earlier keys: S in TMEM (fp32, M = d_k rows) and z in the prep warps'
+// registers (fp32, one entry per thread), both seeded from the block's
+// prefix record. For chunk c (C keys) and each tile of up to C queries
+// answered there:
+//   [S_prev | z_prev] -> bf16 operand, N = d + 16: S_prev, then a swizzle
+//      atom whose columns 0, 1 hold z_prev as hi + lo parts     [prep warps]
+//   z += column sums of phi(K_c) (fp32, CUDA cores)            [prep warps]
+//   S += phi(K_c)^T V_c                                        [MMA]
 //   P  = phi(Q) phi(K_c)^T                                     [MMA, M = C]
 //   P~ = P with keys j > lim_i zeroed, bf16; den_i = rowsum   [mask warps]
-//   O  = phi(Q) S_prev + P~ V_c ; den_i += phi(Q) z_prev       [MMA]
-//   out_i = O_i / den_i                                        [mask warps]
+//   [O | Oz] = phi(Q) [S_prev | z_prev] ; O += P~ V_c          [MMA]
+//   out_i = O_i / (den_i + Oz_i)                               [mask warps]
 // Causal: the queries of chunk c are its own tokens, lim_i = i - cC.
 // Prefix mask: the queries of bin c (floor((m_i+1)/C) = c) are gathered
 // rows, lim_i = m_i - cC in [-1, C-2].
@@ -47,25 +49,25 @@ struct SwCfg {
     static constexpr int STAGES = 2;
     static constexpr int STAGE = NT * TILE;
     static constexpr int PT = C * C * 2;             // P~, K-major (x2)
-    static constexpr int B3 = D * D * 2;             // S_prev, MN-major (x2)
-    static constexpr int BZ = 16 * D * 2;            // z_hi, z_lo, 14 zero rows; K-major (x2)
-    static constexpr int ONES = 16 * C * 2;          // all-ones B operand, 16 x C, K-major
+    static constexpr int ATOM = D * D * 2;           // one [d x 64] bf16 swizzle atom (d = 64)
+    static constexpr int B3 = 2 * ATOM;              // [S_prev | z_prev], MN-major, N = d + 16 (x2)
+    static constexpr int RED = 2 * 4 * D * 4;        // z column-sum partials [parity][warp][d]
     static constexpr int QG = GATHER ? 2 * TILE : 0; // gathered queries (x2)
     static constexpr int ROWS = GATHER ? 2 * 2 * C * 4 : 0;  // token / limit per row (x2)
     static constexpr int STG = TILE;                 // output staging tile
-    // TMEM columns: S, z, then P, O, Oz (two slots each; see above)
+    // TMEM columns: S, then P and O (two slots each; see above). O has
+    // d + 16 columns: the outputs, then phi(Q).z_prev hi and lo in d, d + 1.
     static constexpr int SLOTC = C == 64 ? 1 : 2;    // column copies per slot pair
-    static constexpr int COL_S = 0, COL_Z = D, COL_P = D + 16, COL_O = COL_P + SLOTC * C,
-                         COL_OZ = COL_O + SLOTC * D, COL_END = COL_OZ + SLOTC * 16;
+    static constexpr int OW = D + 16;
+    static constexpr int COL_S = 0, COL_P = D, COL_O = COL_P + SLOTC * C, COL_END = COL_O + SLOTC * OW;
     static constexpr uint32_t TMEM_COLS = COL_END <= 256 ? 256u : 512u;
     static_assert(COL_END <= 512, "TMEM");
     static constexpr int NBAR = 2 * STAGES + 2 + 6 * 2;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 2 * PT + 2 * B3 + 2 * BZ + ONES + QG +
-                                   STG + ROWS + 8 * NBAR + 16;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 2 * PT + 2 * B3 + QG + STG + ROWS + RED +
+                                   8 * NBAR + 16;
     // TMEM address offsets of slot j for P, O and Oz
     __device__ static constexpr uint32_t p_slot(int j) { return C == 64 ? (uint32_t)j * (16u << 16) : (uint32_t)j * C; }
-    __device__ static constexpr uint32_t o_slot(int j) { return C == 64 ? (uint32_t)j * (16u << 16) : (uint32_t)j * D; }
-    __device__ static constexpr uint32_t oz_slot(int j) { return C == 64 ? (uint32_t)j * (16u << 16) : (uint32_t)j * 16; }
+    __device__ static constexpr uint32_t o_slot(int j) { return C == 64 ? (uint32_t)j * (16u << 16) : (uint32_t)j * OW; }
     static constexpr int THREADS = 320;
     static constexpr int MIN_BLOCKS = (D == 64 && C == 64) ? 2 : 1;
     static_assert(C == 64 || C == 128, "chunk");
@@ -87,12 +89,11 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     uint8_t* stages = align1024(smem_raw);
     uint8_t* pt = stages + CF::STAGES * CF::STAGE;
     uint8_t* b3 = pt + 2 * CF::PT;
-    uint8_t* bz = b3 + 2 * CF::B3;
-    uint8_t* ones = bz + 2 * CF::BZ;
-    uint8_t* qg = ones + CF::ONES;
+    uint8_t* qg = b3 + 2 * CF::B3;
     uint8_t* stg = qg + CF::QG;
     int* rows = reinterpret_cast<int*>(stg + CF::STG);  // [slot][srow C | slim C]
-    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(rows) + CF::ROWS);
+    float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(rows) + CF::ROWS);
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + CF::RED);
     uint64_t* empty = full + CF::STAGES;
     uint64_t* bprep = empty + CF::STAGES;
     uint64_t* bsdone = bprep + 1;
@@ -229,13 +230,13 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            constexpr uint32_t id1 = idesc_bf16(C, C, false, false);   // P = Q K^T
-            constexpr uint32_t id3 = idesc_bf16(C, D, false, true);    // O = Q S
-            constexpr uint32_t idz = idesc_bf16(C, 16, false, false);  // Oz = Q [z]
-            constexpr uint32_t id2 = idesc_bf16(C, D, false, true);    // O += P~ V
-            constexpr uint32_t id4 = idesc_bf16(D, D, true, true);     // S += K^T V
-            constexpr uint32_t id5 = idesc_bf16(D, 16, true, false);   // Z += K^T 1
-            const uint32_t pta = smem_u32(pt), onesa = smem_u32(ones);
+            constexpr uint32_t id1 = idesc_bf16(C, C, false, false);       // P = Q K^T
+            constexpr uint32_t id2 = idesc_bf16(C, D, false, true);        // O += P~ V
+            constexpr uint32_t id4 = idesc_bf16(D, D, true, true);         // S += K^T V
+            // [O | Oz] = Q [S | z]: the state operand spans two swizzle atoms
+            // along N (the z atom second); unnormalized, O = Q S alone
+            const uint32_t id3 = normalize ? idesc_bf16(C, D + 16, false, true) : idesc_bf16(C, D, false, true);
+            const uint32_t pta = smem_u32(pt);
             int tq = 0;
             bool ok = true;
             for (int ci = 0; ci < nci && ok; ++ci) {
@@ -247,16 +248,11 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk) {
-                    const uint64_t a = sdesc(kt + kk * 2048, C * 128, 1024);
-                    mma_bf16(tmem + CF::COL_S, a, sdesc(vt + kk * 2048, C * 128, 1024), id4, 1u);
-                    if (normalize)
-                        mma_bf16(tmem + CF::COL_Z, a, sdesc(onesa + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024),
-                                 id5, 1u);
-                }
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_bf16(tmem + CF::COL_S, sdesc(kt + kk * 2048, C * 128, 1024),
+                             sdesc(vt + kk * 2048, C * 128, 1024), id4, 1u);
                 mma_commit(bsdone);
                 const uint32_t b3a = smem_u32(b3 + (ci & 1) * CF::B3);
-                const uint32_t bza = smem_u32(bz + (ci & 1) * CF::BZ);
                 const int ntq = q_tiles(c_begin + ci);
                 for (int t = 0; t < ntq && ok; ++t, ++tq) {
                     const int j = tq & 1, k = tq >> 1;  // slot, use of the slot
@@ -278,11 +274,8 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t a = sdesc(qt + (kk / 4) * (C * 128) + (kk % 4) * 32, 16, 1024);
-                        mma_bf16(tmem + CF::COL_O + CF::o_slot(j), a, sdesc(b3a + kk * 2048, D * 128, 1024), id3,
+                        mma_bf16(tmem + CF::COL_O + CF::o_slot(j), a, sdesc(b3a + kk * 2048, CF::ATOM, 1024), id3,
                                  kk > 0);
-                        if (normalize)
-                            mma_bf16(tmem + CF::COL_OZ + CF::oz_slot(j), a,
-                                     sdesc(bza + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024), idz, kk > 0);
                     }
                     ok = mbar_wait(bptready + j, k & 1, err);
                     if (!ok) break;
@@ -304,16 +297,17 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
         constexpr int RS = D == 128 ? 32 : 16;  // S rows per sub-partition
         const float* pre = prefix + ((size_t)bh * nblk + blk) * (size_t)(D * D + D);
+        // z_prev entry d_k = et (threads et < D), seeded from the prefix
+        float zp = (normalize && et < D) ? pre[(size_t)D * D + et] : 0.f;
+        // column group (of 8) of the K tiles this thread transforms: the
+        // 128-byte swizzle maps 16-byte chunk (et & 7) of its rows (all with
+        // the same row & 7) to logical columns 8 * g .. 8 * g + 7
+        const int zg = (et & 7) ^ ((et >> 3) & 7);
         {
-            const uint4 one8 = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-            for (int c = et; c < CF::ONES / 16; c += 128) reinterpret_cast<uint4*>(ones)[c] = one8;
-            for (int c = et; c < 2 * 16 * D / 8; c += 128) {  // z operand rows 2..15 stay zero
-                const int buf = c / (16 * D / 8), cc = c % (16 * D / 8);
-                const int n = cc / (D / 8), col = (cc % (D / 8)) * 8;
-                if (n >= 2)
-                    *reinterpret_cast<uint4*>(bz + buf * CF::BZ + (col / 64) * 2048 + sw128_off(n, col % 64)) =
-                        make_uint4(0, 0, 0, 0);
-            }
+            // the z atoms start zero (columns 2..15 stay so)
+            for (int c = et; c < 2 * CF::ATOM / 16; c += 128)
+                reinterpret_cast<uint4*>(b3 + (c / (CF::ATOM / 16)) * CF::B3 + CF::ATOM)[c % (CF::ATOM / 16)] =
+                    make_uint4(0, 0, 0, 0);
             // seed the TMEM state with the block's prefix
             const int a = sp * RS + lane;
             const bool own = lane < RS;
@@ -331,13 +325,6 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 }
                 tmem_st16(tmem + CF::COL_S + lane_base + c0, r);
             }
-            if (normalize) {
-                uint32_t r[16];
-                const uint32_t zv = own ? __float_as_uint(pre[(size_t)D * D + a]) : 0u;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) r[e] = zv;
-                tmem_st16(tmem + CF::COL_Z + lane_base, r);
-            }
             tmem_st_wait();
         }
         // No early exit in this warpgroup: after a failed wait the loops run on
@@ -350,6 +337,9 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             uint8_t* st = stages + s * CF::STAGE;
             uint4* kt = reinterpret_cast<uint4*>(st + (GATHER ? 0 : CF::TILE));
             mbar_wait(full + s, u & 1, err);
+            float cs[8];  // column sums of phi(K) over this thread's rows, group zg
+#pragma unroll
+            for (int e = 0; e < 8; ++e) cs[e] = 0.f;
             // in groups of 4 chunks, all loads of a group first: a load placed
             // after a shared store could not be moved ahead of it (aliasing)
 #pragma unroll
@@ -366,9 +356,31 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 for (int i = 0; i < 4; ++i) {
                     const int p = et + 128 * (i0 + i);
                     const int r = (p % (C * 8)) >> 3;
-                    kt[p] = r < kvalid ? (mapped ? phi8<PHI>(kx[i]) : kx[i]) : make_uint4(0, 0, 0, 0);
+                    const uint4 kn = r < kvalid ? (mapped ? phi8<PHI>(kx[i]) : kx[i]) : make_uint4(0, 0, 0, 0);
+                    kt[p] = kn;
                     if (!GATHER && mapped) qt[p] = phi8<PHI>(qx[i]);
+                    if (normalize) {
+                        float f[8];
+                        unpack8(kn, f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) cs[e] += f[e];
+                    }
                 }
+            }
+            if (normalize) {
+                // lanes l, l ^ 9, l ^ 18, l ^ 27 hold the same column group;
+                // lanes 0..7 then publish the warp's sums of all eight groups
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 9);
+                    cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 18);
+                }
+                if (lane < 8) {
+                    float4* dst = reinterpret_cast<float4*>(red + (ci & 1) * 4 * D + (warp - 2) * D + zg * 8);
+                    dst[0] = make_float4(cs[0], cs[1], cs[2], cs[3]);
+                    dst[1] = make_float4(cs[4], cs[5], cs[6], cs[7]);
+                }
+                named_bar(2, 128);
             }
             if (ci > 0) {
                 mbar_wait(bsdone, (ci - 1) & 1, err);
@@ -408,20 +420,16 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                     *reinterpret_cast<uint4*>(b3b + sw128_off(a, cb + 8 * g)) = pack8(f);
                 }
             }
-            // z_prev -> rows 0 (hi) and 1 (lo) of the z operand
-            if (normalize) {
-                uint32_t r[16];
-                tmem_ld16(tmem + CF::COL_Z + lane_base, r);
-                tmem_ld_wait();
-                if (lane < RS) {
-                    const int a = sp * RS + lane;
-                    const float zv = __uint_as_float(r[0]);
-                    const __nv_bfloat16 hi = __float2bfloat16_rn(zv);
-                    const __nv_bfloat16 lo = __float2bfloat16_rn(zv - __bfloat162float(hi));
-                    uint8_t* base = bz + (ci & 1) * CF::BZ + (a / 64) * 2048;
-                    *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(0, a % 64)) = hi;
-                    *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(1, a % 64)) = lo;
-                }
+            // z_prev -> columns 0 (hi) and 1 (lo) of row d_k of the z atom;
+            // then z += the chunk's column sums
+            if (normalize && et < D) {
+                const __nv_bfloat16 hi = __float2bfloat16_rn(zp);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(zp - __bfloat162float(hi));
+                uint8_t* za = b3b + CF::ATOM;
+                *reinterpret_cast<__nv_bfloat16*>(za + sw128_off(et, 0)) = hi;
+                *reinterpret_cast<__nv_bfloat16*>(za + sw128_off(et, 1)) = lo;
+                const float* rp = red + (ci & 1) * 4 * D;
+                zp += (rp[et] + rp[D + et]) + (rp[2 * D + et] + rp[3 * D + et]);
             }
             fence_async_smem();
             tc_fence_before();
@@ -534,7 +542,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 // base; with 64-row chunks slot 1 sits in lanes 16..31 and is
                 // picked out below with a shuffle
                 uint32_t oz[2];
-                tmem_ld2(tmem + CF::COL_OZ + lane_base + (C == 64 ? 0u : CF::oz_slot(slot)), oz);
+                tmem_ld2(tmem + CF::COL_O + D + lane_base + (C == 64 ? 0u : CF::o_slot(slot)), oz);
                 tmem_ld_wait();
                 tc_fence_before();
                 // gathered rows: this thread's copy-out rows, read before the

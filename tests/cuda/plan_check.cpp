@@ -35,6 +35,9 @@ static void check_split(const Problem& p, int sms) {
     // the splits cover [0, N) and none is empty
     EXPECT((long long)s.nsplit * s.tps >= p.N && (long long)(s.nsplit - 1) * s.tps < p.N,
            "kv_plan cover N=%d nsplit=%d tps=%d sms=%d", p.N, s.nsplit, s.tps, sms);
+    // one wave at two CTAs per SM, unless the heads alone are more
+    EXPECT((long long)s.nsplit * p.bh() <= 2LL * sms || s.nsplit == 1, "kv_plan wave nsplit=%d bh=%lld sms=%d",
+           s.nsplit, p.bh(), sms);
 }
 
 static void check_blocks(const Problem& p, int sms) {
