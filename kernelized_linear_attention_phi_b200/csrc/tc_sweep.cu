@@ -18,13 +18,12 @@ using namespace tc;
 // registers (fp32, one entry per thread), both seeded from the block's
 // prefix record. For chunk c (C keys) and each tile of up to C queries
 // answered there:
-//   [S_prev | z_prev] -> bf16 operand, N = d + 16: S_prev, then a swizzle
-//      atom whose columns 0, 1 hold z_prev as hi + lo parts     [prep warps]
+//   S_prev, z_prev -> bf16 operands (z as hi + lo rows)      [prep warps]
 //   z += column sums of phi(K_c) (fp32, CUDA cores)            [prep warps]
 //   S += phi(K_c)^T V_c                                        [MMA]
 //   P  = phi(Q) phi(K_c)^T                                     [MMA, M = C]
 //   P~ = P with keys j > lim_i zeroed, bf16; den_i = rowsum   [mask warps]
-//   [O | Oz] = phi(Q) [S_prev | z_prev] ; O += P~ V_c          [MMA]
+//   O  = phi(Q) S_prev + P~ V_c ; Oz = phi(Q) z_prev           [MMA]
 //   out_i = O_i / (den_i + Oz_i)                               [mask warps]
 // Causal: the queries of chunk c are its own tokens, lim_i = i - cC.
 // Prefix mask: the queries of bin c (floor((m_i+1)/C) = c) are gathered
@@ -35,7 +34,9 @@ using namespace tc;
 // row map of Q, and the tile's row table), warp 1 MMA + TMEM, warps 2-5
 // "prep" (phi on the K / Q tiles, state -> operands), warps 6-9 "mask" (P~,
 // epilogue). Prep runs one chunk ahead of mask; the S / z operands are
-// double-buffered, the gathered query tiles too. The per-tile accumulators
+// double-buffered. Gathered query tiles sit in a ring of QS slots of their
+// own, so that each tile's gather (scattered rows, the longest load of the
+// kernel) is issued QS - 1 tiles before its use. The per-tile accumulators
 // (P, O, Oz) and the P~ operand are double-buffered by tile parity ("slot"),
 // so the tensor core starts tile t+1 while the mask warps finish tile t: with
 // 64-row chunks (M = 64 accumulators, which use TMEM lanes 0..15 of each
@@ -49,25 +50,26 @@ struct SwCfg {
     static constexpr int STAGES = 2;
     static constexpr int STAGE = NT * TILE;
     static constexpr int PT = C * C * 2;             // P~, K-major (x2)
-    static constexpr int ATOM = D * D * 2;           // one [d x 64] bf16 swizzle atom (d = 64)
-    static constexpr int B3 = 2 * ATOM;              // [S_prev | z_prev], MN-major, N = d + 16 (x2)
+    static constexpr int B3 = D * D * 2;             // S_prev, MN-major (x2)
+    static constexpr int BZ = 16 * D * 2;            // z_hi, z_lo, 14 zero rows; K-major (x2)
     static constexpr int RED = 2 * 4 * D * 4;        // z column-sum partials [parity][warp][d]
-    static constexpr int QG = GATHER ? 2 * TILE : 0; // gathered queries (x2)
-    static constexpr int ROWS = GATHER ? 2 * 2 * C * 4 : 0;  // token / limit per row (x2)
+    static constexpr int QS = GATHER ? 3 : 1;        // gathered query slots
+    static constexpr int QG = GATHER ? QS * TILE : 0;
+    static constexpr int ROWS = GATHER ? QS * 2 * C * 4 : 0;  // token / limit per row, per query slot
     static constexpr int STG = TILE;                 // output staging tile
-    // TMEM columns: S, then P and O (two slots each; see above). O has
-    // d + 16 columns: the outputs, then phi(Q).z_prev hi and lo in d, d + 1.
+    // TMEM columns: S, then P, O, Oz (two slots each; see above)
     static constexpr int SLOTC = C == 64 ? 1 : 2;    // column copies per slot pair
-    static constexpr int OW = D + 16;
-    static constexpr int COL_S = 0, COL_P = D, COL_O = COL_P + SLOTC * C, COL_END = COL_O + SLOTC * OW;
+    static constexpr int COL_S = 0, COL_P = D, COL_O = COL_P + SLOTC * C, COL_OZ = COL_O + SLOTC * D,
+                         COL_END = COL_OZ + SLOTC * 16;
     static constexpr uint32_t TMEM_COLS = COL_END <= 256 ? 256u : 512u;
     static_assert(COL_END <= 512, "TMEM");
-    static constexpr int NBAR = 2 * STAGES + 2 + 6 * 2;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 2 * PT + 2 * B3 + QG + STG + ROWS + RED +
-                                   8 * NBAR + 16;
+    static constexpr int NBAR = 2 * STAGES + 2 + 4 * 2 + 3 * QS;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 2 * PT + 2 * B3 + 2 * BZ + QG + STG + ROWS +
+                                   RED + 8 * NBAR + 16;
     // TMEM address offsets of slot j for P, O and Oz
     __device__ static constexpr uint32_t p_slot(int j) { return C == 64 ? (uint32_t)j * (16u << 16) : (uint32_t)j * C; }
-    __device__ static constexpr uint32_t o_slot(int j) { return C == 64 ? (uint32_t)j * (16u << 16) : (uint32_t)j * OW; }
+    __device__ static constexpr uint32_t o_slot(int j) { return C == 64 ? (uint32_t)j * (16u << 16) : (uint32_t)j * D; }
+    __device__ static constexpr uint32_t oz_slot(int j) { return C == 64 ? (uint32_t)j * (16u << 16) : (uint32_t)j * 16; }
     static constexpr int THREADS = 320;
     static constexpr int MIN_BLOCKS = (D == 64 && C == 64) ? 2 : 1;
     static_assert(C == 64 || C == 128, "chunk");
@@ -89,9 +91,10 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     uint8_t* stages = align1024(smem_raw);
     uint8_t* pt = stages + CF::STAGES * CF::STAGE;
     uint8_t* b3 = pt + 2 * CF::PT;
-    uint8_t* qg = b3 + 2 * CF::B3;
+    uint8_t* bz = b3 + 2 * CF::B3;
+    uint8_t* qg = bz + 2 * CF::BZ;
     uint8_t* stg = qg + CF::QG;
-    int* rows = reinterpret_cast<int*>(stg + CF::STG);  // [slot][srow C | slim C]
+    int* rows = reinterpret_cast<int*>(stg + CF::STG);  // [query slot][srow C | slim C]
     float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(rows) + CF::ROWS);
     uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + CF::RED);
     uint64_t* empty = full + CF::STAGES;
@@ -99,15 +102,17 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     uint64_t* bsdone = bprep + 1;
     // Per-tile barriers are kept per slot (tile t uses slot t % 2, phase t / 2),
     // so that no waiter is ever two phases behind its barrier (parity waits
-    // would alias): P ready, P~ written (P read), O ready, O read, queries
-    // transformed, and (prefix mask) query rows landed with their row table.
+    // would alias): P ready, P~ written (P read), O ready, O read. Gathered
+    // query tiles, per query slot (tile t uses t % QS, phase t / QS): rows
+    // landed with their row table, queries transformed, slot read out.
     uint64_t* bpfull = bsdone + 1;     // [2]
     uint64_t* bptready = bpfull + 2;   // [2]
     uint64_t* bofull = bptready + 2;   // [2]
     uint64_t* bofree = bofull + 2;     // [2]
-    uint64_t* bqready = bofree + 2;    // [2]
-    uint64_t* qfull = bqready + 2;     // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qfull + 2);
+    uint64_t* qfull = bofree + 2;      // [QS]
+    uint64_t* bqready = qfull + CF::QS;  // [QS]
+    uint64_t* qfree = bqready + CF::QS;  // [QS]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qfree + CF::QS);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int blk = blockIdx.x;
@@ -139,8 +144,11 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             mbar_init(bptready + j, 128);
             mbar_init(bofull + j, 1);
             mbar_init(bofree + j, 128);
-            mbar_init(bqready + j, 128);
+        }
+        for (int j = 0; j < CF::QS; ++j) {
             mbar_init(qfull + j, 1);
+            mbar_init(bqready + j, 128);
+            mbar_init(qfree + j, 128);
         }
         fence_mbar_init();
     }
@@ -197,7 +205,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 const int qend = bin_start[(size_t)b * (nbins + 1) + c + 1];
                 for (int t = 0; qbase + t * C < qend; ++t, ++tq) {
                     constexpr int R = C / 32;  // rows of the tile per lane
-                    const int slot = tq & 1;
+                    const int slot = tq % CF::QS, use = tq / CF::QS;
                     int tok[R], lim[R];
 #pragma unroll
                     for (int e = 0; e < R; ++e) {
@@ -206,7 +214,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                         lim[e] = idx < qend ? msort[(size_t)b * N + idx] - c * C : -1;
                     }
                     // the slot's previous tile has been read out (and its row table with it)
-                    if (tq >= 2) ok = __all_sync(0xffffffffu, mbar_wait(bofree + slot, ((tq >> 1) - 1) & 1, err));
+                    if (use > 0) ok = __all_sync(0xffffffffu, mbar_wait(qfree + slot, (use - 1) & 1, err));
                     if (!ok) break;
                     int* srow = rows + slot * 2 * C;
 #pragma unroll
@@ -225,17 +233,17 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         if (lane == 0) {
             for (int c2 = max(0, nld - CF::STAGES); c2 < nld; ++c2)
                 mbar_wait(full + c2 % CF::STAGES, (c2 / CF::STAGES) & 1, err, false);
-            for (int t2 = max(0, tq - 2); t2 < tq; ++t2) mbar_wait(qfull + (t2 & 1), (t2 >> 1) & 1, err, false);
+            for (int t2 = max(0, tq - CF::QS); t2 < tq; ++t2)
+                mbar_wait(qfull + t2 % CF::QS, (t2 / CF::QS) & 1, err, false);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            constexpr uint32_t id1 = idesc_bf16(C, C, false, false);       // P = Q K^T
-            constexpr uint32_t id2 = idesc_bf16(C, D, false, true);        // O += P~ V
-            constexpr uint32_t id4 = idesc_bf16(D, D, true, true);         // S += K^T V
-            // [O | Oz] = Q [S | z]: the state operand spans two swizzle atoms
-            // along N (the z atom second); unnormalized, O = Q S alone
-            const uint32_t id3 = normalize ? idesc_bf16(C, D + 16, false, true) : idesc_bf16(C, D, false, true);
+            constexpr uint32_t id1 = idesc_bf16(C, C, false, false);   // P = Q K^T
+            constexpr uint32_t id3 = idesc_bf16(C, D, false, true);    // O = Q S
+            constexpr uint32_t idz = idesc_bf16(C, 16, false, false);  // Oz = Q [z]
+            constexpr uint32_t id2 = idesc_bf16(C, D, false, true);    // O += P~ V
+            constexpr uint32_t id4 = idesc_bf16(D, D, true, true);     // S += K^T V
             const uint32_t pta = smem_u32(pt);
             int tq = 0;
             bool ok = true;
@@ -253,11 +261,13 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                              sdesc(vt + kk * 2048, C * 128, 1024), id4, 1u);
                 mma_commit(bsdone);
                 const uint32_t b3a = smem_u32(b3 + (ci & 1) * CF::B3);
+                const uint32_t bza = smem_u32(bz + (ci & 1) * CF::BZ);
                 const int ntq = q_tiles(c_begin + ci);
                 for (int t = 0; t < ntq && ok; ++t, ++tq) {
                     const int j = tq & 1, k = tq >> 1;  // slot, use of the slot
-                    const uint32_t qt = GATHER ? smem_u32(qg + j * CF::TILE) : st;
-                    if (GATHER) ok = mbar_wait(bqready + j, k & 1, err);
+                    const int qs = tq % CF::QS;  // query slot (gathered tiles)
+                    const uint32_t qt = GATHER ? smem_u32(qg + qs * CF::TILE) : st;
+                    if (GATHER) ok = mbar_wait(bqready + qs, (tq / CF::QS) & 1, err);
                     if (ok && k > 0) ok = mbar_wait(bptready + j, (k - 1) & 1, err);  // P[j] read two tiles ago
                     if (!ok) break;
                     tc_fence_after();
@@ -274,8 +284,11 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t a = sdesc(qt + (kk / 4) * (C * 128) + (kk % 4) * 32, 16, 1024);
-                        mma_bf16(tmem + CF::COL_O + CF::o_slot(j), a, sdesc(b3a + kk * 2048, CF::ATOM, 1024), id3,
+                        mma_bf16(tmem + CF::COL_O + CF::o_slot(j), a, sdesc(b3a + kk * 2048, D * 128, 1024), id3,
                                  kk > 0);
+                        if (normalize)
+                            mma_bf16(tmem + CF::COL_OZ + CF::oz_slot(j), a,
+                                     sdesc(bza + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024), idz, kk > 0);
                     }
                     ok = mbar_wait(bptready + j, k & 1, err);
                     if (!ok) break;
@@ -304,10 +317,9 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         // the same row & 7) to logical columns 8 * g .. 8 * g + 7
         const int zg = (et & 7) ^ ((et >> 3) & 7);
         {
-            // the z atoms start zero (columns 2..15 stay so)
-            for (int c = et; c < 2 * CF::ATOM / 16; c += 128)
-                reinterpret_cast<uint4*>(b3 + (c / (CF::ATOM / 16)) * CF::B3 + CF::ATOM)[c % (CF::ATOM / 16)] =
-                    make_uint4(0, 0, 0, 0);
+            // z operand rows 2..15 stay zero (both buffers; rows of 128 bytes)
+            for (int c = et; c < 2 * 14 * 8; c += 128)
+                reinterpret_cast<uint4*>(bz + (c / 112) * CF::BZ + 2 * 128)[c % 112] = make_uint4(0, 0, 0, 0);
             // seed the TMEM state with the block's prefix
             const int a = sp * RS + lane;
             const bool own = lane < RS;
@@ -420,14 +432,14 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                     *reinterpret_cast<uint4*>(b3b + sw128_off(a, cb + 8 * g)) = pack8(f);
                 }
             }
-            // z_prev -> columns 0 (hi) and 1 (lo) of row d_k of the z atom;
+            // z_prev -> rows 0 (hi) and 1 (lo) of the z operand (column d_k);
             // then z += the chunk's column sums
             if (normalize && et < D) {
                 const __nv_bfloat16 hi = __float2bfloat16_rn(zp);
                 const __nv_bfloat16 lo = __float2bfloat16_rn(zp - __bfloat162float(hi));
-                uint8_t* za = b3b + CF::ATOM;
-                *reinterpret_cast<__nv_bfloat16*>(za + sw128_off(et, 0)) = hi;
-                *reinterpret_cast<__nv_bfloat16*>(za + sw128_off(et, 1)) = lo;
+                uint8_t* zb = bz + (ci & 1) * CF::BZ;
+                *reinterpret_cast<__nv_bfloat16*>(zb + sw128_off(0, et)) = hi;
+                *reinterpret_cast<__nv_bfloat16*>(zb + sw128_off(1, et)) = lo;
                 const float* rp = red + (ci & 1) * 4 * D;
                 zp += (rp[et] + rp[D + et]) + (rp[2 * D + et] + rp[3 * D + et]);
             }
@@ -439,8 +451,8 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 // the gathered query rows of the chunk's tiles: phi in place
                 const int ntq = q_tiles(c);
                 for (int t = 0; t < ntq; ++t, ++tq) {
-                    const int slot = tq & 1;
-                    mbar_wait(qfull + slot, (tq >> 1) & 1, err);
+                    const int slot = tq % CF::QS;
+                    mbar_wait(qfull + slot, (tq / CF::QS) & 1, err);
                     if (mapped) {
                         constexpr int NL = C * D / 8 / 128;
                         uint4* q = reinterpret_cast<uint4*>(qg + slot * CF::TILE);
@@ -477,9 +489,10 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 uint8_t* pts = pt + slot * CF::PT;
                 ok = mbar_wait(bpfull + slot, use & 1, err) && ok;
                 // the row table of a gathered tile (written by the TMA warp)
-                if (GATHER) ok = mbar_wait(qfull + slot, use & 1, err) && ok;
+                const int qs = tq % CF::QS;
+                if (GATHER) ok = mbar_wait(qfull + qs, (tq / CF::QS) & 1, err) && ok;
                 tc_fence_after();
-                const int* srow = rows + slot * 2 * C;
+                const int* srow = rows + qs * 2 * C;
                 const int lim = GATHER ? srow[C + i] : i;
                 const int tok = GATHER ? srow[i] : (i < kvalid ? c * C + i : -1);
                 float rs = 0.f;
@@ -542,7 +555,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                 // base; with 64-row chunks slot 1 sits in lanes 16..31 and is
                 // picked out below with a shuffle
                 uint32_t oz[2];
-                tmem_ld2(tmem + CF::COL_O + D + lane_base + (C == 64 ? 0u : CF::o_slot(slot)), oz);
+                tmem_ld2(tmem + CF::COL_OZ + lane_base + (C == 64 ? 0u : CF::oz_slot(slot)), oz);
                 tmem_ld_wait();
                 tc_fence_before();
                 // gathered rows: this thread's copy-out rows, read before the
@@ -554,6 +567,7 @@ tc_sweep_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
                     for (int j = 0; j < NC; ++j) dst_row[j] = srow[(threadIdx.x - 192 + 128 * j) / (D / 8)];
                 }
                 mbar_arrive(bofree + slot);
+                if (GATHER) mbar_arrive(qfree + qs);  // the query slot and its row table are read
                 float den = rs + __uint_as_float(oz[0]) + __uint_as_float(oz[1]);
                 if (C == 64) den = __shfl_sync(0xffffffffu, den, (lane & 15) + 16 * slot);
                 const float inv = normalize ? __frcp_rn(den) : 1.0f;
