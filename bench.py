@@ -29,7 +29,10 @@ steps in one graph) and the graphs are replayed. Timing: CUDA events around
 every call on the launching stream, L2 flushed (a 256 MiB write) before
 every call outside the events, W untimed warm-up steps, max over ranks.
 ``e2e`` repeats the step through the plain API calls with pinned host inputs
-copied in and the outputs copied back inside the timed region.
+copied in and the outputs copied back inside the timed region, the copies of
+one step overlapped with the calls of the previous (separate copy streams,
+double-buffered device tensors); ``e2e.serial_value`` runs every copy and
+call of a step back to back.
 ``roofline`` is the dominant kernel's: after the timed steps every call is
 replayed from a graph captured with the library's per-kernel timing events
 (la_timing_enable), L2 flushed before each replay, and the kernel with the
@@ -353,6 +356,19 @@ class Call:
         outs = list(self.grads) if self.form.endswith("_bwd") else [self.out]
         return ins, outs
 
+    def bind_io(self, ins, outs):
+        """Point the call at other device tensors of the same shapes (the
+        order of device_io)."""
+        self.q, self.k, self.v = ins[:3]
+        rest = ins[3:]
+        if self.form == "prefix":
+            self.m, rest = rest[0], rest[1:]
+        if self.form.endswith("_bwd"):
+            self.dout = rest[0]
+            self.grads = tuple(outs)
+        else:
+            self.out = outs[0]
+
     def algorithmic_bytes(self):
         """Bytes the call must move at least: its inputs once and outputs once."""
         t = self.B * self.H * self.N * self.d * self.elem     # one [B,H,N,d] tensor
@@ -375,6 +391,56 @@ class Call:
             if nblk >= 2:
                 kb = kb * min(self.N, (nblk - 1) * bt) // self.N
         return kb
+
+
+def e2e_pipelined(calls, h_io, steps, stream):
+    """Seconds for `steps` steps through the public API with every step's
+    inputs copied in from pinned host memory and its outputs copied back, the
+    copies overlapped with the calls: host-to-device copies on one stream, the
+    calls on `stream`, device-to-host copies on a third; each call's device
+    tensors are double-buffered, and a buffer is refilled only after the call
+    that read it, and emptied only after the copy that read it, are done.
+    Timed on the device from before the first copy in to after the last copy
+    out."""
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    bufs = []
+    for c in calls:
+        ins, outs = c.device_io()
+        bufs.append(([ins, [torch.empty_like(t) for t in ins]], [outs, [torch.empty_like(t) for t in outs]]))
+    ev = lambda: torch.cuda.Event()
+    done, freed = {}, {}
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(s_in)
+    for i in range(steps):
+        for j, (c, (h_ins, h_outs)) in enumerate(zip(calls, h_io)):
+            (ins, outs), b = bufs[j], i % 2
+            if i >= 2:
+                s_in.wait_event(done[j, i - 2])
+            with torch.cuda.stream(s_in):
+                for d_t, h_t in zip(ins[b], h_ins):
+                    d_t.copy_(h_t, non_blocking=True)
+            loaded = ev()
+            loaded.record(s_in)
+            stream.wait_event(loaded)
+            if i >= 2:
+                stream.wait_event(freed[j, i - 2])
+            c.bind_io(ins[b], outs[b])
+            with torch.cuda.stream(stream):
+                c.run()
+            done[j, i] = ev()
+            done[j, i].record(stream)
+            s_out.wait_event(done[j, i])
+            with torch.cuda.stream(s_out):
+                for h_t, d_t in zip(h_outs, outs[b]):
+                    h_t.copy_(d_t, non_blocking=True)
+            freed[j, i] = ev()
+            freed[j, i].record(s_out)
+    t1.record(s_out)
+    torch.cuda.synchronize()
+    for j, c in enumerate(calls):
+        c.bind_io(*[x[0] for x in bufs[j]])
+    return t0.elapsed_time(t1) / 1e3
 
 
 def kernel_bytes(form, kernel, B, H, N, d, elem):
@@ -512,6 +578,7 @@ def measure_case(case, args, rank, world, device, flush, sampler, peak, heads=0)
         d2h += sum(t.numel() * t.element_size() for t in h_outs)
         h_io.append((h_ins, h_outs))
     Ke = max(1, min(K, 20))
+    # serial: each step's copies in, calls and copies out back to back on one stream
     e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
     torch.cuda.synchronize()
     for i in range(Ke):
@@ -521,7 +588,9 @@ def measure_case(case, args, rank, world, device, flush, sampler, peak, heads=0)
             c.run_from_host(h_ins, h_outs)
         e_ev[i][1].record(stream)
     torch.cuda.synchronize()
-    e2e_s = sum(a.elapsed_time(b) for a, b in e_ev) / 1e3
+    e2e_serial_s = sum(a.elapsed_time(b) for a, b in e_ev) / 1e3
+    # pipelined: step i+1's copies in overlap step i's calls and copies out
+    e2e_s = e2e_pipelined(calls, h_io, Ke, stream) if all(c.form != "decode" for c in calls) else e2e_serial_s
     del h_io
 
     # each kernel's own duration (per-kernel timing events)
@@ -536,10 +605,11 @@ def measure_case(case, args, rank, world, device, flush, sampler, peak, heads=0)
                 bad_flags[f"{c.name}/{c.form}"] = f
 
     step_ms = sum(per_call_ms)
-    t_s, e2e_s = max_over_ranks([step_ms / 1e3 * K, e2e_s], device)
+    t_s, e2e_s, e2e_serial_s = max_over_ranks([step_ms / 1e3 * K, e2e_s, e2e_serial_s], device)
     tokens = sum(c.tokens for c in calls)
     value = aggregate_tokens_per_s(tokens, K, world, t_s)
     e2e_value = aggregate_tokens_per_s(tokens, Ke, world, e2e_s)
+    e2e_serial = aggregate_tokens_per_s(tokens, Ke, world, e2e_serial_s)
 
     per_call, cands, launches = {}, [], 0
     for c, ms, ktimes in zip(calls, per_call_ms, kt):
@@ -578,7 +648,13 @@ def measure_case(case, args, rank, world, device, flush, sampler, peak, heads=0)
                    "launch": "one CUDA graph per call" + (" (decode: 1024 steps in one graph)"
                                                           if any(c.form == "decode" for c in calls) else ""),
                    "tokens_per_step_per_gpu": tokens},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "serial_value": e2e_serial,
+                "mode": ("pipelined: copies in on one stream, the calls on another, copies out on a third, "
+                         "device tensors double-buffered, so step i+1's inputs load while step i computes and "
+                         "copies out; serial_value runs every copy and call of a step back to back"
+                         if all(c.form != "decode" for c in calls) else
+                         "per decode step: its token copied in, the step, its output copied out")},
         "gpu_launches": launches * K,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
