@@ -116,13 +116,14 @@ SIMT_KERNELS = {
     "causal_bwd": {5: ["kv_partial_kernel", "state_scan_kernel", "bwd_q_kernel", "state_scan_kernel",
                        "bwd_kv_kernel"]},
 }
-# fp32 at d = 64: the split-precision tensor-core kernel in its three modes
-# (block / split states, causal sweep, readout); the prefix mask and decode
-# stay on the CUDA cores
+# fp32 at d = 64: the split-precision tensor-core kernel in its four modes
+# (block / split states, causal sweep, readout, prefix-mask sweep); decode and
+# the gradient sweeps stay on the CUDA cores
 F32_TC_KERNELS = dict(SIMT_KERNELS)
 F32_TC_KERNELS.update({
     "noncausal": {3: ["tc_f32_kernel<0", "state_reduce_kernel", "tc_f32_kernel<2"]},
     "causal": {3: ["tc_f32_kernel<0", "state_scan_kernel", "tc_f32_kernel<1"]},
+    "prefix": {4: ["tc_f32_kernel<0", "bin_kernel", "state_scan_kernel", "tc_f32_kernel<3"]},
     "noncausal_bwd": {5: ["tc_f32_kernel<0", "state_reduce_kernel", "bwd_q_kernel", "state_reduce_kernel",
                           "bwd_kv_kernel"]},
     "causal_bwd": {5: ["tc_f32_kernel<0", "state_scan_kernel", "bwd_q_kernel", "state_scan_kernel",
@@ -137,7 +138,7 @@ KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balan
                "bwd_kv_kernel": "bwd_kv", "tc_bwd_q_kernel": "bwd_q", "tc_bwd_kv_kernel": "bwd_kv",
                "tc_bwd_causal_q_kernel": "bwd_q", "tc_bwd_causal_kv_kernel": "bwd_kv",
                "tc_noncausal_cluster_kernel": "fused", "tc_f32_kernel<0": "kv", "tc_f32_kernel<1": "sweep",
-               "tc_f32_kernel<2": "readout"}
+               "tc_f32_kernel<2": "readout", "tc_f32_kernel<3": "sweep"}
 
 
 def block_plan(B, H, N, d, dtype, sms):

@@ -461,6 +461,8 @@ la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, cons
         LA_TRY(cuda_status(tc_kv_blocks_scan(p, k, v, bp.block_tokens, bp.nblk, part, nullptr, nullptr, flags, st)));
     } else if (tc) {
         LA_TRY(cuda_status(tc_kv_blocks(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
+    } else if (tc_f32_supported(p)) {
+        LA_TRY(cuda_status(tc_f32_states(p, k, v, bp.block_tokens, bp.nblk, part, flags, st)));
     } else {
         LA_TRY(cuda_status(simt_kv_partial(p, k, v, bp.block_tokens, bp.nblk, part, st)));
     }
@@ -469,6 +471,9 @@ la_status la_prefix_mask(const la_desc* desc, int32_t chunk, const void* q, cons
     if (tc)
         return cuda_status(tc_chunked(p, chunk, q, k, v, part, bp.block_tokens, bp.nblk, perm, bins,
                                       msort, nbins, out, flags, st));
+    if (tc_f32_supported(p))  // 64-token chunks, like the CUDA-core kernel
+        return cuda_status(tc_f32_prefix(p, q, k, v, part, bp.block_tokens, bp.nblk, perm, bins, msort, nbins, out,
+                                         flags, st));
     return cuda_status(simt_chunked(p, q, k, v, part, bp.block_tokens, bp.nblk, perm, bins, msort,
                                     nbins, out, st));
 }

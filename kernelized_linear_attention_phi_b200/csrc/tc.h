@@ -113,11 +113,21 @@ cudaError_t tc_f32_states(const Problem& p, const void* k, const void* v, int bl
 // Causal outputs of each block from its exclusive prefix record in `prefix`.
 cudaError_t tc_f32_chunked(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
                            int block_tokens, int nblk, void* out, uint32_t* err, cudaStream_t st);
+// Prefix-mask outputs: the queries of bin c (from the binning tables perm,
+// bins, msort of bin_queries with 64-token chunks) answered at chunk c from
+// the block's exclusive prefix record in `prefix`.
+cudaError_t tc_f32_prefix(const Problem& p, const void* q, const void* k, const void* v, const float* prefix,
+                          int block_tokens, int nblk, const int32_t* perm, const int32_t* bins, const int32_t* msort,
+                          int nbins, void* out, uint32_t* err, cudaStream_t st);
 // Non-causal outputs from each head's total S [bh][d][d] and z [bh][d].
 cudaError_t tc_f32_readout(const Problem& p, const void* q, const float* S, const float* z, int block_tokens,
                            int nblk, void* out, uint32_t* err, cudaStream_t st);
 // The same tensor viewed as 2-D [rows = BH * N, d] for row gathers
 // (tile::gather4): 64-column x 1-row boxes, 128-byte swizzle.
 cudaError_t make_row_map(CUtensorMap* map, const void* base, int d, long long rows);
+// Same, for any element type: one-row boxes of box_cols elements (box_cols *
+// elem_bytes = 128 for the 128-byte swizzle).
+cudaError_t make_row_map_box(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes, int d,
+                             long long rows, int box_cols);
 
 }  // namespace la

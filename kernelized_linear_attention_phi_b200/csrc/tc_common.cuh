@@ -127,14 +127,15 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, u
         "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
         : "memory");
 }
-// One gathered query tile of C rows x 64*NB columns, issued by a whole warp:
+// One gathered query tile of C rows x BOXW*NB columns (boxes of 128 bytes:
+// 64 bf16 or 32 fp32 columns), issued by a whole warp:
 // lane l holds the token indices of rows (C/32)*l .. (C/32)*l + C/32 - 1 in
 // tok[] (-1 for a padding row, which fetches token 0 instead), and lanes
-// 0 .. NB*C/4 - 1 each issue one gather4 of four rows of one 64-column box.
-// `dst` is the 1024-byte aligned tile, one [C x 64] box after another;
+// 0 .. NB*C/4 - 1 each issue one gather4 of four rows of one box.
+// `dst` is the 1024-byte aligned tile, one [C x BOXW] box after another;
 // `row0` is the map row of token 0 of the head. The caller posts the
-// expected bytes (C * 64 * NB * 2) on `bar` before calling.
-template <int C, int NB>
+// expected bytes (C * 128 * NB) on `bar` before calling.
+template <int C, int NB, int BOXW = 64>
 __device__ __forceinline__ void gather_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row0,
                                             const int (&tok)[C / 32], int lane) {
     constexpr int R = C / 32, G = C / 4;  // rows per lane, gathers per box
@@ -145,7 +146,7 @@ __device__ __forceinline__ void gather_tile(uint8_t* dst, const CUtensorMap* map
     for (int e = 0; e < 4; ++e) r[e] = __shfl_sync(0xffffffffu, tok[e % R], (4 * g + e) / R);
     if (lane < NB * G) {
         const int bx = lane / G;
-        tma_gather4(dst + bx * (C * 128) + g * 512, map, bar, bx * 64, row0 + max(r[0], 0), row0 + max(r[1], 0),
+        tma_gather4(dst + bx * (C * 128) + g * 512, map, bar, bx * BOXW, row0 + max(r[0], 0), row0 + max(r[1], 0),
                     row0 + max(r[2], 0), row0 + max(r[3], 0));
     }
 }

@@ -54,6 +54,20 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int d, int N, long long
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t make_row_map_box(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes, int d,
+                             long long rows, int box_cols) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return cudaErrorNotSupported;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * elem_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, 1};
+    cuuint32_t es[2] = {1, 1};
+    const CUresult r = fn(map, type, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t make_row_map(CUtensorMap* map, const void* base, int d, long long rows) {
     auto fn = encode_fn();
     if (fn == nullptr) return cudaErrorNotSupported;

@@ -30,11 +30,12 @@ def test_kernel_names_follow_the_count_of_launches():
     assert kn("causal", "bf16", 128, 3) == ["tc_kv_kernel", "state_scan_kernel", "tc_sweep"]
     assert kn("causal", "bf16", 64, 2) == ["tc_kv_kernel", "tc_sweep"]
     assert kn("prefix", "bf16", 64, 3)[-1] == "tc_sweep"
-    # fp32 at d = 64: the split-precision tensor-core kernel's modes; the
-    # fp32 prefix mask, other fp32 sizes and small d run on the CUDA cores
+    # fp32 at d = 64: the split-precision tensor-core kernel's modes; other
+    # fp32 sizes and small d run on the CUDA cores
     assert kn("causal", "f32", 64, 3) == ["tc_f32_kernel<0", "state_scan_kernel", "tc_f32_kernel<1"]
     assert kn("noncausal", "f32", 64, 3) == ["tc_f32_kernel<0", "state_reduce_kernel", "tc_f32_kernel<2"]
-    assert kn("prefix", "f32", 64, 4)[-1] == "chunked_kernel"
+    assert kn("prefix", "f32", 64, 4) == ["tc_f32_kernel<0", "bin_kernel", "state_scan_kernel", "tc_f32_kernel<3"]
+    assert kn("prefix", "f32", 128, 4)[-1] == "chunked_kernel"
     assert kn("causal", "f32", 128, 3) == ["kv_partial_kernel", "state_scan_kernel", "chunked_kernel"]
     assert kn("noncausal", "bf16", 16, 3)[0] == "kv_partial_kernel"
     # a count the table does not know keeps neutral labels
