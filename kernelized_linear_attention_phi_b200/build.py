@@ -24,7 +24,7 @@ LIB = os.path.join(LIBDIR, "libla_b200.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 SOURCES = ["la_api.cu", "device.cu", "simt.cu", "bin.cu", "decode.cu", "tc_host.cu", "tc_kv.cu", "tc_sweep.cu", "tc_sweep_t.cu", "tc_f32.cu",
-           "static_scratch.cu", "timing.cu", "bwd.cu", "tc_bwd.cu", "tc_bwd_causal.cu", "tc_fused.cu"]
+           "static_scratch.cu", "timing.cu", "bwd.cu", "tc_bwd.cu", "tc_bwd_causal.cu", "tc_bwd_causal_t.cu", "tc_fused.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

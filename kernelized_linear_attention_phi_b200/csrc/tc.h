@@ -83,8 +83,9 @@ cudaError_t tc_noncausal_backward(const Problem& p, const void* q, const void* k
                                   const float* S, const float* z, float* part, float* G, float* h, void* dq,
                                   void* dk, void* dv, uint32_t* err, cudaStream_t st);
 
-// First sweep of the causal gradients on tensor cores (tc_bwd_causal.cu;
-// bf16, d = 64, block_tokens a multiple of 64): from the forward's exclusive
+// First sweep of the causal gradients on tensor cores (tc_bwd_causal.cu,
+// tc_bwd_causal_t.cu at d = 128; bf16, d = 64 or 128, block_tokens a
+// multiple of 64): from the forward's exclusive
 // block prefixes, writes dq, gn (bf16 [bh][N][d]), gden (fp32 [bh][N]) and
 // the blocks' own (G, h) records grec[bh*nblk + blk], as bwd_q does.
 bool tc_causal_backward_supported(const Problem& p, int block_tokens);
@@ -96,6 +97,13 @@ cudaError_t tc_causal_backward_q(const Problem& p, const void* q, const void* k,
 cudaError_t tc_causal_backward_kv(const Problem& p, const void* q, const void* k, const void* v, const void* gn,
                                   const float* gden, const float* suffix, int block_tokens, int nblk, void* dk,
                                   void* dv, uint32_t* err, cudaStream_t st);
+// The same two sweeps at d = 128 (tc_bwd_causal_t.cu), bf16, 64-token chunks.
+cudaError_t tc_causal_backward_q_t(const Problem& p, const void* q, const void* k, const void* v, const void* dout,
+                                   const float* prefix, int block_tokens, int nblk, void* dq, void* gn, float* gden,
+                                   float* grec, uint32_t* err, cudaStream_t st);
+cudaError_t tc_causal_backward_kv_t(const Problem& p, const void* q, const void* k, const void* v, const void* gn,
+                                    const float* gden, const float* suffix, int block_tokens, int nblk, void* dk,
+                                    void* dv, uint32_t* err, cudaStream_t st);
 
 // [BH, N, d] bf16 viewed as 3-D for TMA: 64-column x `rows` boxes, 128-byte
 // swizzle, zero fill outside the tensor.

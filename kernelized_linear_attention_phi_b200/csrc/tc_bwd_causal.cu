@@ -971,13 +971,15 @@ cudaError_t launch_cq(const Problem& p, const void* q, const void* k, const void
 }  // namespace
 
 bool tc_causal_backward_supported(const Problem& p, int block_tokens) {
-    return p.dtype == DT_BF16 && p.d == CqCfg::D && block_tokens % CqCfg::C == 0;
+    return p.dtype == DT_BF16 && (p.d == 64 || p.d == 128) && block_tokens % CqCfg::C == 0;
 }
 
 cudaError_t tc_causal_backward_q(const Problem& p, const void* q, const void* k, const void* v, const void* dout,
                                  const float* prefix, int block_tokens, int nblk, void* dq, void* gn, float* gden,
                                  float* grec, uint32_t* err, cudaStream_t st) {
     if (!tc_causal_backward_supported(p, block_tokens)) return cudaErrorInvalidValue;
+    if (p.d == 128)
+        return tc_causal_backward_q_t(p, q, k, v, dout, prefix, block_tokens, nblk, dq, gn, gden, grec, err, st);
     switch (p.phi) {  // one kernel per feature map (see phi8)
         case PHI_RELU1:
             return launch_cq<PHI_RELU1>(p, q, k, v, dout, prefix, block_tokens, nblk, dq, gn, gden, grec, err, st);
@@ -993,6 +995,8 @@ cudaError_t tc_causal_backward_kv(const Problem& p, const void* q, const void* k
                                   const float* gden, const float* suffix, int block_tokens, int nblk, void* dk,
                                   void* dv, uint32_t* err, cudaStream_t st) {
     if (!tc_causal_backward_supported(p, block_tokens)) return cudaErrorInvalidValue;
+    if (p.d == 128)
+        return tc_causal_backward_kv_t(p, q, k, v, gn, gden, suffix, block_tokens, nblk, dk, dv, err, st);
     switch (p.phi) {  // one kernel per feature map (see phi8)
         case PHI_RELU1:
             return launch_ck<PHI_RELU1>(p, q, k, v, gn, gden, suffix, block_tokens, nblk, dk, dv, err, st);
