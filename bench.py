@@ -31,8 +31,8 @@ every call outside the events, W untimed warm-up steps, max over ranks.
 ``e2e`` repeats the step through the plain API calls with pinned host inputs
 copied in and the outputs copied back inside the timed region, the copies of
 one step overlapped with the calls of the previous (separate copy streams,
-double-buffered device tensors); ``e2e.serial_value`` runs every copy and
-call of a step back to back.
+double-buffered device tensors) or run back to back on one stream
+(``e2e.serial_value``), whichever is faster (``e2e.schedule``).
 ``roofline`` is the dominant kernel's: after the timed steps every call is
 replayed from a graph captured with the library's per-kernel timing events
 (la_timing_enable), L2 flushed before each replay, and the kernel with the
@@ -107,7 +107,7 @@ TC_KERNELS = {
                        "tc_bwd_causal_kv_kernel"]},
 }
 SIMT_KERNELS = {
-    "noncausal": {3: ["kv_partial_kernel", "state_reduce_kernel", "readout_kernel"]},
+    "noncausal": {1: ["noncausal_small_kernel"], 3: ["kv_partial_kernel", "state_reduce_kernel", "readout_kernel"]},
     "causal": {3: ["kv_partial_kernel", "state_scan_kernel", "chunked_kernel"]},
     "prefix": {4: ["kv_partial_kernel", "bin_kernel", "state_scan_kernel", "chunked_kernel"]},
     "decode": {1: ["decode_kernel"]},
@@ -137,7 +137,7 @@ KERNEL_ROLE = {"tc_kv_kernel": "kv", "kv_partial_kernel": "kv", "kv_reduce_balan
                "bin_kernel": "bin", "decode_kernel": "decode", "bwd_q_kernel": "bwd_q",
                "bwd_kv_kernel": "bwd_kv", "tc_bwd_q_kernel": "bwd_q", "tc_bwd_kv_kernel": "bwd_kv",
                "tc_bwd_causal_q_kernel": "bwd_q", "tc_bwd_causal_kv_kernel": "bwd_kv",
-               "tc_noncausal_cluster_kernel": "fused", "tc_f32_kernel<0": "kv", "tc_f32_kernel<1": "sweep",
+               "tc_noncausal_cluster_kernel": "fused", "noncausal_small_kernel": "fused", "tc_f32_kernel<0": "kv", "tc_f32_kernel<1": "sweep",
                "tc_f32_kernel<2": "readout", "tc_f32_kernel<3": "sweep"}
 
 
@@ -591,7 +591,8 @@ def measure_case(case, args, rank, world, device, flush, sampler, peak, heads=0)
     torch.cuda.synchronize()
     e2e_serial_s = sum(a.elapsed_time(b) for a, b in e_ev) / 1e3
     # pipelined: step i+1's copies in overlap step i's calls and copies out
-    e2e_s = e2e_pipelined(calls, h_io, Ke, stream) if all(c.form != "decode" for c in calls) else e2e_serial_s
+    pipelinable = all(c.form != "decode" for c in calls)
+    e2e_pipe_s = e2e_pipelined(calls, h_io, Ke, stream) if pipelinable else e2e_serial_s
     del h_io
 
     # each kernel's own duration (per-kernel timing events)
@@ -606,11 +607,15 @@ def measure_case(case, args, rank, world, device, flush, sampler, peak, heads=0)
                 bad_flags[f"{c.name}/{c.form}"] = f
 
     step_ms = sum(per_call_ms)
-    t_s, e2e_s, e2e_serial_s = max_over_ranks([step_ms / 1e3 * K, e2e_s, e2e_serial_s], device)
+    t_s, e2e_pipe_s, e2e_serial_s = max_over_ranks([step_ms / 1e3 * K, e2e_pipe_s, e2e_serial_s], device)
     tokens = sum(c.tokens for c in calls)
     value = aggregate_tokens_per_s(tokens, K, world, t_s)
-    e2e_value = aggregate_tokens_per_s(tokens, Ke, world, e2e_s)
+    # e2e: the faster of the two schedules (small steps: the serial one, whose
+    # single stream has no cross-stream event waits)
+    e2e_value = aggregate_tokens_per_s(tokens, Ke, world, min(e2e_pipe_s, e2e_serial_s))
     e2e_serial = aggregate_tokens_per_s(tokens, Ke, world, e2e_serial_s)
+    e2e_pipe = aggregate_tokens_per_s(tokens, Ke, world, e2e_pipe_s)
+    e2e_schedule = "pipelined" if pipelinable and e2e_pipe_s < e2e_serial_s else "serial"
 
     per_call, cands, launches = {}, [], 0
     for c, ms, ktimes in zip(calls, per_call_ms, kt):
@@ -650,11 +655,13 @@ def measure_case(case, args, rank, world, device, flush, sampler, peak, heads=0)
                                                           if any(c.form == "decode" for c in calls) else ""),
                    "tokens_per_step_per_gpu": tokens},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "serial_value": e2e_serial,
-                "mode": ("pipelined: copies in on one stream, the calls on another, copies out on a third, "
-                         "device tensors double-buffered, so step i+1's inputs load while step i computes and "
-                         "copies out; serial_value runs every copy and call of a step back to back"
-                         if all(c.form != "decode" for c in calls) else
+                "serial_value": e2e_serial, "pipelined_value": e2e_pipe if pipelinable else None,
+                "schedule": e2e_schedule,
+                "mode": ("value = the faster of two schedules of the same copies and calls: pipelined (copies in "
+                         "on one stream, the calls on another, copies out on a third, device tensors "
+                         "double-buffered, so step i+1's inputs load while step i computes and copies out) and "
+                         "serial (every copy and call of a step back to back on one stream)"
+                         if pipelinable else
                          "per decode step: its token copied in, the step, its output copied out")},
         "gpu_launches": launches * K,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",

@@ -110,6 +110,11 @@ __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Hint: moves the 128-byte line holding p towards L2 (no data returned).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Streaming 16-byte global load (read once: do not keep in L1).
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
     uint4 r;

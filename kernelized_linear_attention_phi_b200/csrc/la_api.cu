@@ -258,7 +258,10 @@ la_status la_noncausal(const la_desc* desc, const void* q, const void* k, const 
     LA_TRY(check_device());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     timing_begin(st);
-    // small problems: one kernel, a thread-block cluster per head
+    // small problems: one kernel, a thread-block cluster per head (bf16,
+    // d = 64) or one CTA per head (d <= 32)
+    if (simt_noncausal_small_supported(p))
+        return cuda_status(simt_noncausal_small(p, q, k, v, out, S_out, z_out, st));
     if (tc_noncausal_fused_supported(p))
         return cuda_status(tc_noncausal_fused(p, q, k, v, out, S_out, z_out, at<uint32_t>(ws, 0), st));
     float* S = S_out;

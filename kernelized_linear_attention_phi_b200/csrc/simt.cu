@@ -42,24 +42,24 @@ __device__ __forceinline__ void lds(const float* p, float* o) {
 // ---------------------------------------------------------------------------
 // Partial KV summary over a token range of one head.
 // ---------------------------------------------------------------------------
+template <int D>
+struct KvRange {
+    static constexpr int R = D / 16;                 // S rows and columns per thread
+    static constexpr int TT = 2048 / D;              // tokens per tile (two tiles of K and V: 32 KB)
+};
+
+// Sums phi(K_t) (x) V_t and phi(K_t) over tokens [t0, t1) of one head, in
+// token order, through two shared tiles of TT tokens (sK, sV: 2 x TT x D
+// floats each). Thread (ta, tb) = (tid / 16, tid % 16) holds the R x R block
+// of S at rows ta*R.., columns tb*R.., and z entries ta*R.. .
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads)
-kv_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int N, int tps, int nsplit,
-                  int phi, float* __restrict__ part) {
-    constexpr int R = D / 16;
-    constexpr int kTT = D == 128 ? 16 : 32;              // tokens per tile (static shared memory <= 32 KB)
+__device__ __forceinline__ void kv_range(const T* __restrict__ Kh, const T* __restrict__ Vh, int t0, int t1,
+                                         int phi, float* sK, float* sV, float (&acc)[KvRange<D>::R][KvRange<D>::R],
+                                         float (&zacc)[KvRange<D>::R]) {
+    constexpr int R = KvRange<D>::R, kTT = KvRange<D>::TT;
     constexpr int EPV = Vec16<T>::N, VPR = D / EPV;
     constexpr int NV = kTT * VPR;                        // 16-byte vectors per tile and tensor
     constexpr int PER = (NV + kThreads - 1) / kThreads;  // of them per thread
-    __shared__ __align__(16) float sK[2][kTT * D];
-    __shared__ __align__(16) float sV[2][kTT * D];
-    const int s = blockIdx.x;
-    const long long bh = blockIdx.y;
-    const int t0 = s * tps;
-    const int t1 = min(N, t0 + tps);
-    pdl_wait();
-    const T* Kh = K + bh * (long long)N * D;
-    const T* Vh = V + bh * (long long)N * D;
     const int ta = threadIdx.x / 16, tb = threadIdx.x % 16;
 
     // this thread's vectors of the tile at `base`, held in registers so that
@@ -88,16 +88,16 @@ kv_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int N, int t
             Vec16<T>::unpack(rv[j], fv);
 #pragma unroll
             for (int e = 0; e < EPV; ++e) fk[e] = r < valid ? phi_apply(fk[e], phi) : 0.f;
+            float* dk = sK + buf * kTT * D + r * D + col;
+            float* dv = sV + buf * kTT * D + r * D + col;
 #pragma unroll
             for (int e = 0; e < EPV; e += 4) {
-                *reinterpret_cast<float4*>(&sK[buf][r * D + col + e]) = make_float4(fk[e], fk[e + 1], fk[e + 2], fk[e + 3]);
-                *reinterpret_cast<float4*>(&sV[buf][r * D + col + e]) = make_float4(fv[e], fv[e + 1], fv[e + 2], fv[e + 3]);
+                *reinterpret_cast<float4*>(dk + e) = make_float4(fk[e], fk[e + 1], fk[e + 2], fk[e + 3]);
+                *reinterpret_cast<float4*>(dv + e) = make_float4(fv[e], fv[e + 1], fv[e + 2], fv[e + 3]);
             }
         }
     };
 
-    float acc[R][R];
-    float zacc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         zacc[r] = 0.f;
@@ -113,8 +113,8 @@ kv_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int N, int t
 #pragma unroll 4
         for (int t = 0; t < kTT; ++t) {
             float a[R], bb[R];
-            lds<R>(&sK[buf][t * D + ta * R], a);
-            lds<R>(&sV[buf][t * D + tb * R], bb);
+            lds<R>(sK + buf * kTT * D + t * D + ta * R, a);
+            lds<R>(sV + buf * kTT * D + t * D + tb * R, bb);
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 zacc[r] += a[r];
@@ -126,6 +126,23 @@ kv_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int N, int t
         __syncthreads();
         buf ^= 1;
     }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+kv_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int N, int tps, int nsplit,
+                  int phi, float* __restrict__ part) {
+    constexpr int R = KvRange<D>::R, kTT = KvRange<D>::TT;
+    __shared__ __align__(16) float sK[2 * kTT * D];
+    __shared__ __align__(16) float sV[2 * kTT * D];
+    const int s = blockIdx.x;
+    const long long bh = blockIdx.y;
+    const int t0 = s * tps;
+    const int t1 = min(N, t0 + tps);
+    pdl_wait();
+    float acc[R][R], zacc[R];
+    kv_range<T, D>(K + bh * (long long)N * D, V + bh * (long long)N * D, t0, t1, phi, sK, sV, acc, zacc);
+    const int ta = threadIdx.x / 16, tb = threadIdx.x % 16;
     float* o = part + ((size_t)bh * nsplit + s) * (size_t)(D * D + D);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -202,24 +219,13 @@ constexpr size_t readout_smem() {
     return sizeof(float) * ((size_t)D * D + D + 64 * (D + 4) + 64);
 }
 
+// Outputs of query rows row0 .. row0 + 63 of one head from S, z in shared
+// memory (sS [D x D], sz [D]); sQ and sDen are the tile's scratch.
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads)
-readout_kernel(const T* __restrict__ Q, const float* __restrict__ S, const float* __restrict__ z,
-               T* __restrict__ out, int N, int phi, int normalize) {
+__device__ __forceinline__ void readout_rows(const T* __restrict__ Qh, T* __restrict__ Oh, int row0, int N,
+                                             int phi, int normalize, const float* sS, const float* sz,
+                                             float* sQ, float* sDen) {
     constexpr int TQ = 64, LDQ = D + 4, RC = D / 16, RT = TQ / 16;
-    extern __shared__ __align__(16) float sm[];
-    float* sS = sm;
-    float* sz = sS + D * D;
-    float* sQ = sz + D;
-    float* sDen = sQ + TQ * LDQ;
-    const int tile = blockIdx.x;
-    const long long bh = blockIdx.y;
-    pdl_wait();
-    const float4* S4 = reinterpret_cast<const float4*>(S + (size_t)bh * D * D);
-    for (int e = threadIdx.x; e < D * D / 4; e += kThreads) reinterpret_cast<float4*>(sS)[e] = S4[e];
-    for (int e = threadIdx.x; e < D; e += kThreads) sz[e] = z[(size_t)bh * D + e];
-    const int row0 = tile * TQ;
-    const T* Qh = Q + bh * (long long)N * D;
     tile_to_smem<T, D, LDQ>(sQ, Qh + (long long)row0 * D, TQ, min(TQ, N - row0), true, phi);
     __syncthreads();
     if (normalize && threadIdx.x < TQ) {
@@ -245,7 +251,6 @@ readout_kernel(const T* __restrict__ Q, const float* __restrict__ S, const float
         }
     }
     __syncthreads();
-    T* Oh = out + bh * (long long)N * D;
 #pragma unroll
     for (int i = 0; i < RT; ++i) {
         const int row = row0 + tt * RT + i;
@@ -254,6 +259,73 @@ readout_kernel(const T* __restrict__ Q, const float* __restrict__ S, const float
 #pragma unroll
         for (int c = 0; c < RC; ++c)
             Oh[(long long)row * D + tc * RC + c] = from_f32<T>(normalize ? acc[i][c] / den : acc[i][c]);
+    }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+readout_kernel(const T* __restrict__ Q, const float* __restrict__ S, const float* __restrict__ z,
+               T* __restrict__ out, int N, int phi, int normalize) {
+    constexpr int TQ = 64, LDQ = D + 4;
+    extern __shared__ __align__(16) float sm[];
+    float* sS = sm;
+    float* sz = sS + D * D;
+    float* sQ = sz + D;
+    float* sDen = sQ + TQ * LDQ;
+    const int tile = blockIdx.x;
+    const long long bh = blockIdx.y;
+    pdl_wait();
+    const float4* S4 = reinterpret_cast<const float4*>(S + (size_t)bh * D * D);
+    for (int e = threadIdx.x; e < D * D / 4; e += kThreads) reinterpret_cast<float4*>(sS)[e] = S4[e];
+    for (int e = threadIdx.x; e < D; e += kThreads) sz[e] = z[(size_t)bh * D + e];
+    readout_rows<T, D>(Q + bh * (long long)N * D, out + bh * (long long)N * D, tile * TQ, N, phi, normalize,
+                       sS, sz, sQ, sDen);
+}
+
+// ---------------------------------------------------------------------------
+// Small non-causal problems in one launch: one CTA per head forms S and z
+// over all of the head's keys (kv_range with a single split), keeps them in
+// shared memory (and writes them out when asked), then reads out all of the
+// head's queries 64 rows at a time (readout_rows). Replaces the three
+// dependent launches (partials, reduction, readout) where a head is short.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+noncausal_small_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V,
+                       T* __restrict__ out, float* __restrict__ S_out, float* __restrict__ z_out, int N,
+                       int phi, int normalize) {
+    constexpr int R = KvRange<D>::R, kTT = KvRange<D>::TT, TQ = 64, LDQ = D + 4;
+    __shared__ __align__(16) float sK[2 * kTT * D];
+    __shared__ __align__(16) float sV[2 * kTT * D];
+    extern __shared__ __align__(16) float sm[];
+    float* sS = sm;
+    float* sz = sS + D * D;
+    float* sQ = sz + D;
+    float* sDen = sQ + TQ * LDQ;
+    const long long bh = blockIdx.x;
+    pdl_wait();
+    const T* Qh = Q + bh * (long long)N * D;
+    // the head's queries (at most 128 KB) move towards L2 while S and z form
+    for (long long off = threadIdx.x * 128LL; off < (long long)N * D * (long long)sizeof(T); off += kThreads * 128LL)
+        prefetch_l2(reinterpret_cast<const char*>(Qh) + off);
+    float acc[R][R], zacc[R];
+    kv_range<T, D>(K + bh * (long long)N * D, V + bh * (long long)N * D, 0, N, phi, sK, sV, acc, zacc);
+    const int ta = threadIdx.x / 16, tb = threadIdx.x % 16;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+        for (int c = 0; c < R; ++c) sS[(ta * R + r) * D + tb * R + c] = acc[r][c];
+        if (tb == 0) sz[ta * R + r] = zacc[r];
+        if (S_out != nullptr) {
+#pragma unroll
+            for (int c = 0; c < R; ++c) S_out[(size_t)bh * D * D + (ta * R + r) * D + tb * R + c] = acc[r][c];
+            if (tb == 0) z_out[(size_t)bh * D + ta * R + r] = zacc[r];
+        }
+    }
+    T* Oh = out + bh * (long long)N * D;
+    for (int row0 = 0; row0 < N; row0 += TQ) {
+        __syncthreads();  // S, z written; the previous tile's sQ and sDen read
+        readout_rows<T, D>(Qh, Oh, row0, N, phi, normalize, sS, sz, sQ, sDen);
     }
 }
 
@@ -492,6 +564,21 @@ cudaError_t launch_readout(const Problem& p, const void* q, const float* S, cons
 }
 
 template <typename T, int D>
+cudaError_t launch_noncausal_small(const Problem& p, const void* q, const void* k, const void* v, void* out,
+                                   float* S_out, float* z_out, cudaStream_t st) {
+    if constexpr (D > 32) {
+        return cudaErrorInvalidValue;
+    } else {
+        constexpr size_t smem = readout_smem<D>();
+        cudaError_t e = ensure_smem<noncausal_small_kernel<T, D>>(smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(noncausal_small_kernel<T, D>, dim3((unsigned)p.bh()), dim3(kThreads), smem, st,
+                          static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+                          static_cast<T*>(out), S_out, z_out, p.N, p.phi, p.normalize);
+    }
+}
+
+template <typename T, int D>
 cudaError_t launch_chunked(const Problem& p, const void* q, const void* k, const void* v,
                            const float* prefix, int block_tokens, int nblk, const int32_t* perm,
                            const int32_t* bin_start, const int32_t* m, int nbins, void* out,
@@ -541,6 +628,14 @@ cudaError_t launch_chunked(const Problem& p, const void* q, const void* k, const
 cudaError_t simt_kv_partial(const Problem& p, const void* k, const void* v, int tps, int nsplit,
                             float* part, cudaStream_t st) {
     LA_DISPATCH(p, launch_kv_partial, p, k, v, tps, nsplit, part, st);
+}
+
+bool simt_noncausal_small_supported(const Problem& p) { return p.d <= 32 && p.N <= kSmallHeadTokens; }
+
+cudaError_t simt_noncausal_small(const Problem& p, const void* q, const void* k, const void* v, void* out,
+                                 float* S_out, float* z_out, cudaStream_t st) {
+    if (!simt_noncausal_small_supported(p)) return cudaErrorInvalidValue;
+    LA_DISPATCH(p, launch_noncausal_small, p, q, k, v, out, S_out, z_out, st);
 }
 
 cudaError_t simt_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,

@@ -38,6 +38,7 @@ def test_kernel_names_follow_the_count_of_launches():
     assert kn("prefix", "f32", 128, 4)[-1] == "chunked_kernel"
     assert kn("causal", "f32", 128, 3) == ["kv_partial_kernel", "state_scan_kernel", "chunked_kernel"]
     assert kn("noncausal", "bf16", 16, 3)[0] == "kv_partial_kernel"
+    assert kn("noncausal", "f32", 16, 1) == ["noncausal_small_kernel"]  # short heads, d <= 32
     # a count the table does not know keeps neutral labels
     assert kn("causal", "bf16", 64, 7) == [f"kernel{i}" for i in range(7)]
 
@@ -63,6 +64,7 @@ def test_kernel_bytes():
     assert kb("causal", "state_scan_kernel") == 0
     assert kb("noncausal", "tc_readout_kernel") == 2 * t + st
     assert kb("noncausal", "tc_noncausal_cluster_kernel") == 4 * t
+    assert kb("noncausal", "noncausal_small_kernel") == 4 * t
     assert kb("prefix", "bin_kernel") == B * N * 4
     assert kb("decode", "decode_kernel") == 2 * st + 4 * B * H * d * e
     assert kb("noncausal_bwd", "tc_noncausal_cluster_kernel") == 2 * t

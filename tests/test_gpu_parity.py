@@ -47,6 +47,34 @@ def test_noncausal(dt, d, N, phi, normalize):
     assert oracle.max_row_rel_err(f64(z)[..., None, :], z_ref[..., None, :]) < _state_tol(dt, phi)
 
 
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [16, 32])
+@pytest.mark.parametrize("N", [64, 1024, 1025, 2500])
+def test_noncausal_short_heads_in_one_launch(dt, d, N):
+    """d <= 32: heads of at most 1024 tokens run in one launch (one CTA per
+    head forms S and z, then reads out its queries), longer heads through the
+    split partials, their reduction and the readout; the launch count says
+    which path ran, and both match the oracle, S and z included."""
+    q, k, v = qkv(3, 5, N, d, dt, seed=7 * N + d)
+    S = torch.empty(3, 5, d, d, device="cuda")
+    z = torch.empty(3, 5, d, device="cuda")
+    la.la_timing_enable(True)
+    try:
+        out = la.la_noncausal(q, k, v, S_out=S, z_out=z)
+        launches = len(la.la_timing_read())
+    finally:
+        la.la_timing_enable(False)
+    assert launches == (1 if N <= 1024 else 3)
+    Q, K, V = f64(q), f64(k), f64(v)
+    ref = oracle.batched(oracle.noncausal, Q, K, V, phi_kind="relu1", normalize=True)
+    assert oracle.max_row_rel_err(f64(out), ref) < TOL[DT[dt]]
+    S_ref, z_ref = oracle.kv_summary_batched(K, V, "relu1")
+    assert oracle.max_row_rel_err(f64(S), S_ref) < _state_tol(dt, "relu1")
+    assert oracle.max_row_rel_err(f64(z)[..., None, :], z_ref[..., None, :]) < _state_tol(dt, "relu1")
+    # without S_out / z_out the outputs are the same, bit for bit
+    assert torch.equal(la.la_noncausal(q, k, v), out)
+
+
 def _state_tol(dt, phi):
     """Tolerance on a KV summary. bf16 inputs: relu+1 and the identity are
     exact in bf16 (relu(K) and K are bf16 values; the +1 is added exactly in
