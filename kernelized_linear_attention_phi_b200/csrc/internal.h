@@ -45,11 +45,10 @@ cudaError_t state_exclusive_scan(const Problem& p, float* part, int nblk, float*
 // out = phi(q) S / (phi(q).z) (or numerator only) for every token.
 cudaError_t simt_readout(const Problem& p, const void* q, const float* S, const float* z, void* out,
                          cudaStream_t st);
-// Non-causal outputs of heads of at most kSmallHeadTokens tokens at d <= 32
-// in one launch (one CTA per head: S and z, then the readout); S_out / z_out
-// (both or neither) also receive S and z. simt_noncausal_small_supported
-// tells whether a problem qualifies.
-constexpr int kSmallHeadTokens = 1024;
+// Non-causal outputs of short heads at d <= 32 in one launch (one CTA per
+// head: S and z, then the readout); S_out / z_out (both or neither) also
+// receive S and z. simt_noncausal_small_supported tells whether a problem
+// qualifies on the current device (plan::small_noncausal).
 bool simt_noncausal_small_supported(const Problem& p);
 cudaError_t simt_noncausal_small(const Problem& p, const void* q, const void* k, const void* v, void* out,
                                  float* S_out, float* z_out, cudaStream_t st);

@@ -62,19 +62,31 @@ cudaError_t launch_cluster_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
     return e;
 }
 
-// Raises a kernel's dynamic shared-memory limit once per device (the
-// attribute is per device context). Safe to call on every launch. The
-// kernel is a template argument so that each kernel keeps its own flag.
+// Raises a kernel's dynamic shared-memory cap once per device (the attribute
+// is per device context) to all of the opt-in shared memory its static
+// shared memory leaves, so that every launch whose static plus dynamic
+// shared memory fits the device passes, whatever the size of earlier
+// launches (the cap is not raised again later). Safe to call on every
+// launch. The kernel is a template argument so that each kernel keeps its
+// own flag.
 template <auto kernel>
 cudaError_t ensure_smem(size_t bytes) {
     static std::atomic<uint64_t> done{0};
-    if (bytes <= 48 * 1024) return cudaSuccess;
+    if (bytes == 0) return cudaSuccess;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const uint64_t bit = 1ull << (dev & 63);
     if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return e;
+    int optin = 0;
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    const int cap = optin - (int)fa.sharedSizeBytes;
+    if (cap < 0 || (size_t)cap < bytes) return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
     if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
     return e;
 }

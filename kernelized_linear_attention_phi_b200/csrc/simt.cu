@@ -13,8 +13,10 @@
 // mask).
 
 #include "common.cuh"
+#include "device.h"
 #include "internal.h"
 #include "launch_util.h"
+#include "plan.h"
 
 namespace la {
 namespace {
@@ -214,18 +216,19 @@ __global__ void state_scan_kernel(float* __restrict__ part, int nblk, int D,
 // ---------------------------------------------------------------------------
 // Readout: out_i = phi(q_i) S / (phi(q_i).z).
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int TQ = 64>
 constexpr size_t readout_smem() {
-    return sizeof(float) * ((size_t)D * D + D + 64 * (D + 4) + 64);
+    return sizeof(float) * ((size_t)D * D + D + TQ * (D + 4) + TQ);
 }
 
-// Outputs of query rows row0 .. row0 + 63 of one head from S, z in shared
-// memory (sS [D x D], sz [D]); sQ and sDen are the tile's scratch.
-template <typename T, int D>
+// Outputs of query rows row0 .. row0 + TQ - 1 of one head from S, z in
+// shared memory (sS [D x D], sz [D]); sQ and sDen are the tile's scratch.
+template <typename T, int D, int TQ = 64>
 __device__ __forceinline__ void readout_rows(const T* __restrict__ Qh, T* __restrict__ Oh, int row0, int N,
                                              int phi, int normalize, const float* sS, const float* sz,
                                              float* sQ, float* sDen) {
-    constexpr int TQ = 64, LDQ = D + 4, RC = D / 16, RT = TQ / 16;
+    constexpr int LDQ = D + 4, RC = D / 16, RT = TQ / 16;
+    static_assert(TQ <= kThreads, "one thread per row for the denominators");
     tile_to_smem<T, D, LDQ>(sQ, Qh + (long long)row0 * D, TQ, min(TQ, N - row0), true, phi);
     __syncthreads();
     if (normalize && threadIdx.x < TQ) {
@@ -289,16 +292,23 @@ readout_kernel(const T* __restrict__ Q, const float* __restrict__ S, const float
 // head's queries 64 rows at a time (readout_rows). Replaces the three
 // dependent launches (partials, reduction, readout) where a head is short.
 // ---------------------------------------------------------------------------
+// query rows per readout pass of the one-launch kernel: all of a 256-token
+// head at d = 16 (16 rows per thread)
+template <int D>
+struct SmallTQ {
+    static constexpr int value = D <= 16 ? 256 : 128;
+};
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 noncausal_small_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V,
                        T* __restrict__ out, float* __restrict__ S_out, float* __restrict__ z_out, int N,
                        int phi, int normalize) {
-    constexpr int R = KvRange<D>::R, kTT = KvRange<D>::TT, TQ = 64, LDQ = D + 4;
-    __shared__ __align__(16) float sK[2 * kTT * D];
-    __shared__ __align__(16) float sV[2 * kTT * D];
+    constexpr int R = KvRange<D>::R, kTT = KvRange<D>::TT, TQ = SmallTQ<D>::value, LDQ = D + 4;
     extern __shared__ __align__(16) float sm[];
-    float* sS = sm;
+    float* sK = sm;                // two K tiles, then two V tiles
+    float* sV = sK + 2 * kTT * D;
+    float* sS = sV + 2 * kTT * D;
     float* sz = sS + D * D;
     float* sQ = sz + D;
     float* sDen = sQ + TQ * LDQ;
@@ -325,7 +335,7 @@ noncausal_small_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T
     T* Oh = out + bh * (long long)N * D;
     for (int row0 = 0; row0 < N; row0 += TQ) {
         __syncthreads();  // S, z written; the previous tile's sQ and sDen read
-        readout_rows<T, D>(Qh, Oh, row0, N, phi, normalize, sS, sz, sQ, sDen);
+        readout_rows<T, D, TQ>(Qh, Oh, row0, N, phi, normalize, sS, sz, sQ, sDen);
     }
 }
 
@@ -569,7 +579,7 @@ cudaError_t launch_noncausal_small(const Problem& p, const void* q, const void* 
     if constexpr (D > 32) {
         return cudaErrorInvalidValue;
     } else {
-        constexpr size_t smem = readout_smem<D>();
+        constexpr size_t smem = 4 * sizeof(float) * KvRange<D>::TT * D + readout_smem<D, SmallTQ<D>::value>();
         cudaError_t e = ensure_smem<noncausal_small_kernel<T, D>>(smem);
         if (e != cudaSuccess) return e;
         return launch_pdl(noncausal_small_kernel<T, D>, dim3((unsigned)p.bh()), dim3(kThreads), smem, st,
@@ -630,7 +640,7 @@ cudaError_t simt_kv_partial(const Problem& p, const void* k, const void* v, int 
     LA_DISPATCH(p, launch_kv_partial, p, k, v, tps, nsplit, part, st);
 }
 
-bool simt_noncausal_small_supported(const Problem& p) { return p.d <= 32 && p.N <= kSmallHeadTokens; }
+bool simt_noncausal_small_supported(const Problem& p) { return plan::small_noncausal(p, device_sms()); }
 
 cudaError_t simt_noncausal_small(const Problem& p, const void* q, const void* k, const void* v, void* out,
                                  float* S_out, float* z_out, cudaStream_t st) {
