@@ -309,18 +309,35 @@ tc_sweep_t_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant_
             *reinterpret_cast<uint4*>(stages + s * CF::STAGE + CF::OFF_K + bx * CF::KBOX + r * 128 + q16 * 16) =
                 make_uint4(0, 0, 0, 0);
         }
-        // seed S^T with the block's prefix record (S stored [d_k][d_v])
+        // seed S^T with the block's prefix record (S stored [d_k][d_v]); the
+        // loads of four records are in flight at a time (one L2 round trip
+        // per four records, not per record), the sum keeps block order
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 16) {
+            float f[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) f[e] = 0.f;
+            int rb = 0;
+#pragma unroll 1
+            for (; rb + 4 <= npre; rb += 4) {
+                float t[4][16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) t[j][e] = pre[(rb + j) * kRec + (size_t)(c0 + e) * D + a];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) f[e] += t[j][e];
+            }
+#pragma unroll 1
+            for (; rb < npre; ++rb) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) f[e] += pre[rb * kRec + (size_t)(c0 + e) * D + a];
+            }
             uint32_t r[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) r[e] = 0u;
-#pragma unroll 1
-            for (int rb = 0; rb < npre; ++rb) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    r[e] = __float_as_uint(__uint_as_float(r[e]) + pre[rb * kRec + (size_t)(c0 + e) * D + a]);
-            }
+            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(f[e]);
             tmem_st16(tmem + CF::COL_S + lane_base + c0, r);
         }
         tmem_st_wait();
