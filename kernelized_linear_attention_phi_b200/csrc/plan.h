@@ -80,12 +80,12 @@ inline KvBalanced kv_balanced_plan(const Problem& p, int sms, int per_sm = 1) {
 
 // Non-causal heads at d <= 32 answered in one launch, one CTA per head (the
 // KV sum, then the readout, each a loop over the head's tokens in its CTA):
-// heads of at most 256 tokens always, heads of at most 1024 tokens when the
-// heads alone fill the GPU (two per SM), where splitting a head would add no
-// parallelism. Other problems take the split partials, their reduction and
-// the readout.
+// heads of at most 256 tokens, whose three-launch form is all fixed cost.
+// Longer heads take the split partials, their reduction and the readout,
+// which spreads a head's queries over many CTAs.
 inline bool small_noncausal(const Problem& p, int sms) {
-    return p.d <= 32 && (p.N <= 256 || (p.N <= 1024 && p.bh() >= 2LL * sms));
+    (void)sms;
+    return p.d <= 32 && p.N <= 256;
 }
 
 }  // namespace plan

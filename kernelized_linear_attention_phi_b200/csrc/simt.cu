@@ -293,7 +293,7 @@ readout_kernel(const T* __restrict__ Q, const float* __restrict__ S, const float
 // dependent launches (partials, reduction, readout) where a head is short.
 // ---------------------------------------------------------------------------
 // query rows per readout pass of the one-launch kernel: all of a 256-token
-// head at d = 16 (16 rows per thread)
+// head at d = 16 (16 rows per thread), half of it at d = 32
 template <int D>
 struct SmallTQ {
     static constexpr int value = D <= 16 ? 256 : 128;
@@ -315,7 +315,7 @@ noncausal_small_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T
     const long long bh = blockIdx.x;
     pdl_wait();
     const T* Qh = Q + bh * (long long)N * D;
-    // the head's queries (at most 128 KB) move towards L2 while S and z form
+    // the head's queries (at most 32 KB) move towards L2 while S and z form
     for (long long off = threadIdx.x * 128LL; off < (long long)N * D * (long long)sizeof(T); off += kThreads * 128LL)
         prefetch_l2(reinterpret_cast<const char*>(Qh) + off);
     float acc[R][R], zacc[R];

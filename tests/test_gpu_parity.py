@@ -49,13 +49,12 @@ def test_noncausal(dt, d, N, phi, normalize):
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
 @pytest.mark.parametrize("d", [16, 32])
-@pytest.mark.parametrize("B,H,N", [(3, 5, 64), (3, 5, 256), (3, 5, 257), (3, 5, 2500), (4, 80, 1000), (4, 80, 1025)])
+@pytest.mark.parametrize("B,H,N", [(3, 5, 64), (3, 5, 256), (3, 5, 257), (3, 5, 2500), (4, 80, 200)])
 def test_noncausal_short_heads_in_one_launch(dt, d, B, H, N):
-    """d <= 32: heads of at most 256 tokens, or of at most 1024 when the heads
-    fill the GPU at two per SM, run in one launch (one CTA per head forms S and
-    z, then reads out its queries); others through the split partials, their
-    reduction and the readout. The launch count says which path ran, and both
-    match the oracle, S and z included."""
+    """d <= 32: heads of at most 256 tokens run in one launch (one CTA per head
+    forms S and z, then reads out its queries); longer heads through the split
+    partials, their reduction and the readout. The launch count says which
+    path ran, and both match the oracle, S and z included."""
     q, k, v = qkv(B, H, N, d, dt, seed=7 * N + d)
     S = torch.empty(B, H, d, d, device="cuda")
     z = torch.empty(B, H, d, device="cuda")
@@ -65,8 +64,7 @@ def test_noncausal_short_heads_in_one_launch(dt, d, B, H, N):
         launches = len(la.la_timing_read())
     finally:
         la.la_timing_enable(False)
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    assert launches == (1 if N <= 256 or (N <= 1024 and B * H >= 2 * sms) else 3)
+    assert launches == (1 if N <= 256 else 3)
     Q, K, V = f64(q), f64(k), f64(v)
     ref = oracle.batched(oracle.noncausal, Q, K, V, phi_kind="relu1", normalize=True)
     assert oracle.max_row_rel_err(f64(out), ref) < TOL[DT[dt]]
