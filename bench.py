@@ -486,6 +486,16 @@ def aggregate_tokens_per_s(tokens_per_step, steps, world, seconds):
     return tokens_per_step * steps * world / seconds
 
 
+def e2e_choice(pipelined_s, serial_s, pipelinable):
+    """The end-to-end figure is the faster of the two schedules of the same
+    copies and calls (small steps: the serial one, whose single stream has no
+    cross-stream event waits); decode steps have only the serial one.
+    Returns (schedule, seconds)."""
+    if pipelinable and pipelined_s < serial_s:
+        return "pipelined", pipelined_s
+    return "serial", serial_s
+
+
 def kernel_times(call, flush, reps):
     """Mean duration (ms) of each kernel the call launches, from the
     library's timing events over `reps` replays of a graph of the call, L2
@@ -610,12 +620,10 @@ def measure_case(case, args, rank, world, device, flush, sampler, peak, heads=0)
     t_s, e2e_pipe_s, e2e_serial_s = max_over_ranks([step_ms / 1e3 * K, e2e_pipe_s, e2e_serial_s], device)
     tokens = sum(c.tokens for c in calls)
     value = aggregate_tokens_per_s(tokens, K, world, t_s)
-    # e2e: the faster of the two schedules (small steps: the serial one, whose
-    # single stream has no cross-stream event waits)
-    e2e_value = aggregate_tokens_per_s(tokens, Ke, world, min(e2e_pipe_s, e2e_serial_s))
+    e2e_schedule, e2e_s = e2e_choice(e2e_pipe_s, e2e_serial_s, pipelinable)
+    e2e_value = aggregate_tokens_per_s(tokens, Ke, world, e2e_s)
     e2e_serial = aggregate_tokens_per_s(tokens, Ke, world, e2e_serial_s)
     e2e_pipe = aggregate_tokens_per_s(tokens, Ke, world, e2e_pipe_s)
-    e2e_schedule = "pipelined" if pipelinable and e2e_pipe_s < e2e_serial_s else "serial"
 
     per_call, cands, launches = {}, [], 0
     for c, ms, ktimes in zip(calls, per_call_ms, kt):

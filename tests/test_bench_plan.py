@@ -75,6 +75,13 @@ def test_kernel_bytes():
     assert kb("causal_bwd", "tc_bwd_causal_kv_kernel") == 5 * t
 
 
+def test_e2e_takes_the_faster_schedule():
+    assert bench.e2e_choice(0.030, 0.040, True) == ("pipelined", 0.030)
+    assert bench.e2e_choice(0.050, 0.040, True) == ("serial", 0.040)
+    # decode: one schedule only, whatever the numbers say
+    assert bench.e2e_choice(0.010, 0.040, False) == ("serial", 0.040)
+
+
 def test_reference_arm_runs_on_the_host_and_prints_one_line():
     """--impl reference times the oracle on a sample of the headline case,
     on the host alone, and prints the contract's JSON line."""
